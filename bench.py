@@ -1,0 +1,409 @@
+#!/usr/bin/env python
+"""Benchmark of the quantized-KV decode path on B200 (one JSON line on rank 0).
+
+Workload (3-bit prod TurboQuant, d = 128): one GQA decode step over a
+compressed cache -- batch 1, 8 KV heads, 32 query heads, context 32768, K and V
+each 2-bit Lloyd-Max MSE + 1-bit QJL sketch (m = 128), fp16 norms and residual
+norms; bf16 K/V with per-(head, channel) std ~ LogNormal(0, 0.5) and 2 outlier
+channels x10 per head. A step is the whole hot path for one new token:
+tq_append(K) -> tq_append(V) (norm, rotate, bucketize, pack, QJL sign-pack of
+the new token) -> tq_attn_decode (query rotation, scores, online softmax,
+value accumulate, combine). The step is captured once in a CUDA graph; each
+timed step replays it. `len` is reset between steps (outside the timed
+bracket) so every step attends over exactly 32768 tokens; L2 is flushed
+between steps (the packed cache, 27 MB, would otherwise sit in the 126 MB L2).
+
+value   = packed K+V bytes read by the attention per step / device time per step (GB/s)
+e2e     = same metric through the C ABI with host buffers: per step the new
+          token and the queries are copied from pinned host memory and the
+          attention output is copied back, inside the timed bracket.
+Multi-GPU (--gpus N under torchrun): every rank runs its own independent
+instance of the workload (weak scaling, no collective on the data path); the
+reported time is the max over ranks.
+"""
+
+import argparse
+import json
+import os
+import subprocess
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+METRIC = "packed-KV GB/s and keys scored/sec (3-bit, d=128) vs HBM roofline; vectors encoded/sec"
+W = dict(B=1, Hkv=8, Hq=32, L=32768, d=128, bits=3, m=128, seed_k_handle=0, seed_v_handle=1,
+         seed_k=2, seed_v=3, seed_q=4)
+PACKED_BYTES_PER_TOKEN = 2 * (32 + 16 + 2 + 2)   # K and V: 2-bit codes + sign bits + fp16 norm + fp16 rnorm
+WORKLOAD_NAME = ("GQA decode step, TurboQuant prod 3-bit (2-bit Lloyd-Max + 1-bit QJL m=128), d=128, "
+                 "B=1, 8 KV heads / 32 query heads, context 32768, bf16 K/V with lognormal channel scales "
+                 "and 2 outlier channels")
+FALLBACK_HBM_GBS = 6650.0
+
+
+def parse_args():
+    p = argparse.ArgumentParser()
+    p.add_argument("--gpus", type=int, default=1)
+    p.add_argument("--steps", type=int, default=200)
+    p.add_argument("--warmup", type=int, default=10)
+    p.add_argument("--impl", choices=["tq", "reference"], default="tq")
+    p.add_argument("--no-cpu-baseline", action="store_true")
+    return p.parse_args()
+
+
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(path):
+        with open(path) as fh:
+            return json.load(fh), "measured"
+    return {"hbm_gbs": FALLBACK_HBM_GBS}, "fallback"
+
+
+# --------------------------------------------------------------------- clocks
+
+class ClockSampler:
+    """Samples SM clocks and throttle reasons with nvidia-smi while running."""
+
+    QUERY = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+             "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+             "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_id):
+        self.gpu_id = gpu_id
+        self.proc = None
+        self.lines = []
+
+    def start(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", self.gpu_id, f"--query-gpu={self.QUERY}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=subprocess.PIPE, stderr=subprocess.DEVNULL, text=True)
+            self.thread = threading.Thread(target=self._read, daemon=True)
+            self.thread.start()
+            time.sleep(0.3)
+        except OSError:
+            self.proc = None
+
+    def _read(self):
+        for line in self.proc.stdout:
+            self.lines.append(line.strip())
+
+    def stop(self):
+        if not self.proc:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        time.sleep(0.2)
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for ln in self.lines:
+            f = [x.strip() for x in ln.split(",")]
+            if len(f) < 7:
+                continue
+            try:
+                sm.append(float(f[0]))
+                mx = float(f[1])
+            except ValueError:
+                continue
+            for name, val in zip(names, f[3:7]):
+                if val.lower() in ("active", "1", "yes"):
+                    reasons.add(name)
+        sm.sort()
+        return {"sm_mhz": sm[len(sm) // 2] if sm else None, "sm_max_mhz": mx, "reasons": sorted(reasons),
+                "samples": len(sm)}
+
+
+# --------------------------------------------------------------------- oracle (CPU) leg
+
+class OracleSample:
+    """The CPU oracle on a bounded sample of the same workload: `group_heads` KV head(s)
+    of the decode step (encode of the new K and V token, then attention of the group's
+    4 query heads over 32768 cached tokens). Setup (the prefill encode) is untimed."""
+
+    def __init__(self, group_heads=1):
+        import numpy as np
+        from embedding_vector_quantization_b200 import synth
+        from oracle import codebook, ops, quant, rotation
+        self.np, self.ops, self.quant = np, ops, quant
+        d, m, L = W["d"], W["m"], W["L"]
+        G = W["Hq"] // W["Hkv"]
+        self.gh, self.d, self.m, self.L = group_heads, d, m, L
+        self.P = [rotation.rotation(d, W["seed_k_handle"], m), rotation.rotation(d, W["seed_v_handle"], m)]
+        self.c, self.beta = codebook.lloyd_max(d, W["bits"] - 1)
+        self.X = [synth.outlier_kv(seed=W["seed_k"])[:, :group_heads].double().numpy(),
+                  synth.outlier_kv(seed=W["seed_v"])[:, :group_heads].double().numpy()]
+        self.q = synth.queries((1, W["Hq"], d), W["seed_q"]).double().numpy()[:, : G * group_heads]
+        self.caches = [self._encode(self.X[i][:, :, : L - 1], *self.P[i]) for i in range(2)]
+
+    def _encode(self, x, P, S):
+        e = self.quant.encode_prod(x.reshape(-1, self.d), P, S, self.c, self.beta, "f16")
+        sh = (1, self.gh, x.shape[2])
+        return {"idx": e["idx"].reshape(sh + (self.d,)), "n": e["n_stored"].reshape(sh),
+                "sigma": e["sigma"].reshape(sh + (self.m,)), "rnorm": e["rnorm_stored"].reshape(sh),
+                "Pi": P, "S": S, "c": self.c}
+
+    def step(self):
+        """One decode step; returns the packed bytes the attention reads."""
+        full = []
+        for i in range(2):
+            new = self._encode(self.X[i][:, :, self.L - 1:self.L], *self.P[i])
+            f = dict(self.caches[i])
+            for key in ("idx", "n", "sigma", "rnorm"):
+                f[key] = self.np.concatenate([self.caches[i][key], new[key]], axis=2)
+            full.append(f)
+        self.ops.decode_attention(self.q, full[0], full[1], [self.L], 1.0 / self.np.sqrt(self.d))
+        return self.L * PACKED_BYTES_PER_TOKEN * self.gh
+
+
+def blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        return max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        return os.cpu_count()
+
+
+def oracle_decode_sample(budget_s=12.0):
+    """Times OracleSample.step repeatedly for about `budget_s` seconds: (GB/s, seconds, steps, threads)."""
+    s = OracleSample()
+    s.step()
+    reps, nbytes, t0 = 0, 0, time.perf_counter()
+    while True:
+        nbytes += s.step()
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return nbytes / el / 1e9, el, reps, blas_threads()
+
+
+def run_reference(args):
+    """--impl reference: the CPU oracle as it stands, on the same workload and metric."""
+    rank = int(os.environ.get("RANK", "0"))
+    if rank != 0:
+        return
+    s = OracleSample()
+    for _ in range(args.warmup):
+        s.step()
+    t_total, nbytes = 0.0, 0
+    for _ in range(args.steps):
+        t0 = time.perf_counter()
+        nbytes += s.step()
+        t_total += time.perf_counter() - t0
+    value = nbytes / t_total / 1e9 if t_total > 0 else 0.0
+    threads = blas_threads()
+    sample = "each step: 1 of 8 KV-head groups (new-token encode + attention of 4 query heads over 32768 tokens)"
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / max(args.steps, 1),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD_NAME, "sample": sample},
+            "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
+            "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    print(json.dumps(line), flush=True)
+
+
+# --------------------------------------------------------------------- GPU leg
+
+def run_tq(args):
+    import torch
+    import torch.distributed as dist
+    import embedding_vector_quantization_b200 as tq
+    from embedding_vector_quantization_b200 import synth
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    torch.cuda.set_device(local)
+    if world > 1:
+        import datetime
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local))
+    dev = torch.device("cuda", local)
+    B, Hkv, Hq, L, d, m = W["B"], W["Hkv"], W["Hq"], W["L"], W["d"], W["m"]
+    L0 = L - 1                                            # prefill; each step appends token L0 -> context L
+    hk = tq.Handle(d, W["bits"], W["seed_k_handle"], qjl_m=m)
+    hv = tq.Handle(d, W["bits"], W["seed_v_handle"], qjl_m=m)
+    K = synth.outlier_kv(seed=W["seed_k"] + 100 * rank).to(dev)
+    V = synth.outlier_kv(seed=W["seed_v"] + 100 * rank).to(dev)
+    kc, vc = tq.Cache(hk, B, Hkv, L, dev), tq.Cache(hv, B, Hkv, L, dev)
+    kc.fill(K[:, :, :L0])
+    vc.fill(V[:, :, :L0])
+    lens = torch.full((B,), L0, dtype=torch.int32, device=dev)
+
+    n_tok = max(args.steps, 1) + args.warmup
+    g = torch.Generator().manual_seed(W["seed_q"] + 100 * rank)
+    q_all = torch.randn(n_tok, B, Hq, d, generator=g).to(dev)
+    k_all = K[:, :, L0].unsqueeze(0).expand(n_tok, B, Hkv, d).contiguous()   # the workload's token 32768
+    v_all = V[:, :, L0].unsqueeze(0).expand(n_tok, B, Hkv, d).contiguous()
+    q_in, k_in, v_in = q_all[0].clone(), k_all[0].clone(), v_all[0].clone()
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device=dev)
+    ws = torch.empty(tq.tq_attn_workspace_bytes(hk.ptr, hv.ptr, B, Hq, Hkv, L), dtype=torch.uint8, device=dev)
+    scale = 1.0 / (d ** 0.5)
+    flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)   # 2x the 126 MB L2
+
+    def step():
+        tq.tq_append(hk.ptr, k_in, B, Hkv, kc.struct, lens, 0)
+        tq.tq_append(hv.ptr, v_in, B, Hkv, vc.struct, lens, 1)
+        tq.tq_attn_decode(hk.ptr, hv.ptr, q_in, B, Hq, Hkv, kc.struct, vc.struct, lens, scale, out, ws)
+
+    # eager warm-up (sets kernel attributes), then capture the step with kernel timers inside
+    s = torch.cuda.Stream(device=dev)
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        for _ in range(3):
+            step()
+            lens.fill_(L0)
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    tq.tq_timer_read(None, forget=True)
+    tq.tq_timer_enable(True)
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    tq.tq_timer_enable(False)
+    lens.fill_(L0)
+    torch.cuda.synchronize()
+    _, kernels_per_step = tq.tq_timer_read(None, forget=False)
+
+    def set_inputs(t):
+        q_in.copy_(q_all[t])
+        k_in.copy_(k_all[t])
+        v_in.copy_(v_all[t])
+
+    for t in range(args.warmup):
+        set_inputs(t)
+        flush.zero_()
+        graph.replay()
+        lens.fill_(L0)
+    torch.cuda.synchronize()
+
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    sampler = ClockSampler("GPU-" + str(torch.cuda.get_device_properties(dev).uuid)) if rank == 0 else None
+    if sampler:
+        sampler.start()
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    split_ms, split_n = 0.0, 0
+    for i in range(args.steps):
+        set_inputs(args.warmup + i)
+        flush.zero_()
+        evs[i][0].record()
+        graph.replay()
+        evs[i][1].record()
+        lens.fill_(L0)
+        evs[i][1].synchronize()                 # captured event pairs are re-recorded by every replay
+        ms_i, n_i = tq.tq_timer_read("attn_split", forget=False)
+        split_ms += ms_i
+        split_n += n_i
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    total_ms = sum(step_ms)
+    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    max_ms = float(t.item())
+
+    # --- end to end through the C ABI with host buffers (pinned), same workload
+    q_h = q_all.cpu().pin_memory()
+    k_h = k_all.cpu().pin_memory()
+    v_h = v_all.cpu().pin_memory()
+    o_h = torch.empty(args.steps, B, Hq, d, dtype=torch.float32).pin_memory()
+    e2e_ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    for i in range(args.steps):
+        flush.zero_()
+        e2e_ev[i][0].record()
+        q_in.copy_(q_h[args.warmup + i], non_blocking=True)
+        k_in.copy_(k_h[args.warmup + i], non_blocking=True)
+        v_in.copy_(v_h[args.warmup + i], non_blocking=True)
+        graph.replay()
+        o_h[i].copy_(out, non_blocking=True)
+        e2e_ev[i][1].record()
+        lens.fill_(L0)
+    torch.cuda.synchronize()
+    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
+    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
+    if world > 1:
+        dist.all_reduce(te, op=dist.ReduceOp.MAX)
+    e2e_ms = float(te.item())
+    h2d = (q_in.numel() * 4 + k_in.numel() * 2 + v_in.numel() * 2)
+    d2h = out.numel() * 4
+
+    # --- encode throughput (vectors encoded / s): prefill encode of the K and V caches
+    enc_ms = 0.0
+    reps = 5
+    for r in range(reps + 1):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record()
+        tq.tq_encode(hk.ptr, K, B * Hkv * L, kc.codes, kc.signs, kc.norms, kc.rnorms)
+        tq.tq_encode(hv.ptr, V, B * Hkv * L, vc.codes, vc.signs, vc.norms, vc.rnorms)
+        b.record()
+        torch.cuda.synchronize()
+        if r:
+            enc_ms += a.elapsed_time(b)
+    enc_vectors = 2 * B * Hkv * L
+    enc_vps = enc_vectors * reps / (enc_ms / 1e3)
+
+    if world > 1:
+        dist.destroy_process_group()
+    if rank != 0:
+        return
+    del graph
+    tokens = B * Hkv * L                               # key (and value) rows read per step per rank
+    bytes_step = tokens * PACKED_BYTES_PER_TOKEN
+    value = world * bytes_step * args.steps / (max_ms / 1e3) / 1e9
+    keys_s = world * tokens * args.steps / (max_ms / 1e3)
+    peaks, peak_src = measured_peaks()
+    peak = float(peaks.get("hbm_gbs", FALLBACK_HBM_GBS))
+    split_avg_ms = split_ms / max(split_n, 1)
+    achieved = bytes_step / (split_avg_ms / 1e3) / 1e9
+    line = {
+        "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
+        "config": {"workload": WORKLOAD_NAME, "B": B, "Hkv": Hkv, "Hq": Hq, "context": L, "d": d,
+                   "bits": "2 MSE + 1 QJL (m=128)", "l2": "flushed between steps (256 MB write)",
+                   "step": "tq_append K + tq_append V + tq_attn_decode, one CUDA graph replay",
+                   "parallelism": f"independent replica per GPU x{world}"},
+        "keys_scored_per_s": keys_s,
+        "query_key_pairs_per_s": keys_s * (Hq // Hkv),
+        "vectors_encoded_per_s": enc_vps,
+        "encode": {"vectors": enc_vectors, "ms_per_pass": enc_ms / reps, "input": "bf16 K and V prefill"},
+        "hbm_frac_nominal_8tbs": value / world / 8000.0,
+        "roofline": {"bound": "hbm", "kernel": "attn_split", "achieved": achieved, "peak": peak,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "peak_source": f"{peak_src} hbm_gbs", "launch_ms": split_avg_ms,
+                     "algorithmic_bytes_per_launch": bytes_step},
+        "e2e": {"value": world * bytes_step * args.steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
+                "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+        "gpu_launches": kernels_per_step * args.steps,
+        "kernels_per_step": kernels_per_step,
+        "clocks": clocks,
+    }
+    if world == 1 and not args.no_cpu_baseline:
+        gbs, el, reps_c, threads = oracle_decode_sample()
+        line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",
+                                "sample": f"{reps_c} decode steps of 1 of 8 KV-head groups (4 query heads, "
+                                          f"32768 tokens) in {el:.1f} s, fp64 NumPy oracle"}
+    print(json.dumps(line), flush=True)
+
+
+def main():
+    args = parse_args()
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_tq(args)
+
+
+if __name__ == "__main__":
+    main()

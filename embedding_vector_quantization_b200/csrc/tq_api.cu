@@ -1,0 +1,663 @@
+// C ABI of libtq.so (declared in include/tq.h): handle lifetime, argument
+// validation, workspace layout and kernel launches. Every entry point returns
+// a status and records a message for tq_last_error(); nothing throws.
+//
+// Fault injection for tests (host side only; no GPU fault is ever caused):
+//   TQ_FAULT=alloc   -> tq_create* fails with TQ_ENOMEM before allocating
+//   TQ_FAULT=launch  -> hot calls fail with TQ_ECUDA before launching
+
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <atomic>
+#include <cmath>
+#include <cstdarg>
+#include <cstdio>
+#include <cstdlib>
+#include <cstring>
+#include <mutex>
+#include <string>
+#include <vector>
+
+#include "tq.h"
+#include "host_math.h"
+#include "common.cuh"
+#include "encode_simt.cuh"
+#include "score_attn_simt.cuh"
+#include "search_simt.cuh"
+
+struct tq_handle {
+  int d = 0, bits = 0, m = 0, norm_dtype = TQ_F32;
+  uint64_t seed = 0;
+  int codes_B = 0, signs_B = 0;
+  int device = 0;
+  std::vector<double> Pi, S, cent, bnd;  // host fp64
+  float* dPi = nullptr;   // [d][d]   y = Pi u
+  float* dPiT = nullptr;  // [d][d]   transpose
+  float* dS = nullptr;    // [m][d]
+  float* dMT = nullptr;   // [d][m]   (S Pi^T)^T
+  float* dcent = nullptr; // [2^bits]
+  float* dbnd = nullptr;  // [2^bits - 1]
+  int* derr = nullptr;    // device error word
+};
+
+namespace {
+
+thread_local std::string g_last_error;
+
+int fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
+
+int ok() {
+  g_last_error.clear();
+  return TQ_OK;
+}
+
+bool fault_is(const char* what) {
+  const char* f = std::getenv("TQ_FAULT");
+  return f && std::strcmp(f, what) == 0;
+}
+
+int cuda_fail(cudaError_t e, const char* where) {
+  return fail(TQ_ECUDA, "%s: %s", where, cudaGetErrorString(e));
+}
+
+#define TQ_CUDA(call)                                   \
+  do {                                                  \
+    cudaError_t e_ = (call);                            \
+    if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
+  } while (0)
+
+int launch_check(const char* what) {
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return ok();
+}
+
+// True the first time (kernel slot, device) is seen: per-device one-time kernel attributes.
+bool once_per_device(int slot, int device) {
+  static std::atomic<uint64_t> seen[16];
+  if (slot < 0 || slot >= 16 || device < 0 || device >= 64) return true;
+  const uint64_t bit = 1ull << device;
+  return (seen[slot].fetch_or(bit) & bit) == 0;
+}
+
+// ---- kernel timer: events recorded around launches while enabled
+struct TimedLaunch {
+  std::string name;
+  cudaEvent_t start, stop;
+};
+std::mutex g_timer_mu;
+std::atomic<bool> g_timer_on{false};
+std::vector<TimedLaunch> g_timer_pending;
+std::vector<cudaEvent_t> g_timer_pool;
+
+cudaEvent_t timer_event() {
+  if (!g_timer_pool.empty()) {
+    cudaEvent_t e = g_timer_pool.back();
+    g_timer_pool.pop_back();
+    return e;
+  }
+  cudaEvent_t e = nullptr;
+  cudaEventCreate(&e);
+  return e;
+}
+
+// Brackets one kernel launch with events when the timer is on.
+struct KernelScope {
+  const char* name;
+  cudaStream_t stream;
+  cudaEvent_t start = nullptr, stop = nullptr;
+  KernelScope(const char* n, cudaStream_t s) : name(n), stream(s) {
+    if (!g_timer_on.load(std::memory_order_relaxed)) return;
+    std::lock_guard<std::mutex> lk(g_timer_mu);
+    start = timer_event();
+    stop = timer_event();
+    cudaEventRecord(start, stream);
+  }
+  ~KernelScope() {
+    if (!start) return;
+    cudaEventRecord(stop, stream);
+    std::lock_guard<std::mutex> lk(g_timer_mu);
+    g_timer_pending.push_back({name, start, stop});
+  }
+};
+
+bool aligned(const void* p, size_t a) { return (reinterpret_cast<uintptr_t>(p) % a) == 0; }
+
+bool valid_dtype(int dt) { return dt == TQ_F32 || dt == TQ_F16 || dt == TQ_BF16; }
+
+size_t round_up(size_t v, size_t a) { return (v + a - 1) / a * a; }
+
+void free_device(tq_handle* h) {
+  cudaFree(h->dPi);
+  cudaFree(h->dPiT);
+  cudaFree(h->dS);
+  cudaFree(h->dMT);
+  cudaFree(h->dcent);
+  cudaFree(h->dbnd);
+  cudaFree(h->derr);
+  h->dPi = h->dPiT = h->dS = h->dMT = h->dcent = h->dbnd = nullptr;
+  h->derr = nullptr;
+}
+
+template <typename T>
+int upload(T** dst, const std::vector<T>& src, const char* what) {
+  if (src.empty()) return TQ_OK;
+  cudaError_t e = cudaMalloc(reinterpret_cast<void**>(dst), src.size() * sizeof(T));
+  if (e != cudaSuccess) return fail(TQ_ENOMEM, "cudaMalloc(%s): %s", what, cudaGetErrorString(e));
+  e = cudaMemcpy(*dst, src.data(), src.size() * sizeof(T), cudaMemcpyHostToDevice);
+  if (e != cudaSuccess) return cuda_fail(e, what);
+  return TQ_OK;
+}
+
+int create_common(int d, int bits_mse, int m, uint64_t seed, int norm_dtype, tq_handle** out) {
+  if (!out) return fail(TQ_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (d < 32 || d > 4096) return fail(TQ_EUNSUPPORTED, "d=%d outside 32..4096", d);
+  if (d % 32 != 0) return fail(TQ_EUNSUPPORTED, "d=%d is not a multiple of 32", d);
+  if (bits_mse < 1 || bits_mse > 4) return fail(TQ_EUNSUPPORTED, "MSE bits=%d outside 1..4", bits_mse);
+  if (m < 0 || m % 32 != 0 || m > 1024) return fail(TQ_EUNSUPPORTED, "qjl_m=%d (needs m %% 32 == 0, m <= 1024)", m);
+  if (m > 0 && d > tqk::kEncBN) return fail(TQ_EUNSUPPORTED, "prod handles need d <= %d", tqk::kEncBN);
+  if (fault_is("alloc")) return fail(TQ_ENOMEM, "injected allocation failure (TQ_FAULT=alloc)");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+
+  tq_handle* h = new tq_handle();
+  h->d = d;
+  h->bits = bits_mse;
+  h->m = m;
+  h->seed = seed;
+  h->norm_dtype = norm_dtype;
+  h->device = dev;
+  h->codes_B = d * bits_mse / 8;
+  h->signs_B = m / 8;
+  const int L = 1 << bits_mse;
+  h->Pi.resize((size_t)d * d);
+  h->S.resize((size_t)m * d);
+  h->cent.resize(L);
+  h->bnd.resize(L - 1);
+  tqhost::rotation(d, m, seed, h->Pi.data(), m ? h->S.data() : nullptr);
+  if (tqhost::codebook(d, bits_mse, h->cent.data(), h->bnd.data()) != 0) {
+    delete h;
+    return fail(TQ_EINVAL, "codebook(d=%d, bits=%d) failed", d, bits_mse);
+  }
+  std::vector<float> Pi(h->Pi.begin(), h->Pi.end()), PiT((size_t)d * d), S(h->S.begin(), h->S.end()),
+      MT((size_t)d * m), cent(h->cent.begin(), h->cent.end()), bnd(h->bnd.begin(), h->bnd.end());
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) PiT[(size_t)j * d + i] = (float)h->Pi[(size_t)i * d + j];
+  // M = S Pi^T (m x d): M[i][k] = sum_j S[i][j] Pi[k][j]; stored transposed MT[k][i].
+  for (int i = 0; i < m; ++i)
+    for (int k = 0; k < d; ++k) {
+      double acc = 0.0;
+      for (int j = 0; j < d; ++j) acc += h->S[(size_t)i * d + j] * h->Pi[(size_t)k * d + j];
+      MT[(size_t)k * m + i] = (float)acc;
+    }
+  int st = TQ_OK;
+  if ((st = upload(&h->dPi, Pi, "Pi")) || (st = upload(&h->dPiT, PiT, "PiT")) ||
+      (st = upload(&h->dS, S, "S")) || (st = upload(&h->dMT, MT, "MT")) ||
+      (st = upload(&h->dcent, cent, "centroids")) || (st = upload(&h->dbnd, bnd, "bounds"))) {
+    free_device(h);
+    delete h;
+    return st;
+  }
+  e = cudaMalloc(&h->derr, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(h->derr, 0, sizeof(int));
+  if (e != cudaSuccess) {
+    free_device(h);
+    delete h;
+    return fail(TQ_ENOMEM, "cudaMalloc(error word): %s", cudaGetErrorString(e));
+  }
+  *out = h;
+  return ok();
+}
+
+tqk::CacheView view_of(const tq_handle* h, const tq_cache* c) {
+  tqk::CacheView v;
+  v.codes = c->codes;
+  v.signs = c->signs;
+  v.norms = c->norms;
+  v.rnorms = static_cast<const __half*>(c->rnorms);
+  v.bits = h->bits;
+  v.m = h->m;
+  v.norm_dtype = h->norm_dtype;
+  v.codes_B = h->codes_B;
+  v.signs_B = h->signs_B;
+  v.cent = h->dcent;
+  return v;
+}
+
+int check_cache(const tq_handle* h, const tq_cache* c, const char* name) {
+  if (!c) return fail(TQ_EINVAL, "%s cache is NULL", name);
+  if (!c->codes || !c->norms) return fail(TQ_EINVAL, "%s cache: codes/norms NULL", name);
+  if (h->m > 0 && (!c->signs || !c->rnorms)) return fail(TQ_EINVAL, "%s cache: prod handle needs signs and rnorms", name);
+  if (c->L_cap < 1) return fail(TQ_EINVAL, "%s cache: L_cap=%lld", name, (long long)c->L_cap);
+  if (!aligned(c->codes, 16) || (c->signs && !aligned(c->signs, 16)) || !aligned(c->norms, 4) ||
+      (c->rnorms && !aligned(c->rnorms, 2)))
+    return fail(TQ_EINVAL, "%s cache: misaligned pointer", name);
+  return TQ_OK;
+}
+
+// Attention split policy: enough CTAs to cover the GPU ~4x, chunks of >= 128 keys.
+void attn_split(int B, int Hkv, int64_t L_cap, int* nsplit, int64_t* chunk) {
+  const int64_t units = (int64_t)B * Hkv;
+  int64_t ns = (4 * 148 + units - 1) / units;
+  const int64_t max_ns = (L_cap + 127) / 128;
+  ns = std::max<int64_t>(1, std::min(ns, max_ns));
+  int64_t ch = (L_cap + ns - 1) / ns;
+  ch = (ch + 127) / 128 * 128;
+  ns = (L_cap + ch - 1) / ch;
+  *nsplit = (int)ns;
+  *chunk = ch;
+}
+
+void search_split(int nq, int64_t n, int* nchunks, int64_t* chunk) {
+  const int64_t qt = (nq + tqk::kSQ - 1) / tqk::kSQ;
+  int64_t nc = (2 * 148 + qt - 1) / qt;
+  nc = std::max<int64_t>(1, std::min<int64_t>(nc, (n + tqk::kSK - 1) / tqk::kSK));
+  int64_t ch = (n + nc - 1) / nc;
+  ch = (ch + tqk::kSK - 1) / tqk::kSK * tqk::kSK;
+  *chunk = ch;
+  *nchunks = (int)((n + ch - 1) / ch);
+}
+
+struct ScoreWs { float* qr; float* qs; };
+size_t score_ws_layout(const tq_handle* h, int rows, char* base, ScoreWs* w) {
+  size_t off = 0;
+  const size_t qr = round_up((size_t)rows * h->d * 4, 256);
+  const size_t qs = round_up((size_t)rows * std::max(h->m, 1) * 4, 256);
+  if (w) { w->qr = reinterpret_cast<float*>(base + off); w->qs = reinterpret_cast<float*>(base + off + qr); }
+  off += qr + qs;
+  return off;
+}
+
+size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, int Hkv, int64_t L_cap,
+                      char* base, ScoreWs* w, float** part, int* nsplit, int64_t* chunk) {
+  size_t off = score_ws_layout(hk, B * Hq, base, w);
+  int ns;
+  int64_t ch;
+  attn_split(B, Hkv, L_cap, &ns, &ch);
+  if (nsplit) *nsplit = ns;
+  if (chunk) *chunk = ch;
+  if (part) *part = reinterpret_cast<float*>(base + off);
+  off += round_up((size_t)B * Hq * ns * (hv->d + hv->m + 2) * 4, 256);
+  return off;
+}
+
+size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base, float** qr, float** cs,
+                        int64_t** ci, int* nchunks, int64_t* chunk) {
+  int nc;
+  int64_t ch;
+  search_split(nq, n, &nc, &ch);
+  if (nchunks) *nchunks = nc;
+  if (chunk) *chunk = ch;
+  size_t off = 0;
+  if (qr) *qr = reinterpret_cast<float*>(base + off);
+  off += round_up((size_t)nq * h->d * 4, 256);
+  if (cs) *cs = reinterpret_cast<float*>(base + off);
+  off += round_up((size_t)nc * nq * k * 4, 256);
+  if (ci) *ci = reinterpret_cast<int64_t*>(base + off);
+  off += round_up((size_t)nc * nq * k * 8, 256);
+  return off;
+}
+
+int launch_qprep(const tq_handle* h, const void* q, int q_dtype, int rows, float* qr, float* qs, cudaStream_t s) {
+  if (rows == 0) return TQ_OK;
+  dim3 grid(rows, std::max(1, std::min(8, (h->d + h->m) / 64)));
+  KernelScope ks("qprep", s);
+  tqk::qprep_kernel<<<grid, 256, h->d * sizeof(float), s>>>(q, q_dtype, rows, h->d, h->dPi, h->dS, h->m, qr, qs);
+  return launch_check("qprep_kernel");
+}
+
+int encode_launch(const tq_handle* h, tqk::EncodeArgs& a, cudaStream_t s) {
+  const size_t smem = tqk::encode_smem_bytes(h->m);
+  if (once_per_device(0, h->device))
+    cudaFuncSetAttribute(tqk::encode_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  dim3 grid((unsigned)((a.rows + tqk::kEncBM - 1) / tqk::kEncBM), (h->d + tqk::kEncBN - 1) / tqk::kEncBN);
+  KernelScope ks(a.len ? "append" : "encode", s);
+  tqk::encode_simt_kernel<<<grid, tqk::kEncThreads, smem, s>>>(a);
+  return launch_check("encode_simt_kernel");
+}
+
+}  // namespace
+
+// ============================================================================
+extern "C" {
+
+int tq_codebook_host(int d, int bits, double* centroids, double* bounds) {
+  if (!centroids || !bounds) return fail(TQ_EINVAL, "NULL output");
+  if (d < 3 || d > 65536 || bits < 1 || bits > 8) return fail(TQ_EINVAL, "d=%d bits=%d out of range", d, bits);
+  if (tqhost::codebook(d, bits, centroids, bounds) != 0) return fail(TQ_EINVAL, "codebook failed");
+  return ok();
+}
+
+int tq_rotation_host(int d, int m, uint64_t seed, double* Pi, double* S) {
+  if (!Pi) return fail(TQ_EINVAL, "Pi is NULL");
+  if (d < 1 || d > 8192 || m < 0 || m > 8192) return fail(TQ_EINVAL, "d=%d m=%d out of range", d, m);
+  if (m > 0 && !S) return fail(TQ_EINVAL, "S is NULL with m > 0");
+  tqhost::rotation(d, m, seed, Pi, S);
+  return ok();
+}
+
+int tq_create(int d, int bits, uint64_t seed, tq_handle** out) {
+  return create_common(d, bits, 0, seed, TQ_F32, out);
+}
+
+int tq_create_prod(int d, int bits, int qjl_m, uint64_t seed, tq_handle** out) {
+  if (bits < 2 || bits > 5) return fail(TQ_EUNSUPPORTED, "prod bits=%d outside 2..5", bits);
+  if (qjl_m < 32) return fail(TQ_EUNSUPPORTED, "qjl_m=%d < 32", qjl_m);
+  return create_common(d, bits - 1, qjl_m, seed, TQ_F16, out);
+}
+
+int tq_set_norm_dtype(tq_handle* h, int dtype) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (dtype != TQ_F32 && dtype != TQ_F16) return fail(TQ_EINVAL, "norm dtype %d (TQ_F32 or TQ_F16)", dtype);
+  h->norm_dtype = dtype;
+  return ok();
+}
+
+void tq_destroy(tq_handle* h) {
+  if (!h) return;
+  free_device(h);
+  delete h;
+}
+
+int tq_get_info(const tq_handle* h, int* d, int* bits_mse, int* qjl_m, int* norm_dtype) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (d) *d = h->d;
+  if (bits_mse) *bits_mse = h->bits;
+  if (qjl_m) *qjl_m = h->m;
+  if (norm_dtype) *norm_dtype = h->norm_dtype;
+  return ok();
+}
+
+int tq_code_bytes(const tq_handle* h, int* codes_B, int* signs_B) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (codes_B) *codes_B = h->codes_B;
+  if (signs_B) *signs_B = h->signs_B;
+  return ok();
+}
+
+int tq_get_codebook(const tq_handle* h, double* centroids, double* bounds) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (centroids) std::memcpy(centroids, h->cent.data(), h->cent.size() * sizeof(double));
+  if (bounds) std::memcpy(bounds, h->bnd.data(), h->bnd.size() * sizeof(double));
+  return ok();
+}
+
+int tq_get_rotation(const tq_handle* h, double* Pi, double* S) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (Pi) std::memcpy(Pi, h->Pi.data(), h->Pi.size() * sizeof(double));
+  if (S && h->m > 0) std::memcpy(S, h->S.data(), h->S.size() * sizeof(double));
+  return ok();
+}
+
+int tq_encode(const tq_handle* h, const void* x, int x_dtype, int64_t n, uint8_t* codes, uint8_t* signs,
+              void* norms, void* rnorms, void* stream) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (n < 0) return fail(TQ_EINVAL, "n=%lld", (long long)n);
+  if (!valid_dtype(x_dtype)) return fail(TQ_EINVAL, "x dtype %d", x_dtype);
+  if (n == 0) return ok();
+  if (!x || !codes || !norms) return fail(TQ_EINVAL, "x/codes/norms NULL");
+  if (h->m > 0 && (!signs || !rnorms)) return fail(TQ_EINVAL, "prod handle needs signs and rnorms");
+  if (!aligned(x, 16) || !aligned(codes, 16) || (signs && !aligned(signs, 16)) || !aligned(norms, 4))
+    return fail(TQ_EINVAL, "misaligned pointer");
+  if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
+  tqk::EncodeArgs a{};
+  a.x = x; a.x_dtype = x_dtype; a.rows = n; a.d = h->d; a.bits = h->bits; a.m = h->m;
+  a.norm_dtype = h->norm_dtype; a.PiT = h->dPiT; a.MT = h->dMT; a.cent = h->dcent; a.bnd = h->dbnd;
+  a.codes = codes; a.codes_B = h->codes_B; a.signs = signs; a.signs_B = h->signs_B;
+  a.norms = norms; a.rnorms = static_cast<__half*>(rnorms); a.len = nullptr; a.err = h->derr;
+  return encode_launch(h, a, static_cast<cudaStream_t>(stream));
+}
+
+int tq_pack_indices(const tq_handle* h, const uint8_t* idx, int64_t n, uint8_t* codes, void* stream) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (n < 0) return fail(TQ_EINVAL, "n=%lld", (long long)n);
+  if (n == 0) return ok();
+  if (!idx || !codes) return fail(TQ_EINVAL, "NULL pointer");
+  if (!aligned(codes, 4)) return fail(TQ_EINVAL, "codes misaligned");
+  const int64_t work = n * (h->d / 32);
+  KernelScope ks("pack", static_cast<cudaStream_t>(stream));
+  tqk::pack_indices_kernel<<<(unsigned)((work + 255) / 256), 256, 0, static_cast<cudaStream_t>(stream)>>>(
+      idx, n, h->d, h->bits, codes, h->codes_B);
+  return launch_check("pack_indices_kernel");
+}
+
+int tq_append(const tq_handle* h, const void* x_new, int x_dtype, int B, int Hkv, const tq_cache* cache,
+              int32_t* len, int advance, void* stream) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (B < 0 || Hkv < 1) return fail(TQ_EINVAL, "B=%d Hkv=%d", B, Hkv);
+  if (!valid_dtype(x_dtype)) return fail(TQ_EINVAL, "x dtype %d", x_dtype);
+  if (B == 0) return ok();
+  int st = check_cache(h, cache, "append");
+  if (st) return st;
+  if (!x_new || !len) return fail(TQ_EINVAL, "x_new/len NULL");
+  if (!aligned(x_new, 16)) return fail(TQ_EINVAL, "x_new misaligned");
+  if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  tqk::EncodeArgs a{};
+  a.x = x_new; a.x_dtype = x_dtype; a.rows = (int64_t)B * Hkv; a.d = h->d; a.bits = h->bits; a.m = h->m;
+  a.norm_dtype = h->norm_dtype; a.PiT = h->dPiT; a.MT = h->dMT; a.cent = h->dcent; a.bnd = h->dbnd;
+  a.codes = cache->codes; a.codes_B = h->codes_B; a.signs = cache->signs; a.signs_B = h->signs_B;
+  a.norms = cache->norms; a.rnorms = static_cast<__half*>(cache->rnorms);
+  a.len = len; a.Hkv = Hkv; a.L_cap = cache->L_cap; a.err = h->derr;
+  st = encode_launch(h, a, s);
+  if (st) return st;
+  if (advance) {
+    KernelScope ks("advance_len", s);
+    tqk::advance_len_kernel<<<(B + 255) / 256, 256, 0, s>>>(len, B, cache->L_cap);
+    return launch_check("advance_len_kernel");
+  }
+  return ok();
+}
+
+size_t tq_score_workspace_bytes(const tq_handle* hk, int B, int Hq) {
+  if (!hk || B < 0 || Hq < 0) return 0;
+  return score_ws_layout(hk, B * Hq, nullptr, nullptr);
+}
+
+size_t tq_attn_workspace_bytes(const tq_handle* hk, const tq_handle* hv, int B, int Hq, int Hkv, int64_t L_cap) {
+  if (!hk || !hv || B < 0 || Hq < 1 || Hkv < 1 || L_cap < 1) return 0;
+  return attn_ws_layout(hk, hv, B, Hq, Hkv, L_cap, nullptr, nullptr, nullptr, nullptr, nullptr);
+}
+
+size_t tq_search_workspace_bytes(const tq_handle* h, int nq, int64_t n, int k) {
+  if (!h || nq < 0 || n < 1 || k < 1) return 0;
+  return search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+}
+
+int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const tq_cache* k, const int32_t* len,
+             float* logits, void* workspace, size_t ws_bytes, void* stream) {
+  if (!hk) return fail(TQ_EINVAL, "handle is NULL");
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return fail(TQ_EINVAL, "B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
+  if (Hq / Hkv > tqk::kMaxGroup) return fail(TQ_EUNSUPPORTED, "group Hq/Hkv=%d > %d", Hq / Hkv, tqk::kMaxGroup);
+  if (hk->d > tqk::kMaxHeadDim) return fail(TQ_EUNSUPPORTED, "score needs d <= %d", tqk::kMaxHeadDim);
+  if (B == 0) return ok();
+  int st = check_cache(hk, k, "key");
+  if (st) return st;
+  if (!q || !len || !logits || !workspace) return fail(TQ_EINVAL, "NULL pointer");
+  const size_t need = tq_score_workspace_bytes(hk, B, Hq);
+  if (ws_bytes < need) return fail(TQ_EINVAL, "workspace %zu < %zu bytes", ws_bytes, need);
+  if (!aligned(workspace, 16)) return fail(TQ_EINVAL, "workspace misaligned");
+  if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ScoreWs w;
+  score_ws_layout(hk, B * Hq, static_cast<char*>(workspace), &w);
+  st = launch_qprep(hk, q, TQ_F32, B * Hq, w.qr, w.qs, s);
+  if (st) return st;
+  tqk::ScoreArgs a{};
+  a.qr = w.qr; a.qs = w.qs; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = hk->d; a.k = view_of(hk, k);
+  a.L_cap = k->L_cap; a.len = len; a.logits = logits;
+  const int64_t units = (int64_t)B * Hkv;
+  int64_t ns = std::max<int64_t>(1, std::min<int64_t>((8 * 148 + units - 1) / units, (k->L_cap + 127) / 128));
+  a.chunk = ((k->L_cap + ns - 1) / ns + 127) / 128 * 128;
+  ns = (k->L_cap + a.chunk - 1) / a.chunk;
+  const int G = Hq / Hkv;
+  const size_t smem = ((size_t)G * (hk->d + hk->m) + 16) * 4;
+  KernelScope ks("score", s);
+  tqk::score_simt_kernel<<<dim3((unsigned)units, (unsigned)ns), tqk::kAttnThreads, smem, s>>>(a);
+  return launch_check("score_simt_kernel");
+}
+
+int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                   const tq_cache* k, const tq_cache* v, const int32_t* len, float scale, float* out,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  if (!hk || !hv) return fail(TQ_EINVAL, "handle is NULL");
+  if (hk->d != hv->d) return fail(TQ_EINVAL, "K and V handles differ in d (%d vs %d)", hk->d, hv->d);
+  if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return fail(TQ_EINVAL, "B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
+  if (Hq / Hkv > tqk::kMaxGroup) return fail(TQ_EUNSUPPORTED, "group Hq/Hkv=%d > %d", Hq / Hkv, tqk::kMaxGroup);
+  if (hk->d > tqk::kMaxHeadDim || hv->m > tqk::kMaxHeadDim)
+    return fail(TQ_EUNSUPPORTED, "attention needs d, m_V <= %d", tqk::kMaxHeadDim);
+  if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_EINVAL, "q dtype %d", q_dtype);
+  if (B == 0) return ok();
+  int st = check_cache(hk, k, "key");
+  if (st) return st;
+  if ((st = check_cache(hv, v, "value"))) return st;
+  if (k->L_cap != v->L_cap) return fail(TQ_EINVAL, "K and V caches differ in L_cap");
+  if (!q || !len || !out || !workspace) return fail(TQ_EINVAL, "NULL pointer");
+  const size_t need = tq_attn_workspace_bytes(hk, hv, B, Hq, Hkv, k->L_cap);
+  if (ws_bytes < need) return fail(TQ_EINVAL, "workspace %zu < %zu bytes", ws_bytes, need);
+  if (!aligned(workspace, 16)) return fail(TQ_EINVAL, "workspace misaligned");
+  if (!std::isfinite(scale)) return fail(TQ_EINVAL, "scale is not finite");
+  if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ScoreWs w;
+  float* part;
+  int nsplit;
+  int64_t chunk;
+  attn_ws_layout(hk, hv, B, Hq, Hkv, k->L_cap, static_cast<char*>(workspace), &w, &part, &nsplit, &chunk);
+  st = launch_qprep(hk, q, q_dtype, B * Hq, w.qr, w.qs, s);
+  if (st) return st;
+  tqk::AttnArgs a{};
+  a.qr = w.qr; a.qs = w.qs; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = hk->d;
+  a.k = view_of(hk, k); a.v = view_of(hv, v); a.L_cap = k->L_cap; a.chunk = chunk; a.nsplit = nsplit;
+  a.len = len; a.scale = scale; a.part = part;
+  const int G = Hq / Hkv;
+  const size_t smem = ((size_t)G * (hk->d + hk->m) + 32 + (size_t)G * tqk::kAttnThreads + 2 * tqk::kAttnThreads +
+                       4 * (size_t)G) * 4;
+  {
+    KernelScope ks("attn_split", s);
+    tqk::attn_split_simt_kernel<<<dim3((unsigned)(B * Hkv), (unsigned)nsplit), tqk::kAttnThreads, smem, s>>>(a);
+  }
+  if ((st = launch_check("attn_split_simt_kernel"))) return st;
+  tqk::CombineArgs c{};
+  c.part = part; c.rows = B * Hq; c.nsplit = nsplit; c.d = hv->d; c.mv = hv->m; c.PiV = hv->dPi; c.SV = hv->dS;
+  c.out = out;
+  const size_t csmem = ((size_t)hv->d + hv->m + nsplit + 2) * 4;
+  KernelScope ks("attn_combine", s);
+  tqk::attn_combine_kernel<<<B * Hq, 128, csmem, s>>>(c);
+  return launch_check("attn_combine_kernel");
+}
+
+int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* codes, const void* norms, int64_t n,
+                   int k, int64_t* idx, float* score, void* workspace, size_t ws_bytes, void* stream) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (h->m > 0) return fail(TQ_EUNSUPPORTED, "search takes MSE handles");
+  if (nq < 0 || n < 1 || k < 1 || k > tqk::kMaxTopK || k > n)
+    return fail(TQ_EINVAL, "nq=%d n=%lld k=%d", nq, (long long)n, k);
+  if (nq == 0) return ok();
+  if (!q || !codes || !norms || !idx || !score || !workspace) return fail(TQ_EINVAL, "NULL pointer");
+  if (!aligned(codes, 16) || !aligned(norms, 4) || !aligned(workspace, 16)) return fail(TQ_EINVAL, "misaligned pointer");
+  const size_t need = tq_search_workspace_bytes(h, nq, n, k);
+  if (ws_bytes < need) return fail(TQ_EINVAL, "workspace %zu < %zu bytes", ws_bytes, need);
+  if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  float *qr, *cs;
+  int64_t* ci;
+  int nchunks;
+  int64_t chunk;
+  search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk);
+  int st = launch_qprep(h, q, TQ_F32, nq, qr, nullptr, s);
+  if (st) return st;
+  tqk::SearchArgs a{};
+  a.qr = qr; a.nq = nq; a.d = h->d; a.bits = h->bits; a.norm_dtype = h->norm_dtype; a.codes_B = h->codes_B;
+  a.k = k; a.codes = codes; a.norms = norms; a.n = n; a.chunk = chunk; a.cent = h->dcent; a.cand_s = cs; a.cand_i = ci;
+  const size_t smem = tqk::search_smem_bytes(k);
+  if (once_per_device(1, h->device))
+    cudaFuncSetAttribute(tqk::search_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  dim3 grid((unsigned)nchunks, (unsigned)((nq + tqk::kSQ - 1) / tqk::kSQ));
+  {
+    KernelScope ks("search", s);
+    tqk::search_simt_kernel<<<grid, tqk::kSearchThreads, smem, s>>>(a);
+  }
+  if ((st = launch_check("search_simt_kernel"))) return st;
+  KernelScope ks("topk_merge", s);
+  tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
+  return launch_check("topk_merge_kernel");
+}
+
+int tq_timer_enable(int on) {
+  if (on) {  // pre-create events so that a stream capture never has to create one
+    std::lock_guard<std::mutex> lk(g_timer_mu);
+    while (g_timer_pool.size() < 64) {
+      cudaEvent_t e = nullptr;
+      cudaError_t err = cudaEventCreate(&e);
+      if (err != cudaSuccess) return cuda_fail(err, "cudaEventCreate");
+      g_timer_pool.push_back(e);
+    }
+  }
+  g_timer_on.store(on != 0);
+  return ok();
+}
+
+int tq_timer_read(const char* name, double* ms, int* launches, int forget) {
+  std::lock_guard<std::mutex> lk(g_timer_mu);
+  double total = 0.0;
+  int count = 0;
+  std::vector<TimedLaunch> keep;
+  for (auto& t : g_timer_pending) {
+    if (name && t.name != name) {
+      keep.push_back(t);
+      continue;
+    }
+    cudaError_t e = cudaEventSynchronize(t.stop);
+    float el = 0.f;
+    if (e == cudaSuccess) e = cudaEventElapsedTime(&el, t.start, t.stop);
+    if (e != cudaSuccess) {
+      g_timer_pending.clear();
+      return cuda_fail(e, "tq_timer_read");
+    }
+    total += el;
+    ++count;
+    if (forget) {
+      g_timer_pool.push_back(t.start);
+      g_timer_pool.push_back(t.stop);
+    } else {
+      keep.push_back(t);
+    }
+  }
+  g_timer_pending.swap(keep);
+  if (ms) *ms += total;
+  if (launches) *launches += count;
+  return ok();
+}
+
+int tq_last_status(const tq_handle* h, void* stream) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaStreamSynchronize(s);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaStreamSynchronize");
+  int word = 0;
+  e = cudaMemcpy(&word, h->derr, sizeof(int), cudaMemcpyDeviceToHost);
+  if (e != cudaSuccess) return cuda_fail(e, "read error word");
+  if (word) {
+    e = cudaMemset(h->derr, 0, sizeof(int));
+    if (e != cudaSuccess) return cuda_fail(e, "clear error word");
+  }
+  if (word & tqk::kErrTimeout) return fail(TQ_ETIMEOUT, "a bounded device wait timed out");
+  if (word & tqk::kErrCapacity) return fail(TQ_ECAPACITY, "append skipped a full sequence (len == L_cap)");
+  return ok();
+}
+
+const char* tq_last_error(void) { return g_last_error.c_str(); }
+
+}  // extern "C"

@@ -1,0 +1,115 @@
+"""GPU parity of the handle constants, encode (MSE and prod), pack and append
+against the oracle ("Google TurboQuant: 6x KV-cache compression", sections
+"Stage 1: PolarQuant" and "Stage 2: QJL residual correction")."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import OracleHandle, check_codes, check_norms, check_signs, to_np64
+from oracle import quant
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tq():
+    from conftest import build_lib
+    m = build_lib()
+    assert torch.cuda.is_available()
+    return m
+
+
+NORM_NP = {0: "f32", 1: "f16"}
+
+
+def _encode_and_check(tq, x_cpu, d, bits, seed, m=0, norm_dtype=None):
+    h = tq.Handle(d, bits, seed, qjl_m=m, norm_dtype=norm_dtype)
+    oh = OracleHandle(d, h.bits_mse, seed, m)
+    out = h.encode(x_cpu.cuda())
+    torch.cuda.synchronize()
+    exp = oh.encode(to_np64(x_cpu), NORM_NP[h.norm_dtype])
+    gidx, bad, frac = check_codes(out["codes"].cpu().numpy().reshape(-1, h.codes_B), exp, oh)
+    check_norms(out["norms"].cpu().numpy().reshape(-1), exp["n_stored"])
+    sfrac = None
+    if m:
+        sfrac = check_signs(out["signs"].cpu().numpy().reshape(-1, h.signs_B), exp, bad)
+        keep = np.ones(len(exp["idx"]), bool)
+        keep[bad] = False
+        check_norms(out["rnorms"].cpu().numpy().reshape(-1)[keep], exp["rnorm_stored"][keep])
+    assert h.status() == tq.TQ_OK
+    return frac, sfrac
+
+
+def test_handle_constants_match_oracle(tq):
+    for d, bits, m, seed in [(128, 3, 0, 0), (128, 3, 128, 2), (1536, 2, 0, 0), (64, 4, 0, 5)]:
+        h = tq.Handle(d, bits, seed, qjl_m=m)
+        oh = OracleHandle(d, h.bits_mse, seed, m)
+        Pi, S = h.rotation()
+        c, b = h.codebook()
+        assert np.abs(Pi - oh.Pi).max() <= 1e-12
+        assert np.abs(c - oh.c).max() <= 1e-12 and np.abs(b - oh.beta).max() <= 1e-12
+        if m:
+            assert np.abs(S - oh.S).max() <= 1e-12
+        assert h.codes_B == d * h.bits_mse // 8 and h.signs_B == m // 8
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("dtype", [torch.float32, torch.bfloat16, torch.float16])
+def test_encode_mse_d128(tq, bits, dtype):
+    x = torch.randn(1001, 128, generator=torch.Generator().manual_seed(bits)).to(dtype)
+    frac, _ = _encode_and_check(tq, x, 128, bits, seed=bits)
+    assert frac < 1e-3
+
+
+@pytest.mark.parametrize("d,bits", [(32, 3), (96, 2), (256, 4), (1536, 2), (1536, 4)])
+def test_encode_mse_other_dims(tq, d, bits):
+    x = torch.randn(257, d, generator=torch.Generator().manual_seed(d))
+    frac, _ = _encode_and_check(tq, x, d, bits, seed=11)
+    assert frac < 1e-3
+
+
+def test_encode_fp16_norms(tq):
+    x = torch.randn(700, 128, generator=torch.Generator().manual_seed(4)) * 7
+    _encode_and_check(tq, x, 128, 3, seed=4, norm_dtype=tq.TQ_F16)
+
+
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float32])
+@pytest.mark.parametrize("bits,m", [(3, 128), (2, 128), (4, 64), (3, 256)])
+def test_encode_prod(tq, dtype, bits, m):
+    x = torch.randn(777, 128, generator=torch.Generator().manual_seed(bits + m)).to(dtype)
+    frac, sfrac = _encode_and_check(tq, x, 128, bits, seed=2, m=m)
+    assert frac < 1e-3 and sfrac < 1e-3
+
+
+def test_encode_edge_rows(tq):
+    """Zero vectors, one-hot rows, huge and tiny scales, n = 1 and n = 65 (ragged tile)."""
+    g = torch.Generator().manual_seed(3)
+    x = torch.randn(65, 128, generator=g)
+    x[0] = 0
+    x[1] = 0
+    x[1, 17] = 3.0
+    x[2] *= 1e4
+    x[3] *= 1e-4
+    _encode_and_check(tq, x, 128, 3, seed=1)
+    _encode_and_check(tq, x, 128, 3, seed=1, m=128)
+    _encode_and_check(tq, x[:1].clone(), 128, 2, seed=1)
+    h = tq.Handle(128, 3, 1)
+    out = h.encode(torch.zeros(0, 128, device="cuda"))     # n = 0 is a no-op
+    assert out["codes"].shape == (0, 48)
+
+
+def test_pack_indices_bit_exact(tq):
+    for d, bits in [(128, 1), (128, 2), (128, 3), (128, 4), (1536, 2), (32, 3)]:
+        h = tq.Handle(d, bits, 0)
+        idx = np.random.default_rng(bits).integers(0, 1 << bits, size=(300, d)).astype(np.uint8)
+        got = h.pack_indices(torch.from_numpy(idx).cuda()).cpu().numpy()
+        assert np.array_equal(got, quant.pack(idx, bits))
+
+
+def test_config1_encode_full(tq):
+    """MSE-only d=128, b=3, 4096 fp32 N(0,1) keys (seed 0): parity and empirical distortion."""
+    from embedding_vector_quantization_b200 import synth
+    x = synth.mse_keys()
+    frac, _ = _encode_and_check(tq, x, 128, 3, seed=0)
+    assert frac < 1e-4

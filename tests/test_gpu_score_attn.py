@@ -1,0 +1,190 @@
+"""GPU parity of scores, decode attention, append and search against the oracle.
+
+Kernel parity: the GPU reads caches filled with the ORACLE's codes (packed by
+the oracle and uploaded), so both sides score identical codes. End-to-end
+parity (GPU encode -> GPU attention vs oracle encode -> oracle attention) is
+checked separately with the same tolerance."""
+
+import numpy as np
+import pytest
+import torch
+
+from gpu_util import ATTN_RTOL, OracleHandle, check_codes, check_norms, score_tolerance, to_np64
+from oracle import ops, quant
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module")
+def tq():
+    from conftest import build_lib
+    m = build_lib()
+    return m
+
+
+NORM_NP = {0: "f32", 1: "f16"}
+
+
+def oracle_cache(tq, h, oh, x):
+    """Oracle-encoded cache for x [B, Hkv, L, d] (np fp64) uploaded into a GPU Cache; returns (cache, odict)."""
+    B, Hkv, L, d = x.shape
+    e = oh.encode(x.reshape(-1, d), NORM_NP[h.norm_dtype])
+    cache = tq.Cache(h, B, Hkv, L)
+    cache.codes.copy_(torch.from_numpy(quant.pack(e["idx"], oh.bits).reshape(B, Hkv, L, -1)))
+    cache.norms.copy_(torch.from_numpy(e["n_stored"].reshape(B, Hkv, L)))
+    od = {"idx": e["idx"].reshape(B, Hkv, L, d), "n": e["n_stored"].reshape(B, Hkv, L), "Pi": oh.Pi, "c": oh.c}
+    if oh.m:
+        cache.signs.copy_(torch.from_numpy(quant.pack(e["sigma"], 1).reshape(B, Hkv, L, -1)))
+        cache.rnorms.copy_(torch.from_numpy(e["rnorm_stored"].reshape(B, Hkv, L)))
+        od.update({"sigma": e["sigma"].reshape(B, Hkv, L, oh.m), "rnorm": e["rnorm_stored"].reshape(B, Hkv, L),
+                   "S": oh.S})
+    return cache, od
+
+
+def _kv(shape, seed, scale=1.0):
+    return np.random.default_rng(seed).standard_normal(shape) * scale
+
+
+@pytest.mark.parametrize("bits,m,G", [(3, 0, 4), (3, 128, 4), (4, 0, 1), (2, 0, 8), (2, 64, 2)])
+def test_score_on_oracle_codes(tq, bits, m, G):
+    B, Hkv, L, d = 2, 2, 1000, 128
+    Hq = Hkv * G
+    h = tq.Handle(d, bits, 3, qjl_m=m)
+    oh = OracleHandle(d, h.bits_mse, 3, m)
+    x = _kv((B, Hkv, L, d), 1, 2.0)
+    cache, od = oracle_cache(tq, h, oh, x)
+    q = torch.randn(B, Hq, d, generator=torch.Generator().manual_seed(5))
+    lens = torch.tensor([L, 617], dtype=torch.int32)
+    logits = tq.score(h, q.cuda(), cache, lens.cuda())
+    got = logits.cpu().numpy()
+    qn = q.double().numpy()
+    for b in range(B):
+        for hq in range(Hq):
+            hk = hq // G
+            Lb = int(lens[b])
+            if m:
+                ref = ops.score_prod(qn[b, hq], od["idx"][b, hk, :Lb], od["n"][b, hk, :Lb], od["sigma"][b, hk, :Lb],
+                                     od["rnorm"][b, hk, :Lb], oh.Pi, oh.S, oh.c)
+            else:
+                ref = ops.score_mse(qn[b, hq], od["idx"][b, hk, :Lb], od["n"][b, hk, :Lb], oh.Pi, oh.c)
+            tol = score_tolerance(ref, np.linalg.norm(qn[b, hq]), od["n"][b, hk, :Lb].astype(np.float64), d)
+            assert np.all(np.abs(got[b, hq, :Lb] - ref) <= tol)
+            assert np.all(got[b, hq, Lb:] == 0)  # untouched tail
+
+
+def _attn_case(tq, kb, km, vb, vm, G, lens, L, B=2, Hkv=2, d=128, q_dtype=torch.float32):
+    Hq = Hkv * G
+    hk = tq.Handle(d, kb, 10, qjl_m=km)
+    hv = tq.Handle(d, vb, 11, qjl_m=vm)
+    ohk, ohv = OracleHandle(d, hk.bits_mse, 10, km), OracleHandle(d, hv.bits_mse, 11, vm)
+    kc, kod = oracle_cache(tq, hk, ohk, _kv((B, Hkv, L, d), 12, 1.5))
+    vc, vod = oracle_cache(tq, hv, ohv, _kv((B, Hkv, L, d), 13))
+    q = (torch.randn(B, Hq, d, generator=torch.Generator().manual_seed(14)) * 2).to(q_dtype)
+    lens_t = torch.tensor(lens, dtype=torch.int32)
+    scale = 1.0 / np.sqrt(d)
+    o = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens_t.cuda(), scale).cpu().numpy()
+    ref = ops.decode_attention(q.double().numpy(), kod, vod, [max(1, l) for l in lens], scale)
+    for b in range(B):
+        for h in range(Hq):
+            if lens[b] == 0:
+                assert np.all(o[b, h] == 0)
+                continue
+            err = np.linalg.norm(o[b, h] - ref[b, h])
+            assert err <= ATTN_RTOL * np.linalg.norm(ref[b, h]), (b, h, err)
+    return o
+
+
+@pytest.mark.parametrize("kb,km,vb,vm,G", [(3, 128, 3, 128, 4), (4, 0, 4, 0, 4), (3, 0, 2, 0, 1),
+                                            (2, 0, 3, 128, 8), (4, 0, 3, 64, 2)])
+def test_attention_on_oracle_codes(tq, kb, km, vb, vm, G):
+    _attn_case(tq, kb, km, vb, vm, G, lens=[1000, 333], L=1000)
+
+
+def test_attention_edge_lengths(tq):
+    _attn_case(tq, 3, 128, 3, 128, 4, lens=[1, 0], L=300)
+    _attn_case(tq, 4, 0, 4, 0, 4, lens=[129, 128], L=129)
+    _attn_case(tq, 4, 0, 4, 0, 4, lens=[2000, 1999], L=2000, q_dtype=torch.bfloat16)
+
+
+def test_attention_end_to_end(tq):
+    """GPU encode -> GPU attention vs oracle encode -> oracle attention (prod 2+1 K and V)."""
+    B, Hkv, G, L, d = 1, 2, 4, 3000, 128
+    hk, hv = tq.Handle(d, 3, 20, qjl_m=128), tq.Handle(d, 3, 21, qjl_m=128)
+    ohk, ohv = OracleHandle(d, 2, 20, 128), OracleHandle(d, 2, 21, 128)
+    k = torch.randn(B, Hkv, L, d, generator=torch.Generator().manual_seed(1)).to(torch.bfloat16)
+    v = torch.randn(B, Hkv, L, d, generator=torch.Generator().manual_seed(2)).to(torch.bfloat16)
+    kc, vc = tq.Cache(hk, B, Hkv, L), tq.Cache(hv, B, Hkv, L)
+    kc.fill(k.cuda())
+    vc.fill(v.cuda())
+    q = torch.randn(B, Hkv * G, d, generator=torch.Generator().manual_seed(3))
+    lens = torch.tensor([L], dtype=torch.int32).cuda()
+    o = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens, 1 / np.sqrt(d)).cpu().numpy()
+    _, kod = oracle_cache(tq, hk, ohk, to_np64(k))
+    _, vod = oracle_cache(tq, hv, ohv, to_np64(v))
+    ref = ops.decode_attention(q.double().numpy(), kod, vod, [L], 1 / np.sqrt(d))
+    for h in range(Hkv * G):
+        assert np.linalg.norm(o[0, h] - ref[0, h]) <= ATTN_RTOL * np.linalg.norm(ref[0, h])
+
+
+@pytest.mark.parametrize("m", [0, 128])
+def test_append_matches_encode_and_capacity(tq, m):
+    B, Hkv, L_cap, d = 3, 2, 40, 128
+    h = tq.Handle(d, 3, 7, qjl_m=m)
+    oh = OracleHandle(d, h.bits_mse, 7, m)
+    cache = tq.Cache(h, B, Hkv, L_cap)
+    cache.codes.zero_()
+    cache.norms.zero_()
+    lens = torch.tensor([0, 5, L_cap - 2], dtype=torch.int32).cuda()
+    toks = []
+    for t in range(3):
+        x = torch.randn(B, Hkv, d, generator=torch.Generator().manual_seed(100 + t)).to(torch.bfloat16)
+        toks.append(x)
+        cache.append(x.cuda(), lens, advance=True)
+    st = h.status()
+    assert st == tq.TQ_ECAPACITY                # third append overflowed sequence 2
+    assert h.status() == tq.TQ_OK               # the error word was cleared
+    assert lens.cpu().tolist() == [3, 8, L_cap]
+    codes = cache.codes.cpu().numpy()
+    norms = cache.norms.cpu().numpy()
+    start = [0, 5, L_cap - 2]
+    for t in range(3):
+        exp = oh.encode(to_np64(toks[t]).reshape(-1, d), "f16" if m else "f32")
+        for b in range(B):
+            pos = start[b] + t
+            if pos >= L_cap:
+                continue
+            for hh in range(Hkv):
+                r = b * Hkv + hh
+                sub = {k: (v[r:r + 1] if isinstance(v, np.ndarray) and v.ndim >= 1 and len(v) == B * Hkv else v)
+                       for k, v in exp.items()}
+                check_codes(codes[b, hh, pos][None], sub, oh)
+                check_norms(norms[b, hh, pos:pos + 1], exp["n_stored"][r:r + 1])
+    # append with advance = 0 writes the slot but leaves len unchanged
+    x = torch.randn(B, Hkv, d).to(torch.bfloat16).cuda()
+    cache.append(x, lens, advance=False)
+    assert lens.cpu().tolist() == [3, 8, L_cap]
+
+
+@pytest.mark.parametrize("bits,d,n,k", [(2, 256, 20000, 10), (4, 256, 9000, 10), (3, 128, 5000, 64),
+                                        (2, 1536, 3000, 10), (4, 128, 70, 1), (2, 128, 33, 33)])
+def test_search_on_oracle_codes(tq, bits, d, n, k):
+    h = tq.Handle(d, bits, 8)
+    oh = OracleHandle(d, bits, 8)
+    db = np.random.default_rng(1).standard_normal((n, d))
+    db /= np.linalg.norm(db, axis=1, keepdims=True)
+    e = oh.encode(db, "f32")
+    codes = torch.from_numpy(quant.pack(e["idx"], bits)).cuda()
+    norms = torch.from_numpy(e["n_stored"]).cuda()
+    nq = 77
+    Q = np.random.default_rng(2).standard_normal((nq, d))
+    idx, sc = h.search_topk(torch.from_numpy(Q).float().cuda(), codes, norms, k)
+    idx, sc = idx.cpu().numpy(), sc.cpu().numpy()
+    S = ops.search_scores(Q.astype(np.float32).astype(np.float64), e["idx"], e["n_stored"], oh.Pi, oh.c)
+    ri, rs = ops.topk(S, k)
+    for i in range(nq):
+        tol = score_tolerance(S[i], np.linalg.norm(Q[i]), 1.0, d)
+        assert len(set(idx[i].tolist())) == k and idx[i].min() >= 0
+        kth = rs[i, -1]
+        assert np.all(S[i, idx[i]] >= kth - tol[idx[i]])
+        assert np.all(np.abs(sc[i] - S[i, idx[i]]) <= tol[idx[i]])
+        assert np.all(np.diff(sc[i]) <= 0)
