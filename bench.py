@@ -267,6 +267,8 @@ def run_tq(args):
         step()
     tq.tq_timer_enable(False)
     lens.fill_(L0)
+    graph.replay()                      # the captured event pairs exist only after a replay
+    lens.fill_(L0)
     torch.cuda.synchronize()
     _, kernels_per_step = tq.tq_timer_read(None, forget=False)
 

@@ -110,21 +110,27 @@ cudaEvent_t timer_event() {
   return e;
 }
 
-// Brackets one kernel launch with events when the timer is on.
+// Brackets one kernel launch with events when the timer is on. Inside a stream
+// capture the records become real event-record nodes of the graph
+// (cudaEventRecordExternal), re-recorded by every replay.
 struct KernelScope {
   const char* name;
   cudaStream_t stream;
   cudaEvent_t start = nullptr, stop = nullptr;
+  unsigned flags = cudaEventRecordDefault;
   KernelScope(const char* n, cudaStream_t s) : name(n), stream(s) {
     if (!g_timer_on.load(std::memory_order_relaxed)) return;
+    cudaStreamCaptureStatus cs = cudaStreamCaptureStatusNone;
+    if (cudaStreamIsCapturing(stream, &cs) == cudaSuccess && cs == cudaStreamCaptureStatusActive)
+      flags = cudaEventRecordExternal;
     std::lock_guard<std::mutex> lk(g_timer_mu);
     start = timer_event();
     stop = timer_event();
-    cudaEventRecord(start, stream);
+    cudaEventRecordWithFlags(start, stream, flags);
   }
   ~KernelScope() {
     if (!start) return;
-    cudaEventRecord(stop, stream);
+    cudaEventRecordWithFlags(stop, stream, flags);
     std::lock_guard<std::mutex> lk(g_timer_mu);
     g_timer_pending.push_back({name, start, stop});
   }

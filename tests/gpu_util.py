@@ -83,6 +83,8 @@ def check_norms(gpu_norms, exp_stored):
     g = np.asarray(gpu_norms).reshape(-1)
     e = np.asarray(exp_stored).reshape(-1)
     assert g.dtype == e.dtype
+    both_inf = np.isinf(e) & (g == e)          # a norm above the fp16 range saturates on both sides
+    g, e = g[~both_inf], e[~both_inf]
     ulp = np.spacing(np.abs(e)).astype(np.float64)
     err = np.abs(g.astype(np.float64) - e.astype(np.float64))
     assert np.all(err <= ulp * (1 + 1e-6)), f"norm off by {np.max(err / np.maximum(ulp, 1e-300)):.2f} ulp"
