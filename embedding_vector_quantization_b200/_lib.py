@@ -63,6 +63,7 @@ _SIGS = {
     "tq_search_workspace_bytes": (_sz, [_vp, _i, _i64, _i]),
     "tq_score": (_i, [_vp, _vp, _i, _i, _i, _cp, _vp, _vp, _vp, _sz, _vp]),
     "tq_attn_decode": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _cp, _cp, _vp, _f, _vp, _vp, _sz, _vp]),
+    "tq_attn_decode_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _cp, _cp, _vp, _f, _vp, _vp]),
     "tq_search_topk": (_i, [_vp, _vp, _i, _vp, _vp, _i64, _i, _vp, _vp, _vp, _sz, _vp]),
     "tq_timer_enable": (_i, [_i]),
     "tq_timer_read": (_i, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), _ip, _i]),
@@ -216,6 +217,13 @@ def tq_attn_decode(hk, hv, q, B, Hq, Hkv, kcache, vcache, len_, scale, out, work
     check(lib.tq_attn_decode(hk, hv, _ptr(q), _dtype_code(q), B, Hq, Hkv, ctypes.byref(kcache),
                              ctypes.byref(vcache), _ptr(len_), float(scale), _ptr(out), _ptr(workspace),
                              workspace.numel() * workspace.element_size(), _stream(stream)), "tq_attn_decode")
+
+
+def tq_attn_decode_noalloc(hk, hv, q, B, Hq, Hkv, kcache, vcache, len_, scale, out, stream=None):
+    """tq_attn_decode without a workspace (scratch from the library's fixed 4 MiB device array)."""
+    check(lib.tq_attn_decode_noalloc(hk, hv, _ptr(q), _dtype_code(q), B, Hq, Hkv, ctypes.byref(kcache),
+                                     ctypes.byref(vcache), _ptr(len_), float(scale), _ptr(out), _stream(stream)),
+          "tq_attn_decode_noalloc")
 
 
 def tq_search_topk(h, q, nq, codes, norms, n, k, idx, score, workspace, stream=None):

@@ -14,7 +14,7 @@ HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
 CSRC = os.path.join(HERE, "csrc")
 LIB = os.path.join(HERE, "libtq.so")
-SOURCES = ["tq_api.cu", "host_math.cpp"]
+SOURCES = ["tq_api.cu", "tq_noalloc.cu", "host_math.cpp"]
 ARCH = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
 

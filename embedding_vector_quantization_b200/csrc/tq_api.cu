@@ -21,6 +21,7 @@
 
 #include "tq.h"
 #include "host_math.h"
+#include "internal.h"
 #include "common.cuh"
 #include "encode_simt.cuh"
 #include "score_attn_simt.cuh"
@@ -334,6 +335,17 @@ int encode_launch(const tq_handle* h, tqk::EncodeArgs& a, cudaStream_t s) {
 }
 
 }  // namespace
+
+// Error reporting for the library's other translation units.
+int tq_internal_fail(int code, const char* fmt, ...) {
+  char buf[512];
+  va_list ap;
+  va_start(ap, fmt);
+  vsnprintf(buf, sizeof(buf), fmt, ap);
+  va_end(ap);
+  g_last_error = buf;
+  return code;
+}
 
 // ============================================================================
 extern "C" {

@@ -185,6 +185,24 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
                    const int32_t* len, float scale, float* out,
                    void* workspace, size_t ws_bytes, void* stream);
 
+/* Same computation, arguments and results as tq_attn_decode, minus the
+ * workspace. The pages have no counterpart to this call; it exists for callers
+ * that cannot allocate device memory at call time -- e.g. a plugin inside an
+ * inference engine that is handed only its input and output buffers, or a
+ * serving loop whose allocator is frozen after start-up. The split-K scratch
+ * comes from a fixed 4 MiB array compiled into libtq.so (every GPU that loads
+ * the library holds it until the process exits); nothing is allocated.
+ *  - A shape whose tq_attn_workspace_bytes exceeds 4 MiB is rejected with
+ *    TQ_EINVAL (e.g. B*Hq*nsplit*(d+m+2)*4 bytes of partial sums too large).
+ *  - The first call on a device looks up the array's device address with that
+ *    device current; make that first call before any stream capture.
+ *  - All calls share the one array and nothing in it needs to start at zero
+ *    (every call rewrites what it reads). Calls that overlap on the GPU (other
+ *    streams, other host threads) race on it: serialise them. */
+int tq_attn_decode_noalloc(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype,
+                           int B, int Hq, int Hkv, const tq_cache* k, const tq_cache* v,
+                           const int32_t* len, float scale, float* out, void* stream);
+
 /* Top-k inner-product search over n packed database vectors [HAKU "Impact on
  * high-dimensional vector search"]: for each of nq queries (device fp32 [nq][d])
  * the k largest estimated scores norm * <Pi q, c[index]> (MSE handles),
