@@ -292,6 +292,8 @@ def run_tq(args):
         dist.barrier()
     torch.cuda.synchronize()
     split_ms, split_n = 0.0, 0
+    names = ("append", "advance_len", "qprep", "attn_split", "attn_combine")
+    kern_ms = {k: 0.0 for k in names}
     for i in range(args.steps):
         set_inputs(args.warmup + i)
         flush.zero_()
@@ -300,9 +302,12 @@ def run_tq(args):
         evs[i][1].record()
         lens.fill_(L0)
         evs[i][1].synchronize()                 # captured event pairs are re-recorded by every replay
-        ms_i, n_i = tq.tq_timer_read("attn_split", forget=False)
-        split_ms += ms_i
-        split_n += n_i
+        for k in names:
+            ms_k, n_k = tq.tq_timer_read(k, forget=False)
+            kern_ms[k] += ms_k
+            if k == "attn_split":
+                split_ms += ms_k
+                split_n += n_k
     torch.cuda.synchronize()
     if world > 1:
         dist.barrier()
@@ -387,6 +392,7 @@ def run_tq(args):
                      "algorithmic_bytes_per_launch": bytes_step},
         "e2e": {"value": world * bytes_step * args.steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
                 "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "ms_per_step": e2e_ms / args.steps},
+        "kernel_us_per_step": {k: round(1e3 * v / args.steps, 3) for k, v in kern_ms.items()},
         "gpu_launches": kernels_per_step * args.steps,
         "kernels_per_step": kernels_per_step,
         "clocks": clocks,

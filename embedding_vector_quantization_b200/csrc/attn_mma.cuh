@@ -1,0 +1,574 @@
+// Decode attention over 3-bit prod caches (2-bit Lloyd-Max codes + 1-bit QJL
+// signs, m = 128) at d = 128 with 4 query heads per KV head, on int8 tensor-core
+// MMAs (mma.sync m16n8k32) fed by TMA bulk copies.
+//
+// What is computed is exactly tq_attn_decode's definition ("TurboQuant / PolarQuant
+// / QJL technical deep dive" (gemilab.net), "Scaled dot-product attention";
+// "Google TurboQuant: 6x KV-cache compression" (ebisuda.net), "Stage 1" and
+// "Stage 2"); only the arithmetic is rearranged so that the packed bits feed the
+// tensor cores directly:
+//
+//  * A symmetric 2-bit codebook is affine in the two index bits:
+//    c[idx] = c0 + (c1 - c0) b0 + (c2 - c0) b1  (the b0*b1 coefficient
+//    c3 - c2 - c1 + c0 vanishes by symmetry). So <q', c[idx]> is c0*sum(q') plus
+//    two 0/1 dot products, and sum_i w_i c[idx_ij] is c0*sum(w) plus two 0/1
+//    weighted sums. Sign bits give <qs, 2 sigma - 1> = 2 <qs, sigma> - sum(qs).
+//  * 0/1 bit planes become int8 MMA operands with one AND per 4 elements:
+//    (word >> s) & 0x01010101 (value 1) or (word >> s) & 0x10101010 (value 16);
+//    every MMA uses one of the two mask families, so its accumulator is exact
+//    after a final division by 16 (kept in separate accumulators for keys).
+//  * Query side (keys as the MMA rows): queries are rotated once, scaled by the
+//    codebook slopes, rounded to 15-bit integers and split into two int8 pieces
+//    (hi * 128 + lo), which fill the 8 MMA columns (4 heads x 2 pieces).
+//  * Value side (bit rows of the value codes as the MMA rows, tokens as the
+//    reduction): softmax weights p * ||v|| (and p * rnorm for the QJL part) are
+//    rounded to 14-bit integers against the chunk maximum and split into two
+//    int8 pieces; ldmatrix .trans.b8 gathers "byte j of 4 consecutive tokens"
+//    into one register.
+//  * Two passes per context chunk: all key scores first (kept in shared memory,
+//    giving the exact chunk maximum), then all values with one fixed weight
+//    scale, so the value sums accumulate in int32 across the whole chunk.
+//
+// Partial results use the layout of the split kernel in score_attn_simt.cuh
+// ([B*Hq][nsplit][d + m + 2]: rotated-domain value sum, QJL sum, max, sum of
+// weights) and are merged by the combine kernel.
+#pragma once
+
+#include "common.cuh"
+#include "small_kernels.cuh"
+
+namespace tqk {
+namespace amma {
+
+constexpr int kD = 128;
+constexpr int kM = 128;
+constexpr int kG = 4;
+constexpr int kBlk = 256;                     // tokens per pipeline block
+constexpr int kStages = 5;
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kCodesB = 32, kSignsB = 16;
+constexpr int kStageCodes = kBlk * kCodesB;   // 8192
+constexpr int kStageSigns = kBlk * kSignsB;   // 4096
+// key block: codes, signs, norms, rnorms + the value norms and rnorms of the same tokens;
+// value block: codes and signs only (its norms came with the key block)
+constexpr int kStageBytes = kStageCodes + kStageSigns + 4 * kBlk * 2;  // 14336
+constexpr int kMaxChunk = 1024;
+
+struct Args {
+  const float* qr;  // [B*Hq][128] Pi_K q
+  const float* qs;  // [B*Hq][128] S_K q
+  int B, Hq, Hkv;
+  const uint8_t* kcodes;
+  const uint8_t* ksigns;
+  const __half* knorm;
+  const __half* krn;
+  const uint8_t* vcodes;
+  const uint8_t* vsigns;
+  const __half* vnorm;
+  const __half* vrn;
+  int64_t L_cap, chunk;
+  int nsplit;
+  const int32_t* len;
+  float kc0, kb0, kb1;  // K codebook: c[idx] = kc0 + kb0*b0 + kb1*b1
+  float vc0, vb0, vb1;  // V codebook
+  float scale;          // softmax scale
+  float* part;          // [B*Hq][nsplit][d + m + 2]
+  int* err;
+};
+
+struct __align__(16) Smem {
+  unsigned char stage[kStages][kStageBytes];
+  // key pass: scaled logits [head][token]; value pass: the integer softmax weights of every
+  // block, [block][0: value weights, 1: QJL weights][col = head*2 + piece][token] (same bytes)
+  float logits[kG][kMaxChunk];
+  uint32_t qfrag[12][2][4][8];  // key-side B fragments: [k-step][register][quad index t][column g]
+  float qconst[kG][4];        // c0*sum(q'), delta_mse, delta_qjl, sum(qs)
+  float red_f[kWarps][kG];
+  float hmax[kG];
+  float nmax[2];
+  int red_i[kWarps][2 * kG];
+  float vacc[3][kG][128];     // value-side sums of the two token halves (rows of each byte group)
+  __half vnorm[kMaxChunk];    // value norms and residual norms of the chunk (copied with the key blocks)
+  __half vrn[kMaxChunk];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];    // one arrival per warp when it is done with the stage
+  int W[2][kG];               // chunk sums of the integer value / QJL weights per head
+  int abort_flag;
+};
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void mbar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_u32(bar)), "r"(bytes)
+               : "memory");
+}
+
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity) { return bar_wait(bar, parity); }
+
+__device__ __forceinline__ void tma_bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(src), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+               "{%0,%1,%2,%3};\n"
+               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ void ldsm_x4(uint32_t (&r)[4], const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x4.shared.b16 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(row_addr)));
+}
+
+__device__ __forceinline__ void ldsm_x2(uint32_t (&r)[2], const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m8n8.x2.shared.b16 {%0,%1}, [%2];\n"
+               : "=r"(r[0]), "=r"(r[1])
+               : "r"(smem_u32(row_addr)));
+}
+
+// Two 16x16 byte tiles, transposed: r[0], r[1] = tile 0 columns g, g+8 of rows
+// 4t..4t+3; r[2], r[3] = the same for tile 1 (g = lane/4, t = lane%4).
+__device__ __forceinline__ void ldsm_t8_x2(uint32_t (&r)[4], const void* row_addr) {
+  asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0,%1,%2,%3}, [%4];\n"
+               : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
+               : "r"(smem_u32(row_addr)));
+}
+
+__device__ __forceinline__ uint32_t pack4(int8_t a, int8_t b, int8_t c, int8_t d) {
+  return (uint32_t)(uint8_t)a | ((uint32_t)(uint8_t)b << 8) | ((uint32_t)(uint8_t)c << 16) |
+         ((uint32_t)(uint8_t)d << 24);
+}
+
+// Where a query-side element sits in the key-side B fragments (inverse of the
+// A-operand construction in the key pass): returns the byte offset within
+// qfrag for column g = 0. Code plane p of code c: k-step 2(c%4)+p, register
+// c/64, quad index (c/16)%4, byte (c%16)/4. Sign bit i: word t = i/32, byte
+// e = (i%32)/8, bit u = i%8 -> k-step 8+u (u<2), 8+u-2 (u=2,3), 10+u-4
+// (u=4,5), 10+u-6 (u=6,7); register 0 for u in {0,1,4,5}, 1 otherwise.
+__device__ __forceinline__ int qfrag_code_offset(int plane, int c) {
+  const int kk = 2 * (c & 3) + plane, slot = c >> 6, t = (c >> 4) & 3, e = (c & 15) >> 2;
+  return (((kk * 2 + slot) * 4 + t) * 8) * 4 + e;
+}
+__device__ __forceinline__ int qfrag_sign_offset(int i) {
+  const int t = i >> 5, e = (i & 31) >> 3, u = i & 7;
+  const int grp = (u < 4) ? 8 : 10, w = u & 3, slot = w >> 1, s = w & 1;
+  const int kk = grp + s;
+  return (((kk * 2 + slot) * 4 + t) * 8) * 4 + e;
+}
+
+__global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int bh = blockIdx.x, split = blockIdx.y;
+  const int b = bh / a.Hkv, hk = bh % a.Hkv, h0 = hk * kG;
+
+  const int64_t L = min((int64_t)max(a.len[b], 0), a.L_cap);
+  const int64_t start = (int64_t)split * a.chunk;
+  const int64_t end = min(L, start + a.chunk);
+  const int ntok = (int)max((int64_t)0, end - start);
+  const int nblk = (ntok + kBlk - 1) / kBlk;
+  const int64_t row0 = (int64_t)bh * a.L_cap + start;  // cache row of the chunk's first token
+
+  // ---------------- setup: barriers, query pieces
+  if (tid == 0) {
+    for (int s = 0; s < kStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kWarps);
+    }
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+
+  auto issue = [&](int j) {  // block j: K block (j < nblk) or V block j - nblk
+    const bool kside = j < nblk;
+    const int jj = kside ? j : j - nblk;
+    const int64_t tok0 = (int64_t)jj * kBlk;
+    const int64_t left = a.L_cap - (start + tok0);
+    const int ncopy = (int)min((int64_t)kBlk, left);   // multiple of 8 (L_cap % 8 == 0)
+    const int64_t r = row0 + tok0;
+    unsigned char* st = sm.stage[j % kStages];
+    uint64_t* bar = &sm.full[j % kStages];
+    const uint32_t bytes = (uint32_t)ncopy * (kCodesB + kSignsB + (kside ? 8 : 0));
+    mbar_expect_tx(bar, bytes);
+    tma_bulk_g2s(st, (kside ? a.kcodes : a.vcodes) + r * kCodesB, ncopy * kCodesB, bar);
+    tma_bulk_g2s(st + kStageCodes, (kside ? a.ksigns : a.vsigns) + r * kSignsB, ncopy * kSignsB, bar);
+    if (kside) {
+      unsigned char* nb = st + kStageCodes + kStageSigns;
+      tma_bulk_g2s(nb, a.knorm + r, ncopy * 2, bar);
+      tma_bulk_g2s(nb + 2 * kBlk, a.krn + r, ncopy * 2, bar);
+      tma_bulk_g2s(nb + 4 * kBlk, a.vnorm + r, ncopy * 2, bar);
+      tma_bulk_g2s(nb + 6 * kBlk, a.vrn + r, ncopy * 2, bar);
+    }
+  };
+  const int njobs = 2 * nblk;
+  constexpr int kAhead = kStages - 2;   // jobs in flight ahead of the one being consumed (3)
+  if (tid == 0)
+    for (int j = 0; j < min(kAhead, njobs); ++j) issue(j);
+
+  // query constants and int8 pieces (one warp per head)
+  if (warp < kG) {
+    const int h = warp;
+    const float* qr = a.qr + ((size_t)b * a.Hq + h0 + h) * kD;
+    const float* qsv = a.qs + ((size_t)b * a.Hq + h0 + h) * kM;
+    float x0[4], x1[4], xs[4], sq = 0.f, ss = 0.f, mx = 0.f, ms = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const float q = qr[lane + 32 * i];
+      const float s = qsv[lane + 32 * i];
+      x0[i] = a.kb0 * q;
+      x1[i] = a.kb1 * q;
+      xs[i] = s;
+      sq += q;
+      ss += s;
+      mx = fmaxf(mx, fmaxf(fabsf(x0[i]), fabsf(x1[i])));
+      ms = fmaxf(ms, fabsf(s));
+    }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      ss += __shfl_xor_sync(0xffffffffu, ss, o);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+      ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
+    }
+    const float dm = mx > 0.f ? mx / 16256.f : 1.f;
+    const float ds = ms > 0.f ? ms / 16256.f : 1.f;
+    int8_t* qf = reinterpret_cast<int8_t*>(&sm.qfrag[0][0][0][0]);
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      const int j = lane + 32 * i;
+      const float v[3] = {x0[i] / dm, x1[i] / dm, xs[i] / ds};
+#pragma unroll
+      for (int c = 0; c < 3; ++c) {
+        const int xi = __float2int_rn(v[c]);
+        const int hi = (xi >= 0) ? (xi + 64) >> 7 : -((-xi + 64) >> 7);
+        const int off = (c < 2) ? qfrag_code_offset(c, j) : qfrag_sign_offset(j);
+        qf[off + (2 * h) * 4] = (int8_t)hi;               // column g = 2h (hi piece)
+        qf[off + (2 * h + 1) * 4] = (int8_t)(xi - 128 * hi);  // column g = 2h + 1 (lo piece)
+      }
+    }
+    if (lane == 0) {
+      sm.qconst[h][0] = a.kc0 * sq;
+      sm.qconst[h][1] = dm;
+      sm.qconst[h][2] = ds;
+      sm.qconst[h][3] = ss;
+    }
+  }
+  __syncthreads();
+
+  // B fragments of the key-side MMAs (constant for the CTA): 12 k-steps x 2 registers
+  uint32_t qb[12][2];
+#pragma unroll
+  for (int kk = 0; kk < 12; ++kk)
+#pragma unroll
+    for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[kk][slot][t][g];
+
+  const float kqjl = kQjlScale / (float)kM;
+  float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
+  float run_max = -INFINITY;   // this thread's max logit of head t
+  float vn_max = 0.f, vr_max = 0.f;
+
+  // value-side accumulators: 8 m-tiles (bit rows 0..7 of bytes g, g+8 of this warp's byte group)
+  int vacc[8][4];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) vacc[u][0] = vacc[u][1] = vacc[u][2] = vacc[u][3] = 0;
+  float lsum = 0.f;            // sum of p for head (P-warps)
+  int wsum[2] = {0, 0};        // sum of integer weights (value, QJL) for head (P-warps)
+
+  const int bg = warp % 3, half = warp / 3;   // value side: byte group and token half (warps 0..5)
+  float dv1 = 1.f, dv2 = 1.f, inv1 = 1.f, inv2 = 1.f;
+
+  // No warp ever leaves this loop early: a wait that runs out sets abort_flag, after
+  // which nothing new is issued and no further waits happen, so every warp still
+  // meets the same CTA barriers; the results are then discarded.
+  int issued = min(kAhead, njobs);
+  for (int j = 0; j < njobs; ++j) {
+    const bool aborted = *(volatile int*)&sm.abort_flag != 0;
+    if (tid == 0 && !aborted && j + kAhead < njobs) {
+      // refill the stage of job j + kAhead - kStages (= j - 2) once every warp has released it
+      const int jo = j + kAhead - kStages;   // = j - 2
+      if (jo >= 0 && !mbar_wait(&sm.empty[jo % kStages], (jo / kStages) & 1)) {
+        sm.abort_flag = 1;
+      } else {
+        issue(j + kAhead);
+        issued = j + kAhead + 1;
+      }
+    }
+    if (!aborted && !mbar_wait(&sm.full[j % kStages], (j / kStages) & 1)) sm.abort_flag = 1;
+    const bool kside = j < nblk;
+    const int jj = kside ? j : j - nblk;
+    const unsigned char* st = sm.stage[j % kStages];
+    const __half* nrm = reinterpret_cast<const __half*>(st + kStageCodes + kStageSigns);
+    const __half* rnm = nrm + kBlk;
+    const int tok_base = jj * kBlk;
+    const int nvalid = min(kBlk, ntok - tok_base);
+
+    if (j == nblk) {
+      // ------------ between the passes: chunk maxima, weight scales, first P block
+      __syncthreads();
+      if (lane == 0) {
+        for (int h = 0; h < kG; ++h) sm.red_f[warp][h] = -INFINITY;
+      }
+      __syncwarp();
+      float m = run_max;
+#pragma unroll
+      for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      if (g == 0) sm.red_f[warp][t] = m;
+      float vn = vn_max, vr = vr_max;
+#pragma unroll
+      for (int o = 1; o < 32; o <<= 1) {
+        vn = fmaxf(vn, __shfl_xor_sync(0xffffffffu, vn, o));
+        vr = fmaxf(vr, __shfl_xor_sync(0xffffffffu, vr, o));
+      }
+      if (lane == 0) sm.red_i[warp][0] = __float_as_int(vn), sm.red_i[warp][1] = __float_as_int(vr);
+      __syncthreads();
+      if (tid < kG) {
+        float mm = -INFINITY;
+        for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.red_f[w][tid]);
+        sm.hmax[tid] = mm;
+      }
+      if (tid == 0) {
+        float n1 = 0.f, n2 = 0.f;
+        for (int w = 0; w < kWarps; ++w) {
+          n1 = fmaxf(n1, __int_as_float(sm.red_i[w][0]));
+          n2 = fmaxf(n2, __int_as_float(sm.red_i[w][1]));
+        }
+        sm.nmax[0] = n1;
+        sm.nmax[1] = n2;
+      }
+      __syncthreads();
+      dv1 = sm.nmax[0] > 0.f ? sm.nmax[0] / 16383.f : 1.f;
+      dv2 = sm.nmax[1] > 0.f ? sm.nmax[1] / 16383.f : 1.f;
+      inv1 = 1.f / dv1;
+      inv2 = 1.f / dv2;
+      // integer weights of the whole chunk; they overwrite the logits, so read first.
+      // thread -> (head h, 4 consecutive tokens) per round; 4-byte stores of 4 tokens.
+      constexpr int kRounds = kMaxChunk * kG / (4 * kThreads);   // 8
+      const int h = tid & 3;
+      float4 lg[kRounds];
+#pragma unroll
+      for (int u = 0; u < kRounds; ++u) {
+        const int tok4 = 4 * ((tid >> 2) + u * (kThreads / 4));
+        lg[u] = (tok4 < nblk * kBlk) ? *reinterpret_cast<const float4*>(&sm.logits[h][tok4])
+                                     : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+      const float hm = sm.hmax[h];
+      __syncthreads();
+      int8_t* pw = reinterpret_cast<int8_t*>(&sm.logits[0][0]);
+#pragma unroll
+      for (int u = 0; u < kRounds; ++u) {
+        const int tok4 = 4 * ((tid >> 2) + u * (kThreads / 4));
+        if (tok4 >= nblk * kBlk) break;
+        const float l4[4] = {lg[u].x, lg[u].y, lg[u].z, lg[u].w};
+        uint32_t w1h = 0, w1l = 0, w2h = 0, w2l = 0;
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const int tok = tok4 + q;
+          const bool ok = tok < ntok;
+          const float p = ok ? __expf(l4[q] - hm) : 0.f;
+          const int w1 = ok ? __float2int_rn(p * __half2float(sm.vnorm[tok]) * inv1) : 0;
+          const int w2 = ok ? __float2int_rn(p * __half2float(sm.vrn[tok]) * inv2) : 0;
+          w1h |= (uint32_t)(w1 >> 7) << (8 * q);
+          w1l |= (uint32_t)(w1 & 127) << (8 * q);
+          w2h |= (uint32_t)(w2 >> 7) << (8 * q);
+          w2l |= (uint32_t)(w2 & 127) << (8 * q);
+          lsum += p;
+          wsum[0] += w1;
+          wsum[1] += w2;
+        }
+        int8_t* blk = pw + (tok4 / kBlk) * (2 * 8 * kBlk);
+        const int tk = tok4 & (kBlk - 1);
+        *reinterpret_cast<uint32_t*>(blk + (2 * h) * kBlk + tk) = w1h;
+        *reinterpret_cast<uint32_t*>(blk + (2 * h + 1) * kBlk + tk) = w1l;
+        *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h) * kBlk + tk) = w2h;
+        *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h + 1) * kBlk + tk) = w2l;
+      }
+      __syncthreads();
+    }
+
+    if (kside) {
+      // ---------------- key pass: warp w scores keys 16w .. 16w+15 and 128+16w .. of the block
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int kbase = 128 * mt + 16 * warp;
+        uint32_t cw[4], sw[2];
+        {
+          const int mat = lane >> 3, r = lane & 7;
+          const int key = kbase + r + 8 * (mat >> 1);
+          ldsm_x4(cw, st + key * kCodesB + 16 * (mat & 1));
+          const int skey = kbase + r + 8 * (mat & 1);
+          ldsm_x2(sw, st + kStageCodes + skey * kSignsB);
+        }
+        // six independent accumulator chains of length two (even / odd shifts)
+        int dm1[2][4] = {}, dm16[2][4] = {}, ds1[4] = {}, ds16[4] = {};
+        // code words: cw[0] = key g word t, cw[1] = key g word 4+t, cw[2] = key g+8 word t, cw[3] = key g+8 word 4+t
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint32_t x0 = cw[0] >> s, x1 = cw[1] >> s, x2 = cw[2] >> s, x3 = cw[3] >> s;
+          mma_s8(dm1[s & 1], x0 & 0x01010101u, x2 & 0x01010101u, x1 & 0x01010101u, x3 & 0x01010101u, qb[s][0],
+                 qb[s][1]);
+          mma_s8(dm16[s & 1], x0 & 0x10101010u, x2 & 0x10101010u, x1 & 0x10101010u, x3 & 0x10101010u,
+                 qb[4 + s][0], qb[4 + s][1]);
+        }
+        // sign words: sw[0] = key g word t, sw[1] = key g+8 word t
+#pragma unroll
+        for (int s = 0; s < 2; ++s) {
+          const uint32_t y0 = sw[0] >> s, y1 = sw[1] >> s, z0 = sw[0] >> (s + 2), z1 = sw[1] >> (s + 2);
+          mma_s8(ds1, y0 & 0x01010101u, y1 & 0x01010101u, z0 & 0x01010101u, z1 & 0x01010101u, qb[8 + s][0],
+                 qb[8 + s][1]);
+          mma_s8(ds16, y0 & 0x10101010u, y1 & 0x10101010u, z0 & 0x10101010u, z1 & 0x10101010u, qb[10 + s][0],
+                 qb[10 + s][1]);
+        }
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
+          const int key = kbase + g + 8 * r;
+          const int hi = 2 * r, lo = 2 * r + 1;
+          const int mse = 128 * (dm1[0][hi] + dm1[1][hi] + ((dm16[0][hi] + dm16[1][hi]) >> 4)) +
+                          (dm1[0][lo] + dm1[1][lo] + ((dm16[0][lo] + dm16[1][lo]) >> 4));
+          const int qjl = 128 * (ds1[hi] + (ds16[hi] >> 4)) + (ds1[lo] + (ds16[lo] >> 4));
+          const float n = __half2float(nrm[key]), rn = __half2float(rnm[key]);
+          float sc = n * (c0h + dmh * (float)mse) + rn * kqjl * (2.f * dsh * (float)qjl - ssh);
+          sc *= a.scale;
+          sc = (key < nvalid) ? sc : -INFINITY;
+          sm.logits[t][tok_base + key] = sc;
+          run_max = fmaxf(run_max, sc);
+        }
+      }
+      // value norms of these tokens (they arrived with the key block): keep for the value pass
+      if (tid < kBlk) {
+        const __half vn = nrm[2 * kBlk + tid], vr = nrm[3 * kBlk + tid];
+        sm.vnorm[tok_base + tid] = vn;
+        sm.vrn[tok_base + tid] = vr;
+        if (tid < nvalid) {
+          vn_max = fmaxf(vn_max, __half2float(vn));
+          vr_max = fmaxf(vr_max, __half2float(vr));
+        }
+      }
+    } else {
+      // ---------------- value pass (warps 0..5: byte group bg, token half)
+      if (warp < 6) {
+        const int8_t* pw = reinterpret_cast<const int8_t*>(&sm.logits[0][0]) + jj * (2 * 8 * kBlk) +
+                           (bg == 2 ? 8 * kBlk : 0);
+#pragma unroll
+        for (int kq = 0; kq < 4; ++kq) {
+          const int tk = 128 * half + 32 * kq;  // first token of this 32-token k-step
+          uint32_t r[4];
+          const int tok = tk + (lane & 15) + 16 * (lane >> 4);
+          const unsigned char* rowp = (bg < 2) ? st + tok * kCodesB + 16 * bg : st + kStageCodes + tok * kSignsB;
+          ldsm_t8_x2(r, rowp);
+          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(pw + g * kBlk + tk + 4 * t);
+          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(pw + g * kBlk + tk + 16 + 4 * t);
+#pragma unroll
+          for (int s = 0; s < 4; ++s) {
+            const uint32_t x0 = r[0] >> s, x1 = r[1] >> s, x2 = r[2] >> s, x3 = r[3] >> s;
+            mma_s8(vacc[s], x0 & 0x01010101u, x1 & 0x01010101u, x2 & 0x01010101u, x3 & 0x01010101u, b0, b1);
+            mma_s8(vacc[4 + s], x0 & 0x10101010u, x1 & 0x10101010u, x2 & 0x10101010u, x3 & 0x10101010u, b0, b1);
+          }
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[j % kStages])) : "memory");
+  }
+
+  __syncthreads();
+  if (sm.abort_flag) {
+    // a copy or a release never completed: record it, then wait (bounded) for the
+    // copies that may still be in flight into this CTA's shared memory before leaving
+    if (tid == 0) {
+      report_error(a.err, kErrTimeout);
+      for (int jx = max(0, issued - kStages); jx < issued; ++jx)
+        (void)mbar_wait(&sm.full[jx % kStages], (jx / kStages) & 1);
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---------------- sums of p and integer weights per head (held by threads with lane & 3 == head)
+  {
+    float l = lsum;
+    int w1 = wsum[0], w2 = wsum[1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l += __shfl_xor_sync(0xffffffffu, l, o);
+      w1 += __shfl_xor_sync(0xffffffffu, w1, o);
+      w2 += __shfl_xor_sync(0xffffffffu, w2, o);
+    }
+    if (lane < kG) {
+      sm.red_f[warp][lane] = l;
+      sm.red_i[warp][lane] = w1;
+      sm.red_i[warp][kG + lane] = w2;
+    }
+  }
+  // value sums of the two token halves -> shared (half 1 writes, half 0 adds); rows are
+  // (byte g, bit u) -> [g * 8 + u] and (byte g + 8, bit u) -> [64 + g * 8 + u]; columns head t (hi, lo)
+  if (warp >= 3 && warp < 6) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int f = (u < 4) ? 0 : 4;
+      const float v0 = 128.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
+      const float v1 = 128.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
+      sm.vacc[bg][t][g * 8 + u] = v0;          // byte g, bit u
+      sm.vacc[bg][t][64 + g * 8 + u] = v1;     // byte g + 8, bit u
+    }
+  }
+  __syncthreads();
+  if (warp < 3) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int f = (u < 4) ? 0 : 4;
+      const float v0 = 128.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
+      const float v1 = 128.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
+      sm.vacc[bg][t][g * 8 + u] += v0;
+      sm.vacc[bg][t][64 + g * 8 + u] += v1;
+    }
+  }
+  __syncthreads();
+
+  // ---------------- partial outputs: rotated-domain value sum, QJL sum, max, sum of p
+  const int stride = partial_stride(kD, kM);
+  for (int i = tid; i < kG * (kD + kM); i += kThreads) {
+    const int h = i / (kD + kM), j = i % (kD + kM);
+    int W1 = 0, W2 = 0;
+    for (int w = 0; w < kWarps; ++w) { W1 += sm.red_i[w][h]; W2 += sm.red_i[w][kG + h]; }
+    float v;
+    if (j < kD) {
+      // code c = j: byte c / 4 (group c / 64), bits 2(c % 4) (plane 0) and 2(c % 4) + 1 (plane 1)
+      const int byte = j >> 2, grp = byte >> 4, bl = byte & 15, u0 = 2 * (j & 3);
+      const int idx = (bl < 8) ? bl * 8 : 64 + (bl - 8) * 8;
+      const float d0 = sm.vacc[grp][h][idx + u0], d1 = sm.vacc[grp][h][idx + u0 + 1];
+      v = dv1 * (a.vc0 * (float)W1 + a.vb0 * d0 + a.vb1 * d1);
+    } else {
+      const int p = j - kD, byte = p >> 3, u = p & 7;
+      const int idx = (byte < 8) ? byte * 8 + u : 64 + (byte - 8) * 8 + u;
+      v = dv2 * (2.f * sm.vacc[2][h][idx] - (float)W2);
+    }
+    a.part[(((size_t)b * a.Hq + h0 + h) * a.nsplit + split) * stride + j] = v;
+  }
+  if (tid < kG) {
+    float l = 0.f;
+    for (int w = 0; w < kWarps; ++w) l += sm.red_f[w][tid];
+    float* o = a.part + (((size_t)b * a.Hq + h0 + tid) * a.nsplit + split) * stride;
+    o[kD + kM] = (ntok > 0) ? sm.hmax[tid] : -INFINITY;
+    o[kD + kM + 1] = (ntok > 0) ? l : 0.f;
+  }
+}
+
+}  // namespace amma
+}  // namespace tqk

@@ -69,4 +69,52 @@ __device__ __forceinline__ uint32_t sign_bit(const uint32_t* row, int j) {
   return (row[j >> 5] >> (j & 31)) & 1u;
 }
 
+// ---- TMA bulk copies (global -> shared) completed on an mbarrier
+
+__device__ __forceinline__ uint32_t smem_addr(const void* p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void bar_init(uint64_t* bar, int count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(count));
+  asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+}
+
+__device__ __forceinline__ void bar_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;\n" ::"r"(smem_addr(bar)), "r"(bytes)
+               : "memory");
+}
+
+// Bounded wait (the thread sleeps between polls); false if the limit was reached.
+__device__ __forceinline__ bool bar_wait(uint64_t* bar, uint32_t parity, int limit = 1 << 16) {
+  const uint32_t addr = smem_addr(bar);
+  for (int it = 0; it < limit; ++it) {
+    uint32_t done;
+    asm volatile(
+        "{\n .reg .pred p;\n mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2, %3;\n selp.u32 %0, 1, 0, p;\n}\n"
+        : "=r"(done)
+        : "r"(addr), "r"(parity), "r"(20000)
+        : "memory");
+    if (done) return true;
+  }
+  return false;
+}
+
+// One contiguous copy; dst, src 16-byte aligned and bytes a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];\n" ::"r"(
+          smem_addr(dst)),
+      "l"(src), "r"(bytes), "r"(smem_addr(bar))
+      : "memory");
+}
+
+// Copies `bytes` (<= 2^20 per call chunk) in pieces the bulk engine accepts.
+__device__ __forceinline__ void bulk_g2s_large(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  const uint32_t piece = 1u << 16;
+  for (uint32_t off = 0; off < bytes; off += piece)
+    bulk_g2s(static_cast<unsigned char*>(dst) + off, static_cast<const unsigned char*>(src) + off,
+             min(piece, bytes - off), bar);
+}
+
 }  // namespace tqk

@@ -43,7 +43,7 @@ struct EncodeArgs {
   __half* rnorms;
   // append mode (len != nullptr): input row r = b * Hkv + h goes to cache row
   // r * L_cap + len[b]; a full sequence is skipped and flagged.
-  const int32_t* len;
+  int32_t* len;
   int Hkv;
   int64_t L_cap;
   int* err;

@@ -19,6 +19,7 @@
 #pragma once
 
 #include "common.cuh"
+#include "small_kernels.cuh"
 
 namespace tqk {
 
@@ -29,26 +30,61 @@ constexpr int kMaxHeadDim = 256;
 // ---------------------------------------------------------------- query prep
 
 // out_r[row][j] = sum_k Pi[j][k] q[row][k];  out_s[row][i] = sum_k S[i][k] q[row][k].
-// One warp per output element; lanes stride over k (coalesced rows of Pi / S).
-__global__ void qprep_kernel(const void* q, int q_dtype, int rows, int d, const float* Pi,
-                             const float* S, int m, float* out_r, float* out_s) {
-  extern __shared__ float qsh[];
-  const int row = blockIdx.x;
-  for (int k = threadIdx.x; k < d; k += blockDim.x) qsh[k] = load_any(q, q_dtype, (int64_t)row * d + k);
+// One CTA per group of up to kQprepRows query rows and 64 output rows of
+// [Pi; S]; four threads share an output row, each loading its quarter of the
+// matrix row at once (16-byte loads, all in flight), then two shuffles combine
+// the quarters. Each loaded element serves every query row of the group.
+constexpr int kQprepRows = 8;
+__global__ void __launch_bounds__(256) qprep_kernel(const void* q, int q_dtype, int rows, int d, const float* Pi,
+                                                    const float* S, int m, float* out_r, float* out_s) {
+  extern __shared__ float qsh[];   // [kQprepRows][d]
+  const int row0 = blockIdx.x * kQprepRows;
+  const int nr = min(kQprepRows, rows - row0);
+  const int o = blockIdx.y * 64 + (threadIdx.x >> 2), part = threadIdx.x & 3;
+  const int q4 = d / 16;           // float4s per quarter row (d % 32 == 0)
+  constexpr int kMaxQ4 = 64;       // d <= 4096
+  float4 mv[kMaxQ4 / 8];
+  const bool active = o < d + m;
+  const float4* mrow = nullptr;
+  if (active) {
+    mrow = reinterpret_cast<const float4*>((o < d) ? (Pi + (size_t)o * d) : (S + (size_t)(o - d) * d)) + part * q4;
+  }
+  for (int i = threadIdx.x; i < nr * d; i += blockDim.x) qsh[i] = load_any(q, q_dtype, (int64_t)row0 * d + i);
   __syncthreads();
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31, nw = blockDim.x >> 5;
-  const int total = d + m;
-  for (int o = blockIdx.y * nw + warp; o < total; o += gridDim.y * nw) {
-    const float* mrow = (o < d) ? (Pi + (size_t)o * d) : (S + (size_t)(o - d) * d);
-    float acc = 0.f;
-    for (int k = lane; k < d; k += 32) acc = fmaf(mrow[k], qsh[k], acc);
+  float acc[kQprepRows];
 #pragma unroll
-    for (int s = 16; s > 0; s >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, s);
-    if (lane == 0) {
+  for (int r = 0; r < kQprepRows; ++r) acc[r] = 0.f;
+  for (int c0 = 0; c0 < q4; c0 += kMaxQ4 / 8) {
+    const int nc = min(kMaxQ4 / 8, q4 - c0);
+#pragma unroll
+    for (int u = 0; u < kMaxQ4 / 8; ++u)
+      mv[u] = (active && u < nc) ? mrow[c0 + u] : make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+    for (int u = 0; u < kMaxQ4 / 8; ++u) {
+      if (u >= nc) break;
+      const int k = 4 * (part * q4 + c0 + u);
+#pragma unroll
+      for (int r = 0; r < kQprepRows; ++r) {
+        if (r < nr) {
+          const float* qq = qsh + r * d + k;
+          acc[r] = fmaf(mv[u].x, qq[0], fmaf(mv[u].y, qq[1], fmaf(mv[u].z, qq[2], fmaf(mv[u].w, qq[3], acc[r]))));
+        }
+      }
+    }
+  }
+#pragma unroll
+  for (int r = 0; r < kQprepRows; ++r) {
+    acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 1);
+    acc[r] += __shfl_xor_sync(0xffffffffu, acc[r], 2);
+  }
+  if (active && part == 0) {
+#pragma unroll
+    for (int r = 0; r < kQprepRows; ++r) {
+      if (r >= nr) break;
       if (o < d)
-        out_r[(size_t)row * d + o] = acc;
+        out_r[(size_t)(row0 + r) * d + o] = acc[r];
       else
-        out_s[(size_t)row * m + (o - d)] = acc;
+        out_s[(size_t)(row0 + r) * m + (o - d)] = acc[r];
     }
   }
 }
@@ -148,7 +184,7 @@ struct AttnArgs {
   int nsplit;
   const int32_t* len;
   float scale;
-  float* part;      // [B*Hq][nsplit][d + mv + 2]
+  float* part;      // [B*Hq][nsplit][partial_stride(d, mv)]
 };
 
 __global__ void __launch_bounds__(kAttnThreads) attn_split_simt_kernel(AttnArgs a) {
@@ -268,7 +304,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_simt_kernel(AttnArgs 
     __syncthreads();
   }
 
-  const int stride = d + mv + 2;
+  const int stride = partial_stride(d, mv);
 #pragma unroll
   for (int g = 0; g < kMaxGroup; ++g) {
     if (g >= G) break;
@@ -284,50 +320,92 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_simt_kernel(AttnArgs 
 }
 
 struct CombineArgs {
-  const float* part;  // [B*Hq][nsplit][d + mv + 2]
-  int rows, nsplit, d, mv;
+  const float* part;  // [B*Hq][nsplit][partial_stride(d, mv)]
+  int Hq, Hkv, nsplit, d, mv;
   const float* PiV;   // [d][d] row-major
   const float* SV;    // [mv][d] row-major
   float* out;         // [B*Hq][d]
 };
 
-__global__ void attn_combine_kernel(CombineArgs a) {
+constexpr int kCombineThreads = 1024;
+
+// One CTA per (sequence, query head). Thread (j, part) first issues its loads
+// of an eighth of column j of [Pi_V; sqrt(pi/2)/m S_V] (so they travel while the
+// chunk weights are merged), then:
+// 1) log-sum-exp weights of the chunks (warp 0);
+// 2) merged rotated-domain sums acc (d) and QJL sums (mv), two threads per entry;
+// 3) o_j = (sum_k Pi_V[k][j] acc_k + sqrt(pi/2)/m sum_k S_V[k][j] acc_s_k) / sum p.
+__global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(CombineArgs a) {
   extern __shared__ float sm[];
-  const int row = blockIdx.x;
-  const int d = a.d, mv = a.mv, stride = d + mv + 2;
-  float* accv = sm;            // [d]
-  float* accs = accv + d;      // [mv]
-  float* w = accs + mv;        // [nsplit]
-  float* red = w + a.nsplit;   // [2]
+  const int d = a.d, mv = a.mv, stride = partial_stride(d, mv), dm = d + mv;
+  const int row = blockIdx.x;                   // b * Hq + h
+  float* w = sm;                                // [nsplit]
+  float* acc = w + a.nsplit;                    // [2][d + mv] (two halves of the splits)
+  float* part_o = acc + 2 * dm;                 // [8][d]
+  float* Ls = part_o + 8 * d;                   // [1]
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const float qscale = (mv > 0) ? kQjlScale / (float)mv : 0.f;
+  constexpr int kMaxRows = 32;                  // per part: (d + mv) / 8 <= 32 (d + mv <= 256)
+  const int quarter = tid >> 7, j = tid & 127;  // quarter = part 0..7
+  const int kq = (dm + 7) / 8, k0 = quarter * kq, k1 = min(dm, k0 + kq);
+  float mcol[kMaxRows];
+#pragma unroll
+  for (int u = 0; u < kMaxRows; ++u) {
+    const int k = k0 + u;
+    float v = 0.f;
+    if (j < d && k < k1) v = (k < d) ? a.PiV[(size_t)k * d + j] : qscale * a.SV[(size_t)(k - d) * d + j];
+    mcol[u] = v;
+  }
   const float* p = a.part + (size_t)row * a.nsplit * stride;
-  if (threadIdx.x == 0) {
+  if (warp == 0) {
     float M = -INFINITY;
-    for (int s = 0; s < a.nsplit; ++s) M = fmaxf(M, p[(size_t)s * stride + d + mv]);
+    for (int s = lane; s < a.nsplit; s += 32) M = fmaxf(M, p[(size_t)s * stride + dm]);
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Lsum = 0.f;
-    for (int s = 0; s < a.nsplit; ++s) {
-      const float ms = p[(size_t)s * stride + d + mv];
+    for (int s = lane; s < a.nsplit; s += 32) {
+      const float ms = p[(size_t)s * stride + dm];
       const float ws = (ms == -INFINITY) ? 0.f : __expf(ms - M);
       w[s] = ws;
-      Lsum += ws * p[(size_t)s * stride + d + mv + 1];
+      Lsum += ws * p[(size_t)s * stride + dm + 1];
     }
-    red[0] = Lsum;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) Lsum += __shfl_xor_sync(0xffffffffu, Lsum, o);
+    if (lane == 0) Ls[0] = Lsum;
   }
   __syncthreads();
-  for (int j = threadIdx.x; j < d + mv; j += blockDim.x) {
-    float acc = 0.f;
-    for (int s = 0; s < a.nsplit; ++s) acc = fmaf(w[s], p[(size_t)s * stride + j], acc);
-    if (j < d) accv[j] = acc; else accs[j - d] = acc;
+  for (int i = tid; i < 2 * dm; i += blockDim.x) {
+    const int half = i / dm, jj = i % dm;
+    const int s0 = half * ((a.nsplit + 1) / 2), s1 = half ? a.nsplit : (a.nsplit + 1) / 2;
+    float v[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    int s = s0;
+    for (; s + 8 <= s1; s += 8) {   // 8 independent loads in flight
+      float x[8];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) x[u] = p[(size_t)(s + u) * stride + jj];
+#pragma unroll
+      for (int u = 0; u < 8; ++u) v[u] = fmaf(w[s + u], x[u], v[u]);
+    }
+    for (; s < s1; ++s) v[0] = fmaf(w[s], p[(size_t)s * stride + jj], v[0]);
+    acc[i] = ((v[0] + v[1]) + (v[2] + v[3])) + ((v[4] + v[5]) + (v[6] + v[7]));
   }
   __syncthreads();
-  const float Lsum = red[0];
-  const float qscale = (mv > 0) ? kQjlScale / (float)mv : 0.f;
-  for (int j = threadIdx.x; j < d; j += blockDim.x) {
+  if (j < d) {
     float o = 0.f;
-    for (int k = 0; k < d; ++k) o = fmaf(a.PiV[(size_t)k * d + j], accv[k], o);
-    float os = 0.f;
-    for (int k = 0; k < mv; ++k) os = fmaf(a.SV[(size_t)k * d + j], accs[k], os);
-    o = fmaf(qscale, os, o);
-    a.out[(size_t)row * d + j] = (Lsum > 0.f) ? o / Lsum : 0.f;
+#pragma unroll
+    for (int u = 0; u < kMaxRows; ++u) {
+      const int k = k0 + u;
+      if (k < k1) o = fmaf(mcol[u], acc[k] + acc[dm + k], o);
+    }
+    part_o[quarter * d + j] = o;
+  }
+  __syncthreads();
+  for (int i = tid; i < d; i += blockDim.x) {
+    float v = 0.f;
+#pragma unroll
+    for (int q = 0; q < 8; ++q) v += part_o[q * d + i];
+    const float L = Ls[0];
+    a.out[(size_t)row * d + i] = (L > 0.f) ? v / L : 0.f;
   }
 }
 

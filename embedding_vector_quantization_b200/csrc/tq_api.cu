@@ -24,8 +24,11 @@
 #include "internal.h"
 #include "common.cuh"
 #include "encode_simt.cuh"
+#include "encode_rows.cuh"
 #include "score_attn_simt.cuh"
 #include "search_simt.cuh"
+#include "attn_mma.cuh"
+#include "small_kernels.cuh"
 
 struct tq_handle {
   int d = 0, bits = 0, m = 0, norm_dtype = TQ_F32;
@@ -36,6 +39,7 @@ struct tq_handle {
   float* dPi = nullptr;   // [d][d]   y = Pi u
   float* dPiT = nullptr;  // [d][d]   transpose
   float* dS = nullptr;    // [m][d]
+  float* dST = nullptr;   // [d][m]   S^T
   float* dMT = nullptr;   // [d][m]   (S Pi^T)^T
   float* dcent = nullptr; // [2^bits]
   float* dbnd = nullptr;  // [2^bits - 1]
@@ -147,11 +151,12 @@ void free_device(tq_handle* h) {
   cudaFree(h->dPi);
   cudaFree(h->dPiT);
   cudaFree(h->dS);
+  cudaFree(h->dST);
   cudaFree(h->dMT);
   cudaFree(h->dcent);
   cudaFree(h->dbnd);
   cudaFree(h->derr);
-  h->dPi = h->dPiT = h->dS = h->dMT = h->dcent = h->dbnd = nullptr;
+  h->dPi = h->dPiT = h->dS = h->dST = h->dMT = h->dcent = h->dbnd = nullptr;
   h->derr = nullptr;
 }
 
@@ -198,7 +203,9 @@ int create_common(int d, int bits_mse, int m, uint64_t seed, int norm_dtype, tq_
     return fail(TQ_EINVAL, "codebook(d=%d, bits=%d) failed", d, bits_mse);
   }
   std::vector<float> Pi(h->Pi.begin(), h->Pi.end()), PiT((size_t)d * d), S(h->S.begin(), h->S.end()),
-      MT((size_t)d * m), cent(h->cent.begin(), h->cent.end()), bnd(h->bnd.begin(), h->bnd.end());
+      ST((size_t)d * m), MT((size_t)d * m), cent(h->cent.begin(), h->cent.end()), bnd(h->bnd.begin(), h->bnd.end());
+  for (int i = 0; i < m; ++i)
+    for (int k = 0; k < d; ++k) ST[(size_t)k * m + i] = (float)h->S[(size_t)i * d + k];
   for (int i = 0; i < d; ++i)
     for (int j = 0; j < d; ++j) PiT[(size_t)j * d + i] = (float)h->Pi[(size_t)i * d + j];
   // M = S Pi^T (m x d): M[i][k] = sum_j S[i][j] Pi[k][j]; stored transposed MT[k][i].
@@ -210,7 +217,7 @@ int create_common(int d, int bits_mse, int m, uint64_t seed, int norm_dtype, tq_
     }
   int st = TQ_OK;
   if ((st = upload(&h->dPi, Pi, "Pi")) || (st = upload(&h->dPiT, PiT, "PiT")) ||
-      (st = upload(&h->dS, S, "S")) || (st = upload(&h->dMT, MT, "MT")) ||
+      (st = upload(&h->dS, S, "S")) || (st = upload(&h->dST, ST, "ST")) || (st = upload(&h->dMT, MT, "MT")) ||
       (st = upload(&h->dcent, cent, "centroids")) || (st = upload(&h->dbnd, bnd, "bounds"))) {
     free_device(h);
     delete h;
@@ -253,17 +260,15 @@ int check_cache(const tq_handle* h, const tq_cache* c, const char* name) {
   return TQ_OK;
 }
 
-// Attention split policy: enough CTAs to cover the GPU ~4x, chunks of >= 128 keys.
+// Attention split policy (shared by every attention kernel): about two CTAs per
+// SM, chunks a multiple of 128 tokens and at most 1024 tokens long.
 void attn_split(int B, int Hkv, int64_t L_cap, int* nsplit, int64_t* chunk) {
-  const int64_t units = (int64_t)B * Hkv;
-  int64_t ns = (4 * 148 + units - 1) / units;
-  const int64_t max_ns = (L_cap + 127) / 128;
-  ns = std::max<int64_t>(1, std::min(ns, max_ns));
+  const int64_t units = std::max<int64_t>(1, (int64_t)B * Hkv);
+  const int64_t ns = std::max<int64_t>(1, (2 * 148 + units - 1) / units);
   int64_t ch = (L_cap + ns - 1) / ns;
-  ch = (ch + 127) / 128 * 128;
-  ns = (L_cap + ch - 1) / ch;
-  *nsplit = (int)ns;
+  ch = std::min<int64_t>(1024, std::max<int64_t>(128, (ch + 127) / 128 * 128));
   *chunk = ch;
+  *nsplit = (int)((L_cap + ch - 1) / ch);
 }
 
 void search_split(int nq, int64_t n, int* nchunks, int64_t* chunk) {
@@ -274,6 +279,21 @@ void search_split(int nq, int64_t n, int* nchunks, int64_t* chunk) {
   ch = (ch + tqk::kSK - 1) / tqk::kSK * tqk::kSK;
   *chunk = ch;
   *nchunks = (int)((n + ch - 1) / ch);
+}
+
+// The int8 tensor-core attention kernel covers 3-bit prod K and V caches (2-bit
+// codes + 128 QJL signs, fp16 norms) at d = 128 with 4 query heads per KV head.
+// TQ_SIMT=1 forces the SIMT kernels (used by tests to cross-check both paths).
+bool attn_prod2_fast_path(const tq_handle* hk, const tq_handle* hv, int G, const tq_cache* k, const tq_cache* v) {
+  if (std::getenv("TQ_SIMT")) return false;
+  auto ok_handle = [](const tq_handle* h) {
+    return h->d == 128 && h->m == 128 && h->bits == 2 && h->norm_dtype == TQ_F16 &&
+           std::fabs(h->cent[3] - h->cent[2] - h->cent[1] + h->cent[0]) < 1e-12;
+  };
+  auto ok_cache = [](const tq_cache* c) {
+    return aligned(c->codes, 16) && aligned(c->signs, 16) && aligned(c->norms, 16) && aligned(c->rnorms, 16);
+  };
+  return G == 4 && ok_handle(hk) && ok_handle(hv) && k->L_cap % 8 == 0 && ok_cache(k) && ok_cache(v);
 }
 
 struct ScoreWs { float* qr; float* qs; };
@@ -295,7 +315,7 @@ size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, i
   if (nsplit) *nsplit = ns;
   if (chunk) *chunk = ch;
   if (part) *part = reinterpret_cast<float*>(base + off);
-  off += round_up((size_t)B * Hq * ns * (hv->d + hv->m + 2) * 4, 256);
+  off += round_up((size_t)B * Hq * ns * tqk::partial_stride(hv->d, hv->m) * 4, 256);
   return off;
 }
 
@@ -318,13 +338,42 @@ size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base
 
 int launch_qprep(const tq_handle* h, const void* q, int q_dtype, int rows, float* qr, float* qs, cudaStream_t s) {
   if (rows == 0) return TQ_OK;
-  dim3 grid(rows, std::max(1, std::min(8, (h->d + h->m) / 64)));
+  if (h->d <= tqk::kSmallMaxD && h->m <= tqk::kSmallMaxD) {
+    const size_t smem = tqk::qprep_staged_smem_bytes(h->d, h->m);
+    if (once_per_device(6, h->device))
+      cudaFuncSetAttribute(tqk::qprep_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    KernelScope ks("qprep", s);
+    tqk::qprep_staged_kernel<<<(rows + tqk::kQRows - 1) / tqk::kQRows, tqk::kSmallThreads, smem, s>>>(
+        q, q_dtype, rows, h->d, h->dPiT, h->dST, h->m, qr, qs, h->derr);
+    return launch_check("qprep_staged_kernel");
+  }
+  const int groups = (rows + tqk::kQprepRows - 1) / tqk::kQprepRows;
+  dim3 grid(groups, (h->d + h->m + 63) / 64);
+  if (once_per_device(5, h->device))
+    cudaFuncSetAttribute(tqk::qprep_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   KernelScope ks("qprep", s);
-  tqk::qprep_kernel<<<grid, 256, h->d * sizeof(float), s>>>(q, q_dtype, rows, h->d, h->dPi, h->dS, h->m, qr, qs);
+  tqk::qprep_kernel<<<grid, 256, (size_t)tqk::kQprepRows * h->d * sizeof(float), s>>>(q, q_dtype, rows, h->d, h->dPi, h->dS, h->m, qr, qs);
   return launch_check("qprep_kernel");
 }
 
+// Small batches (and every append) go to the latency-oriented kernel: one CTA per
+// <= 16 rows (or per sequence), every thread one output coordinate.
+bool rows_kernel_ok(const tq_handle* h, int64_t rows_per_cta) {
+  return h->d <= tqk::kRowsMaxD && rows_per_cta <= tqk::kRowsMax;
+}
+
+int encode_rows_launch(const tq_handle* h, tqk::EncodeArgs& a, unsigned grid, int advance, cudaStream_t s) {
+  const size_t smem = tqk::encode_rows_smem_bytes(h->d, h->m);
+  if (once_per_device(4, h->device))
+    cudaFuncSetAttribute(tqk::encode_rows_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  KernelScope ks(a.len ? "append" : "encode", s);
+  tqk::encode_rows_kernel<<<grid, tqk::kRowsThreads, smem, s>>>(a, advance);
+  return launch_check("encode_rows_kernel");
+}
+
 int encode_launch(const tq_handle* h, tqk::EncodeArgs& a, cudaStream_t s) {
+  if (a.len == nullptr && a.rows <= 256 && rows_kernel_ok(h, 1))
+    return encode_rows_launch(h, a, (unsigned)((a.rows + tqk::kRowsMax - 1) / tqk::kRowsMax), 0, s);
   const size_t smem = tqk::encode_smem_bytes(h->m);
   if (once_per_device(0, h->device))
     cudaFuncSetAttribute(tqk::encode_simt_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
@@ -468,6 +517,30 @@ int tq_append(const tq_handle* h, const void* x_new, int x_dtype, int B, int Hkv
   a.codes = cache->codes; a.codes_B = h->codes_B; a.signs = cache->signs; a.signs_B = h->signs_B;
   a.norms = cache->norms; a.rnorms = static_cast<__half*>(cache->rnorms);
   a.len = len; a.Hkv = Hkv; a.L_cap = cache->L_cap; a.err = h->derr;
+  if (h->d <= tqk::kSmallMaxD && h->m <= tqk::kSmallMaxD && Hkv <= 8) {
+    // one CTA per (sequence, head); the Hkv CTAs of a sequence form a cluster
+    const size_t smem = tqk::append_cluster_smem_bytes(h->d, h->m);
+    if (once_per_device(8, h->device))
+      cudaFuncSetAttribute(tqk::append_cluster_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3((unsigned)Hkv, (unsigned)B, 1);
+    cfg.blockDim = dim3(tqk::kSmallThreads, 1, 1);
+    cfg.dynamicSmemBytes = smem;
+    cfg.stream = s;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeClusterDimension;
+    attr[0].val.clusterDim.x = (unsigned)Hkv;
+    attr[0].val.clusterDim.y = 1;
+    attr[0].val.clusterDim.z = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    const int adv = advance ? 1 : 0;
+    KernelScope ks("append", s);
+    cudaError_t e = cudaLaunchKernelEx(&cfg, tqk::append_cluster_kernel, a, adv);
+    if (e != cudaSuccess) return cuda_fail(e, "append_cluster_kernel");
+    return launch_check("append_cluster_kernel");
+  }
+  if (rows_kernel_ok(h, Hkv)) return encode_rows_launch(h, a, (unsigned)B, advance ? 1 : 0, s);
   st = encode_launch(h, a, s);
   if (st) return st;
   if (advance) {
@@ -533,8 +606,8 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
   if (hk->d != hv->d) return fail(TQ_EINVAL, "K and V handles differ in d (%d vs %d)", hk->d, hv->d);
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return fail(TQ_EINVAL, "B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
   if (Hq / Hkv > tqk::kMaxGroup) return fail(TQ_EUNSUPPORTED, "group Hq/Hkv=%d > %d", Hq / Hkv, tqk::kMaxGroup);
-  if (hk->d > tqk::kMaxHeadDim || hv->m > tqk::kMaxHeadDim)
-    return fail(TQ_EUNSUPPORTED, "attention needs d, m_V <= %d", tqk::kMaxHeadDim);
+  if (hk->d > tqk::kMaxHeadDim || hv->m > tqk::kMaxHeadDim || hv->d + hv->m > 256)
+    return fail(TQ_EUNSUPPORTED, "attention needs d <= %d and d + m_V <= 256", tqk::kMaxHeadDim);
   if (q_dtype != TQ_F32 && q_dtype != TQ_BF16) return fail(TQ_EINVAL, "q dtype %d", q_dtype);
   if (B == 0) return ok();
   int st = check_cache(hk, k, "key");
@@ -560,19 +633,55 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
   a.k = view_of(hk, k); a.v = view_of(hv, v); a.L_cap = k->L_cap; a.chunk = chunk; a.nsplit = nsplit;
   a.len = len; a.scale = scale; a.part = part;
   const int G = Hq / Hkv;
-  const size_t smem = ((size_t)G * (hk->d + hk->m) + 32 + (size_t)G * tqk::kAttnThreads + 2 * tqk::kAttnThreads +
-                       4 * (size_t)G) * 4;
-  {
-    KernelScope ks("attn_split", s);
-    tqk::attn_split_simt_kernel<<<dim3((unsigned)(B * Hkv), (unsigned)nsplit), tqk::kAttnThreads, smem, s>>>(a);
+  if (attn_prod2_fast_path(hk, hv, G, k, v)) {
+    tqk::amma::Args m{};
+    m.qr = w.qr; m.qs = w.qs; m.B = B; m.Hq = Hq; m.Hkv = Hkv;
+    m.kcodes = k->codes; m.ksigns = k->signs; m.knorm = static_cast<const __half*>(k->norms);
+    m.krn = static_cast<const __half*>(k->rnorms);
+    m.vcodes = v->codes; m.vsigns = v->signs; m.vnorm = static_cast<const __half*>(v->norms);
+    m.vrn = static_cast<const __half*>(v->rnorms);
+    m.L_cap = k->L_cap; m.chunk = chunk; m.nsplit = nsplit; m.len = len;
+    m.kc0 = (float)hk->cent[0]; m.kb0 = (float)(hk->cent[1] - hk->cent[0]); m.kb1 = (float)(hk->cent[2] - hk->cent[0]);
+    m.vc0 = (float)hv->cent[0]; m.vb0 = (float)(hv->cent[1] - hv->cent[0]); m.vb1 = (float)(hv->cent[2] - hv->cent[0]);
+    m.scale = scale; m.part = part; m.err = hk->derr;
+    const size_t msmem = sizeof(tqk::amma::Smem);
+    if (once_per_device(2, hk->device)) {
+      cudaFuncSetAttribute(tqk::amma::attn_prod2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+      cudaFuncSetAttribute(tqk::amma::attn_prod2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    }
+    {
+      KernelScope ks("attn_split", s);
+      tqk::amma::attn_prod2_kernel<<<dim3((unsigned)(B * Hkv), (unsigned)nsplit), tqk::amma::kThreads, msmem, s>>>(m);
+    }
+    if ((st = launch_check("attn_prod2_kernel"))) return st;
+  } else {
+    const size_t smem = ((size_t)G * (hk->d + hk->m) + 32 + (size_t)G * tqk::kAttnThreads +
+                         2 * tqk::kAttnThreads + 4 * (size_t)G) * 4;
+    {
+      KernelScope ks("attn_split", s);
+      tqk::attn_split_simt_kernel<<<dim3((unsigned)(B * Hkv), (unsigned)nsplit), tqk::kAttnThreads, smem, s>>>(a);
+    }
+    if ((st = launch_check("attn_split_simt_kernel"))) return st;
   }
-  if ((st = launch_check("attn_split_simt_kernel"))) return st;
+  if (tqk::combine_staged_smem_bytes(nsplit, hv->d, hv->m) <= 200 * 1024) {
+    tqk::CombineStagedArgs cs{};
+    cs.part = part; cs.nsplit = nsplit; cs.d = hv->d; cs.mv = hv->m; cs.PiV = hv->dPi; cs.SV = hv->dS;
+    cs.out = out; cs.err = hv->derr;
+    if (once_per_device(7, hv->device))
+      cudaFuncSetAttribute(tqk::combine_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    KernelScope ks("attn_combine", s);
+    tqk::combine_staged_kernel<<<B * Hq, tqk::kSmallThreads, tqk::combine_staged_smem_bytes(nsplit, hv->d, hv->m),
+                                 s>>>(cs);
+    return launch_check("combine_staged_kernel");
+  }
   tqk::CombineArgs c{};
-  c.part = part; c.rows = B * Hq; c.nsplit = nsplit; c.d = hv->d; c.mv = hv->m; c.PiV = hv->dPi; c.SV = hv->dS;
-  c.out = out;
-  const size_t csmem = ((size_t)hv->d + hv->m + nsplit + 2) * 4;
+  c.part = part; c.Hq = Hq; c.Hkv = Hkv; c.nsplit = nsplit; c.d = hv->d; c.mv = hv->m; c.PiV = hv->dPi;
+  c.SV = hv->dS; c.out = out;
+  const size_t csmem = ((size_t)nsplit + 2 * (size_t)(hv->d + hv->m) + 8 * (size_t)hv->d + 4) * 4;
+  if (once_per_device(3, hv->device))
+    cudaFuncSetAttribute(tqk::attn_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   KernelScope ks("attn_combine", s);
-  tqk::attn_combine_kernel<<<B * Hq, 128, csmem, s>>>(c);
+  tqk::attn_combine_kernel<<<B * Hq, tqk::kCombineThreads, csmem, s>>>(c);
   return launch_check("attn_combine_kernel");
 }
 

@@ -188,3 +188,37 @@ def test_search_on_oracle_codes(tq, bits, d, n, k):
         assert np.all(S[i, idx[i]] >= kth - tol[idx[i]])
         assert np.all(np.abs(sc[i] - S[i, idx[i]]) <= tol[idx[i]])
         assert np.all(np.diff(sc[i]) <= 0)
+
+
+@pytest.mark.parametrize("B,Hkv,L,lens", [(1, 2, 5000, [4999]), (2, 3, 2048, [2048, 1]), (3, 1, 800, [0, 800, 129])])
+def test_attention_tensor_core_path_matches_simt_and_oracle(tq, B, Hkv, L, lens):
+    """3-bit prod K/V at d=128, 4 query heads per KV head: the int8 tensor-core kernel, the
+    SIMT kernel (TQ_SIMT=1) and the oracle agree (caches hold the oracle's codes)."""
+    import os
+    G, d = 4, 128
+    hk = tq.Handle(d, 3, 30, qjl_m=128)
+    hv = tq.Handle(d, 3, 31, qjl_m=128)
+    ohk, ohv = OracleHandle(d, 2, 30, 128), OracleHandle(d, 2, 31, 128)
+    rs = np.random.default_rng(B * 100 + L)
+    std = np.exp(0.5 * rs.standard_normal((1, Hkv, 1, d)))
+    kc, kod = oracle_cache(tq, hk, ohk, rs.standard_normal((B, Hkv, L, d)) * std)
+    vc, vod = oracle_cache(tq, hv, ohv, rs.standard_normal((B, Hkv, L, d)) * std)
+    q = torch.from_numpy(rs.standard_normal((B, Hkv * G, d))).float()
+    lens_t = torch.tensor(lens, dtype=torch.int32).cuda()
+    scale = 1 / np.sqrt(d)
+    o_fast = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens_t, scale).cpu().numpy()
+    os.environ["TQ_SIMT"] = "1"
+    try:
+        o_simt = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens_t, scale).cpu().numpy()
+    finally:
+        del os.environ["TQ_SIMT"]
+    ref = ops.decode_attention(q.double().numpy(), kod, vod, [max(1, x) for x in lens], scale)
+    for b in range(B):
+        for h in range(Hkv * G):
+            if lens[b] == 0:
+                assert np.all(o_fast[b, h] == 0) and np.all(o_simt[b, h] == 0)
+                continue
+            nr = np.linalg.norm(ref[b, h])
+            assert np.linalg.norm(o_fast[b, h] - ref[b, h]) <= ATTN_RTOL * nr, (b, h)
+            assert np.linalg.norm(o_simt[b, h] - ref[b, h]) <= ATTN_RTOL * nr, (b, h)
+    assert hk.status() == tq.TQ_OK
