@@ -79,10 +79,10 @@ struct Args {
 
 struct __align__(16) Smem {
   unsigned char stage[kStages][kStageBytes];
-  // key pass: scaled logits [head][token]; value pass: the integer softmax weights of every
-  // block, [block][0: value weights, 1: QJL weights][col = head*2 + piece][token] (same bytes)
-  float logits[kG][kMaxChunk];
+  float logits[kG][kMaxChunk];  // key pass output: scaled logits in log2 units [head][token]
   uint32_t qfrag[12][2][4][8];  // key-side B fragments: [k-step][register][quad index t][column g]
+  int8_t pw[2][2][8][kBlk];     // integer softmax weights of a value block, double buffered:
+                                // [buffer][0: value weights, 1: QJL weights][col = head*2+piece][token]
   float qconst[kG][4];        // c0*sum(q'), delta_mse, delta_qjl, sum(qs)
   float red_f[kWarps][kG];
   float hmax[kG];
@@ -146,6 +146,14 @@ __device__ __forceinline__ void ldsm_t8_x2(uint32_t (&r)[4], const void* row_add
   asm volatile("ldmatrix.sync.aligned.m16n16.x2.trans.shared.b8 {%0,%1,%2,%3}, [%4];\n"
                : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3])
                : "r"(smem_u32(row_addr)));
+}
+
+// 2^x by the hardware's approximate base-2 exponential (flushes subnormal results to 0);
+// the weights it feeds are rounded to 14 bits right after.
+__device__ __forceinline__ float exp2_approx(float x) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;\n" : "=f"(y) : "f"(x));
+  return y;
 }
 
 __device__ __forceinline__ uint32_t pack4(int8_t a, int8_t b, int8_t c, int8_t d) {
@@ -280,6 +288,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
     for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[kk][slot][t][g];
 
   const float kqjl = kQjlScale / (float)kM;
+  const float scale2 = a.scale * 1.4426950408889634f;
   float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
   float run_max = -INFINITY;   // this thread's max logit of head t
   float vn_max = 0.f, vr_max = 0.f;
@@ -293,6 +302,42 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 
   const int bg = warp % 3, half = warp / 3;   // value side: byte group and token half (warps 0..5)
   float dv1 = 1.f, dv2 = 1.f, inv1 = 1.f, inv2 = 1.f;
+
+  // Integer weights of value block jj into pw[jj & 1]: thread -> (head, 4 consecutive tokens)
+  // per round; w1 = round(p * ||v|| / dv1), w2 = round(p * rnorm / dv2) with p = exp2(logit - max),
+  // each split into 7-bit pieces (hi * 128 + lo). Also accumulates sum p and the integer sums.
+  auto prepare_weights = [&](int jj, int tix, int nthreads) {
+    const int tb = jj * kBlk;
+    const int nval = min(kBlk, ntok - tb);
+    const int h = tix & 3;
+    const float hm = sm.hmax[h];
+    for (int q4 = (tix >> 2) * 4; q4 < kBlk; q4 += (nthreads >> 2) * 4) {
+      const float4 l4 = *reinterpret_cast<const float4*>(&sm.logits[h][tb + q4]);
+      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+      uint32_t w1h = 0, w1l = 0, w2h = 0, w2l = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int tok = q4 + q;
+        if (tok < nval) {
+          const float p = exp2_approx(lv[q] - hm);
+          const int w1 = __float2int_rn(p * __half2float(sm.vnorm[tb + tok]) * inv1);
+          const int w2 = __float2int_rn(p * __half2float(sm.vrn[tb + tok]) * inv2);
+          w1h |= (uint32_t)(w1 >> 7) << (8 * q);
+          w1l |= (uint32_t)(w1 & 127) << (8 * q);
+          w2h |= (uint32_t)(w2 >> 7) << (8 * q);
+          w2l |= (uint32_t)(w2 & 127) << (8 * q);
+          lsum += p;
+          wsum[0] += w1;
+          wsum[1] += w2;
+        }
+      }
+      int8_t* blk = &sm.pw[jj & 1][0][0][0];
+      *reinterpret_cast<uint32_t*>(blk + (2 * h) * kBlk + q4) = w1h;
+      *reinterpret_cast<uint32_t*>(blk + (2 * h + 1) * kBlk + q4) = w1l;
+      *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h) * kBlk + q4) = w2h;
+      *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h + 1) * kBlk + q4) = w2l;
+    }
+  };
 
   // No warp ever leaves this loop early: a wait that runs out sets abort_flag, after
   // which nothing new is issued and no further waits happen, so every warp still
@@ -357,48 +402,9 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
       dv2 = sm.nmax[1] > 0.f ? sm.nmax[1] / 16383.f : 1.f;
       inv1 = 1.f / dv1;
       inv2 = 1.f / dv2;
-      // integer weights of the whole chunk; they overwrite the logits, so read first.
-      // thread -> (head h, 4 consecutive tokens) per round; 4-byte stores of 4 tokens.
-      constexpr int kRounds = kMaxChunk * kG / (4 * kThreads);   // 8
-      const int h = tid & 3;
-      float4 lg[kRounds];
-#pragma unroll
-      for (int u = 0; u < kRounds; ++u) {
-        const int tok4 = 4 * ((tid >> 2) + u * (kThreads / 4));
-        lg[u] = (tok4 < nblk * kBlk) ? *reinterpret_cast<const float4*>(&sm.logits[h][tok4])
-                                     : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
-      }
-      const float hm = sm.hmax[h];
-      __syncthreads();
-      int8_t* pw = reinterpret_cast<int8_t*>(&sm.logits[0][0]);
-#pragma unroll
-      for (int u = 0; u < kRounds; ++u) {
-        const int tok4 = 4 * ((tid >> 2) + u * (kThreads / 4));
-        if (tok4 >= nblk * kBlk) break;
-        const float l4[4] = {lg[u].x, lg[u].y, lg[u].z, lg[u].w};
-        uint32_t w1h = 0, w1l = 0, w2h = 0, w2l = 0;
-#pragma unroll
-        for (int q = 0; q < 4; ++q) {
-          const int tok = tok4 + q;
-          const bool ok = tok < ntok;
-          const float p = ok ? __expf(l4[q] - hm) : 0.f;
-          const int w1 = ok ? __float2int_rn(p * __half2float(sm.vnorm[tok]) * inv1) : 0;
-          const int w2 = ok ? __float2int_rn(p * __half2float(sm.vrn[tok]) * inv2) : 0;
-          w1h |= (uint32_t)(w1 >> 7) << (8 * q);
-          w1l |= (uint32_t)(w1 & 127) << (8 * q);
-          w2h |= (uint32_t)(w2 >> 7) << (8 * q);
-          w2l |= (uint32_t)(w2 & 127) << (8 * q);
-          lsum += p;
-          wsum[0] += w1;
-          wsum[1] += w2;
-        }
-        int8_t* blk = pw + (tok4 / kBlk) * (2 * 8 * kBlk);
-        const int tk = tok4 & (kBlk - 1);
-        *reinterpret_cast<uint32_t*>(blk + (2 * h) * kBlk + tk) = w1h;
-        *reinterpret_cast<uint32_t*>(blk + (2 * h + 1) * kBlk + tk) = w1l;
-        *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h) * kBlk + tk) = w2h;
-        *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h + 1) * kBlk + tk) = w2l;
-      }
+      // integer weights of the first value block (all threads); later blocks are prepared
+      // by warps 6 and 7 while warps 0..5 run the value MMAs of the block before
+      prepare_weights(0, tid, kThreads);
       __syncthreads();
     }
 
@@ -444,7 +450,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
           const int qjl = 128 * (ds1[hi] + (ds16[hi] >> 4)) + (ds1[lo] + (ds16[lo] >> 4));
           const float n = __half2float(nrm[key]), rn = __half2float(rnm[key]);
           float sc = n * (c0h + dmh * (float)mse) + rn * kqjl * (2.f * dsh * (float)qjl - ssh);
-          sc *= a.scale;
+          sc *= scale2;   // softmax scale * log2(e): the weights are exp2(logit - max)
           sc = (key < nvalid) ? sc : -INFINITY;
           sm.logits[t][tok_base + key] = sc;
           run_max = fmaxf(run_max, sc);
@@ -463,8 +469,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
     } else {
       // ---------------- value pass (warps 0..5: byte group bg, token half)
       if (warp < 6) {
-        const int8_t* pw = reinterpret_cast<const int8_t*>(&sm.logits[0][0]) + jj * (2 * 8 * kBlk) +
-                           (bg == 2 ? 8 * kBlk : 0);
+        const int8_t* pw = &sm.pw[jj & 1][bg == 2 ? 1 : 0][0][0];
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
           const int tk = 128 * half + 32 * kq;  // first token of this 32-token k-step
@@ -481,7 +486,10 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
             mma_s8(vacc[4 + s], x0 & 0x10101010u, x1 & 0x10101010u, x2 & 0x10101010u, x3 & 0x10101010u, b0, b1);
           }
         }
+      } else if (jj + 1 < nblk) {
+        prepare_weights(jj + 1, tid - 6 * 32, 64);
       }
+      __syncthreads();   // the next block's weights are ready; this block's are no longer read
     }
     __syncwarp();
     if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[j % kStages])) : "memory");
@@ -543,10 +551,15 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 
   // ---------------- partial outputs: rotated-domain value sum, QJL sum, max, sum of p
   const int stride = partial_stride(kD, kM);
+  if (tid < 2 * kG) {
+    int W = 0;
+    for (int w = 0; w < kWarps; ++w) W += sm.red_i[w][tid];
+    sm.W[tid / kG][tid % kG] = W;
+  }
+  __syncthreads();
   for (int i = tid; i < kG * (kD + kM); i += kThreads) {
     const int h = i / (kD + kM), j = i % (kD + kM);
-    int W1 = 0, W2 = 0;
-    for (int w = 0; w < kWarps; ++w) { W1 += sm.red_i[w][h]; W2 += sm.red_i[w][kG + h]; }
+    const int W1 = sm.W[0][h], W2 = sm.W[1][h];
     float v;
     if (j < kD) {
       // code c = j: byte c / 4 (group c / 64), bits 2(c % 4) (plane 0) and 2(c % 4) + 1 (plane 1)
@@ -565,7 +578,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
     float l = 0.f;
     for (int w = 0; w < kWarps; ++w) l += sm.red_f[w][tid];
     float* o = a.part + (((size_t)b * a.Hq + h0 + tid) * a.nsplit + split) * stride;
-    o[kD + kM] = (ntok > 0) ? sm.hmax[tid] : -INFINITY;
+    o[kD + kM] = (ntok > 0) ? sm.hmax[tid] * 0.6931471805599453f : -INFINITY;   // back to natural-log units
     o[kD + kM + 1] = (ntok > 0) ? l : 0.f;
   }
 }
