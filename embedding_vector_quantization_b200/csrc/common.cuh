@@ -15,6 +15,7 @@ constexpr float kQjlScale = 1.2533141373155002512f;  // sqrt(pi / 2)
 // Error bits OR-ed into a handle's device error word (decoded by the host).
 constexpr int kErrCapacity = 1;
 constexpr int kErrTimeout = 2;
+constexpr int kErrInternal = 4;   // a kernel found its own launch state unusable (e.g. shared memory alignment)
 
 __device__ __forceinline__ void report_error(int* err, int bit) {
   if (err) atomicOr(err, bit);

@@ -6,6 +6,8 @@
 //   TQ_FAULT=alloc   -> tq_create* fails with TQ_ENOMEM before allocating
 //   TQ_FAULT=launch  -> hot calls fail with TQ_ECUDA before launching
 
+#include <cuda.h>
+#include <cudaTypedefs.h>
 #include <cuda_runtime.h>
 
 #include <algorithm>
@@ -29,6 +31,7 @@
 #include "search_simt.cuh"
 #include "attn_mma.cuh"
 #include "small_kernels.cuh"
+#include "encode_tc.cuh"
 
 struct tq_handle {
   int d = 0, bits = 0, m = 0, norm_dtype = TQ_F32;
@@ -44,6 +47,7 @@ struct tq_handle {
   float* dcent = nullptr; // [2^bits]
   float* dbnd = nullptr;  // [2^bits - 1]
   int* derr = nullptr;    // device error word
+  uint8_t* dOps = nullptr; // d = 128: pre-swizzled 16-bit hi/lo operands of the tensor-core encode
 };
 
 namespace {
@@ -156,8 +160,10 @@ void free_device(tq_handle* h) {
   cudaFree(h->dcent);
   cudaFree(h->dbnd);
   cudaFree(h->derr);
+  cudaFree(h->dOps);
   h->dPi = h->dPiT = h->dS = h->dST = h->dMT = h->dcent = h->dbnd = nullptr;
   h->derr = nullptr;
+  h->dOps = nullptr;
 }
 
 template <typename T>
@@ -168,6 +174,52 @@ int upload(T** dst, const std::vector<T>& src, const char* what) {
   e = cudaMemcpy(*dst, src.data(), src.size() * sizeof(T), cudaMemcpyHostToDevice);
   if (e != cudaSuccess) return cuda_fail(e, what);
   return TQ_OK;
+}
+
+// One [128][128] matrix of 16-bit values (row n, reduction index k) in the 128-byte-swizzled
+// K-major layout the tensor-core encode reads: two atoms of K 0..63 and 64..127, row n at
+// byte 128 n of its atom, 16-byte chunk c at chunk position c ^ (n % 8).
+void swizzle_k128(const std::vector<uint16_t>& src, uint8_t* dst) {
+  for (int n = 0; n < 128; ++n)
+    for (int k = 0; k < 128; ++k) {
+      const int atom = k >> 6, chunk = (k & 63) >> 3, e = k & 7;
+      const size_t off = (size_t)atom * tqk::etc::kAtom + (size_t)n * 128 + (size_t)((chunk ^ (n & 7)) << 4) + e * 2;
+      std::memcpy(dst + off, &src[(size_t)n * 128 + k], 2);
+    }
+}
+
+// Tensor-core operands of a d = 128 handle: Pi (bf16 and f16 hi/lo pairs) and, for prod
+// with m = 128, M = S Pi^T (bf16 hi/lo): value = hi + lo with lo the rounded remainder.
+std::vector<uint8_t> tc_operands(const std::vector<double>& Pi, const std::vector<double>& M) {
+  const size_t mat = tqk::etc::kMat;
+  std::vector<uint8_t> ops(mat * tqk::etc::kOpCount, 0);
+  std::vector<uint16_t> hi(128 * 128), lo(128 * 128);
+  auto split_bf16 = [&](const std::vector<double>& A) {
+    for (size_t i = 0; i < A.size(); ++i) {
+      const __nv_bfloat16 h = __float2bfloat16((float)A[i]);
+      hi[i] = __bfloat16_as_ushort(h);
+      lo[i] = __bfloat16_as_ushort(__float2bfloat16((float)(A[i] - (double)__bfloat162float(h))));
+    }
+  };
+  auto split_f16 = [&](const std::vector<double>& A) {
+    for (size_t i = 0; i < A.size(); ++i) {
+      const __half h = __float2half((float)A[i]);
+      hi[i] = __half_as_ushort(h);
+      lo[i] = __half_as_ushort(__float2half((float)(A[i] - (double)__half2float(h))));
+    }
+  };
+  split_bf16(Pi);
+  swizzle_k128(hi, ops.data() + tqk::etc::kOpPiBf16Hi * mat);
+  swizzle_k128(lo, ops.data() + tqk::etc::kOpPiBf16Lo * mat);
+  split_f16(Pi);
+  swizzle_k128(hi, ops.data() + tqk::etc::kOpPiF16Hi * mat);
+  swizzle_k128(lo, ops.data() + tqk::etc::kOpPiF16Lo * mat);
+  if (!M.empty()) {
+    split_bf16(M);
+    swizzle_k128(hi, ops.data() + tqk::etc::kOpMHi * mat);
+    swizzle_k128(lo, ops.data() + tqk::etc::kOpMLo * mat);
+  }
+  return ops;
 }
 
 int create_common(int d, int bits_mse, int m, uint64_t seed, int norm_dtype, tq_handle** out) {
@@ -209,16 +261,21 @@ int create_common(int d, int bits_mse, int m, uint64_t seed, int norm_dtype, tq_
   for (int i = 0; i < d; ++i)
     for (int j = 0; j < d; ++j) PiT[(size_t)j * d + i] = (float)h->Pi[(size_t)i * d + j];
   // M = S Pi^T (m x d): M[i][k] = sum_j S[i][j] Pi[k][j]; stored transposed MT[k][i].
+  std::vector<double> M((size_t)m * d);
   for (int i = 0; i < m; ++i)
     for (int k = 0; k < d; ++k) {
       double acc = 0.0;
       for (int j = 0; j < d; ++j) acc += h->S[(size_t)i * d + j] * h->Pi[(size_t)k * d + j];
+      M[(size_t)i * d + k] = acc;
       MT[(size_t)k * m + i] = (float)acc;
     }
+  std::vector<uint8_t> ops;
+  if (d == tqk::etc::kD && (m == 0 || m == tqk::etc::kD)) ops = tc_operands(h->Pi, M);
   int st = TQ_OK;
   if ((st = upload(&h->dPi, Pi, "Pi")) || (st = upload(&h->dPiT, PiT, "PiT")) ||
       (st = upload(&h->dS, S, "S")) || (st = upload(&h->dST, ST, "ST")) || (st = upload(&h->dMT, MT, "MT")) ||
-      (st = upload(&h->dcent, cent, "centroids")) || (st = upload(&h->dbnd, bnd, "bounds"))) {
+      (st = upload(&h->dcent, cent, "centroids")) || (st = upload(&h->dbnd, bnd, "bounds")) ||
+      (st = upload(&h->dOps, ops, "tensor-core operands"))) {
     free_device(h);
     delete h;
     return st;
@@ -371,7 +428,92 @@ int encode_rows_launch(const tq_handle* h, tqk::EncodeArgs& a, unsigned grid, in
   return launch_check("encode_rows_kernel");
 }
 
+// ---- tensor-core encode (d = 128, bf16 / f16 input)
+
+PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
+  static PFN_cuTensorMapEncodeTiled fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q = cudaDriverEntryPointSymbolNotFound;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
+  });
+  return fn;
+}
+
+int sm_count(int device) {
+  static std::atomic<int> counts[64];
+  if (device < 0 || device >= 64) return 148;
+  int c = counts[device].load();
+  if (c == 0) {
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || c <= 0) c = 148;
+    counts[device].store(c);
+  }
+  return c;
+}
+
+bool tc_encode_ok(const tq_handle* h, const tqk::EncodeArgs& a) {
+  if (std::getenv("TQ_SIMT")) return false;
+  return h->dOps && a.len == nullptr && (a.x_dtype == TQ_BF16 || a.x_dtype == TQ_F16) && a.rows >= 1024 &&
+         a.rows < (int64_t)1 << 31;
+}
+
+template <int BITS, bool PROD, bool NORM32>
+int tc_launch_one(const tq_handle* h, const CUtensorMap& map, const tqk::etc::Args& ea, int f16in, unsigned grid,
+                  cudaStream_t s) {
+  auto kern = tqk::etc::encode_tc_kernel<BITS, PROD, NORM32>;
+  const size_t smem = tqk::etc::Layout<PROD>::kBytes;
+  static std::atomic<uint64_t> attr_done{0};
+  const uint64_t bit = 1ull << (h->device & 63);
+  if ((attr_done.fetch_or(bit) & bit) == 0) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem);
+    if (e != cudaSuccess) return cuda_fail(e, "cudaFuncSetAttribute(encode_tc_kernel)");
+  }
+  KernelScope ks("encode", s);
+  kern<<<grid, tqk::etc::Layout<PROD>::kThreads, smem, s>>>(map, ea, f16in);
+  return launch_check("encode_tc_kernel");
+}
+
+template <bool PROD, bool NORM32>
+int tc_launch_bits(const tq_handle* h, const CUtensorMap& map, const tqk::etc::Args& ea, int f16in, unsigned grid,
+                   cudaStream_t s) {
+  switch (h->bits) {
+    case 1: return tc_launch_one<1, PROD, NORM32>(h, map, ea, f16in, grid, s);
+    case 2: return tc_launch_one<2, PROD, NORM32>(h, map, ea, f16in, grid, s);
+    case 3: return tc_launch_one<3, PROD, NORM32>(h, map, ea, f16in, grid, s);
+    default: return tc_launch_one<4, PROD, NORM32>(h, map, ea, f16in, grid, s);
+  }
+}
+
+int encode_tc_launch(const tq_handle* h, const tqk::EncodeArgs& a, cudaStream_t s) {
+  PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+  if (!enc) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  CUtensorMap map;
+  const cuuint64_t dims[2] = {(cuuint64_t)h->d, (cuuint64_t)a.rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)h->d * 2};
+  const cuuint32_t box[2] = {64, 128};
+  const cuuint32_t estr[2] = {1, 1};
+  CUresult r = enc(&map, a.x_dtype == TQ_F16 ? CU_TENSOR_MAP_DATA_TYPE_FLOAT16 : CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2,
+                   const_cast<void*>(a.x), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                   CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  tqk::etc::Args ea{};
+  ea.rows = a.rows; ea.norm_dtype = a.norm_dtype; ea.ops = h->dOps; ea.cent = a.cent; ea.bnd = a.bnd;
+  ea.codes = a.codes; ea.codes_B = a.codes_B; ea.signs = a.signs; ea.signs_B = a.signs_B;
+  ea.norms = a.norms; ea.rnorms = a.rnorms; ea.err = a.err;
+  const int64_t tiles = (a.rows + tqk::etc::kTile - 1) / tqk::etc::kTile;
+  const unsigned grid = (unsigned)std::min<int64_t>(tiles, sm_count(h->device));
+  const int f16 = a.x_dtype == TQ_F16 ? 1 : 0;
+  const bool n32 = a.norm_dtype == TQ_F32;
+  if (h->m > 0)
+    return n32 ? tc_launch_bits<true, true>(h, map, ea, f16, grid, s) : tc_launch_bits<true, false>(h, map, ea, f16, grid, s);
+  return n32 ? tc_launch_bits<false, true>(h, map, ea, f16, grid, s) : tc_launch_bits<false, false>(h, map, ea, f16, grid, s);
+}
+
 int encode_launch(const tq_handle* h, tqk::EncodeArgs& a, cudaStream_t s) {
+  if (tc_encode_ok(h, a)) return encode_tc_launch(h, a, s);
   if (a.len == nullptr && a.rows <= 256 && rows_kernel_ok(h, 1))
     return encode_rows_launch(h, a, (unsigned)((a.rows + tqk::kRowsMax - 1) / tqk::kRowsMax), 0, s);
   const size_t smem = tqk::encode_smem_bytes(h->m);
@@ -780,6 +922,7 @@ int tq_last_status(const tq_handle* h, void* stream) {
     e = cudaMemset(h->derr, 0, sizeof(int));
     if (e != cudaSuccess) return cuda_fail(e, "clear error word");
   }
+  if (word & tqk::kErrInternal) return fail(TQ_ECUDA, "a kernel found its shared memory misaligned");
   if (word & tqk::kErrTimeout) return fail(TQ_ETIMEOUT, "a bounded device wait timed out");
   if (word & tqk::kErrCapacity) return fail(TQ_ECAPACITY, "append skipped a full sequence (len == L_cap)");
   return ok();

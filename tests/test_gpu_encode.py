@@ -113,3 +113,70 @@ def test_config1_encode_full(tq):
     x = synth.mse_keys()
     frac, _ = _encode_and_check(tq, x, 128, 3, seed=0)
     assert frac < 1e-4
+
+
+# ---- tensor-core encode (d = 128, bf16 / f16 input, >= 1024 rows): persistent CTAs over
+# 128-vector tiles, taken in turn by 4 (MSE) or 2 (prod) epilogue groups. 170,365 rows =
+# 1330 full tiles + a ragged tile of 125: on a 148-SM B200 every CTA runs 9 or 10 tiles, so
+# every group and every pipeline stage is reused at least twice.
+
+TC_ROWS = 148 * 128 * 9 - 128 * 2 + 125
+
+
+@pytest.mark.parametrize("bits", [1, 2, 3, 4])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_encode_tc_mse(tq, bits, dtype):
+    x = torch.randn(TC_ROWS, 128, generator=torch.Generator().manual_seed(40 + bits)).to(dtype)
+    frac, _ = _encode_and_check(tq, x, 128, bits, seed=bits)
+    assert frac < 1e-4
+
+
+@pytest.mark.parametrize("bits", [2, 3])
+@pytest.mark.parametrize("dtype", [torch.bfloat16, torch.float16])
+def test_encode_tc_prod(tq, bits, dtype):
+    x = torch.randn(TC_ROWS, 128, generator=torch.Generator().manual_seed(50 + bits)).to(dtype)
+    frac, sfrac = _encode_and_check(tq, x, 128, bits, seed=2, m=128)
+    assert frac < 1e-4 and sfrac < 1e-4
+
+
+def test_encode_tc_prod_fp32_norms(tq):
+    """prod with fp32 norms: the two epilogue groups share one staged x tile (the fp64 norm
+    pass reads it), in tile order."""
+    x = torch.randn(TC_ROWS, 128, generator=torch.Generator().manual_seed(61)).to(torch.bfloat16)
+    frac, sfrac = _encode_and_check(tq, x, 128, 3, seed=3, m=128, norm_dtype=tq.TQ_F32)
+    assert frac < 1e-4 and sfrac < 1e-4
+
+
+def test_encode_tc_edge_rows(tq):
+    """Zero, one-hot and extreme-scale rows inside a tensor-core batch, fp32 and fp16 norms."""
+    g = torch.Generator().manual_seed(6)
+    x = torch.randn(3000, 128, generator=g)
+    x[5] = 0
+    x[130] = 0
+    x[131, 3] = 2.0
+    x[1000] *= 1e3
+    x[2999] *= 1e-3
+    xb = x.to(torch.bfloat16)
+    _encode_and_check(tq, xb, 128, 3, seed=1)
+    _encode_and_check(tq, xb, 128, 3, seed=1, m=128)
+    _encode_and_check(tq, xb, 128, 2, seed=1, m=128, norm_dtype=tq.TQ_F32)
+    _encode_and_check(tq, x.to(torch.float16), 128, 4, seed=1, norm_dtype=tq.TQ_F16)
+    _encode_and_check(tq, xb, 128, 2, seed=1, norm_dtype=tq.TQ_F16)
+    _encode_and_check(tq, x.to(torch.float16), 128, 1, seed=1, m=0)
+
+
+def test_encode_tc_matches_simt(tq, monkeypatch):
+    """The tensor-core and SIMT kernels agree on codes and signs away from decision
+    boundaries (both are checked against the oracle above; here against each other)."""
+    x = torch.randn(4096 + 61, 128, generator=torch.Generator().manual_seed(8)).to(torch.bfloat16).cuda()
+    h = tq.Handle(128, 3, 2, qjl_m=128)
+    a = h.encode(x)
+    monkeypatch.setenv("TQ_SIMT", "1")
+    b = h.encode(x)
+    torch.cuda.synchronize()
+    same_codes = (a["codes"] == b["codes"]).all(dim=1).float().mean().item()
+    same_signs = (a["signs"] == b["signs"]).all(dim=1).float().mean().item()
+    assert same_codes > 0.999 and same_signs > 0.999
+    # fp16 norms: the tensor-core path takes ||(Pi_hi + Pi_lo) x||, within 1 ulp of ||x||
+    ulp = (a["norms"].float() - b["norms"].float()).abs() / torch.finfo(torch.float16).eps / b["norms"].float().abs()
+    assert ulp.max().item() <= 1.0
