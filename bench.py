@@ -5,11 +5,11 @@ Workload (3-bit prod TurboQuant, d = 128): one GQA decode step over a
 compressed cache -- batch 1, 8 KV heads, 32 query heads, context 32768, K and V
 each 2-bit Lloyd-Max MSE + 1-bit QJL sketch (m = 128), fp16 norms and residual
 norms; bf16 K/V with per-(head, channel) std ~ LogNormal(0, 0.5) and 2 outlier
-channels x10 per head. A step is the whole hot path for one new token:
-tq_append(K) -> tq_append(V) (norm, rotate, bucketize, pack, QJL sign-pack of
-the new token) -> tq_attn_decode (query rotation, scores, online softmax,
-value accumulate, combine). The step is captured once in a CUDA graph; each
-timed step replays it. `len` is reset between steps (outside the timed
+channels x10 per head. A step is the whole hot path for one new token, one
+tq_decode_step call: append of the new key and value (norm, rotate, bucketize,
+pack, QJL sign-pack) together with the query rotation, then scores, online
+softmax and value accumulate, then the combine that also advances len. The
+step is captured once in a CUDA graph; each timed step replays it. `len` is reset between steps (outside the timed
 bracket) so every step attends over exactly 32768 tokens; L2 is flushed
 between steps (the packed cache, 27 MB, would otherwise sit in the 126 MB L2).
 
@@ -246,10 +246,8 @@ def run_tq(args):
     scale = 1.0 / (d ** 0.5)
     flush = torch.empty(256 * 1024 * 1024 // 4, dtype=torch.float32, device=dev)   # 2x the 126 MB L2
 
-    def step():
-        tq.tq_append(hk.ptr, k_in, B, Hkv, kc.struct, lens, 0)
-        tq.tq_append(hv.ptr, v_in, B, Hkv, vc.struct, lens, 1)
-        tq.tq_attn_decode(hk.ptr, hv.ptr, q_in, B, Hq, Hkv, kc.struct, vc.struct, lens, scale, out, ws)
+    def step():   # append the new key and value of every head at slot len[b], attend over len[b] + 1 tokens
+        tq.tq_decode_step(hk.ptr, hv.ptr, q_in, k_in, v_in, B, Hq, Hkv, kc.struct, vc.struct, lens, scale, out, ws)
 
     # eager warm-up (sets kernel attributes), then capture the step with kernel timers inside
     s = torch.cuda.Stream(device=dev)
@@ -260,14 +258,19 @@ def run_tq(args):
             lens.fill_(L0)
     torch.cuda.current_stream().wait_stream(s)
     torch.cuda.synchronize()
-    tq.tq_timer_read(None, forget=True)
-    tq.tq_timer_enable(True)
+    # two captures of the same step: `graph` (timed, nothing but the step's kernels) and
+    # `graph_k` (the same with an event pair around every kernel, for the per-kernel split)
     graph = torch.cuda.CUDAGraph()
     with torch.cuda.graph(graph):
         step()
+    tq.tq_timer_read(None, forget=True)
+    tq.tq_timer_enable(True)
+    graph_k = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_k):
+        step()
     tq.tq_timer_enable(False)
     lens.fill_(L0)
-    graph.replay()                      # the captured event pairs exist only after a replay
+    graph_k.replay()                    # the captured event pairs exist only after a replay
     lens.fill_(L0)
     torch.cuda.synchronize()
     _, kernels_per_step = tq.tq_timer_read(None, forget=False)
@@ -292,7 +295,7 @@ def run_tq(args):
         dist.barrier()
     torch.cuda.synchronize()
     split_ms, split_n = 0.0, 0
-    names = ("append", "advance_len", "qprep", "attn_split", "attn_combine")
+    names = ("prologue", "attn_split", "attn_combine")
     kern_ms = {k: 0.0 for k in names}
     for i in range(args.steps):
         set_inputs(args.warmup + i)
@@ -301,18 +304,24 @@ def run_tq(args):
         graph.replay()
         evs[i][1].record()
         lens.fill_(L0)
-        evs[i][1].synchronize()                 # captured event pairs are re-recorded by every replay
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clocks = sampler.stop() if sampler else None
+    step_ms = [a.elapsed_time(b) for a, b in evs]
+    # per-kernel device time: the same steps replayed through the instrumented capture
+    for i in range(args.steps):
+        set_inputs(args.warmup + i)
+        flush.zero_()
+        graph_k.replay()
+        lens.fill_(L0)
+        torch.cuda.synchronize()                # captured event pairs are re-recorded by every replay
         for k in names:
             ms_k, n_k = tq.tq_timer_read(k, forget=False)
             kern_ms[k] += ms_k
             if k == "attn_split":
                 split_ms += ms_k
                 split_n += n_k
-    torch.cuda.synchronize()
-    if world > 1:
-        dist.barrier()
-    clocks = sampler.stop() if sampler else None
-    step_ms = [a.elapsed_time(b) for a, b in evs]
     total_ms = sum(step_ms)
     t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
     if world > 1:
@@ -364,7 +373,7 @@ def run_tq(args):
         dist.destroy_process_group()
     if rank != 0:
         return
-    del graph
+    del graph, graph_k
     tokens = B * Hkv * L                               # key (and value) rows read per step per rank
     bytes_step = tokens * PACKED_BYTES_PER_TOKEN
     value = world * bytes_step * args.steps / (max_ms / 1e3) / 1e9
@@ -379,7 +388,7 @@ def run_tq(args):
         "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": WORKLOAD_NAME, "B": B, "Hkv": Hkv, "Hq": Hq, "context": L, "d": d,
                    "bits": "2 MSE + 1 QJL (m=128)", "l2": "flushed between steps (256 MB write)",
-                   "step": "tq_append K + tq_append V + tq_attn_decode, one CUDA graph replay",
+                   "step": "tq_decode_step (append K and V, rotate q, attend, advance len), one CUDA graph replay",
                    "parallelism": f"independent replica per GPU x{world}"},
         "keys_scored_per_s": keys_s,
         "query_key_pairs_per_s": keys_s * (Hq // Hkv),

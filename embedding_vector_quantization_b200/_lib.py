@@ -64,6 +64,7 @@ _SIGS = {
     "tq_score": (_i, [_vp, _vp, _i, _i, _i, _cp, _vp, _vp, _vp, _sz, _vp]),
     "tq_attn_decode": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _cp, _cp, _vp, _f, _vp, _vp, _sz, _vp]),
     "tq_attn_decode_noalloc": (_i, [_vp, _vp, _vp, _i, _i, _i, _i, _cp, _cp, _vp, _f, _vp, _vp]),
+    "tq_decode_step": (_i, [_vp, _vp, _vp, _i, _vp, _vp, _i, _i, _i, _i, _cp, _cp, _vp, _f, _vp, _vp, _sz, _vp]),
     "tq_search_topk": (_i, [_vp, _vp, _i, _vp, _vp, _i64, _i, _vp, _vp, _vp, _sz, _vp]),
     "tq_timer_enable": (_i, [_i]),
     "tq_timer_read": (_i, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), _ip, _i]),
@@ -224,6 +225,16 @@ def tq_attn_decode_noalloc(hk, hv, q, B, Hq, Hkv, kcache, vcache, len_, scale, o
     check(lib.tq_attn_decode_noalloc(hk, hv, _ptr(q), _dtype_code(q), B, Hq, Hkv, ctypes.byref(kcache),
                                      ctypes.byref(vcache), _ptr(len_), float(scale), _ptr(out), _stream(stream)),
           "tq_attn_decode_noalloc")
+
+
+def tq_decode_step(hk, hv, q, k_new, v_new, B, Hq, Hkv, kcache, vcache, len_, scale, out, workspace, stream=None):
+    """Append k_new / v_new [B, Hkv, d] at slot len[b], attend over len[b] + 1 tokens, advance len."""
+    if k_new.dtype != v_new.dtype:
+        raise TQError(1, "tq_decode_step", "k_new and v_new must have one dtype")
+    check(lib.tq_decode_step(hk, hv, _ptr(q), _dtype_code(q), _ptr(k_new), _ptr(v_new), _dtype_code(k_new), B, Hq,
+                             Hkv, ctypes.byref(kcache), ctypes.byref(vcache), _ptr(len_), float(scale), _ptr(out),
+                             _ptr(workspace), workspace.numel() * workspace.element_size(), _stream(stream)),
+          "tq_decode_step")
 
 
 def tq_search_topk(h, q, nq, codes, norms, n, k, idx, score, workspace, stream=None):

@@ -70,6 +70,7 @@ struct Args {
   int64_t L_cap, chunk;
   int nsplit;
   const int32_t* len;
+  int len_extra;        // 1 inside a decode step: the token appended at slot len[b] counts
   float kc0, kb0, kb1;  // K codebook: c[idx] = kc0 + kb0*b0 + kb1*b1
   float vc0, vb0, vb1;  // V codebook
   float scale;          // softmax scale
@@ -178,6 +179,105 @@ __device__ __forceinline__ int qfrag_sign_offset(int i) {
   return (((kk * 2 + slot) * 4 + t) * 8) * 4 + e;
 }
 
+// Query side of the key MMAs for the kG heads h0 .. h0 + 3 of sequence b (one warp per
+// head, warps 0..3): rotated queries scaled by the codebook slopes and S q, rounded to
+// 15-bit integers against their maxima and split into int8 hi/lo pieces in B-fragment
+// order; qconst[h] = {c0 sum(q'), step of the code pieces, step of the sign pieces, sum(S q)}.
+__device__ __forceinline__ void prepare_query(const float* qr_rows, const float* qs_rows, float kb0, float kb1,
+                                              float kc0, uint32_t (&qfrag)[12][2][4][8], float (&qconst)[kG][4]) {
+  const int lane = threadIdx.x & 31, h = threadIdx.x >> 5;
+  if (h >= kG) return;
+  const float* qr = qr_rows + (size_t)h * kD;
+  const float* qsv = qs_rows + (size_t)h * kM;
+  float x0[4], x1[4], xs[4], sq = 0.f, ss = 0.f, mx = 0.f, ms = 0.f;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float q = qr[lane + 32 * i];
+    const float s = qsv[lane + 32 * i];
+    x0[i] = kb0 * q;
+    x1[i] = kb1 * q;
+    xs[i] = s;
+    sq += q;
+    ss += s;
+    mx = fmaxf(mx, fmaxf(fabsf(x0[i]), fabsf(x1[i])));
+    ms = fmaxf(ms, fabsf(s));
+  }
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sq += __shfl_xor_sync(0xffffffffu, sq, o);
+    ss += __shfl_xor_sync(0xffffffffu, ss, o);
+    mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
+  }
+  const float dm = mx > 0.f ? mx / 16256.f : 1.f;
+  const float ds = ms > 0.f ? ms / 16256.f : 1.f;
+  int8_t* qf = reinterpret_cast<int8_t*>(&qfrag[0][0][0][0]);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const int j = lane + 32 * i;
+    const float v[3] = {x0[i] / dm, x1[i] / dm, xs[i] / ds};
+#pragma unroll
+    for (int c = 0; c < 3; ++c) {
+      const int xi = __float2int_rn(v[c]);
+      const int hi = (xi >= 0) ? (xi + 64) >> 7 : -((-xi + 64) >> 7);
+      const int off = (c < 2) ? qfrag_code_offset(c, j) : qfrag_sign_offset(j);
+      qf[off + (2 * h) * 4] = (int8_t)hi;                   // column g = 2h (hi piece)
+      qf[off + (2 * h + 1) * 4] = (int8_t)(xi - 128 * hi);  // column g = 2h + 1 (lo piece)
+    }
+  }
+  if (lane == 0) {
+    qconst[h][0] = kc0 * sq;
+    qconst[h][1] = dm;
+    qconst[h][2] = ds;
+    qconst[h][3] = ss;
+  }
+}
+
+// Raw scores (tq_score's formula) of keys kbase + g and kbase + g + 8 of a staged key block
+// for query head t = lane % 4: twelve int8 MMAs over the code and sign bit planes.
+__device__ __forceinline__ void mtile_scores(const unsigned char* st, const __half* nrm, const __half* rnm, int kbase,
+                                             const uint32_t (&qb)[12][2], float c0h, float dmh, float dsh, float ssh,
+                                             float (&sc)[2]) {
+  const int lane = threadIdx.x & 31, g = lane >> 2;
+  uint32_t cw[4], sw[2];
+  {
+    const int mat = lane >> 3, r = lane & 7;
+    const int key = kbase + r + 8 * (mat >> 1);
+    ldsm_x4(cw, st + key * kCodesB + 16 * (mat & 1));
+    const int skey = kbase + r + 8 * (mat & 1);
+    ldsm_x2(sw, st + kStageCodes + skey * kSignsB);
+  }
+  // six independent accumulator chains of length two (even / odd shifts)
+  int dm1[2][4] = {}, dm16[2][4] = {}, ds1[4] = {}, ds16[4] = {};
+  // code words: cw[0] = key g word t, cw[1] = key g word 4+t, cw[2] = key g+8 word t, cw[3] = key g+8 word 4+t
+#pragma unroll
+  for (int s = 0; s < 4; ++s) {
+    const uint32_t x0 = cw[0] >> s, x1 = cw[1] >> s, x2 = cw[2] >> s, x3 = cw[3] >> s;
+    mma_s8(dm1[s & 1], x0 & 0x01010101u, x2 & 0x01010101u, x1 & 0x01010101u, x3 & 0x01010101u, qb[s][0], qb[s][1]);
+    mma_s8(dm16[s & 1], x0 & 0x10101010u, x2 & 0x10101010u, x1 & 0x10101010u, x3 & 0x10101010u, qb[4 + s][0],
+           qb[4 + s][1]);
+  }
+  // sign words: sw[0] = key g word t, sw[1] = key g+8 word t
+#pragma unroll
+  for (int s = 0; s < 2; ++s) {
+    const uint32_t y0 = sw[0] >> s, y1 = sw[1] >> s, z0 = sw[0] >> (s + 2), z1 = sw[1] >> (s + 2);
+    mma_s8(ds1, y0 & 0x01010101u, y1 & 0x01010101u, z0 & 0x01010101u, z1 & 0x01010101u, qb[8 + s][0], qb[8 + s][1]);
+    mma_s8(ds16, y0 & 0x10101010u, y1 & 0x10101010u, z0 & 0x10101010u, z1 & 0x10101010u, qb[10 + s][0],
+           qb[10 + s][1]);
+  }
+  const float kqjl = kQjlScale / (float)kM;
+#pragma unroll
+  for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
+    const int key = kbase + g + 8 * r;
+    const int hi = 2 * r, lo = 2 * r + 1;
+    const int mse = 128 * (dm1[0][hi] + dm1[1][hi] + ((dm16[0][hi] + dm16[1][hi]) >> 4)) +
+                    (dm1[0][lo] + dm1[1][lo] + ((dm16[0][lo] + dm16[1][lo]) >> 4));
+    const int qjl = 128 * (ds1[hi] + (ds16[hi] >> 4)) + (ds1[lo] + (ds16[lo] >> 4));
+    const float n = __half2float(nrm[key]), rn = __half2float(rnm[key]);
+    sc[r] = n * (c0h + dmh * (float)mse) + rn * kqjl * (2.f * dsh * (float)qjl - ssh);
+  }
+}
+
 __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
@@ -186,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
   const int bh = blockIdx.x, split = blockIdx.y;
   const int b = bh / a.Hkv, hk = bh % a.Hkv, h0 = hk * kG;
 
-  const int64_t L = min((int64_t)max(a.len[b], 0), a.L_cap);
+  const int64_t L = min((int64_t)max(a.len[b], 0) + a.len_extra, a.L_cap);
   const int64_t start = (int64_t)split * a.chunk;
   const int64_t end = min(L, start + a.chunk);
   const int ntok = (int)max((int64_t)0, end - start);
@@ -227,57 +327,20 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
   };
   const int njobs = 2 * nblk;
   constexpr int kAhead = kStages - 2;   // jobs in flight ahead of the one being consumed (3)
+  grid_dep_launch();
+  // The kernel before this one in a decode step (append + query rotation) writes only the
+  // slot len[b] and the rotated queries: a chunk that does not hold the slot may start
+  // streaming its cache blocks before waiting for it.
+  const int64_t slot = (int64_t)max(a.len[b], 0);
+  const bool holds_new = a.len_extra && slot >= start && slot < start + a.chunk;
+  if (holds_new) grid_dep_wait();
   if (tid == 0)
     for (int j = 0; j < min(kAhead, njobs); ++j) issue(j);
+  if (!holds_new) grid_dep_wait();
 
   // query constants and int8 pieces (one warp per head)
-  if (warp < kG) {
-    const int h = warp;
-    const float* qr = a.qr + ((size_t)b * a.Hq + h0 + h) * kD;
-    const float* qsv = a.qs + ((size_t)b * a.Hq + h0 + h) * kM;
-    float x0[4], x1[4], xs[4], sq = 0.f, ss = 0.f, mx = 0.f, ms = 0.f;
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const float q = qr[lane + 32 * i];
-      const float s = qsv[lane + 32 * i];
-      x0[i] = a.kb0 * q;
-      x1[i] = a.kb1 * q;
-      xs[i] = s;
-      sq += q;
-      ss += s;
-      mx = fmaxf(mx, fmaxf(fabsf(x0[i]), fabsf(x1[i])));
-      ms = fmaxf(ms, fabsf(s));
-    }
-#pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      sq += __shfl_xor_sync(0xffffffffu, sq, o);
-      ss += __shfl_xor_sync(0xffffffffu, ss, o);
-      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
-      ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
-    }
-    const float dm = mx > 0.f ? mx / 16256.f : 1.f;
-    const float ds = ms > 0.f ? ms / 16256.f : 1.f;
-    int8_t* qf = reinterpret_cast<int8_t*>(&sm.qfrag[0][0][0][0]);
-#pragma unroll
-    for (int i = 0; i < 4; ++i) {
-      const int j = lane + 32 * i;
-      const float v[3] = {x0[i] / dm, x1[i] / dm, xs[i] / ds};
-#pragma unroll
-      for (int c = 0; c < 3; ++c) {
-        const int xi = __float2int_rn(v[c]);
-        const int hi = (xi >= 0) ? (xi + 64) >> 7 : -((-xi + 64) >> 7);
-        const int off = (c < 2) ? qfrag_code_offset(c, j) : qfrag_sign_offset(j);
-        qf[off + (2 * h) * 4] = (int8_t)hi;               // column g = 2h (hi piece)
-        qf[off + (2 * h + 1) * 4] = (int8_t)(xi - 128 * hi);  // column g = 2h + 1 (lo piece)
-      }
-    }
-    if (lane == 0) {
-      sm.qconst[h][0] = a.kc0 * sq;
-      sm.qconst[h][1] = dm;
-      sm.qconst[h][2] = ds;
-      sm.qconst[h][3] = ss;
-    }
-  }
+  prepare_query(a.qr + ((size_t)b * a.Hq + h0) * kD, a.qs + ((size_t)b * a.Hq + h0) * kM, a.kb0, a.kb1, a.kc0,
+                sm.qfrag, sm.qconst);
   __syncthreads();
 
   // B fragments of the key-side MMAs (constant for the CTA): 12 k-steps x 2 registers
@@ -287,7 +350,6 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 #pragma unroll
     for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[kk][slot][t][g];
 
-  const float kqjl = kQjlScale / (float)kM;
   const float scale2 = a.scale * 1.4426950408889634f;
   float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
   float run_max = -INFINITY;   // this thread's max logit of head t
@@ -413,47 +475,15 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
         const int kbase = 128 * mt + 16 * warp;
-        uint32_t cw[4], sw[2];
-        {
-          const int mat = lane >> 3, r = lane & 7;
-          const int key = kbase + r + 8 * (mat >> 1);
-          ldsm_x4(cw, st + key * kCodesB + 16 * (mat & 1));
-          const int skey = kbase + r + 8 * (mat & 1);
-          ldsm_x2(sw, st + kStageCodes + skey * kSignsB);
-        }
-        // six independent accumulator chains of length two (even / odd shifts)
-        int dm1[2][4] = {}, dm16[2][4] = {}, ds1[4] = {}, ds16[4] = {};
-        // code words: cw[0] = key g word t, cw[1] = key g word 4+t, cw[2] = key g+8 word t, cw[3] = key g+8 word 4+t
-#pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const uint32_t x0 = cw[0] >> s, x1 = cw[1] >> s, x2 = cw[2] >> s, x3 = cw[3] >> s;
-          mma_s8(dm1[s & 1], x0 & 0x01010101u, x2 & 0x01010101u, x1 & 0x01010101u, x3 & 0x01010101u, qb[s][0],
-                 qb[s][1]);
-          mma_s8(dm16[s & 1], x0 & 0x10101010u, x2 & 0x10101010u, x1 & 0x10101010u, x3 & 0x10101010u,
-                 qb[4 + s][0], qb[4 + s][1]);
-        }
-        // sign words: sw[0] = key g word t, sw[1] = key g+8 word t
-#pragma unroll
-        for (int s = 0; s < 2; ++s) {
-          const uint32_t y0 = sw[0] >> s, y1 = sw[1] >> s, z0 = sw[0] >> (s + 2), z1 = sw[1] >> (s + 2);
-          mma_s8(ds1, y0 & 0x01010101u, y1 & 0x01010101u, z0 & 0x01010101u, z1 & 0x01010101u, qb[8 + s][0],
-                 qb[8 + s][1]);
-          mma_s8(ds16, y0 & 0x10101010u, y1 & 0x10101010u, z0 & 0x10101010u, z1 & 0x10101010u, qb[10 + s][0],
-                 qb[10 + s][1]);
-        }
+        float sc[2];
+        mtile_scores(st, nrm, rnm, kbase, qb, c0h, dmh, dsh, ssh, sc);
 #pragma unroll
         for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
           const int key = kbase + g + 8 * r;
-          const int hi = 2 * r, lo = 2 * r + 1;
-          const int mse = 128 * (dm1[0][hi] + dm1[1][hi] + ((dm16[0][hi] + dm16[1][hi]) >> 4)) +
-                          (dm1[0][lo] + dm1[1][lo] + ((dm16[0][lo] + dm16[1][lo]) >> 4));
-          const int qjl = 128 * (ds1[hi] + (ds16[hi] >> 4)) + (ds1[lo] + (ds16[lo] >> 4));
-          const float n = __half2float(nrm[key]), rn = __half2float(rnm[key]);
-          float sc = n * (c0h + dmh * (float)mse) + rn * kqjl * (2.f * dsh * (float)qjl - ssh);
-          sc *= scale2;   // softmax scale * log2(e): the weights are exp2(logit - max)
-          sc = (key < nvalid) ? sc : -INFINITY;
-          sm.logits[t][tok_base + key] = sc;
-          run_max = fmaxf(run_max, sc);
+          // softmax scale * log2(e): the weights are exp2(logit - max)
+          const float v = (key < nvalid) ? sc[r] * scale2 : -INFINITY;
+          sm.logits[t][tok_base + key] = v;
+          run_max = fmaxf(run_max, v);
         }
       }
       // value norms of these tokens (they arrived with the key block): keep for the value pass
@@ -580,6 +610,146 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
     float* o = a.part + (((size_t)b * a.Hq + h0 + tid) * a.nsplit + split) * stride;
     o[kD + kM] = (ntok > 0) ? sm.hmax[tid] * 0.6931471805599453f : -INFINITY;   // back to natural-log units
     o[kD + kM + 1] = (ntok > 0) ? l : 0.f;
+  }
+}
+
+// ================================================================ scores (tq_score)
+//
+// The key pass above on its own: raw scores s = ||k|| <q', c[idx]> + rnorm sqrt(pi/2)/m
+// <S q, 2 sigma - 1> of every key of the chunk for the 4 query heads of a KV head,
+// written to logits [B][Hq][L_cap] ("TurboQuant: redefining AI efficiency", "QJL";
+// "Google TurboQuant", "Stage 2"). Key blocks of 256 stream through a 4-stage TMA ring;
+// each block's scores are staged in shared memory and leave as full 16-byte rows.
+
+constexpr int kSStages = 4;
+constexpr int kSStageBytes = kStageCodes + kStageSigns + 2 * kBlk * 2;  // codes, signs, norms, rnorms: 13312
+
+struct ScoreArgs {
+  const float* qr;  // [B*Hq][128] Pi q
+  const float* qs;  // [B*Hq][128] S q
+  int B, Hq, Hkv;
+  const uint8_t* kcodes;
+  const uint8_t* ksigns;
+  const __half* knorm;
+  const __half* krn;
+  int64_t L_cap, chunk;
+  const int32_t* len;
+  float kc0, kb0, kb1;
+  float* logits;    // [B][Hq][L_cap]
+  int* err;
+};
+
+struct __align__(16) ScoreSmem {
+  unsigned char stage[kSStages][kSStageBytes];
+  float out[2][kG][kBlk];         // scores of a block, double buffered: [buffer][head][key]
+  uint32_t qfrag[12][2][4][8];
+  float qconst[kG][4];
+  uint64_t full[kSStages];
+  uint64_t empty[kSStages];
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int bh = blockIdx.x, split = blockIdx.y;
+  const int b = bh / a.Hkv, hk = bh % a.Hkv, h0 = hk * kG;
+  const int64_t L = min((int64_t)max(a.len[b], 0), a.L_cap);
+  const int64_t start = (int64_t)split * a.chunk;
+  const int64_t end = min(L, start + a.chunk);
+  const int ntok = (int)max((int64_t)0, end - start);
+  const int nblk = (ntok + kBlk - 1) / kBlk;
+  const int64_t row0 = (int64_t)bh * a.L_cap + start;
+  if (nblk == 0) return;
+
+  if (tid == 0) {
+    for (int s = 0; s < kSStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kWarps);
+    }
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+  auto issue = [&](int j) {
+    const int64_t tok0 = (int64_t)j * kBlk;
+    const int ncopy = (int)min((int64_t)kBlk, a.L_cap - (start + tok0));   // multiple of 8 (L_cap % 8 == 0)
+    const int64_t r = row0 + tok0;
+    unsigned char* st = sm.stage[j % kSStages];
+    uint64_t* bar = &sm.full[j % kSStages];
+    mbar_expect_tx(bar, (uint32_t)ncopy * (kCodesB + kSignsB + 4));
+    tma_bulk_g2s(st, a.kcodes + r * kCodesB, ncopy * kCodesB, bar);
+    tma_bulk_g2s(st + kStageCodes, a.ksigns + r * kSignsB, ncopy * kSignsB, bar);
+    tma_bulk_g2s(st + kStageCodes + kStageSigns, a.knorm + r, ncopy * 2, bar);
+    tma_bulk_g2s(st + kStageCodes + kStageSigns + 2 * kBlk, a.krn + r, ncopy * 2, bar);
+  };
+  constexpr int kAhead = kSStages - 2;
+  if (tid == 0)
+    for (int j = 0; j < min(kAhead, nblk); ++j) issue(j);
+  int issued = min(kAhead, nblk);
+  grid_dep_wait();   // the rotated queries come from the kernel before this one
+
+  prepare_query(a.qr + ((size_t)b * a.Hq + h0) * kD, a.qs + ((size_t)b * a.Hq + h0) * kM, a.kb0, a.kb1, a.kc0,
+                sm.qfrag, sm.qconst);
+  __syncthreads();
+  uint32_t qb[12][2];
+#pragma unroll
+  for (int kk = 0; kk < 12; ++kk)
+#pragma unroll
+    for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[kk][slot][t][g];
+  const float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
+  const bool vec_ok = (a.L_cap % 4) == 0;   // 16-byte rows of logits
+
+  // No thread leaves this loop early (see attn_prod2_kernel): a wait that runs out stops
+  // new copies and further waits, and the remaining blocks are skipped uniformly.
+  for (int j = 0; j < nblk; ++j) {
+    const bool aborted = *(volatile int*)&sm.abort_flag != 0;
+    if (tid == 0 && !aborted && j + kAhead < nblk) {
+      const int jo = j + kAhead - kSStages;   // the stage's previous block (j - 2)
+      if (jo >= 0 && !mbar_wait(&sm.empty[jo % kSStages], (jo / kSStages) & 1)) {
+        sm.abort_flag = 1;
+      } else {
+        issue(j + kAhead);
+        issued = j + kAhead + 1;
+      }
+    }
+    if (!aborted && !mbar_wait(&sm.full[j % kSStages], (j / kSStages) & 1)) sm.abort_flag = 1;
+    const unsigned char* st = sm.stage[j % kSStages];
+    const __half* nrm = reinterpret_cast<const __half*>(st + kStageCodes + kStageSigns);
+    const __half* rnm = nrm + kBlk;
+    float* ob = &sm.out[j & 1][0][0];
+    if (!aborted) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt) {
+        const int kbase = 128 * mt + 16 * warp;
+        float sc[2];
+        mtile_scores(st, nrm, rnm, kbase, qb, c0h, dmh, dsh, ssh, sc);
+        ob[t * kBlk + kbase + g] = sc[0];
+        ob[t * kBlk + kbase + g + 8] = sc[1];
+      }
+    }
+    __syncwarp();
+    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[j % kSStages])) : "memory");
+    __syncthreads();   // the block's scores are staged (and the other buffer is free again)
+    if (!*(volatile int*)&sm.abort_flag) {
+      const int tb = j * kBlk, nvalid = min(kBlk, ntok - tb);
+      const int h = tid >> 6, k4 = 4 * (tid & 63);
+      float* dst = a.logits + ((size_t)b * a.Hq + h0 + h) * a.L_cap + start + tb + k4;
+      const float4 v4 = *reinterpret_cast<const float4*>(ob + h * kBlk + k4);
+      if (vec_ok && k4 + 4 <= nvalid) {
+        *reinterpret_cast<float4*>(dst) = v4;
+      } else {
+        const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
+        for (int i = 0; i < 4 && k4 + i < nvalid; ++i) dst[i] = vv[i];
+      }
+    }
+  }
+  __syncthreads();
+  if (sm.abort_flag && tid == 0) {
+    report_error(a.err, kErrTimeout);
+    for (int jx = max(0, issued - kSStages); jx < issued; ++jx) (void)mbar_wait(&sm.full[jx % kSStages], (jx / kSStages) & 1);
   }
 }
 

@@ -70,6 +70,13 @@ __device__ __forceinline__ uint32_t sign_bit(const uint32_t* row, int j) {
   return (row[j >> 5] >> (j & 31)) & 1u;
 }
 
+// ---- programmatic dependent launch: a kernel launched with programmatic stream
+// serialization may start while the previous kernel of the stream still runs; it must
+// wait (grid_dep_wait) before touching that kernel's outputs. Both are no-ops for a
+// kernel launched without the attribute.
+__device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
+__device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
+
 // ---- TMA bulk copies (global -> shared) completed on an mbarrier
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

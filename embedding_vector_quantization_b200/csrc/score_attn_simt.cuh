@@ -183,12 +183,15 @@ struct AttnArgs {
   int64_t L_cap, chunk;
   int nsplit;
   const int32_t* len;
+  int len_extra;    // 1 inside a decode step: the token appended at slot len[b] counts
   float scale;
   float* part;      // [B*Hq][nsplit][partial_stride(d, mv)]
 };
 
 __global__ void __launch_bounds__(kAttnThreads) attn_split_simt_kernel(AttnArgs a) {
   extern __shared__ float sm[];
+  grid_dep_launch();
+  grid_dep_wait();
   const int G = a.Hq / a.Hkv;
   const int d = a.d, mk = a.k.m, mv = a.v.m;
   const int bh = blockIdx.x, split = blockIdx.y;
@@ -216,7 +219,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_simt_kernel(AttnArgs 
 #pragma unroll
   for (int g = 0; g < kMaxGroup; ++g) { acc[g][0] = acc[g][1] = 0.f; accs[g][0] = accs[g][1] = 0.f; }
 
-  const int64_t L = min((int64_t)max(a.len[b], 0), a.L_cap);  // never read past the cache
+  const int64_t L = min((int64_t)max(a.len[b], 0) + a.len_extra, a.L_cap);  // never read past the cache
   const int64_t start = (int64_t)split * a.chunk;
   const int64_t end = min(L, start + a.chunk);
   const int64_t base = (int64_t)bh * a.L_cap;

@@ -1,19 +1,17 @@
-// Latency-oriented kernels of the decode step for head dimensions up to 128:
-// streaming append, query rotation and the split-K combine. Each stages the
-// small constant matrices it needs (Pi^T, (S Pi^T)^T, S^T, Pi_V, S_V) and its
-// other inputs with one TMA bulk copy -- a single memory round trip -- and then
-// works from shared memory, one thread per output coordinate.
+// Latency-oriented kernels of the decode step: streaming append, query rotation
+// and the split-K combine.
 //
 //  * append_cluster_kernel: one CTA per (sequence, KV head) vector, the Hkv CTAs
 //    of a sequence form a thread-block cluster. Encode as in "Google TurboQuant:
-//    6x KV-cache compression" (ebisuda.net), "Stage 1" / "Stage 2"; every CTA
-//    reads len[b] before a cluster barrier, after which rank 0 advances len[b]
-//    ("Fractal KV-cache archive" (gist.science), "Problem statement": O(1)
-//    append to a growing cache).
-//  * qprep_staged_kernel: q' = Pi q and q_s = S q for a group of query rows.
-//  * combine_staged_kernel: log-sum-exp merge of one query head's chunk partials
-//    and the map back from the rotated domain,
-//    o = (Pi_V^T acc + sqrt(pi/2)/m S_V^T acc_s) / sum p.
+//    6x KV-cache compression" (ebisuda.net), "Stage 1" / "Stage 2", with Pi^T and
+//    (S Pi^T)^T staged by one TMA bulk copy; every CTA reads len[b] before a
+//    cluster barrier, after which rank 0 advances len[b] ("Fractal KV-cache
+//    archive" (gist.science), "Problem statement": O(1) append to a growing cache).
+//  * qprep_wide_kernel: q' = Pi q and q_s = S q; each CTA owns 32 output columns of
+//    a group of query rows and stages only those columns of Pi^T / S^T.
+//  * combine_wide_kernel: log-sum-exp merge of one query head's chunk partials and
+//    the map back from the rotated domain, o = (Pi_V^T acc + sqrt(pi/2)/m S_V^T acc_s)
+//    / sum p; each CTA owns 32 output coordinates.
 #pragma once
 
 #include <cooperative_groups.h>
@@ -32,11 +30,10 @@ __host__ __device__ inline size_t append_cluster_smem_bytes(int d, int m) {
   return (size_t)d * (d + m) * 4 + (size_t)3 * d * 4 + 64 + 4 * 16 + 64;
 }
 
-__global__ void __launch_bounds__(kSmallThreads) append_cluster_kernel(EncodeArgs a, int advance) {
-  namespace cg = cooperative_groups;
-  extern __shared__ __align__(16) unsigned char smem_raw[];
+// Encodes input row b * Hkv + h into slot len[b] of KV head h (len itself is not changed);
+// a full sequence is skipped and flagged once (by head 0). Returns the slot, or -1 if skipped.
+__device__ __forceinline__ int32_t append_vector(const EncodeArgs& a, int b, int h, unsigned char* smem_raw) {
   const int d = a.d, m = a.m, bits = a.bits, L = 1 << bits;
-  const int h = blockIdx.x, b = blockIdx.y;
   const int64_t r = (int64_t)b * a.Hkv + h;   // input row
   float* mat = reinterpret_cast<float*>(smem_raw);          // [d][d] Pi^T, then [d][m] (S Pi^T)^T
   float* xs = mat + (size_t)d * (d + m);                    // [d] input, then e
@@ -121,10 +118,18 @@ __global__ void __launch_bounds__(kSmallThreads) append_cluster_kernel(EncodeArg
       }
     }
   }
+  return full ? -1 : pos;
+}
+
+__global__ void __launch_bounds__(kSmallThreads) append_cluster_kernel(EncodeArgs a, int advance) {
+  namespace cg = cooperative_groups;
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int32_t pos = append_vector(a, b, h, smem_raw);
   if (advance) {
     // every CTA of the sequence has read len[b]; then rank 0 moves it on
     cg::this_cluster().sync();
-    if (!full && h == 0 && tid == 0) a.len[b] = pos + 1;
+    if (pos >= 0 && h == 0 && threadIdx.x == 0) a.len[b] = pos + 1;
   }
 }
 
@@ -132,55 +137,81 @@ __global__ void __launch_bounds__(kSmallThreads) append_cluster_kernel(EncodeArg
 
 constexpr int kQRows = 8;
 
-__host__ __device__ inline size_t qprep_staged_smem_bytes(int d, int m) {
-  return (size_t)d * (d + m) * 4 + (size_t)kQRows * d * 4 + 16;
+// q' = Pi q and q_s = S q for d <= kWideMaxD: CTA (row group, column block) computes 32 of the d + m
+// outputs (q' = Pi q for o < d, q_s = S q after) of up to kQRows query rows. It stages
+// only its 32 columns of Pi^T (or S^T), d x 32 floats, with every thread's vector loads in
+// flight at once, then forms the dot products from shared memory.
+constexpr int kWideMaxD = 512;
+constexpr int kWideCols = 32;
+
+__host__ __device__ inline size_t qprep_wide_smem_bytes(int d) {
+  return (size_t)d * kWideCols * 4 + (size_t)kQRows * d * 4;
 }
 
-// mats = [Pi^T | S^T] as two row-major blocks [d][d] and [d][m].
-__global__ void __launch_bounds__(kSmallThreads) qprep_staged_kernel(const void* q, int q_dtype, int rows, int d,
-                                                                     const float* PiT, const float* ST, int m,
-                                                                     float* out_r, float* out_s, int* err) {
-  extern __shared__ __align__(16) unsigned char smem_raw[];
-  float* mat = reinterpret_cast<float*>(smem_raw);
-  float* qsh = mat + (size_t)d * (d + m);
-  uint64_t* bar = reinterpret_cast<uint64_t*>(qsh + kQRows * d);
-  const int row0 = blockIdx.x * kQRows, nr = min(kQRows, rows - row0);
+__device__ __forceinline__ void qprep_tile(const void* q, int q_dtype, int rows, int d, const float* PiT,
+                                           const float* ST, int m, float* out_r, float* out_s, int rg, int cb,
+                                           unsigned char* smem_raw) {
+  float* sub = reinterpret_cast<float*>(smem_raw);   // [d][32]
+  float* qsh = sub + (size_t)d * kWideCols;           // [kQRows][d]
+  const int row0 = rg * kQRows, nr = min(kQRows, rows - row0);
+  const int o0 = cb * kWideCols;
+  const bool rot = o0 < d;
+  const float* src = rot ? PiT + o0 : ST + (o0 - d);
+  const int ld = rot ? d : m;
   const int tid = threadIdx.x;
-  if (tid == 0) {
-    bar_init(bar, 1);
-    const uint32_t b1 = (uint32_t)d * d * 4, b2 = (uint32_t)d * m * 4;
-    bar_expect_tx(bar, b1 + b2);
-    bulk_g2s_large(mat, PiT, b1, bar);
-    if (m > 0) bulk_g2s_large(mat + (size_t)d * d, ST, b2, bar);
+  for (int i = tid; i < d * (kWideCols / 4); i += blockDim.x) {
+    const int k = i / (kWideCols / 4), c4 = i % (kWideCols / 4);
+    reinterpret_cast<float4*>(sub)[i] = *reinterpret_cast<const float4*>(src + (size_t)k * ld + 4 * c4);
   }
   for (int i = tid; i < nr * d; i += blockDim.x) qsh[i] = load_any(q, q_dtype, (int64_t)row0 * d + i);
   __syncthreads();
-  const bool arrived = bar_wait(bar, 0);
-  if (__syncthreads_or(!arrived)) {
-    if (tid == 0) { report_error(err, kErrTimeout); (void)bar_wait(bar, 0); }
-    return;
+  const int c = tid % kWideCols;
+  for (int r = tid / kWideCols; r < nr; r += blockDim.x / kWideCols) {
+    float acc[4] = {0.f, 0.f, 0.f, 0.f};
+#pragma unroll 8
+    for (int k = 0; k < d; ++k) acc[k & 3] = fmaf(sub[k * kWideCols + c], qsh[r * d + k], acc[k & 3]);
+    const float v = (acc[0] + acc[1]) + (acc[2] + acc[3]);
+    if (rot)
+      out_r[(size_t)(row0 + r) * d + o0 + c] = v;
+    else
+      out_s[(size_t)(row0 + r) * m + (o0 - d) + c] = v;
   }
-  for (int o = tid; o < d + m; o += blockDim.x) {
-    const bool rot = o < d;
-    const float* col = rot ? mat + o : mat + (size_t)d * d + (o - d);
-    const int ld = rot ? d : m;
-    float acc[kQRows];
-#pragma unroll
-    for (int r = 0; r < kQRows; ++r) acc[r] = 0.f;
-#pragma unroll 4
-    for (int k = 0; k < d; ++k) {
-      const float v = col[(size_t)k * ld];
-#pragma unroll
-      for (int r = 0; r < kQRows; ++r) acc[r] = fmaf(v, qsh[r * d + k], acc[r]);
-    }
-#pragma unroll
-    for (int r = 0; r < kQRows; ++r) {
-      if (r >= nr) break;
-      if (rot)
-        out_r[(size_t)(row0 + r) * d + o] = acc[r];
-      else
-        out_s[(size_t)(row0 + r) * m + (o - d)] = acc[r];
-    }
+}
+
+__global__ void __launch_bounds__(kSmallThreads) qprep_wide_kernel(const void* q, int q_dtype, int rows, int d,
+                                                                   const float* PiT, const float* ST, int m,
+                                                                   float* out_r, float* out_s) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  grid_dep_launch();
+  qprep_tile(q, q_dtype, rows, d, PiT, ST, m, out_r, out_s, blockIdx.x, blockIdx.y, smem_raw);
+}
+
+// ---------------------------------------------------------------- decode-step prologue
+
+// One launch for the independent first half of a decode step: CTAs [0, nvec) append the
+// new keys, [nvec, 2 nvec) the new values (slot len[b], len unchanged: the combine that
+// ends the step advances it), and the rest rotate the queries (qprep_tile).
+struct PrologueArgs {
+  EncodeArgs k, v;
+  int nvec;          // B * Hkv
+  const void* q;
+  int q_dtype, rows, d, m, qcols;
+  const float* PiT;
+  const float* ST;
+  float* qr;
+  float* qs;
+};
+
+__global__ void __launch_bounds__(kSmallThreads) decode_prologue_kernel(PrologueArgs p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  grid_dep_launch();
+  const int bid = blockIdx.x;
+  if (bid < 2 * p.nvec) {
+    const int v = bid % p.nvec;
+    (void)append_vector(bid < p.nvec ? p.k : p.v, v / p.k.Hkv, v % p.k.Hkv, smem_raw);
+  } else {
+    const int t = bid - 2 * p.nvec;
+    qprep_tile(p.q, p.q_dtype, p.rows, p.d, p.PiT, p.ST, p.m, p.qr, p.qs, t / p.qcols, t % p.qcols, smem_raw);
   }
 }
 
@@ -190,12 +221,10 @@ __global__ void __launch_bounds__(kSmallThreads) qprep_staged_kernel(const void*
 // rotated-domain value sum (d), QJL sum (mv), chunk max, chunk sum of p.
 __host__ __device__ inline int partial_stride(int d, int mv) { return (d + mv + 2 + 3) / 4 * 4; }
 
-__host__ __device__ inline size_t combine_staged_smem_bytes(int nsplit, int d, int mv) {
-  return 16 + (size_t)nsplit * partial_stride(d, mv) * 4 + (size_t)d * (d + mv) * 4 + (size_t)nsplit * 4 +
-         (size_t)(d + mv) * 4 + 64;
-}
-
-struct CombineStagedArgs {
+struct CombineWideArgs {
+  int32_t* len_advance;   // decode step: len[b] += 1 (below L_cap) once the step is done, else NULL
+  int Hq;
+  int64_t L_cap;
   const float* part;
   int nsplit, d, mv;
   const float* PiV;   // [d][d]
@@ -204,41 +233,47 @@ struct CombineStagedArgs {
   int* err;
 };
 
-__global__ void __launch_bounds__(kSmallThreads) combine_staged_kernel(CombineStagedArgs a) {
+// Wide combine for d <= kWideMaxD: CTA (query row, 32-coordinate block) merges all chunk
+// partials of its row by log-sum-exp (w_s = exp(max_s - M), L = sum_s w_s l_s), forms the
+// rotated-domain sums acc = sum_s w_s part_s, and applies its 32 columns of the inverse map:
+// o_j = (sum_k Pi_V[k][j] acc[k] + sqrt(pi/2)/m sum_k S_V[k][j] acc_s[k]) / L.
+__host__ __device__ inline size_t combine_wide_smem_bytes(int nsplit, int d, int mv) {
+  return (size_t)(d + mv) * kWideCols * 4 + (size_t)nsplit * 4 + (size_t)(d + mv) * 4 + 64 +
+         (size_t)nsplit * partial_stride(d, mv) * 4;
+}
+
+__global__ void __launch_bounds__(kSmallThreads) combine_wide_kernel(CombineWideArgs a) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   const int d = a.d, mv = a.mv, dm = d + mv, stride = partial_stride(d, mv), ns = a.nsplit;
-  uint64_t* bar = reinterpret_cast<uint64_t*>(smem_raw);  // [2] (16 bytes, keeps the copies 16-byte aligned)
-  float* P = reinterpret_cast<float*>(smem_raw + 16);     // [ns][stride]
-  float* mats = P + (size_t)ns * stride;                  // [d][d] Pi_V then [mv][d] S_V
-  float* w = mats + (size_t)d * dm;                       // [ns]
-  float* acc = w + ns;                                    // [d + mv]
-  float* misc = acc + dm;                                 // [16]
-  const int row = blockIdx.x, tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  if (tid == 0) {
-    bar_init(bar, 1);
-    const uint32_t bp = (uint32_t)ns * stride * 4, b1 = (uint32_t)d * d * 4, b2 = (uint32_t)mv * d * 4;
-    bar_expect_tx(bar, bp + b1 + b2);
-    bulk_g2s_large(P, a.part + (size_t)row * ns * stride, bp, bar);
-    bulk_g2s_large(mats, a.PiV, b1, bar);
-    if (mv > 0) bulk_g2s_large(mats + (size_t)d * d, a.SV, b2, bar);
+  float* P = reinterpret_cast<float*>(smem_raw);      // [ns][stride]: this row's partials (stride % 4 == 0)
+  float* cols = P + (size_t)ns * stride;               // [d + mv][32]: Pi_V rows k, then S_V rows k
+  float* w = cols + (size_t)dm * kWideCols;            // [ns]
+  float* acc = w + ns;                                 // [d + mv]
+  float* misc = acc + dm;                              // [16]
+  const int row = blockIdx.x, j0 = blockIdx.y * kWideCols;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  for (int i = tid; i < dm * (kWideCols / 4); i += blockDim.x) {
+    const int k = i / (kWideCols / 4), c4 = i % (kWideCols / 4);
+    const float* src = (k < d) ? a.PiV + (size_t)k * d : a.SV + (size_t)(k - d) * d;
+    reinterpret_cast<float4*>(cols)[i] = *reinterpret_cast<const float4*>(src + j0 + 4 * c4);
+  }
+  grid_dep_wait();   // the partials (and, in a decode step, len) come from the attention kernel
+  {  // all of the row's partials at once, independent 16-byte loads (stride is a multiple of 4)
+    const float4* src = reinterpret_cast<const float4*>(a.part + (size_t)row * ns * stride);
+    for (int i = tid; i < ns * stride / 4; i += blockDim.x) reinterpret_cast<float4*>(P)[i] = src[i];
   }
   __syncthreads();
-  const bool arrived = bar_wait(bar, 0);
-  if (__syncthreads_or(!arrived)) {
-    if (tid == 0) { report_error(a.err, kErrTimeout); (void)bar_wait(bar, 0); }
-    return;
-  }
   if (warp == 0) {
     float M = -INFINITY;
-    for (int s = lane; s < ns; s += 32) M = fmaxf(M, P[s * stride + dm]);
+    for (int s = lane; s < ns; s += 32) M = fmaxf(M, P[(size_t)s * stride + dm]);
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
     float Ls = 0.f;
     for (int s = lane; s < ns; s += 32) {
-      const float ms = P[s * stride + dm];
+      const float ms = P[(size_t)s * stride + dm];
       const float ws = (ms == -INFINITY) ? 0.f : __expf(ms - M);
       w[s] = ws;
-      Ls += ws * P[s * stride + dm + 1];
+      Ls += ws * P[(size_t)s * stride + dm + 1];
     }
 #pragma unroll
     for (int o = 16; o > 0; o >>= 1) Ls += __shfl_xor_sync(0xffffffffu, Ls, o);
@@ -246,20 +281,37 @@ __global__ void __launch_bounds__(kSmallThreads) combine_staged_kernel(CombineSt
   }
   __syncthreads();
   for (int j = tid; j < dm; j += blockDim.x) {
-    float v = 0.f;
-    for (int s = 0; s < ns; ++s) v = fmaf(w[s], P[s * stride + j], v);
-    acc[j] = v;
+    float v0 = 0.f, v1 = 0.f;
+    int s = 0;
+    for (; s + 1 < ns; s += 2) {
+      v0 = fmaf(w[s], P[(size_t)s * stride + j], v0);
+      v1 = fmaf(w[s + 1], P[(size_t)(s + 1) * stride + j], v1);
+    }
+    if (s < ns) v0 = fmaf(w[s], P[(size_t)s * stride + j], v0);
+    acc[j] = v0 + v1;
   }
   __syncthreads();
+  // thread (c, slice): partial dot over k = slice, slice + 8, ... for column c, then a shuffle-free
+  // reduction through shared memory (the 8 slices of a column are 8 warps)
   const float qscale = (mv > 0) ? kQjlScale / (float)mv : 0.f;
-  for (int j = tid; j < d; j += blockDim.x) {
-    float o = 0.f, os = 0.f;
-#pragma unroll 8
-    for (int k = 0; k < d; ++k) o = fmaf(mats[k * d + j], acc[k], o);
-    for (int k = 0; k < mv; ++k) os = fmaf(mats[(size_t)(d + k) * d + j], acc[d + k], os);
-    o = fmaf(qscale, os, o);
+  const int c = tid % kWideCols, sl = tid / kWideCols, nsl = blockDim.x / kWideCols;
+  float o = 0.f, os = 0.f;
+  for (int k = sl; k < d; k += nsl) o = fmaf(cols[k * kWideCols + c], acc[k], o);
+  for (int k = sl; k < mv; k += nsl) os = fmaf(cols[(d + k) * kWideCols + c], acc[d + k], os);
+  __syncthreads();
+  float* red = cols;   // reuse: [nsl][32]
+  red[sl * kWideCols + c] = fmaf(qscale, os, o);
+  __syncthreads();
+  if (tid < kWideCols) {
+    float t = 0.f;
+    for (int i = 0; i < nsl; ++i) t += red[i * kWideCols + tid];
     const float Ls = misc[0];
-    a.out[(size_t)row * d + j] = (Ls > 0.f) ? o / Ls : 0.f;
+    a.out[(size_t)row * d + j0 + tid] = (Ls > 0.f) ? t / Ls : 0.f;
+  }
+  if (a.len_advance && blockIdx.y == 0 && row % a.Hq == 0 && tid == 0) {
+    const int b = row / a.Hq;
+    const int32_t cur = a.len_advance[b];
+    if (cur >= 0 && cur < a.L_cap) a.len_advance[b] = cur + 1;
   }
 }
 

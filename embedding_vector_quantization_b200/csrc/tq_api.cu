@@ -19,6 +19,7 @@
 #include <cstring>
 #include <mutex>
 #include <string>
+#include <utility>
 #include <vector>
 
 #include "tq.h"
@@ -353,6 +354,15 @@ bool attn_prod2_fast_path(const tq_handle* hk, const tq_handle* hv, int G, const
   return G == 4 && ok_handle(hk) && ok_handle(hv) && k->L_cap % 8 == 0 && ok_cache(k) && ok_cache(v);
 }
 
+// tq_score on the int8 tensor cores: the same key formats as the attention fast path.
+bool score_prod2_fast_path(const tq_handle* hk, int G, const tq_cache* k) {
+  if (std::getenv("TQ_SIMT")) return false;
+  const bool fmt = hk->d == 128 && hk->m == 128 && hk->bits == 2 && hk->norm_dtype == TQ_F16 &&
+                   std::fabs(hk->cent[3] - hk->cent[2] - hk->cent[1] + hk->cent[0]) < 1e-12;
+  return G == 4 && fmt && k->L_cap % 8 == 0 && aligned(k->codes, 16) && aligned(k->signs, 16) &&
+         aligned(k->norms, 16) && aligned(k->rnorms, 16);
+}
+
 struct ScoreWs { float* qr; float* qs; };
 size_t score_ws_layout(const tq_handle* h, int rows, char* base, ScoreWs* w) {
   size_t off = 0;
@@ -395,14 +405,15 @@ size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base
 
 int launch_qprep(const tq_handle* h, const void* q, int q_dtype, int rows, float* qr, float* qs, cudaStream_t s) {
   if (rows == 0) return TQ_OK;
-  if (h->d <= tqk::kSmallMaxD && h->m <= tqk::kSmallMaxD) {
-    const size_t smem = tqk::qprep_staged_smem_bytes(h->d, h->m);
+  if (h->d <= tqk::kWideMaxD && h->m <= tqk::kWideMaxD) {
+    const size_t smem = tqk::qprep_wide_smem_bytes(h->d);
     if (once_per_device(6, h->device))
-      cudaFuncSetAttribute(tqk::qprep_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+      cudaFuncSetAttribute(tqk::qprep_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+    dim3 grid((unsigned)((rows + tqk::kQRows - 1) / tqk::kQRows), (unsigned)((h->d + h->m) / tqk::kWideCols));
     KernelScope ks("qprep", s);
-    tqk::qprep_staged_kernel<<<(rows + tqk::kQRows - 1) / tqk::kQRows, tqk::kSmallThreads, smem, s>>>(
-        q, q_dtype, rows, h->d, h->dPiT, h->dST, h->m, qr, qs, h->derr);
-    return launch_check("qprep_staged_kernel");
+    tqk::qprep_wide_kernel<<<grid, tqk::kSmallThreads, smem, s>>>(q, q_dtype, rows, h->d, h->dPiT, h->dST, h->m,
+                                                                   qr, qs);
+    return launch_check("qprep_wide_kernel");
   }
   const int groups = (rows + tqk::kQprepRows - 1) / tqk::kQprepRows;
   dim3 grid(groups, (h->d + h->m + 63) / 64);
@@ -426,6 +437,23 @@ int encode_rows_launch(const tq_handle* h, tqk::EncodeArgs& a, unsigned grid, in
   KernelScope ks(a.len ? "append" : "encode", s);
   tqk::encode_rows_kernel<<<grid, tqk::kRowsThreads, smem, s>>>(a, advance);
   return launch_check("encode_rows_kernel");
+}
+
+// Launch with programmatic stream serialization: the kernel may start while the previous
+// kernel of the stream finishes, and waits (griddepcontrol.wait) before reading its outputs.
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg{};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute at[1];
+  at[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  at[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = at;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
 }
 
 // ---- tensor-core encode (d = 128, bf16 / f16 input)
@@ -727,10 +755,32 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const 
   score_ws_layout(hk, B * Hq, static_cast<char*>(workspace), &w);
   st = launch_qprep(hk, q, TQ_F32, B * Hq, w.qr, w.qs, s);
   if (st) return st;
+  const int64_t units = (int64_t)B * Hkv;
+  if (score_prod2_fast_path(hk, Hq / Hkv, k)) {
+    // about eight waves of 3 CTAs per SM; chunks are whole 256-key blocks
+    const int64_t target = 8 * 3 * (int64_t)sm_count(hk->device);
+    int64_t chunk = ((units * k->L_cap + target - 1) / target + 255) / 256 * 256;
+    chunk = std::max<int64_t>(256, std::min<int64_t>(chunk, (k->L_cap + 255) / 256 * 256));
+    const int64_t nsp = (k->L_cap + chunk - 1) / chunk;
+    tqk::amma::ScoreArgs m{};
+    m.qr = w.qr; m.qs = w.qs; m.B = B; m.Hq = Hq; m.Hkv = Hkv;
+    m.kcodes = k->codes; m.ksigns = k->signs; m.knorm = static_cast<const __half*>(k->norms);
+    m.krn = static_cast<const __half*>(k->rnorms);
+    m.L_cap = k->L_cap; m.chunk = chunk; m.len = len;
+    m.kc0 = (float)hk->cent[0]; m.kb0 = (float)(hk->cent[1] - hk->cent[0]); m.kb1 = (float)(hk->cent[2] - hk->cent[0]);
+    m.logits = logits; m.err = hk->derr;
+    const size_t msmem = sizeof(tqk::amma::ScoreSmem);
+    if (once_per_device(10, hk->device))
+      cudaFuncSetAttribute(tqk::amma::score_prod2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    KernelScope ks("score", s);
+    const cudaError_t e = launch_pdl(tqk::amma::score_prod2_kernel, dim3((unsigned)units, (unsigned)nsp),
+                                     dim3(tqk::amma::kThreads), msmem, s, m);
+    if (e != cudaSuccess) return cuda_fail(e, "score_prod2_kernel");
+    return launch_check("score_prod2_kernel");
+  }
   tqk::ScoreArgs a{};
   a.qr = w.qr; a.qs = w.qs; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = hk->d; a.k = view_of(hk, k);
   a.L_cap = k->L_cap; a.len = len; a.logits = logits;
-  const int64_t units = (int64_t)B * Hkv;
   int64_t ns = std::max<int64_t>(1, std::min<int64_t>((8 * 148 + units - 1) / units, (k->L_cap + 127) / 128));
   a.chunk = ((k->L_cap + ns - 1) / ns + 127) / 128 * 128;
   ns = (k->L_cap + a.chunk - 1) / a.chunk;
@@ -741,9 +791,14 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const 
   return launch_check("score_simt_kernel");
 }
 
-int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
-                   const tq_cache* k, const tq_cache* v, const int32_t* len, float scale, float* out,
-                   void* workspace, size_t ws_bytes, void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Argument checks shared by tq_attn_decode and tq_decode_step (TQ_OK also for B == 0).
+int attn_check(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
+               const tq_cache* k, const tq_cache* v, const int32_t* len, float scale, float* out, void* workspace,
+               size_t ws_bytes) {
   if (!hk || !hv) return fail(TQ_EINVAL, "handle is NULL");
   if (hk->d != hv->d) return fail(TQ_EINVAL, "K and V handles differ in d (%d vs %d)", hk->d, hv->d);
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return fail(TQ_EINVAL, "B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
@@ -762,18 +817,26 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
   if (!aligned(workspace, 16)) return fail(TQ_EINVAL, "workspace misaligned");
   if (!std::isfinite(scale)) return fail(TQ_EINVAL, "scale is not finite");
   if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
-  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  return ok();
+}
+
+// Query rotation (unless a decode-step prologue did it), split attention and combine.
+// fused: the token appended at slot len[b] by the prologue counts, and the combine
+// advances len[b] once everything that reads it is done.
+int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
+              const tq_cache* k, const tq_cache* v, int32_t* len, float scale, float* out, void* workspace,
+              cudaStream_t s, bool fused) {
   ScoreWs w;
   float* part;
   int nsplit;
   int64_t chunk;
   attn_ws_layout(hk, hv, B, Hq, Hkv, k->L_cap, static_cast<char*>(workspace), &w, &part, &nsplit, &chunk);
-  st = launch_qprep(hk, q, q_dtype, B * Hq, w.qr, w.qs, s);
-  if (st) return st;
+  int st = TQ_OK;
+  if (!fused && (st = launch_qprep(hk, q, q_dtype, B * Hq, w.qr, w.qs, s))) return st;
   tqk::AttnArgs a{};
   a.qr = w.qr; a.qs = w.qs; a.B = B; a.Hq = Hq; a.Hkv = Hkv; a.d = hk->d;
   a.k = view_of(hk, k); a.v = view_of(hv, v); a.L_cap = k->L_cap; a.chunk = chunk; a.nsplit = nsplit;
-  a.len = len; a.scale = scale; a.part = part;
+  a.len = len; a.len_extra = fused ? 1 : 0; a.scale = scale; a.part = part;
   const int G = Hq / Hkv;
   if (attn_prod2_fast_path(hk, hv, G, k, v)) {
     tqk::amma::Args m{};
@@ -782,7 +845,7 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
     m.krn = static_cast<const __half*>(k->rnorms);
     m.vcodes = v->codes; m.vsigns = v->signs; m.vnorm = static_cast<const __half*>(v->norms);
     m.vrn = static_cast<const __half*>(v->rnorms);
-    m.L_cap = k->L_cap; m.chunk = chunk; m.nsplit = nsplit; m.len = len;
+    m.L_cap = k->L_cap; m.chunk = chunk; m.nsplit = nsplit; m.len = len; m.len_extra = fused ? 1 : 0;
     m.kc0 = (float)hk->cent[0]; m.kb0 = (float)(hk->cent[1] - hk->cent[0]); m.kb1 = (float)(hk->cent[2] - hk->cent[0]);
     m.vc0 = (float)hv->cent[0]; m.vb0 = (float)(hv->cent[1] - hv->cent[0]); m.vb1 = (float)(hv->cent[2] - hv->cent[0]);
     m.scale = scale; m.part = part; m.err = hk->derr;
@@ -793,7 +856,9 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
     }
     {
       KernelScope ks("attn_split", s);
-      tqk::amma::attn_prod2_kernel<<<dim3((unsigned)(B * Hkv), (unsigned)nsplit), tqk::amma::kThreads, msmem, s>>>(m);
+      const cudaError_t e = launch_pdl(tqk::amma::attn_prod2_kernel, dim3((unsigned)(B * Hkv), (unsigned)nsplit),
+                                       dim3(tqk::amma::kThreads), msmem, s, m);
+      if (e != cudaSuccess) return cuda_fail(e, "attn_prod2_kernel");
     }
     if ((st = launch_check("attn_prod2_kernel"))) return st;
   } else {
@@ -801,20 +866,25 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
                          2 * tqk::kAttnThreads + 4 * (size_t)G) * 4;
     {
       KernelScope ks("attn_split", s);
-      tqk::attn_split_simt_kernel<<<dim3((unsigned)(B * Hkv), (unsigned)nsplit), tqk::kAttnThreads, smem, s>>>(a);
+      const cudaError_t e = launch_pdl(tqk::attn_split_simt_kernel, dim3((unsigned)(B * Hkv), (unsigned)nsplit),
+                                       dim3(tqk::kAttnThreads), smem, s, a);
+      if (e != cudaSuccess) return cuda_fail(e, "attn_split_simt_kernel");
     }
     if ((st = launch_check("attn_split_simt_kernel"))) return st;
   }
-  if (tqk::combine_staged_smem_bytes(nsplit, hv->d, hv->m) <= 200 * 1024) {
-    tqk::CombineStagedArgs cs{};
+  if (hv->d <= tqk::kWideMaxD && hv->m <= tqk::kWideMaxD &&
+      tqk::combine_wide_smem_bytes(nsplit, hv->d, hv->m) <= 200 * 1024) {
+    tqk::CombineWideArgs cs{};
     cs.part = part; cs.nsplit = nsplit; cs.d = hv->d; cs.mv = hv->m; cs.PiV = hv->dPi; cs.SV = hv->dS;
     cs.out = out; cs.err = hv->derr;
+    cs.len_advance = fused ? len : nullptr; cs.Hq = Hq; cs.L_cap = k->L_cap;
     if (once_per_device(7, hv->device))
-      cudaFuncSetAttribute(tqk::combine_staged_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+      cudaFuncSetAttribute(tqk::combine_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
     KernelScope ks("attn_combine", s);
-    tqk::combine_staged_kernel<<<B * Hq, tqk::kSmallThreads, tqk::combine_staged_smem_bytes(nsplit, hv->d, hv->m),
-                                 s>>>(cs);
-    return launch_check("combine_staged_kernel");
+    const cudaError_t e = launch_pdl(tqk::combine_wide_kernel, dim3((unsigned)(B * Hq), (unsigned)(hv->d / tqk::kWideCols)),
+                                     dim3(tqk::kSmallThreads), tqk::combine_wide_smem_bytes(nsplit, hv->d, hv->m), s, cs);
+    if (e != cudaSuccess) return cuda_fail(e, "combine_wide_kernel");
+    return launch_check("combine_wide_kernel");
   }
   tqk::CombineArgs c{};
   c.part = part; c.Hq = Hq; c.Hkv = Hkv; c.nsplit = nsplit; c.d = hv->d; c.mv = hv->m; c.PiV = hv->dPi;
@@ -822,10 +892,76 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
   const size_t csmem = ((size_t)nsplit + 2 * (size_t)(hv->d + hv->m) + 8 * (size_t)hv->d + 4) * 4;
   if (once_per_device(3, hv->device))
     cudaFuncSetAttribute(tqk::attn_combine_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-  KernelScope ks("attn_combine", s);
-  tqk::attn_combine_kernel<<<B * Hq, tqk::kCombineThreads, csmem, s>>>(c);
-  return launch_check("attn_combine_kernel");
+  {
+    KernelScope ks("attn_combine", s);
+    tqk::attn_combine_kernel<<<B * Hq, tqk::kCombineThreads, csmem, s>>>(c);
+  }
+  if ((st = launch_check("attn_combine_kernel"))) return st;
+  if (fused) {
+    KernelScope ks("advance_len", s);
+    tqk::advance_len_kernel<<<(B + 255) / 256, 256, 0, s>>>(len, B, k->L_cap);
+    return launch_check("advance_len_kernel");
+  }
+  return TQ_OK;
 }
+
+}  // namespace
+
+extern "C" {
+
+int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
+                   const tq_cache* k, const tq_cache* v, const int32_t* len, float scale, float* out,
+                   void* workspace, size_t ws_bytes, void* stream) {
+  int st = attn_check(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, len, scale, out, workspace, ws_bytes);
+  if (st || B == 0) return st;
+  return attn_impl(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, const_cast<int32_t*>(len), scale, out, workspace,
+                   static_cast<cudaStream_t>(stream), false);
+}
+
+int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, const void* k_new,
+                   const void* v_new, int x_dtype, int B, int Hq, int Hkv, const tq_cache* k, const tq_cache* v,
+                   int32_t* len, float scale, float* out, void* workspace, size_t ws_bytes, void* stream) {
+  int st = attn_check(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, len, scale, out, workspace, ws_bytes);
+  if (st || B == 0) return st;
+  if (!valid_dtype(x_dtype)) return fail(TQ_EINVAL, "x dtype %d", x_dtype);
+  if (!k_new || !v_new) return fail(TQ_EINVAL, "k_new/v_new NULL");
+  if (!aligned(k_new, 16) || !aligned(v_new, 16)) return fail(TQ_EINVAL, "k_new/v_new misaligned");
+  if (hk->d > tqk::kSmallMaxD || hk->m > tqk::kSmallMaxD || hv->m > tqk::kSmallMaxD || hk->d > tqk::kWideMaxD)
+    return fail(TQ_EUNSUPPORTED, "tq_decode_step needs d <= %d and m <= %d", tqk::kSmallMaxD, tqk::kSmallMaxD);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  ScoreWs w;
+  float* part;
+  int nsplit;
+  int64_t chunk;
+  attn_ws_layout(hk, hv, B, Hq, Hkv, k->L_cap, static_cast<char*>(workspace), &w, &part, &nsplit, &chunk);
+  auto enc = [&](const tq_handle* h, const void* x, const tq_cache* c) {
+    tqk::EncodeArgs a{};
+    a.x = x; a.x_dtype = x_dtype; a.rows = (int64_t)B * Hkv; a.d = h->d; a.bits = h->bits; a.m = h->m;
+    a.norm_dtype = h->norm_dtype; a.PiT = h->dPiT; a.MT = h->dMT; a.cent = h->dcent; a.bnd = h->dbnd;
+    a.codes = c->codes; a.codes_B = h->codes_B; a.signs = c->signs; a.signs_B = h->signs_B;
+    a.norms = c->norms; a.rnorms = static_cast<__half*>(c->rnorms);
+    a.len = len; a.Hkv = Hkv; a.L_cap = c->L_cap; a.err = h->derr;
+    return a;
+  };
+  tqk::PrologueArgs p{};
+  p.k = enc(hk, k_new, k);
+  p.v = enc(hv, v_new, v);
+  p.nvec = B * Hkv;
+  p.q = q; p.q_dtype = q_dtype; p.rows = B * Hq; p.d = hk->d; p.m = hk->m; p.qcols = (hk->d + hk->m) / tqk::kWideCols;
+  p.PiT = hk->dPiT; p.ST = hk->dST; p.qr = w.qr; p.qs = w.qs;
+  const size_t smem = std::max({tqk::append_cluster_smem_bytes(hk->d, hk->m), tqk::append_cluster_smem_bytes(hv->d, hv->m),
+                                tqk::qprep_wide_smem_bytes(hk->d)});
+  if (once_per_device(9, hk->device))
+    cudaFuncSetAttribute(tqk::decode_prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  const unsigned grid = (unsigned)(2 * p.nvec + ((B * Hq + tqk::kQRows - 1) / tqk::kQRows) * p.qcols);
+  {
+    KernelScope ks("prologue", s);
+    tqk::decode_prologue_kernel<<<grid, tqk::kSmallThreads, smem, s>>>(p);
+  }
+  if ((st = launch_check("decode_prologue_kernel"))) return st;
+  return attn_impl(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, len, scale, out, workspace, s, true);
+}
+
 
 int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* codes, const void* norms, int64_t n,
                    int k, int64_t* idx, float* score, void* workspace, size_t ws_bytes, void* stream) {

@@ -203,6 +203,25 @@ int tq_attn_decode_noalloc(const tq_handle* hk, const tq_handle* hv, const void*
                            int B, int Hq, int Hkv, const tq_cache* k, const tq_cache* v,
                            const int32_t* len, float scale, float* out, void* stream);
 
+/* One whole decode step in three launches: append the new key and value of every
+ * (sequence, KV head) at slot len[b] (as tq_append on hk and hv), attend over the
+ * len[b] + 1 tokens (as tq_attn_decode), then advance len[b] by one. Same results
+ * as tq_append(hk, k_new, .., advance 0), tq_append(hv, v_new, .., advance 1) and
+ * tq_attn_decode called in that order; the query rotation runs in the same launch
+ * as the appends, and len[b] is advanced by the last launch, after every read of it.
+ * [Google TurboQuant "Stage 1", "Stage 2"; gemilab "Scaled dot-product attention";
+ * gist.science "Problem statement": O(1) append to a growing cache]
+ *  k_new, v_new  device [B][Hkv][d] of x_dtype (16-byte aligned)
+ *  len           device int32 [B]; a sequence already at L_cap is not appended
+ *                (TQ_ECAPACITY is recorded in hk's error word), attends over its
+ *                L_cap tokens and keeps len[b] == L_cap
+ *  other arguments as tq_attn_decode; needs d <= 128 and m <= 128 for both handles.
+ *  Calls sharing len or a cache must be stream-ordered. */
+int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype,
+                   const void* k_new, const void* v_new, int x_dtype, int B, int Hq, int Hkv,
+                   const tq_cache* k, const tq_cache* v, int32_t* len, float scale, float* out,
+                   void* workspace, size_t ws_bytes, void* stream);
+
 /* Top-k inner-product search over n packed database vectors [HAKU "Impact on
  * high-dimensional vector search"]: for each of nq queries (device fp32 [nq][d])
  * the k largest estimated scores norm * <Pi q, c[index]> (MSE handles),
