@@ -77,6 +77,18 @@ __device__ __forceinline__ uint32_t sign_bit(const uint32_t* row, int j) {
 __device__ __forceinline__ void grid_dep_wait() { asm volatile("griddepcontrol.wait;\n" ::: "memory"); }
 __device__ __forceinline__ void grid_dep_launch() { asm volatile("griddepcontrol.launch_dependents;\n" ::: "memory"); }
 
+// ---- asynchronous 16-byte copies (global -> shared): every thread issues all of its
+// copies, then waits once, so a staging loop costs one memory latency, not one per element.
+__device__ __forceinline__ void cp_async16(void* smem_dst, const void* gmem_src) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;\n" ::"r"(
+                   static_cast<uint32_t>(__cvta_generic_to_shared(smem_dst))),
+               "l"(gmem_src)
+               : "memory");
+}
+__device__ __forceinline__ void cp_async_wait_all() {
+  asm volatile("cp.async.commit_group;\ncp.async.wait_group 0;\n" ::: "memory");
+}
+
 // ---- TMA bulk copies (global -> shared) completed on an mbarrier
 
 __device__ __forceinline__ uint32_t smem_addr(const void* p) {

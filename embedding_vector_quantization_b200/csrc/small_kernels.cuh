@@ -161,9 +161,16 @@ __device__ __forceinline__ void qprep_tile(const void* q, int q_dtype, int rows,
   const int tid = threadIdx.x;
   for (int i = tid; i < d * (kWideCols / 4); i += blockDim.x) {
     const int k = i / (kWideCols / 4), c4 = i % (kWideCols / 4);
-    reinterpret_cast<float4*>(sub)[i] = *reinterpret_cast<const float4*>(src + (size_t)k * ld + 4 * c4);
+    cp_async16(reinterpret_cast<float4*>(sub) + i, src + (size_t)k * ld + 4 * c4);
   }
-  for (int i = tid; i < nr * d; i += blockDim.x) qsh[i] = load_any(q, q_dtype, (int64_t)row0 * d + i);
+  if (q_dtype == TQ_F32 && (d % 4) == 0 && (reinterpret_cast<uintptr_t>(q) & 15) == 0) {
+    const float* qf = static_cast<const float*>(q) + (size_t)row0 * d;
+    for (int i = tid; i < nr * d / 4; i += blockDim.x) cp_async16(reinterpret_cast<float4*>(qsh) + i, qf + 4 * i);
+  } else {
+#pragma unroll 4
+    for (int i = tid; i < nr * d; i += blockDim.x) qsh[i] = load_any(q, q_dtype, (int64_t)row0 * d + i);
+  }
+  cp_async_wait_all();
   __syncthreads();
   const int c = tid % kWideCols;
   for (int r = tid / kWideCols; r < nr; r += blockDim.x / kWideCols) {
@@ -255,13 +262,14 @@ __global__ void __launch_bounds__(kSmallThreads) combine_wide_kernel(CombineWide
   for (int i = tid; i < dm * (kWideCols / 4); i += blockDim.x) {
     const int k = i / (kWideCols / 4), c4 = i % (kWideCols / 4);
     const float* src = (k < d) ? a.PiV + (size_t)k * d : a.SV + (size_t)(k - d) * d;
-    reinterpret_cast<float4*>(cols)[i] = *reinterpret_cast<const float4*>(src + j0 + 4 * c4);
+    cp_async16(reinterpret_cast<float4*>(cols) + i, src + j0 + 4 * c4);
   }
   grid_dep_wait();   // the partials (and, in a decode step, len) come from the attention kernel
-  {  // all of the row's partials at once, independent 16-byte loads (stride is a multiple of 4)
-    const float4* src = reinterpret_cast<const float4*>(a.part + (size_t)row * ns * stride);
-    for (int i = tid; i < ns * stride / 4; i += blockDim.x) reinterpret_cast<float4*>(P)[i] = src[i];
+  {  // all of the row's partials (stride is a multiple of 4 floats)
+    const float* src = a.part + (size_t)row * ns * stride;
+    for (int i = tid; i < ns * stride / 4; i += blockDim.x) cp_async16(reinterpret_cast<float4*>(P) + i, src + 4 * i);
   }
+  cp_async_wait_all();
   __syncthreads();
   if (warp == 0) {
     float M = -INFINITY;
