@@ -41,6 +41,10 @@ WORKLOAD_NAME = ("GQA decode step, TurboQuant prod 3-bit (2-bit Lloyd-Max + 1-bi
                  "B=1, 8 KV heads / 32 query heads, context 32768, bf16 K/V with lognormal channel scales "
                  "and 2 outlier channels")
 FALLBACK_HBM_GBS = 6650.0
+# DRAM bytes (read + write) of one attn_prod2_kernel launch on this workload, from
+# `ncu --set full` (profiles/attn_prod2_decode_prod3_ctx32768.md); set to None whenever
+# that kernel changes until it is captured again.
+ATTN_TRAFFIC_BYTES = 27350272
 
 
 def parse_args():
@@ -50,6 +54,9 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["tq", "reference"], default="tq")
     p.add_argument("--no-cpu-baseline", action="store_true")
+    p.add_argument("--workload", choices=["decode", "score", "encode", "attn4", "search"], default="decode",
+                   help="decode: the headline decode step (default); the others measure the remaining hot-path "
+                        "rows on their own workloads, one JSON line each")
     return p.parse_args()
 
 
@@ -396,7 +403,7 @@ def run_tq(args):
         "encode": {"vectors": enc_vectors, "ms_per_pass": enc_ms / reps, "input": "bf16 K and V prefill"},
         "hbm_frac_nominal_8tbs": value / world / 8000.0,
         "roofline": {"bound": "hbm", "kernel": "attn_split", "achieved": achieved, "peak": peak,
-                     "unit": "GB/s", "frac": achieved / peak, "traffic": None,
+                     "unit": "GB/s", "frac": achieved / peak, "traffic": ATTN_TRAFFIC_BYTES,
                      "peak_source": f"{peak_src} hbm_gbs", "launch_ms": split_avg_ms,
                      "algorithmic_bytes_per_launch": bytes_step},
         "e2e": {"value": world * bytes_step * args.steps / (e2e_ms / 1e3) / 1e9, "unit": "GB/s",
@@ -418,8 +425,11 @@ def main():
     args = parse_args()
     if args.impl == "reference":
         run_reference(args)
-    else:
+    elif args.workload == "decode":
         run_tq(args)
+    else:
+        import bench_rows
+        bench_rows.run(args)
 
 
 if __name__ == "__main__":

@@ -1,0 +1,514 @@
+"""Measurement of the hot-path rows other than the headline decode step (`bench.py
+--workload score|encode|attn4|search`): one JSON line each, same keys as the headline
+line (metric, value, roofline of the row's dominant kernel, clocks, launches) plus the CPU
+oracle timed on a bounded sample of the same workload.
+
+Workloads (all synthetic, seeded; the big inputs are drawn on the GPU):
+  score   64 sequences x 8 KV heads, context 16384 growing by one token per step; prod
+          2+1 keys (m = 128), fp16 norms; a step appends one bf16 token per (sequence,
+          head) and scores 32 query heads (4 per KV head) over every key.
+  encode  the prefill of that cache: 8,388,608 bf16 vectors, prod 2+1, d = 128.
+  attn4   4 sequences x 8 KV heads x context 131072, K and V 4-bit MSE, fp16 norms, bf16
+          K/V with a per-(sequence, head) scale ~ U(0.5, 2); one tq_decode_step per step.
+  search  1,000,000 x 1536 L2-normalised fp32 database vectors, 2-bit MSE codes, 1024
+          queries, top-10.
+"""
+
+import json
+import time
+
+import bench
+
+ROWS = ("score", "encode", "attn4", "search")
+
+
+def _events(torch):
+    return torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+
+
+def _peak(kind):
+    peaks, src = bench.measured_peaks()
+    if kind == "hbm":
+        return float(peaks.get("hbm_gbs", bench.FALLBACK_HBM_GBS)), f"{src} hbm_gbs"
+    return float(peaks.get("bf16_tflops", 1590.0)), f"{src} bf16_tflops"
+
+
+def _line(args, metric, value, unit, ms_per_step, config, roofline, launches, clocks, extra=None, cpu=None):
+    line = {"metric": metric, "value": value, "unit": unit, "n_gpus": 1, "steps": args.steps,
+            "warmup": args.warmup, "ms_per_step": ms_per_step, "higher_is_better": True, "scaling": "weak",
+            "vs_baseline": None, "dtype": config.pop("dtype"), "data": "synthetic", "config": config,
+            "roofline": roofline, "gpu_launches": launches, "clocks": clocks}
+    if extra:
+        line.update(extra)
+    if cpu:
+        line["cpu_baseline"] = cpu
+    print(json.dumps(line), flush=True)
+
+
+def _encode_into(tq, h, cache, x_of, L, slice_len, torch):
+    """Encodes the cache prefill in slices of `slice_len` tokens (x_of(l0, n) -> [B, Hkv, n, d]);
+    returns the device milliseconds spent in the encode calls."""
+    ms = 0.0
+    for l0 in range(0, L, slice_len):
+        n = min(slice_len, L - l0)
+        x = x_of(l0, n)
+        a, b = _events(torch)
+        a.record()
+        out = h.encode(x)
+        b.record()
+        torch.cuda.synchronize()
+        ms += a.elapsed_time(b)
+        cache.codes[:, :, l0:l0 + n].copy_(out["codes"])
+        cache.norms[:, :, l0:l0 + n].copy_(out["norms"])
+        if h.m:
+            cache.signs[:, :, l0:l0 + n].copy_(out["signs"])
+            cache.rnorms[:, :, l0:l0 + n].copy_(out["rnorms"])
+        del x, out
+    return ms
+
+
+# ------------------------------------------------------------------ score (cfg 5)
+
+S5 = dict(B=64, Hkv=8, Hq=32, L0=16384, d=128, bits=3, m=128, seed_handle=0, seed_prefill=10, seed_step=11)
+
+
+def run_score(args):
+    import torch
+    import embedding_vector_quantization_b200 as tq
+    B, Hkv, Hq, L0, d = S5["B"], S5["Hkv"], S5["Hq"], S5["L0"], S5["d"]
+    T = min(args.steps, 256)
+    L_cap = L0 + 256
+    h = tq.Handle(d, S5["bits"], S5["seed_handle"], qjl_m=S5["m"])
+    cache = tq.Cache(h, B, Hkv, L_cap)
+    g = torch.Generator(device="cuda").manual_seed(S5["seed_prefill"])
+    enc_ms = _encode_into(tq, h, cache,
+                          lambda l0, n: torch.randn(B, Hkv, n, d, generator=g, device="cuda").to(torch.bfloat16),
+                          L0, 2048, torch)
+    gs = torch.Generator(device="cuda").manual_seed(S5["seed_step"])
+    W = args.warmup
+    toks = torch.randn(T + W, B, Hkv, d, generator=gs, device="cuda").to(torch.bfloat16)
+    qs = torch.randn(T + W, B, Hq, d, generator=gs, device="cuda")
+    lens = torch.full((B,), L0, dtype=torch.int32, device="cuda")
+    logits = torch.empty(B, Hq, L_cap, dtype=torch.float32, device="cuda")
+    ws = torch.empty(tq.tq_score_workspace_bytes(h.ptr, B, Hq), dtype=torch.uint8, device="cuda")
+    k_in, q_in = toks[0].clone(), qs[0].clone()
+
+    def step():
+        tq.tq_append(h.ptr, k_in, B, Hkv, cache.struct, lens, 1)
+        tq.tq_score(h.ptr, q_in, B, Hq, Hkv, cache.struct, lens, logits, ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    tq.tq_timer_read(None, forget=True)
+    tq.tq_timer_enable(True)
+    graph_k = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_k):
+        step()
+    tq.tq_timer_enable(False)
+    return _score_timed(args, torch, tq, h, graph, graph_k, step, toks, qs, k_in, q_in, lens, T, W, L0, enc_ms)
+
+
+def _score_timed(args, torch, tq, h, graph, graph_k, step, toks, qs, k_in, q_in, lens, T, W, L0, enc_ms):
+    B, Hkv, Hq = S5["B"], S5["Hkv"], S5["Hq"]
+    G = Hq // Hkv
+
+    def run(gr, t0, timed):
+        evs = []
+        for t in range(t0, t0 + T):
+            k_in.copy_(toks[W + t - t0])
+            q_in.copy_(qs[W + t - t0])
+            ev = _events(torch)
+            ev[0].record()
+            gr.replay()
+            ev[1].record()
+            evs.append(ev)
+            if not timed:
+                torch.cuda.synchronize()
+                yield t
+        torch.cuda.synchronize()
+        if timed:
+            yield sum(a.elapsed_time(b) for a, b in evs)
+
+    lens.fill_(L0 - W)
+    for t in range(W):
+        k_in.copy_(toks[t])
+        q_in.copy_(qs[t])
+        graph.replay()
+    torch.cuda.synchronize()
+    sampler = bench.ClockSampler("GPU-" + str(torch.cuda.get_device_properties(0).uuid))
+    sampler.start()
+    total_ms = next(run(graph, 0, True))
+    clocks = sampler.stop()
+    # score-kernel time per launch from the instrumented capture (same steps again)
+    lens.fill_(L0)
+    score_ms, score_n = 0.0, 0
+    for _ in run(graph_k, 0, False):
+        ms_k, n_k = tq.tq_timer_read("score", forget=False)
+        score_ms += ms_k
+        score_n += n_k
+    _, kernels_per_step = tq.tq_timer_read(None, forget=False)
+    keys = sum(B * Hkv * (L0 + t + 1) for t in range(T))          # KV-head keys scored
+    packed = keys * 52                                              # codes 32 + signs 16 + norm 2 + rnorm 2
+    written = keys * G * 4                                          # fp32 logits of 4 query heads
+    peak, src = _peak("hbm")
+    ach = (packed + written) / (score_ms / 1e3) / 1e9
+    cfg = {"workload": "score step, TurboQuant prod 3-bit (2-bit Lloyd-Max + 1-bit QJL m=128), d=128, "
+                       "64 sequences x 8 KV heads, 32 query heads, context 16384 growing by 1 per step",
+           "B": B, "Hkv": Hkv, "Hq": Hq, "context_start": L0, "d": 128, "dtype": "int8 mma / f32",
+           "l2": "not flushed: each step reads 440 MB of packed keys and writes 135 MB of logits (> 126 MB L2)",
+           "step": "tq_append (one bf16 token per sequence and head, len += 1) + tq_score, one CUDA graph replay"}
+    roof = {"bound": "hbm", "kernel": "score_prod2_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
+            "frac": ach / peak, "traffic": None, "peak_source": src, "launch_ms": score_ms / max(score_n, 1),
+            "algorithmic_bytes_per_launch": (packed + written) / T}
+    extra = {"keys_scored_per_s": keys / (total_ms / 1e3), "query_key_pairs_per_s": keys * G / (total_ms / 1e3),
+             "packed_gb_per_s": packed / (total_ms / 1e3) / 1e9,
+             "prefill_encode": {"vectors": B * Hkv * L0, "ms": enc_ms,
+                                "vectors_per_s": B * Hkv * L0 / (enc_ms / 1e3)}}
+    cpu = None if args.no_cpu_baseline else oracle_score_sample()
+    _line(args, "keys scored/sec (cfg 5 score step)", extra["keys_scored_per_s"], "keys/s", total_ms / T, cfg, roof,
+          kernels_per_step * T, clocks, extra, cpu)
+
+
+def oracle_score_sample(budget_s=12.0):
+    """The oracle scoring 4 query heads over 16384 prod-encoded keys of one (sequence, KV
+    head), repeated for about budget_s seconds (setup untimed); keys/s."""
+    import numpy as np
+    import torch
+    from oracle import codebook, ops, quant, rotation
+    d, m, L = 128, 128, S5["L0"]
+    Pi, S = rotation.rotation(d, S5["seed_handle"], m)
+    c, beta = codebook.lloyd_max(d, 2)
+    x = torch.randn(L, d, generator=torch.Generator().manual_seed(S5["seed_prefill"])).to(torch.bfloat16).double().numpy()
+    e = quant.encode_prod(x, Pi, S, c, beta, "f16")
+    q = torch.randn(4, d, generator=torch.Generator().manual_seed(S5["seed_step"])).double().numpy()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        for hq in range(4):
+            ops.score_prod(q[hq], e["idx"], e["n_stored"], e["sigma"], e["rnorm_stored"], Pi, S, c)
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": reps * L / el, "unit": "keys/s", "cores": bench.blas_threads(), "kind": "oracle",
+            "sample": f"{reps} x (4 query heads over 16384 keys of one sequence and KV head) in {el:.1f} s, "
+                      f"fp64 NumPy oracle"}
+
+
+# ------------------------------------------------------------------ encode (cfg 5 prefill)
+
+def run_encode(args):
+    """Prefill encode of the score workload's cache: 8,388,608 bf16 vectors, prod 2+1, in
+    launches of 1,048,576 vectors (each pass re-encodes the whole prefill)."""
+    import torch
+    import embedding_vector_quantization_b200 as tq
+    B, Hkv, L0, d, m = S5["B"], S5["Hkv"], S5["L0"], S5["d"], S5["m"]
+    h = tq.Handle(d, S5["bits"], S5["seed_handle"], qjl_m=m)
+    n_all = B * Hkv * L0
+    per = 1 << 20
+    g = torch.Generator(device="cuda").manual_seed(S5["seed_prefill"])
+    x = torch.randn(n_all, d, generator=g, device="cuda").to(torch.bfloat16)      # 2.15 GB
+    out = h.alloc_rows((per,), x.device)
+    passes = max(1, args.steps)
+
+    def one_pass():
+        for r0 in range(0, n_all, per):
+            h.encode(x[r0:r0 + per], out=out)
+
+    for _ in range(max(1, args.warmup)):
+        one_pass()
+    torch.cuda.synchronize()
+    tq.tq_timer_read(None, forget=True)
+    sampler = bench.ClockSampler("GPU-" + str(torch.cuda.get_device_properties(0).uuid))
+    sampler.start()
+    a, b = _events(torch)
+    a.record()
+    for _ in range(passes):
+        one_pass()
+    b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = a.elapsed_time(b) / passes
+    # per-launch kernel time, timed separately with the library's event pairs
+    tq.tq_timer_enable(True)
+    one_pass()
+    torch.cuda.synchronize()
+    tq.tq_timer_enable(False)
+    k_ms, k_n = tq.tq_timer_read("encode", forget=True)
+    launches_per_pass = (n_all + per - 1) // per
+    flops = 2 * d * d + 2 * m * d                     # algorithmic: rotation + QJL projection, per vector
+    peak, src = _peak("tensor")
+    ach = per * flops / (k_ms / max(k_n, 1) / 1e3) / 1e12
+    cfg = {"workload": "prefill encode, TurboQuant prod 3-bit (2-bit Lloyd-Max + 1-bit QJL m=128), d=128, "
+                       "bf16 input, 8,388,608 vectors (64 sequences x 8 KV heads x 16384)",
+           "vectors": n_all, "launch_vectors": per, "d": d, "dtype": "bf16 hi/lo tcgen05, f32 accumulate",
+           "l2": "not flushed: each pass reads 2.15 GB of input (> 126 MB L2)"}
+    roof = {"bound": "tensor", "kernel": "encode_tc_kernel", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+            "frac": ach / peak, "traffic": None, "peak_source": src, "launch_ms": k_ms / max(k_n, 1),
+            "algorithmic_flops_per_launch": per * flops,
+            "note": "algorithmic flops (2d^2 + 2md per vector); the hi/lo split runs 5 MMA passes of that size"}
+    hbm_bytes = n_all * (2 * d + 32 + 16 + 2 + 2)
+    extra = {"vectors_encoded_per_s": n_all / (ms / 1e3), "hbm_gb_per_s": hbm_bytes / (ms / 1e3) / 1e9}
+    cpu = None if args.no_cpu_baseline else oracle_encode_sample()
+    _line(args, "vectors encoded/sec (cfg 5 prefill encode)", extra["vectors_encoded_per_s"], "vectors/s", ms, cfg,
+          roof, launches_per_pass * passes, clocks, extra, cpu)
+
+
+def oracle_encode_sample(budget_s=12.0, rows=16384):
+    """The oracle's prod encode of `rows` bf16 vectors, repeated for about budget_s seconds."""
+    import torch
+    from oracle import codebook, quant, rotation
+    Pi, S = rotation.rotation(128, S5["seed_handle"], 128)
+    c, beta = codebook.lloyd_max(128, 2)
+    x = torch.randn(rows, 128, generator=torch.Generator().manual_seed(S5["seed_prefill"])).to(torch.bfloat16)
+    x = x.double().numpy()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        quant.encode_prod(x, Pi, S, c, beta, "f16")
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": reps * rows / el, "unit": "vectors/s", "cores": bench.blas_threads(), "kind": "oracle",
+            "sample": f"{reps} x {rows} bf16 vectors, prod 2+1, d=128, in {el:.1f} s, fp64 NumPy oracle"}
+
+
+# ------------------------------------------------------------------ attention, 4-bit MSE (cfg 3)
+
+S3 = dict(B=4, Hkv=8, Hq=32, L=131072, d=128, bits=4, seed_k=5, seed_v=6, seed_q=7)
+
+
+def run_attn4(args):
+    import torch
+    import embedding_vector_quantization_b200 as tq
+    B, Hkv, Hq, L, d = S3["B"], S3["Hkv"], S3["Hq"], S3["L"], S3["d"]
+    hk = tq.Handle(d, S3["bits"], 0, norm_dtype=tq.TQ_F16)
+    hv = tq.Handle(d, S3["bits"], 1, norm_dtype=tq.TQ_F16)
+    kc, vc = tq.Cache(hk, B, Hkv, L), tq.Cache(hv, B, Hkv, L)
+    enc_ms = 0.0
+    for h, cache, seed in ((hk, kc, S3["seed_k"]), (hv, vc, S3["seed_v"])):
+        g = torch.Generator(device="cuda").manual_seed(seed)
+        scl = (0.5 + 1.5 * torch.rand(B, Hkv, 1, 1, generator=g, device="cuda"))      # U(0.5, 2) per (b, head)
+        enc_ms += _encode_into(tq, h, cache, lambda l0, n: (torch.randn(B, Hkv, n, d, generator=g, device="cuda")
+                                                           * scl).to(torch.bfloat16), L, 8192, torch)
+    gq = torch.Generator(device="cuda").manual_seed(S3["seed_q"])
+    W, T = args.warmup, args.steps
+    qs = torch.randn(T + W, B, Hq, d, generator=gq, device="cuda")
+    kn = torch.randn(T + W, B, Hkv, d, generator=gq, device="cuda").to(torch.bfloat16)
+    vn = torch.randn(T + W, B, Hkv, d, generator=gq, device="cuda").to(torch.bfloat16)
+    L0 = L - 1
+    lens = torch.full((B,), L0, dtype=torch.int32, device="cuda")
+    out = torch.empty(B, Hq, d, dtype=torch.float32, device="cuda")
+    ws = torch.empty(tq.tq_attn_workspace_bytes(hk.ptr, hv.ptr, B, Hq, Hkv, L), dtype=torch.uint8, device="cuda")
+    q_in, k_in, v_in = qs[0].clone(), kn[0].clone(), vn[0].clone()
+
+    def step():
+        tq.tq_decode_step(hk.ptr, hv.ptr, q_in, k_in, v_in, B, Hq, Hkv, kc.struct, vc.struct, lens, 1 / d ** 0.5,
+                          out, ws)
+
+    s = torch.cuda.Stream()
+    s.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s):
+        step()
+    torch.cuda.current_stream().wait_stream(s)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    tq.tq_timer_read(None, forget=True)
+    tq.tq_timer_enable(True)
+    graph_k = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_k):
+        step()
+    tq.tq_timer_enable(False)
+
+    def set_inputs(t):
+        q_in.copy_(qs[t])
+        k_in.copy_(kn[t])
+        v_in.copy_(vn[t])
+        lens.fill_(L0)
+
+    for t in range(W):
+        set_inputs(t)
+        graph.replay()
+    torch.cuda.synchronize()
+    sampler = bench.ClockSampler("GPU-" + str(torch.cuda.get_device_properties(0).uuid))
+    sampler.start()
+    evs = []
+    for t in range(T):
+        set_inputs(W + t)
+        ev = _events(torch)
+        ev[0].record()
+        graph.replay()
+        ev[1].record()
+        evs.append(ev)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    total_ms = sum(a.elapsed_time(b) for a, b in evs)
+    split_ms, split_n = 0.0, 0
+    for t in range(T):
+        set_inputs(W + t)
+        graph_k.replay()
+        torch.cuda.synchronize()
+        ms_k, n_k = tq.tq_timer_read("attn_split", forget=False)
+        split_ms += ms_k
+        split_n += n_k
+    _, kernels_per_step = tq.tq_timer_read(None, forget=False)
+    bytes_step = B * Hkv * L * 2 * (64 + 2)        # K and V: 4-bit codes (64 B) + fp16 norm per token
+    peak, src = _peak("hbm")
+    ach = bytes_step / (split_ms / max(split_n, 1) / 1e3) / 1e9
+    cfg = {"workload": "GQA decode step, TurboQuant MSE 4-bit K and V, d=128, B=4, 8 KV heads / 32 query heads, "
+                       "context 131072, bf16 K/V N(0,1) x U(0.5,2) per (sequence, head)",
+           "B": B, "Hkv": Hkv, "Hq": Hq, "context": L, "d": d, "dtype": "f32",
+           "l2": "not flushed: each step reads 553.6 MB of packed K/V (> 126 MB L2)",
+           "step": "tq_decode_step, one CUDA graph replay; len reset outside the timed bracket"}
+    roof = {"bound": "hbm", "kernel": "attn_mse4_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
+            "frac": ach / peak, "traffic": None, "peak_source": src, "launch_ms": split_ms / max(split_n, 1),
+            "algorithmic_bytes_per_launch": bytes_step}
+    value = bytes_step * T / (total_ms / 1e3) / 1e9
+    extra = {"tokens_per_s": B * Hkv * L * T / (total_ms / 1e3),
+             "prefill_encode": {"vectors": 2 * B * Hkv * L, "ms": enc_ms,
+                                "vectors_per_s": 2 * B * Hkv * L / (enc_ms / 1e3)}}
+    cpu = None if args.no_cpu_baseline else oracle_attn4_sample()
+    _line(args, "packed-KV GB/s (cfg 3 decode step, 4-bit MSE)", value, "GB/s", total_ms / T, cfg, roof,
+          kernels_per_step * T, clocks, extra, cpu)
+
+
+def oracle_attn4_sample(budget_s=12.0, L=32768):
+    """The oracle's decode attention of 4 query heads over L tokens of one (sequence, KV head)
+    of 4-bit MSE K/V (encoded once, untimed); packed GB/s."""
+    import numpy as np
+    import torch
+    from oracle import codebook, ops, quant, rotation
+    d = 128
+    c, beta = codebook.lloyd_max(d, 4)
+    caches = []
+    for seed, hseed in ((S3["seed_k"], 0), (S3["seed_v"], 1)):
+        Pi = rotation.rotation(d, hseed, 0)[0]
+        x = torch.randn(L, d, generator=torch.Generator().manual_seed(seed)).to(torch.bfloat16).double().numpy()
+        e = quant.encode_mse(x, Pi, c, beta, "f16")
+        caches.append({"idx": e["idx"].reshape(1, 1, L, d), "n": e["n_stored"].reshape(1, 1, L), "Pi": Pi, "c": c})
+    q = torch.randn(1, 4, d, generator=torch.Generator().manual_seed(S3["seed_q"])).double().numpy()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        ops.decode_attention(q, caches[0], caches[1], [L], 1 / np.sqrt(d))
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    return {"value": reps * L * 2 * 66 / el / 1e9, "unit": "GB/s", "cores": bench.blas_threads(), "kind": "oracle",
+            "sample": f"{reps} x (4 query heads over {L} tokens of one sequence and KV head) in {el:.1f} s, "
+                      f"fp64 NumPy oracle"}
+
+
+# ------------------------------------------------------------------ search (cfg 4)
+
+S4 = dict(n=1_000_000, nq=1024, d=1536, bits=2, k=10, seed_handle=0, seed_db=8, seed_q=9)
+FP32_LANES_PER_SM = 128   # fp32 FMA lanes per B200 SM (4 partitions x 32)
+
+
+def run_search(args):
+    import torch
+    import embedding_vector_quantization_b200 as tq
+    n, nq, d, k = S4["n"], S4["nq"], S4["d"], S4["k"]
+    h = tq.Handle(d, S4["bits"], S4["seed_handle"])
+    g = torch.Generator(device="cuda").manual_seed(S4["seed_db"])
+    db = torch.randn(n, d, generator=g, device="cuda")
+    db /= db.norm(dim=1, keepdim=True)
+    gq = torch.Generator(device="cuda").manual_seed(S4["seed_q"])
+    q = torch.randn(nq, d, generator=gq, device="cuda")
+    q /= q.norm(dim=1, keepdim=True)
+    a, b = _events(torch)
+    a.record()
+    enc = h.encode(db)
+    b.record()
+    torch.cuda.synchronize()
+    enc_ms = a.elapsed_time(b)
+    ws = torch.empty(tq.tq_search_workspace_bytes(h.ptr, nq, n, k), dtype=torch.uint8, device="cuda")
+    T = max(1, min(args.steps, 5))
+    for _ in range(max(1, min(args.warmup, 3))):
+        idx, sc = h.search_topk(q, enc["codes"], enc["norms"], k, workspace=ws)
+    torch.cuda.synchronize()
+    sampler = bench.ClockSampler("GPU-" + str(torch.cuda.get_device_properties(0).uuid))
+    sampler.start()
+    a.record()
+    for _ in range(T):
+        idx, sc = h.search_topk(q, enc["codes"], enc["norms"], k, workspace=ws)
+    b.record()
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    ms = a.elapsed_time(b) / T
+    tq.tq_timer_read(None, forget=True)
+    tq.tq_timer_enable(True)
+    h.search_topk(q, enc["codes"], enc["norms"], k, workspace=ws)
+    torch.cuda.synchronize()
+    tq.tq_timer_enable(False)
+    s_ms, s_n = tq.tq_timer_read("search", forget=False)
+    _, launches = tq.tq_timer_read(None, forget=True)
+    # recall@10 against exact fp32 inner products (no TF32), in database chunks
+    prev = torch.backends.cuda.matmul.allow_tf32
+    torch.backends.cuda.matmul.allow_tf32 = False
+    best_s = torch.full((nq, k), -float("inf"), device="cuda")
+    best_i = torch.zeros((nq, k), dtype=torch.int64, device="cuda")
+    for r0 in range(0, n, 131072):
+        s_ = q @ db[r0:r0 + 131072].T
+        ts, ti = s_.topk(k, dim=1)
+        cs, ci = torch.cat([best_s, ts], 1), torch.cat([best_i, ti + r0], 1)
+        best_s, sel = cs.topk(k, dim=1)
+        best_i = ci.gather(1, sel)
+    torch.backends.cuda.matmul.allow_tf32 = prev
+    hits = sum(len(set(x.tolist()) & set(y.tolist())) for x, y in zip(idx.cpu(), best_i.cpu()))
+    recall = hits / (nq * k)
+    flops = 2.0 * d * nq * n
+    sm_mhz = clocks.get("sm_mhz") or 1965.0
+    peak = torch.cuda.get_device_properties(0).multi_processor_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+    ach = flops / (s_ms / max(s_n, 1) / 1e3) / 1e12
+    cfg = {"workload": "top-10 inner-product search, TurboQuant MSE 2-bit, d=1536, 1,000,000 L2-normalised "
+                       "N(0,I) database vectors, 1024 queries (stands in for the pages' vector-search benchmarks)",
+           "n": n, "nq": nq, "d": d, "k": k, "dtype": "f32 SIMT",
+           "l2": "not flushed: the 384 MB of codes exceed the 126 MB L2"}
+    roof = {"bound": "alu", "kernel": "search_simt_kernel", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+            "frac": ach / peak, "traffic": None,
+            "peak_source": "derived: SMs x 128 fp32 lanes x 2 flop x median sampled SM clock",
+            "launch_ms": s_ms / max(s_n, 1), "algorithmic_flops_per_launch": flops}
+    extra = {"queries_per_s": nq / (ms / 1e3), "recall_at_10": recall,
+             "db_encode": {"vectors": n, "ms": enc_ms, "vectors_per_s": n / (enc_ms / 1e3), "input": "fp32"}}
+    cpu = None if args.no_cpu_baseline else oracle_search_sample()
+    _line(args, "queries/sec (cfg 4 top-10 search, 1M x 1536, 2-bit)", extra["queries_per_s"], "queries/s", ms, cfg,
+          roof, launches * T, clocks, extra, cpu)
+
+
+def oracle_search_sample(budget_s=12.0, n=32768, nq=64):
+    """The oracle's top-10 search of nq queries over n 2-bit vectors (d = 1536; encode untimed)."""
+    import torch
+    from oracle import codebook, ops, quant, rotation
+    d = S4["d"]
+    Pi = rotation.rotation(d, S4["seed_handle"], 0)[0]
+    c, beta = codebook.lloyd_max(d, S4["bits"])
+    x = torch.randn(n, d, generator=torch.Generator().manual_seed(S4["seed_db"])).double()
+    x = (x / x.norm(dim=1, keepdim=True)).numpy()
+    e = quant.encode_mse(x, Pi, c, beta, "f32")
+    q = torch.randn(nq, d, generator=torch.Generator().manual_seed(S4["seed_q"])).double()
+    q = (q / q.norm(dim=1, keepdim=True)).numpy()
+    reps, t0 = 0, time.perf_counter()
+    while True:
+        s = ops.search_scores(q, e["idx"], e["n_stored"], Pi, c)
+        ops.topk(s, S4["k"])
+        reps += 1
+        el = time.perf_counter() - t0
+        if el >= budget_s:
+            break
+    scale = S4["n"] / n
+    return {"value": reps * nq / el / scale, "unit": "queries/s", "cores": bench.blas_threads(), "kind": "oracle",
+            "sample": f"{reps} x ({nq} queries over {n} vectors) in {el:.1f} s, scaled to 1,000,000 vectors; "
+                      f"fp64 NumPy oracle"}
+
+
+def run(args):
+    {"score": run_score, "encode": run_encode, "attn4": run_attn4, "search": run_search}[args.workload](args)

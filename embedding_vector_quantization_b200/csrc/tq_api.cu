@@ -33,6 +33,7 @@
 #include "attn_mma.cuh"
 #include "small_kernels.cuh"
 #include "encode_tc.cuh"
+#include "attn_mse4.cuh"
 
 struct tq_handle {
   int d = 0, bits = 0, m = 0, norm_dtype = TQ_F32;
@@ -361,6 +362,45 @@ bool score_prod2_fast_path(const tq_handle* hk, int G, const tq_cache* k) {
                    std::fabs(hk->cent[3] - hk->cent[2] - hk->cent[1] + hk->cent[0]) < 1e-12;
   return G == 4 && fmt && k->L_cap % 8 == 0 && aligned(k->codes, 16) && aligned(k->signs, 16) &&
          aligned(k->norms, 16) && aligned(k->rnorms, 16);
+}
+
+// Walsh-plane form of a symmetric 16-level codebook (the int8 tensor-core 4-bit
+// attention): c[idx] = c[0] + sum_S w[S] beta_S(idx) over the planes {0}, {1}, {2}, {3},
+// {0,1,2}, {0,1,3}, {0,2,3}, {1,2,3} (beta = bit, or parity of three bits). In the +-1
+// variables s_i = 2 b_i - 1 the coefficients are a_T = mean_idx c[idx] prod_{i in T} s_i;
+// w[S] = 2 a_S. False if an even-degree coefficient does not vanish (no symmetry).
+bool plane_coeffs4(const std::vector<double>& c, float* c0, float* w) {
+  if (c.size() != 16) return false;
+  static const int kMasks[8] = {1, 2, 4, 8, 7, 11, 13, 14};
+  double cmax = 0.0;
+  for (double v : c) cmax = std::max(cmax, std::fabs(v));
+  double a[16];
+  for (int T = 0; T < 16; ++T) {
+    double acc = 0.0;
+    for (int idx = 0; idx < 16; ++idx) {
+      double prod = 1.0;
+      for (int i = 0; i < 4; ++i)
+        if (T >> i & 1) prod *= ((idx >> i) & 1) ? 1.0 : -1.0;
+      acc += c[idx] * prod;
+    }
+    a[T] = acc / 16.0;
+    if (__builtin_popcount(T) % 2 == 0 && std::fabs(a[T]) > 1e-12 * cmax) return false;
+  }
+  for (int p = 0; p < 8; ++p) w[p] = (float)(2.0 * a[kMasks[p]]);
+  *c0 = (float)c[0];
+  return true;
+}
+
+// The int8 tensor-core kernel for 4-bit MSE K and V caches (fp16 norms) at d = 128 with
+// 4 query heads per KV head.
+bool attn_mse4_fast_path(const tq_handle* hk, const tq_handle* hv, int G, const tq_cache* k, const tq_cache* v) {
+  if (std::getenv("TQ_SIMT")) return false;
+  float c0, w[8];
+  auto ok_handle = [&](const tq_handle* h) {
+    return h->d == 128 && h->m == 0 && h->bits == 4 && h->norm_dtype == TQ_F16 && plane_coeffs4(h->cent, &c0, w);
+  };
+  auto ok_cache = [](const tq_cache* c) { return aligned(c->codes, 16) && aligned(c->norms, 16); };
+  return G == 4 && ok_handle(hk) && ok_handle(hv) && k->L_cap % 8 == 0 && ok_cache(k) && ok_cache(v);
 }
 
 struct ScoreWs { float* qr; float* qs; };
@@ -861,6 +901,27 @@ int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dty
       if (e != cudaSuccess) return cuda_fail(e, "attn_prod2_kernel");
     }
     if ((st = launch_check("attn_prod2_kernel"))) return st;
+  } else if (attn_mse4_fast_path(hk, hv, G, k, v)) {
+    tqk::am4::Args m4{};
+    m4.qr = w.qr; m4.B = B; m4.Hq = Hq; m4.Hkv = Hkv;
+    m4.kcodes = k->codes; m4.knorm = static_cast<const __half*>(k->norms);
+    m4.vcodes = v->codes; m4.vnorm = static_cast<const __half*>(v->norms);
+    m4.L_cap = k->L_cap; m4.chunk = chunk; m4.nsplit = nsplit; m4.len = len; m4.len_extra = fused ? 1 : 0;
+    plane_coeffs4(hk->cent, &m4.kc0, m4.kw);
+    plane_coeffs4(hv->cent, &m4.vc0, m4.vw);
+    m4.scale = scale; m4.part = part; m4.err = hk->derr;
+    const size_t msmem = sizeof(tqk::am4::Smem);
+    if (once_per_device(11, hk->device)) {
+      cudaFuncSetAttribute(tqk::am4::attn_mse4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+      cudaFuncSetAttribute(tqk::am4::attn_mse4_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    }
+    {
+      KernelScope ks("attn_split", s);
+      const cudaError_t e = launch_pdl(tqk::am4::attn_mse4_kernel, dim3((unsigned)(B * Hkv), (unsigned)nsplit),
+                                       dim3(tqk::am4::kThreads), msmem, s, m4);
+      if (e != cudaSuccess) return cuda_fail(e, "attn_mse4_kernel");
+    }
+    if ((st = launch_check("attn_mse4_kernel"))) return st;
   } else {
     const size_t smem = ((size_t)G * (hk->d + hk->m) + 32 + (size_t)G * tqk::kAttnThreads +
                          2 * tqk::kAttnThreads + 4 * (size_t)G) * 4;

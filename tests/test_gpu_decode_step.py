@@ -21,10 +21,10 @@ def tq():
     return m
 
 
-def _setup(tq, bits, m, B, Hkv, G, L_cap, L0, seed):
+def _setup(tq, bits, m, B, Hkv, G, L_cap, L0, seed, norm_dtype=None):
     d = 128
-    hk = tq.Handle(d, bits, seed, qjl_m=m)
-    hv = tq.Handle(d, bits, seed + 1, qjl_m=m)
+    hk = tq.Handle(d, bits, seed, qjl_m=m, norm_dtype=norm_dtype)
+    hv = tq.Handle(d, bits, seed + 1, qjl_m=m, norm_dtype=norm_dtype)
     g = torch.Generator().manual_seed(seed)
     K = (torch.randn(B, Hkv, L_cap, d, generator=g) * 1.5).to(torch.bfloat16).cuda()
     V = torch.randn(B, Hkv, L_cap, d, generator=g).to(torch.bfloat16).cuda()
@@ -49,14 +49,16 @@ def _step(tq, hk, hv, q, k_new, v_new, kc, vc, lens, scale):
     return out
 
 
-@pytest.mark.parametrize("bits,m,B,Hkv,G,L_cap,L0", [
-    (3, 128, 2, 8, 4, 4096, [4000, 0]),      # int8 tensor-core attention, an empty sequence
-    (3, 128, 3, 4, 4, 2048, [2047, 1500, 2048]),  # last slot, middle, a full sequence
-    (3, 0, 2, 2, 4, 1024, [700, 1023]),      # MSE-only K/V: the SIMT attention kernel
-    (4, 0, 1, 2, 2, 512, [3]),
+@pytest.mark.parametrize("bits,m,B,Hkv,G,L_cap,L0,f16", [
+    (3, 128, 2, 8, 4, 4096, [4000, 0], False),      # int8 tensor-core attention, an empty sequence
+    (3, 128, 3, 4, 4, 2048, [2047, 1500, 2048], False),  # last slot, middle, a full sequence
+    (3, 0, 2, 2, 4, 1024, [700, 1023], False),      # MSE-only K/V: the SIMT attention kernel
+    (4, 0, 1, 2, 2, 512, [3], False),
+    (4, 0, 2, 2, 4, 3072, [3000, 1024], True),       # 4-bit MSE, fp16 norms: the Walsh-plane kernel
 ])
-def test_decode_step_equals_separate_calls(tq, bits, m, B, Hkv, G, L_cap, L0):
-    hk, hv, caches, q, k_new, v_new = _setup(tq, bits, m, B, Hkv, G, L_cap, L0, seed=bits * 10 + B)
+def test_decode_step_equals_separate_calls(tq, bits, m, B, Hkv, G, L_cap, L0, f16):
+    hk, hv, caches, q, k_new, v_new = _setup(tq, bits, m, B, Hkv, G, L_cap, L0, seed=bits * 10 + B,
+                                             norm_dtype=tq.TQ_F16 if f16 else None)
     scale = 1.0 / np.sqrt(128)
     (kc1, vc1), (kc2, vc2) = caches
     lens1 = torch.tensor(L0, dtype=torch.int32).cuda()

@@ -274,3 +274,37 @@ def test_score_tensor_core_path_matches_simt_and_oracle(tq, B, Hkv, L, lens):
             assert np.all(np.abs(fast[b, hq, :Lb] - ref) <= tol), (b, hq)
             assert np.all(np.abs(simt[b, hq, :Lb] - ref) <= tol), (b, hq)
     assert h.status() == tq.TQ_OK
+
+
+@pytest.mark.parametrize("B,Hkv,L,lens", [(2, 2, 5000, [5000, 2001]), (2, 1, 600, [1, 0])])
+def test_attention_mse4_tensor_core_path_matches_simt_and_oracle(tq, B, Hkv, L, lens):
+    """4-bit MSE K/V with fp16 norms at d=128, 4 query heads per KV head: the int8 tensor-core
+    kernel (codebook in Walsh-plane form), the SIMT kernel (TQ_SIMT=1) and the oracle agree."""
+    import os
+    G, d = 4, 128
+    hk = tq.Handle(d, 4, 40, norm_dtype=tq.TQ_F16)
+    hv = tq.Handle(d, 4, 41, norm_dtype=tq.TQ_F16)
+    ohk, ohv = OracleHandle(d, 4, 40, 0), OracleHandle(d, 4, 41, 0)
+    rs = np.random.default_rng(L + 7 * B)
+    scl = rs.uniform(0.5, 2.0, size=(B, Hkv, 1, 1))
+    kc, kod = oracle_cache(tq, hk, ohk, rs.standard_normal((B, Hkv, L, d)) * scl)
+    vc, vod = oracle_cache(tq, hv, ohv, rs.standard_normal((B, Hkv, L, d)) * scl[:, ::-1])
+    q = torch.from_numpy(rs.standard_normal((B, Hkv * G, d)) * 2).float()
+    lens_t = torch.tensor(lens, dtype=torch.int32).cuda()
+    scale = 1 / np.sqrt(d)
+    o_fast = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens_t, scale).cpu().numpy()
+    os.environ["TQ_SIMT"] = "1"
+    try:
+        o_simt = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens_t, scale).cpu().numpy()
+    finally:
+        del os.environ["TQ_SIMT"]
+    ref = ops.decode_attention(q.double().numpy(), kod, vod, [max(1, x) for x in lens], scale)
+    for b in range(B):
+        for h in range(Hkv * G):
+            if lens[b] == 0:
+                assert np.all(o_fast[b, h] == 0) and np.all(o_simt[b, h] == 0)
+                continue
+            nr = np.linalg.norm(ref[b, h])
+            assert np.linalg.norm(o_fast[b, h] - ref[b, h]) <= ATTN_RTOL * nr, (b, h)
+            assert np.linalg.norm(o_simt[b, h] - ref[b, h]) <= ATTN_RTOL * nr, (b, h)
+    assert hk.status() == tq.TQ_OK
