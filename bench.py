@@ -57,6 +57,9 @@ def parse_args():
     p.add_argument("--workload", choices=["decode", "score", "encode", "attn4", "search"], default="decode",
                    help="decode: the headline decode step (default); the others measure the remaining hot-path "
                         "rows on their own workloads, one JSON line each")
+    p.add_argument("--small", action="store_true",
+                   help="row workloads only: a reduced size (still above the 126 MB L2, a few hundred MB in "
+                        "all) for profiler captures; the numbers of such a run are not bench values")
     return p.parse_args()
 
 

@@ -75,6 +75,8 @@ S5 = dict(B=64, Hkv=8, Hq=32, L0=16384, d=128, bits=3, m=128, seed_handle=0, see
 def run_score(args):
     import torch
     import embedding_vector_quantization_b200 as tq
+    if args.small:
+        S5["B"] = 16        # 109 MB of packed keys + 34 MB of logits
     B, Hkv, Hq, L0, d = S5["B"], S5["Hkv"], S5["Hq"], S5["L0"], S5["d"]
     T = min(args.steps, 256)
     L_cap = L0 + 256
@@ -172,6 +174,8 @@ def _score_timed(args, torch, tq, h, graph, graph_k, step, toks, qs, k_in, q_in,
              "prefill_encode": {"vectors": B * Hkv * L0, "ms": enc_ms,
                                 "vectors_per_s": B * Hkv * L0 / (enc_ms / 1e3)}}
     cpu = None if args.no_cpu_baseline else oracle_score_sample()
+    if args.small:
+        cfg["workload"] += " [reduced for profiling: 16 sequences]"
     _line(args, "keys scored/sec (cfg 5 score step)", extra["keys_scored_per_s"], "keys/s", total_ms / T, cfg, roof,
           kernels_per_step * T, clocks, extra, cpu)
 
@@ -210,7 +214,7 @@ def run_encode(args):
     import embedding_vector_quantization_b200 as tq
     B, Hkv, L0, d, m = S5["B"], S5["Hkv"], S5["L0"], S5["d"], S5["m"]
     h = tq.Handle(d, S5["bits"], S5["seed_handle"], qjl_m=m)
-    n_all = B * Hkv * L0
+    n_all = B * Hkv * L0 if not args.small else 1 << 20   # small: one launch, 268 MB of input
     per = 1 << 20
     g = torch.Generator(device="cuda").manual_seed(S5["seed_prefill"])
     x = torch.randn(n_all, d, generator=g, device="cuda").to(torch.bfloat16)      # 2.15 GB
@@ -256,6 +260,8 @@ def run_encode(args):
     hbm_bytes = n_all * (2 * d + 32 + 16 + 2 + 2)
     extra = {"vectors_encoded_per_s": n_all / (ms / 1e3), "hbm_gb_per_s": hbm_bytes / (ms / 1e3) / 1e9}
     cpu = None if args.no_cpu_baseline else oracle_encode_sample()
+    if args.small:
+        cfg["workload"] += " [reduced for profiling: 1,048,576 vectors]"
     _line(args, "vectors encoded/sec (cfg 5 prefill encode)", extra["vectors_encoded_per_s"], "vectors/s", ms, cfg,
           roof, launches_per_pass * passes, clocks, extra, cpu)
 
@@ -287,6 +293,8 @@ S3 = dict(B=4, Hkv=8, Hq=32, L=131072, d=128, bits=4, seed_k=5, seed_v=6, seed_q
 def run_attn4(args):
     import torch
     import embedding_vector_quantization_b200 as tq
+    if args.small:
+        S3["B"] = 1         # 138 MB of packed K/V
     B, Hkv, Hq, L, d = S3["B"], S3["Hkv"], S3["Hq"], S3["L"], S3["d"]
     hk = tq.Handle(d, S3["bits"], 0, norm_dtype=tq.TQ_F16)
     hv = tq.Handle(d, S3["bits"], 1, norm_dtype=tq.TQ_F16)
@@ -376,6 +384,8 @@ def run_attn4(args):
              "prefill_encode": {"vectors": 2 * B * Hkv * L, "ms": enc_ms,
                                 "vectors_per_s": 2 * B * Hkv * L / (enc_ms / 1e3)}}
     cpu = None if args.no_cpu_baseline else oracle_attn4_sample()
+    if args.small:
+        cfg["workload"] += " [reduced for profiling: 1 sequence]"
     _line(args, "packed-KV GB/s (cfg 3 decode step, 4-bit MSE)", value, "GB/s", total_ms / T, cfg, roof,
           kernels_per_step * T, clocks, extra, cpu)
 
@@ -416,6 +426,8 @@ FP32_LANES_PER_SM = 128   # fp32 FMA lanes per B200 SM (4 partitions x 32)
 def run_search(args):
     import torch
     import embedding_vector_quantization_b200 as tq
+    if args.small:
+        S4["n"] = 400_000   # 154 MB of codes
     n, nq, d, k = S4["n"], S4["nq"], S4["d"], S4["k"]
     h = tq.Handle(d, S4["bits"], S4["seed_handle"])
     g = torch.Generator(device="cuda").manual_seed(S4["seed_db"])
@@ -480,6 +492,8 @@ def run_search(args):
     extra = {"queries_per_s": nq / (ms / 1e3), "recall_at_10": recall,
              "db_encode": {"vectors": n, "ms": enc_ms, "vectors_per_s": n / (enc_ms / 1e3), "input": "fp32"}}
     cpu = None if args.no_cpu_baseline else oracle_search_sample()
+    if args.small:
+        cfg["workload"] += " [reduced for profiling: 400,000 vectors]"
     _line(args, "queries/sec (cfg 4 top-10 search, 1M x 1536, 2-bit)", extra["queries_per_s"], "queries/s", ms, cfg,
           roof, launches * T, clocks, extra, cpu)
 

@@ -619,7 +619,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 // <S q, 2 sigma - 1> of every key of the chunk for the 4 query heads of a KV head,
 // written to logits [B][Hq][L_cap] ("TurboQuant: redefining AI efficiency", "QJL";
 // "Google TurboQuant", "Stage 2"). Key blocks of 256 stream through a 4-stage TMA ring;
-// each block's scores are staged in shared memory and leave as full 16-byte rows.
+// every thread stores its scores directly: per store instruction a warp writes 8
+// consecutive keys of each of the 4 heads, i.e. whole 32-byte sectors.
 
 constexpr int kSStages = 4;
 constexpr int kSStageBytes = kStageCodes + kStageSigns + 2 * kBlk * 2;  // codes, signs, norms, rnorms: 13312
@@ -641,7 +642,6 @@ struct ScoreArgs {
 
 struct __align__(16) ScoreSmem {
   unsigned char stage[kSStages][kSStageBytes];
-  float out[2][kG][kBlk];         // scores of a block, double buffered: [buffer][head][key]
   uint32_t qfrag[12][2][4][8];
   float qconst[kG][4];
   uint64_t full[kSStages];
@@ -700,7 +700,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
 #pragma unroll
     for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[kk][slot][t][g];
   const float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
-  const bool vec_ok = (a.L_cap % 4) == 0;   // 16-byte rows of logits
+  float* lrow = a.logits + ((size_t)b * a.Hq + h0 + t) * a.L_cap + start;   // head t's scores of the chunk
 
   // No thread leaves this loop early (see attn_prod2_kernel): a wait that runs out stops
   // new copies and further waits, and the remaining blocks are skipped uniformly.
@@ -719,31 +719,22 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
     const unsigned char* st = sm.stage[j % kSStages];
     const __half* nrm = reinterpret_cast<const __half*>(st + kStageCodes + kStageSigns);
     const __half* rnm = nrm + kBlk;
-    float* ob = &sm.out[j & 1][0][0];
+    const int tb = j * kBlk, nvalid = min(kBlk, ntok - tb);
+    float sc[2][2];
     if (!aborted) {
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const int kbase = 128 * mt + 16 * warp;
-        float sc[2];
-        mtile_scores(st, nrm, rnm, kbase, qb, c0h, dmh, dsh, ssh, sc);
-        ob[t * kBlk + kbase + g] = sc[0];
-        ob[t * kBlk + kbase + g + 8] = sc[1];
-      }
+      for (int mt = 0; mt < 2; ++mt) mtile_scores(st, nrm, rnm, 128 * mt + 16 * warp, qb, c0h, dmh, dsh, ssh, sc[mt]);
     }
     __syncwarp();
     if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[j % kSStages])) : "memory");
-    __syncthreads();   // the block's scores are staged (and the other buffer is free again)
-    if (!*(volatile int*)&sm.abort_flag) {
-      const int tb = j * kBlk, nvalid = min(kBlk, ntok - tb);
-      const int h = tid >> 6, k4 = 4 * (tid & 63);
-      float* dst = a.logits + ((size_t)b * a.Hq + h0 + h) * a.L_cap + start + tb + k4;
-      const float4 v4 = *reinterpret_cast<const float4*>(ob + h * kBlk + k4);
-      if (vec_ok && k4 + 4 <= nvalid) {
-        *reinterpret_cast<float4*>(dst) = v4;
-      } else {
-        const float vv[4] = {v4.x, v4.y, v4.z, v4.w};
-        for (int i = 0; i < 4 && k4 + i < nvalid; ++i) dst[i] = vv[i];
-      }
+    if (!aborted) {
+#pragma unroll
+      for (int mt = 0; mt < 2; ++mt)
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int key = 128 * mt + 16 * warp + g + 8 * r;
+          if (key < nvalid) lrow[tb + key] = sc[mt][r];
+        }
     }
   }
   __syncthreads();

@@ -135,7 +135,8 @@ __global__ void __launch_bounds__(kSmallThreads) append_cluster_kernel(EncodeArg
 
 // ---------------------------------------------------------------- query rotation
 
-constexpr int kQRows = 8;
+constexpr int kQRows = 8;      // query rows per CTA (small batches)
+constexpr int kQRowsBig = 64;  // query rows per CTA from 512 rows on: the column slice is staged once per 64 rows
 
 // q' = Pi q and q_s = S q for d <= kWideMaxD: CTA (row group, column block) computes 32 of the d + m
 // outputs (q' = Pi q for o < d, q_s = S q after) of up to kQRows query rows. It stages
@@ -144,16 +145,16 @@ constexpr int kQRows = 8;
 constexpr int kWideMaxD = 512;
 constexpr int kWideCols = 32;
 
-__host__ __device__ inline size_t qprep_wide_smem_bytes(int d) {
-  return (size_t)d * kWideCols * 4 + (size_t)kQRows * d * 4;
+__host__ __device__ inline size_t qprep_wide_smem_bytes(int d, int rpc) {
+  return (size_t)d * kWideCols * 4 + (size_t)rpc * d * 4;
 }
 
 __device__ __forceinline__ void qprep_tile(const void* q, int q_dtype, int rows, int d, const float* PiT,
                                            const float* ST, int m, float* out_r, float* out_s, int rg, int cb,
-                                           unsigned char* smem_raw) {
+                                           int rpc, unsigned char* smem_raw) {
   float* sub = reinterpret_cast<float*>(smem_raw);   // [d][32]
-  float* qsh = sub + (size_t)d * kWideCols;           // [kQRows][d]
-  const int row0 = rg * kQRows, nr = min(kQRows, rows - row0);
+  float* qsh = sub + (size_t)d * kWideCols;           // [rpc][d]
+  const int row0 = rg * rpc, nr = min(rpc, rows - row0);
   const int o0 = cb * kWideCols;
   const bool rot = o0 < d;
   const float* src = rot ? PiT + o0 : ST + (o0 - d);
@@ -187,10 +188,10 @@ __device__ __forceinline__ void qprep_tile(const void* q, int q_dtype, int rows,
 
 __global__ void __launch_bounds__(kSmallThreads) qprep_wide_kernel(const void* q, int q_dtype, int rows, int d,
                                                                    const float* PiT, const float* ST, int m,
-                                                                   float* out_r, float* out_s) {
+                                                                   float* out_r, float* out_s, int rpc) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   grid_dep_launch();
-  qprep_tile(q, q_dtype, rows, d, PiT, ST, m, out_r, out_s, blockIdx.x, blockIdx.y, smem_raw);
+  qprep_tile(q, q_dtype, rows, d, PiT, ST, m, out_r, out_s, blockIdx.x, blockIdx.y, rpc, smem_raw);
 }
 
 // ---------------------------------------------------------------- decode-step prologue
@@ -207,18 +208,24 @@ struct PrologueArgs {
   const float* ST;
   float* qr;
   float* qs;
+  const void* pf[2];       // prefetched into L2 for a later kernel of the step (may be NULL)
+  uint32_t pf_bytes[2];    // multiples of 16
 };
 
 __global__ void __launch_bounds__(kSmallThreads) decode_prologue_kernel(PrologueArgs p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   grid_dep_launch();
   const int bid = blockIdx.x;
+  if (bid == 0 && threadIdx.x < 2 && p.pf[threadIdx.x] && p.pf_bytes[threadIdx.x])
+    asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p.pf[threadIdx.x]), "r"(p.pf_bytes[threadIdx.x])
+                 : "memory");
   if (bid < 2 * p.nvec) {
     const int v = bid % p.nvec;
     (void)append_vector(bid < p.nvec ? p.k : p.v, v / p.k.Hkv, v % p.k.Hkv, smem_raw);
   } else {
     const int t = bid - 2 * p.nvec;
-    qprep_tile(p.q, p.q_dtype, p.rows, p.d, p.PiT, p.ST, p.m, p.qr, p.qs, t / p.qcols, t % p.qcols, smem_raw);
+    qprep_tile(p.q, p.q_dtype, p.rows, p.d, p.PiT, p.ST, p.m, p.qr, p.qs, t / p.qcols, t % p.qcols, kQRows,
+               smem_raw);
   }
 }
 

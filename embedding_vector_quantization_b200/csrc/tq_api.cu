@@ -446,13 +446,13 @@ size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base
 int launch_qprep(const tq_handle* h, const void* q, int q_dtype, int rows, float* qr, float* qs, cudaStream_t s) {
   if (rows == 0) return TQ_OK;
   if (h->d <= tqk::kWideMaxD && h->m <= tqk::kWideMaxD) {
-    const size_t smem = tqk::qprep_wide_smem_bytes(h->d);
     if (once_per_device(6, h->device))
       cudaFuncSetAttribute(tqk::qprep_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
-    dim3 grid((unsigned)((rows + tqk::kQRows - 1) / tqk::kQRows), (unsigned)((h->d + h->m) / tqk::kWideCols));
+    const int rpc = rows >= 512 ? tqk::kQRowsBig : tqk::kQRows;   // query rows per CTA
+    dim3 grid((unsigned)((rows + rpc - 1) / rpc), (unsigned)((h->d + h->m) / tqk::kWideCols));
     KernelScope ks("qprep", s);
-    tqk::qprep_wide_kernel<<<grid, tqk::kSmallThreads, smem, s>>>(q, q_dtype, rows, h->d, h->dPiT, h->dST, h->m,
-                                                                   qr, qs);
+    tqk::qprep_wide_kernel<<<grid, tqk::kSmallThreads, tqk::qprep_wide_smem_bytes(h->d, rpc), s>>>(
+        q, q_dtype, rows, h->d, h->dPiT, h->dST, h->m, qr, qs, rpc);
     return launch_check("qprep_wide_kernel");
   }
   const int groups = (rows + tqk::kQprepRows - 1) / tqk::kQprepRows;
@@ -1010,8 +1010,11 @@ int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int 
   p.nvec = B * Hkv;
   p.q = q; p.q_dtype = q_dtype; p.rows = B * Hq; p.d = hk->d; p.m = hk->m; p.qcols = (hk->d + hk->m) / tqk::kWideCols;
   p.PiT = hk->dPiT; p.ST = hk->dST; p.qr = w.qr; p.qs = w.qs;
+  p.pf[0] = hv->dPi; p.pf[1] = hv->dS;   // the combine's matrices: into L2 while the step runs
+  p.pf_bytes[0] = (uint32_t)((size_t)hv->d * hv->d * 4);
+  p.pf_bytes[1] = (uint32_t)((size_t)hv->m * hv->d * 4);
   const size_t smem = std::max({tqk::append_cluster_smem_bytes(hk->d, hk->m), tqk::append_cluster_smem_bytes(hv->d, hv->m),
-                                tqk::qprep_wide_smem_bytes(hk->d)});
+                                tqk::qprep_wide_smem_bytes(hk->d, tqk::kQRows)});
   if (once_per_device(9, hk->device))
     cudaFuncSetAttribute(tqk::decode_prologue_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
   const unsigned grid = (unsigned)(2 * p.nvec + ((B * Hq + tqk::kQRows - 1) / tqk::kQRows) * p.qcols);
