@@ -223,6 +223,7 @@ def run_tq(args):
     import torch
     import torch.distributed as dist
     import embedding_vector_quantization_b200 as tq
+    from embedding_vector_quantization_b200 import dist as tqdist
     from embedding_vector_quantization_b200 import synth
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
@@ -332,11 +333,7 @@ def run_tq(args):
             if k == "attn_split":
                 split_ms += ms_k
                 split_n += n_k
-    total_ms = sum(step_ms)
-    t = torch.tensor([total_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    max_ms = float(t.item())
+    max_ms = tqdist.max_over_ranks(sum(step_ms))   # the job's time: the slowest rank
 
     # --- end to end through the C ABI with host buffers (pinned), same workload
     q_h = q_all.cpu().pin_memory()
@@ -355,11 +352,7 @@ def run_tq(args):
         e2e_ev[i][1].record()
         lens.fill_(L0)
     torch.cuda.synchronize()
-    e2e_ms = sum(a.elapsed_time(b) for a, b in e2e_ev)
-    te = torch.tensor([e2e_ms], dtype=torch.float64, device=dev)
-    if world > 1:
-        dist.all_reduce(te, op=dist.ReduceOp.MAX)
-    e2e_ms = float(te.item())
+    e2e_ms = tqdist.max_over_ranks(sum(a.elapsed_time(b) for a, b in e2e_ev))
     h2d = (q_in.numel() * 4 + k_in.numel() * 2 + v_in.numel() * 2)
     d2h = out.numel() * 4
 
