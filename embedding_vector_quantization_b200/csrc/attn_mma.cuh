@@ -705,7 +705,8 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
   // No thread leaves this loop early (see attn_prod2_kernel): a wait that runs out stops
   // new copies and further waits, and the remaining blocks are skipped uniformly.
   for (int j = 0; j < nblk; ++j) {
-    const bool aborted = *(volatile int*)&sm.abort_flag != 0;
+    // warp-uniform (the guarded code is warp-collective)
+    const bool aborted = __any_sync(0xffffffffu, *(volatile int*)&sm.abort_flag != 0);
     if (tid == 0 && !aborted && j + kAhead < nblk) {
       const int jo = j + kAhead - kSStages;   // the stage's previous block (j - 2)
       if (jo >= 0 && !mbar_wait(&sm.empty[jo % kSStages], (jo / kSStages) & 1)) {

@@ -1,0 +1,262 @@
+// Top-k inner-product search over 2-bit MSE codes on int8 tensor-core MMAs.
+//
+// "TurboQuant: redefining AI efficiency" (hakusoku.com), "Impact on high-dimensional
+// vector search": scores s = ||x|| <Pi q, c[idx]> on the compressed vectors, ranked by
+// score (equal scores: lower index first). A symmetric 2-bit codebook is affine in its
+// index bits, c[idx] = c0 + (c1 - c0) b0 + (c2 - c0) b1, so
+//   <q', c[idx]> = c0 sum(q') + <(c1 - c0) q', b0> + <(c2 - c0) q', b1>,
+// two 0/1 bit-plane dot products. Database vectors are the MMA rows (their packed code
+// words, shifted and masked into 0/1 bytes), queries the columns: the scaled query values
+// are rounded to 15-bit integers against one step per query and split into int8 hi/lo
+// pieces, so every dot product accumulates exactly in int32.
+//
+// One CTA owns 16 queries (their B fragments stay in shared memory: 64 d bytes) and a
+// contiguous chunk of the database, streamed in blocks of 128 vectors by TMA bulk copies
+// into two stages. Warp w scores vectors 16w .. 16w+15 of a block against the 16 queries;
+// the block's scores go through shared memory to the warps that own the queries (two each),
+// which keep a running top-k (k <= 32) with one list entry per lane. At the end each query's
+// list goes to the per-chunk candidate arrays, which topk_merge_kernel reduces.
+#pragma once
+
+#include "attn_mma.cuh"
+#include "search_simt.cuh"
+
+namespace tqk {
+namespace sm2 {
+
+using amma::ldsm_x4;
+using amma::mbar_expect_tx;
+using amma::mbar_init;
+using amma::mbar_wait;
+using amma::mma_s8;
+using amma::smem_u32;
+using amma::tma_bulk_g2s;
+
+constexpr int kQT = 16;          // queries per CTA (4 MMA column tiles of 4 queries x hi/lo)
+constexpr int kVB = 128;         // vectors per block
+constexpr int kWarps = 8;
+constexpr int kThreads = kWarps * 32;
+constexpr int kMaxD = 1536;      // codes_B = d / 4 <= 384
+constexpr int kMaxCodesB = kMaxD / 4;
+constexpr int kMaxK = 32;        // one list entry per lane
+constexpr int kMaxSteps = kMaxCodesB / 32 * 8;   // k-steps: 32-byte chunks x (4 shifts x 2 masks)
+
+struct Args {
+  const float* qr;       // [nq][d] rotated queries
+  int nq, d, codes_B, k, norm_dtype;
+  const uint8_t* codes;  // [n][codes_B]
+  const void* norms;     // [n]
+  int64_t n, chunk;
+  float c0, w0, w1;      // c[idx] = c0 + w0 b0 + w1 b1
+  float* cand_s;         // [nchunks][nq][k]
+  int64_t* cand_i;       // [nchunks][nq][k]
+  int* err;
+};
+
+struct __align__(16) Smem {
+  unsigned char stage[2][kVB * kMaxCodesB];   // code rows of a block
+  uint32_t qfrag[kMaxSteps][4][4][8][2];      // [k-step][column tile][quad t][column g][register]
+  float sc[kQT][kVB];                         // a block's scores [query][vector]
+  float qc0[kQT], qstep[kQT];                 // c0 sum(q'), integer step of the query pieces
+  uint64_t full[2];
+  int abort_flag;
+};
+
+// Where the query value of coordinate c, plane p sits: byte c / 4 of the code row (chunk
+// byte / 32, k index byte % 32), bit 2 (c % 4) + p -> shift s = bit % 4, mask family bit / 4.
+__device__ __forceinline__ int q_offset(int c, int p, int nt) {
+  const int byte = c >> 2, bit = 2 * (c & 3) + p;
+  const int kk = (byte >> 5) * 8 + (bit >> 2) * 4 + (bit & 3);
+  const int kb = byte & 31, slot = kb >> 4, t = (kb & 15) >> 2, e = kb & 3;
+  return ((((kk * 4 + nt) * 4 + t) * 8) * 2 + slot) * 4 + e;   // byte offset for column g = 0
+}
+
+__device__ __forceinline__ size_t smem_bytes() { return sizeof(Smem); }
+
+// (s, i) ranks before (t, j): higher score, or equal score and lower index.
+__device__ __forceinline__ bool before(float s, int64_t i, float t, int64_t j) { return s > t || (s == t && i < j); }
+
+// Offers candidate (s, i) to a warp-held sorted list (lane j < k holds entry j, best first).
+__device__ __forceinline__ void list_insert(float& ls, int64_t& li, int k, float s, int64_t i) {
+  const int lane = threadIdx.x & 31;
+  const bool b = lane < k && before(s, i, ls, li);
+  const uint32_t m = __ballot_sync(0xffffffffu, b);
+  if (m == 0) return;
+  const int pos = __ffs(m) - 1;
+  const float ps = __shfl_up_sync(0xffffffffu, ls, 1);
+  const int64_t pi = __shfl_up_sync(0xffffffffu, li, 1);
+  if (lane > pos && lane < k) { ls = ps; li = pi; }
+  if (lane == pos) { ls = s; li = i; }
+}
+
+__global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(Args a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int q0 = blockIdx.y * kQT;
+  const int64_t c0 = (int64_t)blockIdx.x * a.chunk, c1 = min(a.n, c0 + a.chunk);
+  const int nblk = (int)((max(c1 - c0, (int64_t)0) + kVB - 1) / kVB);
+  const int nch = a.codes_B / 32;   // 32-byte chunks of a code row
+  const int nsteps = nch * 8;
+
+  if (tid == 0) {
+    mbar_init(&sm.full[0], 1);
+    mbar_init(&sm.full[1], 1);
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  for (int i = tid; i < nsteps * 4 * 4 * 8 * 2; i += kThreads) (&sm.qfrag[0][0][0][0][0])[i] = 0u;
+  __syncthreads();
+  int issued = 0;
+  auto issue = [&](int j) {
+    const int64_t v0 = c0 + (int64_t)j * kVB;
+    const int nv = (int)min((int64_t)kVB, c1 - v0);
+    mbar_expect_tx(&sm.full[j & 1], (uint32_t)nv * a.codes_B);
+    tma_bulk_g2s(sm.stage[j & 1], a.codes + v0 * a.codes_B, (uint32_t)nv * a.codes_B, &sm.full[j & 1]);
+    issued = j + 1;
+  };
+  if (tid == 0)
+    for (int j = 0; j < min(2, nblk); ++j) issue(j);
+  grid_dep_wait();   // the rotated queries come from the kernel before this one
+
+  // query pieces: warp w prepares queries 2w and 2w + 1 of the tile
+#pragma unroll
+  for (int qq = 0; qq < 2; ++qq) {
+    const int ql = 2 * warp + qq, q = q0 + ql;
+    const float* qv = a.qr + (size_t)q * a.d;
+    float sq = 0.f, mx = 0.f;
+    if (q < a.nq)
+      for (int c = lane; c < a.d; c += 32) {
+        const float v = qv[c];
+        sq += v;
+        mx = fmaxf(mx, fmaxf(fabsf(a.w0 * v), fabsf(a.w1 * v)));
+      }
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sq += __shfl_xor_sync(0xffffffffu, sq, o);
+      mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+    }
+    const float step = mx > 0.f ? mx / 16256.f : 1.f;
+    if (q < a.nq) {
+      int8_t* qf = reinterpret_cast<int8_t*>(&sm.qfrag[0][0][0][0][0]);
+      const int nt = ql >> 2, col = 2 * (ql & 3);
+      for (int c = lane; c < a.d; c += 32) {
+        const float v = qv[c];
+#pragma unroll
+        for (int p = 0; p < 2; ++p) {
+          const int xi = __float2int_rn((p ? a.w1 : a.w0) * v / step);
+          const int hi = (xi >= 0) ? (xi + 64) >> 7 : -((-xi + 64) >> 7);
+          const int off = q_offset(c, p, nt);
+          qf[off + col * 8] = (int8_t)hi;                 // column 2 (q % 4): hi piece
+          qf[off + (col + 1) * 8] = (int8_t)(xi - 128 * hi);  // column 2 (q % 4) + 1: lo piece
+        }
+      }
+    }
+    if (lane == 0) {
+      sm.qc0[ql] = a.c0 * sq;
+      sm.qstep[ql] = step;
+    }
+  }
+  __syncthreads();
+
+  float ls[2] = {-INFINITY, -INFINITY};   // running top-k of queries 2w, 2w+1: lane j holds entry j
+  int64_t li[2] = {-1, -1};
+  for (int j = 0; j < nblk; ++j) {
+    // warp-uniform (the guarded code is warp-collective)
+    const bool aborted = __any_sync(0xffffffffu, *(volatile int*)&sm.abort_flag != 0);
+    if (!aborted && !mbar_wait(&sm.full[j & 1], (j >> 1) & 1)) sm.abort_flag = 1;
+    const unsigned char* st = sm.stage[j & 1];
+    const int64_t v0 = c0 + (int64_t)j * kVB;
+    const int nv = (int)min((int64_t)kVB, c1 - v0);
+    int acc1[4][4] = {}, acc16[4][4] = {};
+    if (!aborted) {
+      const int mat = lane >> 3, r = lane & 7;
+      const unsigned char* rowp = st + (16 * warp + r + 8 * (mat >> 1)) * a.codes_B + 16 * (mat & 1);
+      for (int ch = 0; ch < nch; ++ch) {
+        // cw[0] = vector g word t, cw[1] = vector g word 4+t, cw[2] = vector g+8 word t, cw[3] = g+8 word 4+t
+        uint32_t cw[4];
+        ldsm_x4(cw, rowp + 32 * ch);
+#pragma unroll
+        for (int s = 0; s < 4; ++s) {
+          const uint32_t x0 = cw[0] >> s, x1 = cw[1] >> s, x2 = cw[2] >> s, x3 = cw[3] >> s;
+#pragma unroll
+          for (int fam = 0; fam < 2; ++fam) {
+            const uint32_t m = fam ? 0x10101010u : 0x01010101u;
+            const uint32_t p0 = x0 & m, p1 = x1 & m, p2 = x2 & m, p3 = x3 & m;
+            const int kk = ch * 8 + fam * 4 + s;
+#pragma unroll
+            for (int nt = 0; nt < 4; ++nt) {
+              const uint2 b = *reinterpret_cast<const uint2*>(&sm.qfrag[kk][nt][t][g][0]);
+              int(&acc)[4] = fam ? acc16[nt] : acc1[nt];
+              mma_s8(acc, p0, p2, p1, p3, b.x, b.y);
+            }
+          }
+        }
+      }
+    }
+    __syncthreads();   // the previous block's top-k pass is done with sm.sc; this stage is read
+    if (tid == 0 && !*(volatile int*)&sm.abort_flag && j + 2 < nblk) issue(j + 2);
+#pragma unroll
+    for (int nt = 0; nt < 4; ++nt) {
+      const int ql = 4 * nt + t;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int hi = 2 * r, lo = 2 * r + 1;
+        const int dot = 128 * (acc1[nt][hi] + (acc16[nt][hi] >> 4)) + (acc1[nt][lo] + (acc16[nt][lo] >> 4));
+        const int vi = 16 * warp + g + 8 * r;
+        const float nrm = vi < nv ? load_norm(a.norms, a.norm_dtype, v0 + vi) : 0.f;
+        sm.sc[ql][vi] = nrm * (sm.qc0[ql] + sm.qstep[ql] * (float)dot);
+      }
+    }
+    __syncthreads();
+    if (!aborted) {
+#pragma unroll
+      for (int qq = 0; qq < 2; ++qq) {
+        const int ql = 2 * warp + qq;
+        if (q0 + ql >= a.nq) continue;   // the same for the whole warp
+#pragma unroll
+        for (int i = 0; i < kVB / 32; ++i) {
+          const int vi = lane + 32 * i;
+          const bool valid = vi < nv;
+          const float s = valid ? sm.sc[ql][vi] : -INFINITY;
+          const int64_t idx = v0 + vi;
+          float ts = __shfl_sync(0xffffffffu, ls[qq], a.k - 1);
+          int64_t ti = __shfl_sync(0xffffffffu, li[qq], a.k - 1);
+          uint32_t mk = __ballot_sync(0xffffffffu, valid && before(s, idx, ts, ti));
+          while (mk) {
+            const int src = __ffs(mk) - 1;
+            const float cs = __shfl_sync(0xffffffffu, s, src);
+            const int64_t ci = __shfl_sync(0xffffffffu, idx, src);
+            list_insert(ls[qq], li[qq], a.k, cs, ci);
+            ts = __shfl_sync(0xffffffffu, ls[qq], a.k - 1);
+            ti = __shfl_sync(0xffffffffu, li[qq], a.k - 1);
+            mk &= ~(1u << src);
+            mk &= __ballot_sync(0xffffffffu, valid && before(s, idx, ts, ti));
+          }
+        }
+      }
+    }
+  }
+
+  __syncthreads();
+  if (sm.abort_flag) {
+    if (tid == 0) {
+      report_error(a.err, kErrTimeout);
+      for (int jx = max(0, issued - 2); jx < issued; ++jx) (void)mbar_wait(&sm.full[jx & 1], (jx >> 1) & 1);
+    }
+    return;
+  }
+#pragma unroll
+  for (int qq = 0; qq < 2; ++qq) {
+    const int q = q0 + 2 * warp + qq;
+    if (q < a.nq && lane < a.k) {
+      const size_t o = ((size_t)blockIdx.x * a.nq + q) * a.k + lane;
+      a.cand_s[o] = ls[qq];
+      a.cand_i[o] = li[qq];
+    }
+  }
+}
+
+}  // namespace sm2
+}  // namespace tqk

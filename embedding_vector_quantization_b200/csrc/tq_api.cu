@@ -34,6 +34,7 @@
 #include "small_kernels.cuh"
 #include "encode_tc.cuh"
 #include "attn_mse4.cuh"
+#include "search_mma.cuh"
 
 struct tq_handle {
   int d = 0, bits = 0, m = 0, norm_dtype = TQ_F32;
@@ -1047,6 +1048,29 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
   search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk);
   int st = launch_qprep(h, q, TQ_F32, nq, qr, nullptr, s);
   if (st) return st;
+  // 2-bit codes, d % 128 == 0, d <= 1536, k <= 32: int8 tensor-core bit-plane scores
+  if (!std::getenv("TQ_SIMT") && h->bits == 2 && h->d % 128 == 0 && h->d <= tqk::sm2::kMaxD && k <= tqk::sm2::kMaxK &&
+      std::fabs(h->cent[3] - h->cent[2] - h->cent[1] + h->cent[0]) < 1e-12) {
+    tqk::sm2::Args m{};
+    m.qr = qr; m.nq = nq; m.d = h->d; m.codes_B = h->codes_B; m.k = k; m.norm_dtype = h->norm_dtype;
+    m.codes = codes; m.norms = norms; m.n = n; m.chunk = chunk;
+    m.c0 = (float)h->cent[0]; m.w0 = (float)(h->cent[1] - h->cent[0]); m.w1 = (float)(h->cent[2] - h->cent[0]);
+    m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
+    const size_t msmem = sizeof(tqk::sm2::Smem);
+    if (once_per_device(12, h->device))
+      cudaFuncSetAttribute(tqk::sm2::search_mma2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    {
+      KernelScope ks("search", s);
+      const cudaError_t e = launch_pdl(tqk::sm2::search_mma2_kernel,
+                                       dim3((unsigned)nchunks, (unsigned)((nq + tqk::sm2::kQT - 1) / tqk::sm2::kQT)),
+                                       dim3(tqk::sm2::kThreads), msmem, s, m);
+      if (e != cudaSuccess) return cuda_fail(e, "search_mma2_kernel");
+    }
+    if ((st = launch_check("search_mma2_kernel"))) return st;
+    KernelScope ks("topk_merge", s);
+    tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
+    return launch_check("topk_merge_kernel");
+  }
   tqk::SearchArgs a{};
   a.qr = qr; a.nq = nq; a.d = h->d; a.bits = h->bits; a.norm_dtype = h->norm_dtype; a.codes_B = h->codes_B;
   a.k = k; a.codes = codes; a.norms = norms; a.n = n; a.chunk = chunk; a.cent = h->dcent; a.cand_s = cs; a.cand_i = ci;

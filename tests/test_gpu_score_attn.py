@@ -308,3 +308,46 @@ def test_attention_mse4_tensor_core_path_matches_simt_and_oracle(tq, B, Hkv, L, 
             assert np.linalg.norm(o_fast[b, h] - ref[b, h]) <= ATTN_RTOL * nr, (b, h)
             assert np.linalg.norm(o_simt[b, h] - ref[b, h]) <= ATTN_RTOL * nr, (b, h)
     assert hk.status() == tq.TQ_OK
+
+
+@pytest.mark.parametrize("d,n,nq,k", [(512, 50000, 40, 32), (1536, 9000, 17, 1), (128, 700, 3, 10)])
+def test_search_tensor_core_path_matches_simt_and_oracle(tq, d, n, nq, k):
+    """2-bit codes: the int8 tensor-core search (several 128-vector blocks and chunks, a
+    partial query tile, k = 1 and 32) and the SIMT kernel (TQ_SIMT=1) against the oracle.
+    Exact duplicate database rows score identically on either path, so the lower index
+    must be returned first."""
+    import os
+    h = tq.Handle(d, 2, 9)
+    oh = OracleHandle(d, 2, 9)
+    rs = np.random.default_rng(d + n)
+    db = rs.standard_normal((n, d))
+    db /= np.linalg.norm(db, axis=1, keepdims=True)
+    Q = rs.standard_normal((nq, d))
+    # plant exact duplicates of the best vector of query 0 at higher indices
+    best = int(np.argmax(db @ Q[0]))
+    for j in (n - 1, n // 2 + 3):
+        if j != best:
+            db[j] = db[best]
+    e = oh.encode(db, "f32")
+    codes = torch.from_numpy(quant.pack(e["idx"], 2)).cuda()
+    norms = torch.from_numpy(e["n_stored"]).cuda()
+    qg = torch.from_numpy(Q).float().cuda()
+    fast = [x.cpu().numpy() for x in h.search_topk(qg, codes, norms, k)]
+    os.environ["TQ_SIMT"] = "1"
+    try:
+        simt = [x.cpu().numpy() for x in h.search_topk(qg, codes, norms, k)]
+    finally:
+        del os.environ["TQ_SIMT"]
+    S = ops.search_scores(Q.astype(np.float32).astype(np.float64), e["idx"], e["n_stored"], oh.Pi, oh.c)
+    ri, rsc = ops.topk(S, k)
+    for idx, sc in (fast, simt):
+        for i in range(nq):
+            tol = score_tolerance(S[i], np.linalg.norm(Q[i]), 1.0, d)
+            assert len(set(idx[i].tolist())) == k and idx[i].min() >= 0
+            assert np.all(S[i, idx[i]] >= rsc[i, -1] - tol[idx[i]])
+            assert np.all(np.abs(sc[i] - S[i, idx[i]]) <= tol[idx[i]])
+            assert np.all(np.diff(sc[i]) <= 0)
+            for a in range(k - 1):   # equal scores: lower index first
+                if sc[i, a] == sc[i, a + 1]:
+                    assert idx[i, a] < idx[i, a + 1]
+    assert h.status() == tq.TQ_OK
