@@ -10,13 +10,19 @@
 // are rounded to 15-bit integers against one step per query and split into int8 hi/lo
 // pieces, so every dot product accumulates exactly in int32.
 //
-// One CTA owns 16 queries (their B fragments stay in shared memory: 64 d bytes) and a
-// contiguous chunk of the database, streamed in blocks of 128 vectors by TMA bulk copies
-// into two stages. Warp w scores vectors 16w .. 16w+15 of a block against the 16 queries;
+// One CTA owns 16 queries (their B fragments stay in shared memory: 64 d bytes, stored in
+// lane order so that a warp's fragment load covers all 32 banks) and a contiguous chunk of
+// the database, streamed in blocks of 128 vectors into two stages by 2-D TMA copies of
+// 128-byte column slices with the 128-byte swizzle (the rows of a slice are 128 bytes apart
+// and the swizzle spreads the 8 rows an ldmatrix reads over all banks; unswizzled code rows
+// of d / 4 bytes would put them in one bank). Warp w scores vectors 16w .. 16w+15 of a block
+// against the 16 queries;
 // the block's scores go through shared memory to the warps that own the queries (two each),
 // which keep a running top-k (k <= 32) with one list entry per lane. At the end each query's
 // list goes to the per-chunk candidate arrays, which topk_merge_kernel reduces.
 #pragma once
+
+#include <cuda.h>
 
 #include "attn_mma.cuh"
 #include "search_simt.cuh"
@@ -40,6 +46,9 @@ constexpr int kMaxD = 1536;      // codes_B = d / 4 <= 384
 constexpr int kMaxCodesB = kMaxD / 4;
 constexpr int kMaxK = 32;        // one list entry per lane
 constexpr int kMaxSteps = kMaxCodesB / 32 * 8;   // k-steps: 32-byte chunks x (4 shifts x 2 masks)
+constexpr int kSlice = 128;                       // bytes of a code row per TMA slice (the swizzle span)
+constexpr int kMaxSlices = kMaxCodesB / kSlice;
+constexpr int kSliceBytes = kVB * kSlice;         // 16 KB
 
 struct Args {
   const float* qr;       // [nq][d] rotated queries
@@ -53,10 +62,10 @@ struct Args {
   int* err;
 };
 
-struct __align__(16) Smem {
-  unsigned char stage[2][kVB * kMaxCodesB];   // code rows of a block
-  uint32_t qfrag[kMaxSteps][4][4][8][2];      // [k-step][column tile][quad t][column g][register]
-  float sc[kQT][kVB];                         // a block's scores [query][vector]
+struct __align__(1024) Smem {
+  unsigned char stage[2][kMaxSlices][kSliceBytes];   // a block's code rows: 128-byte slices, swizzled
+  uint32_t qfrag[kMaxSteps][4][8][4][2];             // [k-step][column tile][column g][quad t][register]
+  float sc[kQT][kVB + 8];                            // a block's scores [query][vector] (rows 8 banks apart)
   float qc0[kQT], qstep[kQT];                 // c0 sum(q'), integer step of the query pieces
   uint64_t full[2];
   int abort_flag;
@@ -68,10 +77,19 @@ __device__ __forceinline__ int q_offset(int c, int p, int nt) {
   const int byte = c >> 2, bit = 2 * (c & 3) + p;
   const int kk = (byte >> 5) * 8 + (bit >> 2) * 4 + (bit & 3);
   const int kb = byte & 31, slot = kb >> 4, t = (kb & 15) >> 2, e = kb & 3;
-  return ((((kk * 4 + nt) * 4 + t) * 8) * 2 + slot) * 4 + e;   // byte offset for column g = 0
+  return ((((kk * 4 + nt) * 8) * 4 + t) * 2 + slot) * 4 + e;   // byte offset for column g = 0 (g adds 32 g)
 }
 
-__device__ __forceinline__ size_t smem_bytes() { return sizeof(Smem); }
+// Dynamic shared memory to request: the Smem block plus room to align it to 1024 bytes.
+__host__ __device__ inline size_t smem_bytes() { return sizeof(Smem) + 1024; }
+
+__device__ __forceinline__ void tma_tile_2d(void* dst, const CUtensorMap* map, int x, int y, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes [%0], [%1, {%2, %3}], [%4];\n" ::"r"(
+          smem_u32(dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(x), "r"(y), "r"(smem_u32(bar))
+      : "memory");
+}
 
 // (s, i) ranks before (t, j): higher score, or equal score and lower index.
 __device__ __forceinline__ bool before(float s, int64_t i, float t, int64_t j) { return s > t || (s == t && i < j); }
@@ -89,9 +107,10 @@ __device__ __forceinline__ void list_insert(float& ls, int64_t& li, int k, float
   if (lane == pos) { ls = s; li = i; }
 }
 
-__global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(Args a) {
-  extern __shared__ __align__(128) unsigned char smem_raw[];
-  Smem& sm = *reinterpret_cast<Smem*>(smem_raw);
+// cmap: the codes as a 2-D uint8 tensor {codes_B, n}, box {128, 128}, 128-byte swizzle.
+__global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_constant__ CUtensorMap cmap, Args a) {
+  extern __shared__ __align__(1024) unsigned char smem_raw[];
+  Smem& sm = *reinterpret_cast<Smem*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int g = lane >> 2, t = lane & 3;
   const int q0 = blockIdx.y * kQT;
@@ -99,6 +118,7 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(Args a) {
   const int nblk = (int)((max(c1 - c0, (int64_t)0) + kVB - 1) / kVB);
   const int nch = a.codes_B / 32;   // 32-byte chunks of a code row
   const int nsteps = nch * 8;
+  const int nsl = (a.codes_B + kSlice - 1) / kSlice;
 
   if (tid == 0) {
     mbar_init(&sm.full[0], 1);
@@ -109,11 +129,10 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(Args a) {
   for (int i = tid; i < nsteps * 4 * 4 * 8 * 2; i += kThreads) (&sm.qfrag[0][0][0][0][0])[i] = 0u;
   __syncthreads();
   int issued = 0;
-  auto issue = [&](int j) {
+  auto issue = [&](int j) {   // whole boxes arrive (rows past n and bytes past codes_B as zeros)
     const int64_t v0 = c0 + (int64_t)j * kVB;
-    const int nv = (int)min((int64_t)kVB, c1 - v0);
-    mbar_expect_tx(&sm.full[j & 1], (uint32_t)nv * a.codes_B);
-    tma_bulk_g2s(sm.stage[j & 1], a.codes + v0 * a.codes_B, (uint32_t)nv * a.codes_B, &sm.full[j & 1]);
+    mbar_expect_tx(&sm.full[j & 1], (uint32_t)(nsl * kSliceBytes));
+    for (int sl = 0; sl < nsl; ++sl) tma_tile_2d(sm.stage[j & 1][sl], &cmap, sl * kSlice, (int)v0, &sm.full[j & 1]);
     issued = j + 1;
   };
   if (tid == 0)
@@ -148,8 +167,8 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(Args a) {
           const int xi = __float2int_rn((p ? a.w1 : a.w0) * v / step);
           const int hi = (xi >= 0) ? (xi + 64) >> 7 : -((-xi + 64) >> 7);
           const int off = q_offset(c, p, nt);
-          qf[off + col * 8] = (int8_t)hi;                 // column 2 (q % 4): hi piece
-          qf[off + (col + 1) * 8] = (int8_t)(xi - 128 * hi);  // column 2 (q % 4) + 1: lo piece
+          qf[off + col * 32] = (int8_t)hi;                     // column 2 (q % 4): hi piece
+          qf[off + (col + 1) * 32] = (int8_t)(xi - 128 * hi);  // column 2 (q % 4) + 1: lo piece
         }
       }
     }
@@ -166,17 +185,20 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(Args a) {
     // warp-uniform (the guarded code is warp-collective)
     const bool aborted = __any_sync(0xffffffffu, *(volatile int*)&sm.abort_flag != 0);
     if (!aborted && !mbar_wait(&sm.full[j & 1], (j >> 1) & 1)) sm.abort_flag = 1;
-    const unsigned char* st = sm.stage[j & 1];
+    const unsigned char* st = &sm.stage[j & 1][0][0];
     const int64_t v0 = c0 + (int64_t)j * kVB;
     const int nv = (int)min((int64_t)kVB, c1 - v0);
     int acc1[4][4] = {}, acc16[4][4] = {};
     if (!aborted) {
       const int mat = lane >> 3, r = lane & 7;
-      const unsigned char* rowp = st + (16 * warp + r + 8 * (mat >> 1)) * a.codes_B + 16 * (mat & 1);
+      const int vr = 16 * warp + r + 8 * (mat >> 1);   // this lane's row of the block
+      const unsigned char* rowp = st + vr * kSlice;
       for (int ch = 0; ch < nch; ++ch) {
         // cw[0] = vector g word t, cw[1] = vector g word 4+t, cw[2] = vector g+8 word t, cw[3] = g+8 word 4+t
+        // (16-byte unit u of a slice row sits at unit u ^ (row % 8))
         uint32_t cw[4];
-        ldsm_x4(cw, rowp + 32 * ch);
+        const int unit = (((ch & 3) << 1) | (mat & 1)) ^ (vr & 7);
+        ldsm_x4(cw, rowp + (ch >> 2) * kSliceBytes + 16 * unit);
 #pragma unroll
         for (int s = 0; s < 4; ++s) {
           const uint32_t x0 = cw[0] >> s, x1 = cw[1] >> s, x2 = cw[2] >> s, x3 = cw[3] >> s;
@@ -187,7 +209,7 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(Args a) {
             const int kk = ch * 8 + fam * 4 + s;
 #pragma unroll
             for (int nt = 0; nt < 4; ++nt) {
-              const uint2 b = *reinterpret_cast<const uint2*>(&sm.qfrag[kk][nt][t][g][0]);
+              const uint2 b = *reinterpret_cast<const uint2*>(&sm.qfrag[kk][nt][g][t][0]);
               int(&acc)[4] = fam ? acc16[nt] : acc1[nt];
               mma_s8(acc, p0, p2, p1, p3, b.x, b.y);
             }

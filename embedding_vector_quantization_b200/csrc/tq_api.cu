@@ -1056,14 +1056,26 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
     m.codes = codes; m.norms = norms; m.n = n; m.chunk = chunk;
     m.c0 = (float)h->cent[0]; m.w0 = (float)(h->cent[1] - h->cent[0]); m.w1 = (float)(h->cent[2] - h->cent[0]);
     m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
-    const size_t msmem = sizeof(tqk::sm2::Smem);
+    // the codes as a 2-D byte tensor {codes_B, n}: 128-byte x 128-row boxes, 128-byte swizzle
+    PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+    if (!enc) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+    CUtensorMap cmap;
+    const cuuint64_t dims[2] = {(cuuint64_t)h->codes_B, (cuuint64_t)n};
+    const cuuint64_t strides[1] = {(cuuint64_t)h->codes_B};
+    const cuuint32_t box[2] = {(cuuint32_t)tqk::sm2::kSlice, (cuuint32_t)tqk::sm2::kVB};
+    const cuuint32_t estr[2] = {1, 1};
+    const CUresult r = enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box,
+                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+    if (r != CUDA_SUCCESS) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    const size_t msmem = tqk::sm2::smem_bytes();
     if (once_per_device(12, h->device))
       cudaFuncSetAttribute(tqk::sm2::search_mma2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
     {
       KernelScope ks("search", s);
       const cudaError_t e = launch_pdl(tqk::sm2::search_mma2_kernel,
                                        dim3((unsigned)nchunks, (unsigned)((nq + tqk::sm2::kQT - 1) / tqk::sm2::kQT)),
-                                       dim3(tqk::sm2::kThreads), msmem, s, m);
+                                       dim3(tqk::sm2::kThreads), msmem, s, cmap, m);
       if (e != cudaSuccess) return cuda_fail(e, "search_mma2_kernel");
     }
     if ((st = launch_check("search_mma2_kernel"))) return st;
