@@ -12,11 +12,12 @@
 //
 // One CTA owns 16 queries (their B fragments stay in shared memory: 64 d bytes, stored in
 // lane order so that a warp's fragment load covers all 32 banks) and a contiguous chunk of
-// the database, streamed in blocks of 128 vectors into two stages by 2-D TMA copies of
-// 128-byte column slices with the 128-byte swizzle (the rows of a slice are 128 bytes apart
-// and the swizzle spreads the 8 rows an ldmatrix reads over all banks; unswizzled code rows
-// of d / 4 bytes would put them in one bank). Warp w scores vectors 16w .. 16w+15 of a block
-// against the 16 queries;
+// the database, in blocks of 256 vectors. A block arrives as d / 512 column slices of
+// 128 bytes per row (2-D TMA tiles with the 128-byte swizzle, one slice per stage of a
+// 3-stage ring): the rows of a slice are 128 bytes apart and the swizzle spreads the 8 rows
+// an ldmatrix reads over all banks (unswizzled code rows of d / 4 bytes would put them in
+// one bank). Warp w scores vectors 32w .. 32w+31 of a block (two MMA row tiles, so each
+// query fragment loaded from shared memory feeds two MMAs) against the 16 queries;
 // the block's scores go through shared memory to the warps that own the queries (two each),
 // which keep a running top-k (k <= 32) with one list entry per lane. At the end each query's
 // list goes to the per-chunk candidate arrays, which topk_merge_kernel reduces.
@@ -39,7 +40,8 @@ using amma::smem_u32;
 using amma::tma_bulk_g2s;
 
 constexpr int kQT = 16;          // queries per CTA (4 MMA column tiles of 4 queries x hi/lo)
-constexpr int kVB = 128;         // vectors per block
+constexpr int kVB = 256;         // vectors per block (two 16-row MMA tiles per warp)
+constexpr int kStages = 3;       // slice stages
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxD = 1536;      // codes_B = d / 4 <= 384
@@ -48,7 +50,7 @@ constexpr int kMaxK = 32;        // one list entry per lane
 constexpr int kMaxSteps = kMaxCodesB / 32 * 8;   // k-steps: 32-byte chunks x (4 shifts x 2 masks)
 constexpr int kSlice = 128;                       // bytes of a code row per TMA slice (the swizzle span)
 constexpr int kMaxSlices = kMaxCodesB / kSlice;
-constexpr int kSliceBytes = kVB * kSlice;         // 16 KB
+constexpr int kSliceBytes = kVB * kSlice;         // 32 KB
 
 struct Args {
   const float* qr;       // [nq][d] rotated queries
@@ -63,11 +65,12 @@ struct Args {
 };
 
 struct __align__(1024) Smem {
-  unsigned char stage[2][kMaxSlices][kSliceBytes];   // a block's code rows: 128-byte slices, swizzled
+  unsigned char stage[kStages][kSliceBytes];         // 128-byte column slices of a block's code rows, swizzled
   uint32_t qfrag[kMaxSteps][4][8][4][2];             // [k-step][column tile][column g][quad t][register]
   float sc[kQT][kVB + 8];                            // a block's scores [query][vector] (rows 8 banks apart)
   float qc0[kQT], qstep[kQT];                 // c0 sum(q'), integer step of the query pieces
-  uint64_t full[2];
+  uint64_t full[kStages];
+  uint64_t empty[kStages];   // one arrival per warp when it is done with the slice
   int abort_flag;
 };
 
@@ -119,24 +122,29 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_c
   const int nch = a.codes_B / 32;   // 32-byte chunks of a code row
   const int nsteps = nch * 8;
   const int nsl = (a.codes_B + kSlice - 1) / kSlice;
+  const int njobs = nblk * nsl;     // job J: slice J % nsl of block J / nsl
 
   if (tid == 0) {
-    mbar_init(&sm.full[0], 1);
-    mbar_init(&sm.full[1], 1);
+    for (int st = 0; st < kStages; ++st) {
+      mbar_init(&sm.full[st], 1);
+      mbar_init(&sm.empty[st], kWarps);
+    }
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   for (int i = tid; i < nsteps * 4 * 4 * 8 * 2; i += kThreads) (&sm.qfrag[0][0][0][0][0])[i] = 0u;
   __syncthreads();
   int issued = 0;
-  auto issue = [&](int j) {   // whole boxes arrive (rows past n and bytes past codes_B as zeros)
-    const int64_t v0 = c0 + (int64_t)j * kVB;
-    mbar_expect_tx(&sm.full[j & 1], (uint32_t)(nsl * kSliceBytes));
-    for (int sl = 0; sl < nsl; ++sl) tma_tile_2d(sm.stage[j & 1][sl], &cmap, sl * kSlice, (int)v0, &sm.full[j & 1]);
-    issued = j + 1;
+  auto issue = [&](int J) {   // whole boxes arrive (rows past n and bytes past codes_B as zeros)
+    const int64_t v0 = c0 + (int64_t)(J / nsl) * kVB;
+    const int sl = J % nsl;
+    uint64_t* bar = &sm.full[J % kStages];
+    mbar_expect_tx(bar, (uint32_t)kSliceBytes);
+    tma_tile_2d(sm.stage[J % kStages], &cmap, sl * kSlice, (int)v0, bar);   // box {128 bytes, 256 rows}
+    issued = J + 1;
   };
   if (tid == 0)
-    for (int j = 0; j < min(2, nblk); ++j) issue(j);
+    for (int J = 0; J < min(kStages, njobs); ++J) issue(J);
   grid_dep_wait();   // the rotated queries come from the kernel before this one
 
   // query pieces: warp w prepares queries 2w and 2w + 1 of the tile
@@ -179,65 +187,84 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_c
   }
   __syncthreads();
 
+  // this lane's rows of ldmatrix: row tile 0 at vr0, row tile 1 at vr0 + 16 (same row mod 8)
+  const int mat = lane >> 3, vr0 = 32 * warp + (lane & 7) + 8 * (mat >> 1);
   float ls[2] = {-INFINITY, -INFINITY};   // running top-k of queries 2w, 2w+1: lane j holds entry j
   int64_t li[2] = {-1, -1};
   for (int j = 0; j < nblk; ++j) {
-    // warp-uniform (the guarded code is warp-collective)
-    const bool aborted = __any_sync(0xffffffffu, *(volatile int*)&sm.abort_flag != 0);
-    if (!aborted && !mbar_wait(&sm.full[j & 1], (j >> 1) & 1)) sm.abort_flag = 1;
-    const unsigned char* st = &sm.stage[j & 1][0][0];
     const int64_t v0 = c0 + (int64_t)j * kVB;
     const int nv = (int)min((int64_t)kVB, c1 - v0);
-    int acc1[4][4] = {}, acc16[4][4] = {};
-    if (!aborted) {
-      const int mat = lane >> 3, r = lane & 7;
-      const int vr = 16 * warp + r + 8 * (mat >> 1);   // this lane's row of the block
-      const unsigned char* rowp = st + vr * kSlice;
-      for (int ch = 0; ch < nch; ++ch) {
-        // cw[0] = vector g word t, cw[1] = vector g word 4+t, cw[2] = vector g+8 word t, cw[3] = g+8 word 4+t
-        // (16-byte unit u of a slice row sits at unit u ^ (row % 8))
-        uint32_t cw[4];
-        const int unit = (((ch & 3) << 1) | (mat & 1)) ^ (vr & 7);
-        ldsm_x4(cw, rowp + (ch >> 2) * kSliceBytes + 16 * unit);
+    int acc1[2][4][4] = {}, acc16[2][4][4] = {};   // [row tile][column tile]
+    for (int sl = 0; sl < nsl; ++sl) {
+      const int J = j * nsl + sl;
+      // warp-uniform (the guarded code is warp-collective)
+      const bool aborted = __any_sync(0xffffffffu, *(volatile int*)&sm.abort_flag != 0);
+      if (tid == 0 && !aborted && J >= 1 && J - 1 + kStages < njobs) {
+        // refill the stage of job J - 1 with job J - 1 + kStages once every warp has released it
+        if (!mbar_wait(&sm.empty[(J - 1) % kStages], ((J - 1) / kStages) & 1)) sm.abort_flag = 1;
+        else issue(J - 1 + kStages);
+      }
+      if (!aborted && !mbar_wait(&sm.full[J % kStages], (J / kStages) & 1)) sm.abort_flag = 1;
+      if (!aborted) {
+        const unsigned char* st = sm.stage[J % kStages];
+        const int nc4 = min(4, nch - 4 * sl);   // 32-byte chunks in this slice
+        for (int c4 = 0; c4 < nc4; ++c4) {
+          // cw[m][0] = vector g word t, [1] = vector g word 4+t, [2] = vector g+8 word t, [3] = g+8 word 4+t
+          // (16-byte unit u of a slice row sits at unit u ^ (row % 8))
+          const int unit = ((c4 << 1) | (mat & 1)) ^ (vr0 & 7);
+          uint32_t cw[2][4];
+          ldsm_x4(cw[0], st + vr0 * kSlice + 16 * unit);
+          ldsm_x4(cw[1], st + (vr0 + 16) * kSlice + 16 * unit);
 #pragma unroll
-        for (int s = 0; s < 4; ++s) {
-          const uint32_t x0 = cw[0] >> s, x1 = cw[1] >> s, x2 = cw[2] >> s, x3 = cw[3] >> s;
+          for (int s = 0; s < 4; ++s) {
+            uint32_t x[2][4];
 #pragma unroll
-          for (int fam = 0; fam < 2; ++fam) {
-            const uint32_t m = fam ? 0x10101010u : 0x01010101u;
-            const uint32_t p0 = x0 & m, p1 = x1 & m, p2 = x2 & m, p3 = x3 & m;
-            const int kk = ch * 8 + fam * 4 + s;
+            for (int m = 0; m < 2; ++m)
 #pragma unroll
-            for (int nt = 0; nt < 4; ++nt) {
-              const uint2 b = *reinterpret_cast<const uint2*>(&sm.qfrag[kk][nt][g][t][0]);
-              int(&acc)[4] = fam ? acc16[nt] : acc1[nt];
-              mma_s8(acc, p0, p2, p1, p3, b.x, b.y);
+              for (int i = 0; i < 4; ++i) x[m][i] = cw[m][i] >> s;
+#pragma unroll
+            for (int fam = 0; fam < 2; ++fam) {
+              const uint32_t mk = fam ? 0x10101010u : 0x01010101u;
+              const int kk = (4 * sl + c4) * 8 + fam * 4 + s;
+#pragma unroll
+              for (int nt = 0; nt < 4; ++nt) {
+                const uint2 b = *reinterpret_cast<const uint2*>(&sm.qfrag[kk][nt][g][t][0]);
+#pragma unroll
+                for (int m = 0; m < 2; ++m) {
+                  int(&acc)[4] = fam ? acc16[m][nt] : acc1[m][nt];
+                  mma_s8(acc, x[m][0] & mk, x[m][2] & mk, x[m][1] & mk, x[m][3] & mk, b.x, b.y);
+                }
+              }
             }
           }
         }
       }
+      __syncwarp();
+      if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[J % kStages])) : "memory");
     }
-    __syncthreads();   // the previous block's top-k pass is done with sm.sc; this stage is read
-    if (tid == 0 && !*(volatile int*)&sm.abort_flag && j + 2 < nblk) issue(j + 2);
+    const bool aborted = __any_sync(0xffffffffu, *(volatile int*)&sm.abort_flag != 0);
+    __syncthreads();   // the previous block's top-k pass is done with sm.sc
 #pragma unroll
-    for (int nt = 0; nt < 4; ++nt) {
-      const int ql = 4 * nt + t;
+    for (int m = 0; m < 2; ++m)
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int hi = 2 * r, lo = 2 * r + 1;
-        const int dot = 128 * (acc1[nt][hi] + (acc16[nt][hi] >> 4)) + (acc1[nt][lo] + (acc16[nt][lo] >> 4));
-        const int vi = 16 * warp + g + 8 * r;
-        const float nrm = vi < nv ? load_norm(a.norms, a.norm_dtype, v0 + vi) : 0.f;
-        sm.sc[ql][vi] = nrm * (sm.qc0[ql] + sm.qstep[ql] * (float)dot);
+      for (int nt = 0; nt < 4; ++nt) {
+        const int ql = 4 * nt + t;
+#pragma unroll
+        for (int r = 0; r < 2; ++r) {
+          const int hi = 2 * r, lo = 2 * r + 1;
+          const int dot = 128 * (acc1[m][nt][hi] + (acc16[m][nt][hi] >> 4)) + (acc1[m][nt][lo] + (acc16[m][nt][lo] >> 4));
+          const int vi = 32 * warp + 16 * m + g + 8 * r;
+          const float nrm = vi < nv ? load_norm(a.norms, a.norm_dtype, v0 + vi) : 0.f;
+          sm.sc[ql][vi] = nrm * (sm.qc0[ql] + sm.qstep[ql] * (float)dot);
+        }
       }
-    }
     __syncthreads();
     if (!aborted) {
 #pragma unroll
       for (int qq = 0; qq < 2; ++qq) {
         const int ql = 2 * warp + qq;
         if (q0 + ql >= a.nq) continue;   // the same for the whole warp
-#pragma unroll
+#pragma unroll 2
         for (int i = 0; i < kVB / 32; ++i) {
           const int vi = lane + 32 * i;
           const bool valid = vi < nv;
@@ -265,7 +292,8 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_c
   if (sm.abort_flag) {
     if (tid == 0) {
       report_error(a.err, kErrTimeout);
-      for (int jx = max(0, issued - 2); jx < issued; ++jx) (void)mbar_wait(&sm.full[jx & 1], (jx >> 1) & 1);
+      for (int jx = max(0, issued - kStages); jx < issued; ++jx)
+        (void)mbar_wait(&sm.full[jx % kStages], (jx / kStages) & 1);
     }
     return;
   }

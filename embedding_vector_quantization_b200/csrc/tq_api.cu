@@ -341,6 +341,33 @@ void search_split(int nq, int64_t n, int* nchunks, int64_t* chunk) {
   *nchunks = (int)((n + ch - 1) / ch);
 }
 
+int sm_count(int device) {
+  static std::atomic<int> counts[64];
+  if (device < 0 || device >= 64) return 148;
+  int c = counts[device].load();
+  if (c == 0) {
+    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || c <= 0) c = 148;
+    counts[device].store(c);
+  }
+  return c;
+}
+
+// Split of the int8 tensor-core search (one CTA per SM, 16 queries per CTA): the number of
+// database chunks makes chunks x query tiles a whole number of waves where it can, chunks a
+// multiple of 256 vectors.
+void search_mma_split(int nq, int64_t n, int sms, int* nchunks, int64_t* chunk) {
+  const int64_t qt = (nq + tqk::sm2::kQT - 1) / tqk::sm2::kQT;
+  int64_t a = sms, bq = qt;   // nc0 = sms / gcd(sms, qt): the fewest chunks giving whole waves
+  while (bq) { const int64_t r = a % bq; a = bq; bq = r; }
+  const int64_t nc0 = sms / a;
+  int64_t nc = nc0 * std::max<int64_t>(1, (8 * (int64_t)sms + nc0 * qt / 2) / (nc0 * qt));
+  nc = std::max<int64_t>(1, std::min<int64_t>(nc, (n + tqk::sm2::kVB - 1) / tqk::sm2::kVB));
+  int64_t ch = (n + nc - 1) / nc;
+  ch = (ch + tqk::sm2::kVB - 1) / tqk::sm2::kVB * tqk::sm2::kVB;
+  *chunk = ch;
+  *nchunks = (int)((n + ch - 1) / ch);
+}
+
 // The int8 tensor-core attention kernel covers 3-bit prod K and V caches (2-bit
 // codes + 128 QJL signs, fp16 norms) at d = 128 with 4 query heads per KV head.
 // TQ_SIMT=1 forces the SIMT kernels (used by tests to cross-check both paths).
@@ -428,10 +455,13 @@ size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, i
 }
 
 size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base, float** qr, float** cs,
-                        int64_t** ci, int* nchunks, int64_t* chunk) {
+                        int64_t** ci, int* nchunks, int64_t* chunk, bool mma) {
   int nc;
   int64_t ch;
-  search_split(nq, n, &nc, &ch);
+  if (mma)
+    search_mma_split(nq, n, sm_count(h->device), &nc, &ch);
+  else
+    search_split(nq, n, &nc, &ch);
   if (nchunks) *nchunks = nc;
   if (chunk) *chunk = ch;
   size_t off = 0;
@@ -510,17 +540,6 @@ PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
   });
   return fn;
-}
-
-int sm_count(int device) {
-  static std::atomic<int> counts[64];
-  if (device < 0 || device >= 64) return 148;
-  int c = counts[device].load();
-  if (c == 0) {
-    if (cudaDeviceGetAttribute(&c, cudaDevAttrMultiProcessorCount, device) != cudaSuccess || c <= 0) c = 148;
-    counts[device].store(c);
-  }
-  return c;
 }
 
 bool tc_encode_ok(const tq_handle* h, const tqk::EncodeArgs& a) {
@@ -774,7 +793,8 @@ size_t tq_attn_workspace_bytes(const tq_handle* hk, const tq_handle* hv, int B, 
 
 size_t tq_search_workspace_bytes(const tq_handle* h, int nq, int64_t n, int k) {
   if (!h || nq < 0 || n < 1 || k < 1) return 0;
-  return search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return std::max(search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, false),
+                  search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, true));
 }
 
 int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const tq_cache* k, const int32_t* len,
@@ -1045,18 +1065,20 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
   int64_t* ci;
   int nchunks;
   int64_t chunk;
-  search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk);
+  // 2-bit codes, d % 128 == 0, d <= 1536, k <= 32: int8 tensor-core bit-plane scores
+  const bool mma = !std::getenv("TQ_SIMT") && h->bits == 2 && h->d % 128 == 0 && h->d <= tqk::sm2::kMaxD &&
+                   k <= tqk::sm2::kMaxK && n < (int64_t(1) << 31) &&
+                   std::fabs(h->cent[3] - h->cent[2] - h->cent[1] + h->cent[0]) < 1e-12;
+  search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk, mma);
   int st = launch_qprep(h, q, TQ_F32, nq, qr, nullptr, s);
   if (st) return st;
-  // 2-bit codes, d % 128 == 0, d <= 1536, k <= 32: int8 tensor-core bit-plane scores
-  if (!std::getenv("TQ_SIMT") && h->bits == 2 && h->d % 128 == 0 && h->d <= tqk::sm2::kMaxD && k <= tqk::sm2::kMaxK &&
-      std::fabs(h->cent[3] - h->cent[2] - h->cent[1] + h->cent[0]) < 1e-12) {
+  if (mma) {
     tqk::sm2::Args m{};
     m.qr = qr; m.nq = nq; m.d = h->d; m.codes_B = h->codes_B; m.k = k; m.norm_dtype = h->norm_dtype;
     m.codes = codes; m.norms = norms; m.n = n; m.chunk = chunk;
     m.c0 = (float)h->cent[0]; m.w0 = (float)(h->cent[1] - h->cent[0]); m.w1 = (float)(h->cent[2] - h->cent[0]);
     m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
-    // the codes as a 2-D byte tensor {codes_B, n}: 128-byte x 128-row boxes, 128-byte swizzle
+    // the codes as a 2-D byte tensor {codes_B, n}: 128-byte x 256-row boxes, 128-byte swizzle
     PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
     if (!enc) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
     CUtensorMap cmap;
