@@ -422,13 +422,18 @@ def oracle_attn4_sample(budget_s=12.0, L=32768):
 S4 = dict(n=1_000_000, nq=1024, d=1536, bits=2, k=10, seed_handle=0, seed_db=8, seed_q=9)
 
 
-def run_search(args):
+FP32_LANES_PER_SM = 128   # fp32 FMA lanes per B200 SM (4 partitions x 32)
+
+
+def run_search(args, bits=None):
+    """cfg-4 search at 2 bits (int8 tensor-core kernel) or 4 bits (SIMT kernel with the centroid table)."""
     import torch
     import embedding_vector_quantization_b200 as tq
+    bits = S4["bits"] if bits is None else bits
     if args.small:
-        S4["n"] = 400_000   # 154 MB of codes
+        S4["n"] = 400_000   # 154 MB of 2-bit codes
     n, nq, d, k = S4["n"], S4["nq"], S4["d"], S4["k"]
-    h = tq.Handle(d, S4["bits"], S4["seed_handle"])
+    h = tq.Handle(d, bits, S4["seed_handle"])
     g = torch.Generator(device="cuda").manual_seed(S4["seed_db"])
     db = torch.randn(n, d, generator=g, device="cuda")
     db /= db.norm(dim=1, keepdim=True)
@@ -478,35 +483,47 @@ def run_search(args):
     recall = hits / (nq * k)
     flops = 2.0 * d * nq * n
     ach = flops / (s_ms / max(s_n, 1) / 1e3) / 1e12
-    # int8 tensor-core contraction: the measured bf16 dense peak x 2 (the nominal int8 : bf16
-    # ratio, 4.5 : 2.25 PFLOP/s)
-    bf16, src = _peak("tensor")
-    peak = 2.0 * bf16
-    cfg = {"workload": "top-10 inner-product search, TurboQuant MSE 2-bit, d=1536, 1,000,000 L2-normalised "
+    cfg = {"workload": f"top-10 inner-product search, TurboQuant MSE {bits}-bit, d=1536, 1,000,000 L2-normalised "
                        "N(0,I) database vectors, 1024 queries (stands in for the pages' vector-search benchmarks)",
-           "n": n, "nq": nq, "d": d, "k": k, "dtype": "int8 mma (bit planes x 15-bit query pieces), s32 accumulate",
-           "l2": "not flushed: the 384 MB of codes exceed the 126 MB L2"}
-    roof = {"bound": "tensor", "kernel": "search_mma2_kernel", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
-            "frac": ach / peak, "traffic": None, "peak_source": f"{src} x 2 (int8 : bf16 nominal ratio)",
-            "launch_ms": s_ms / max(s_n, 1), "algorithmic_flops_per_launch": flops,
-            "note": "algorithmic 2d flops per (query, vector); the int8 bit-plane form executes 4x that in MMA "
-                    "operations (2 planes x hi/lo query pieces)"}
+           "n": n, "nq": nq, "d": d, "k": k,
+           "l2": f"not flushed: the {n * d * bits // 8 // 1000000} MB of codes exceed the 126 MB L2"}
+    if bits == 2:
+        # int8 tensor-core contraction: the measured bf16 dense peak x 2 (the nominal int8 : bf16
+        # ratio, 4.5 : 2.25 PFLOP/s)
+        bf16, src = _peak("tensor")
+        peak = 2.0 * bf16
+        cfg["dtype"] = "int8 mma (bit planes x 15-bit query pieces), s32 accumulate"
+        roof = {"bound": "tensor", "kernel": "search_mma2_kernel", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": None, "peak_source": f"{src} x 2 (int8 : bf16 nominal ratio)",
+                "launch_ms": s_ms / max(s_n, 1), "algorithmic_flops_per_launch": flops,
+                "note": "algorithmic 2d flops per (query, vector); the int8 bit-plane form executes 4x that in MMA "
+                        "operations (2 planes x hi/lo query pieces)"}
+    else:
+        # fp32 FMAs on the CUDA cores: SMs x 128 lanes x 2 flop x the median sampled SM clock
+        sm_mhz = clocks.get("sm_mhz") or 1965.0
+        peak = torch.cuda.get_device_properties(0).multi_processor_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+        cfg["dtype"] = "f32 SIMT (centroid table in shared memory)"
+        roof = {"bound": "alu", "kernel": "search_simt_kernel", "achieved": ach, "peak": peak, "unit": "TFLOP/s",
+                "frac": ach / peak, "traffic": None,
+                "peak_source": "derived: SMs x 128 fp32 FMA lanes x 2 flop x median sampled SM clock",
+                "launch_ms": s_ms / max(s_n, 1), "algorithmic_flops_per_launch": flops}
     extra = {"queries_per_s": nq / (ms / 1e3), "recall_at_10": recall,
              "db_encode": {"vectors": n, "ms": enc_ms, "vectors_per_s": n / (enc_ms / 1e3), "input": "fp32"}}
-    cpu = None if args.no_cpu_baseline else oracle_search_sample()
+    cpu = None if args.no_cpu_baseline else oracle_search_sample(bits=bits)
     if args.small:
         cfg["workload"] += " [reduced for profiling: 400,000 vectors]"
-    _line(args, "queries/sec (cfg 4 top-10 search, 1M x 1536, 2-bit)", extra["queries_per_s"], "queries/s", ms, cfg,
-          roof, launches * T, clocks, extra, cpu)
+    _line(args, f"queries/sec (cfg 4 top-10 search, 1M x 1536, {bits}-bit)", extra["queries_per_s"], "queries/s", ms,
+          cfg, roof, launches * T, clocks, extra, cpu)
 
 
-def oracle_search_sample(budget_s=12.0, n=32768, nq=64):
-    """The oracle's top-10 search of nq queries over n 2-bit vectors (d = 1536; encode untimed)."""
+def oracle_search_sample(budget_s=12.0, n=32768, nq=64, bits=None):
+    """The oracle's top-10 search of nq queries over n vectors (d = 1536; encode untimed)."""
     import torch
     from oracle import codebook, ops, quant, rotation
     d = S4["d"]
+    bits = S4["bits"] if bits is None else bits
     Pi = rotation.rotation(d, S4["seed_handle"], 0)[0]
-    c, beta = codebook.lloyd_max(d, S4["bits"])
+    c, beta = codebook.lloyd_max(d, bits)
     x = torch.randn(n, d, generator=torch.Generator().manual_seed(S4["seed_db"])).double()
     x = (x / x.norm(dim=1, keepdim=True)).numpy()
     e = quant.encode_mse(x, Pi, c, beta, "f32")
@@ -527,4 +544,7 @@ def oracle_search_sample(budget_s=12.0, n=32768, nq=64):
 
 
 def run(args):
+    if args.workload == "search4":
+        run_search(args, bits=4)
+        return
     {"score": run_score, "encode": run_encode, "attn4": run_attn4, "search": run_search}[args.workload](args)
