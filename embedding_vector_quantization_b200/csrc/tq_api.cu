@@ -35,6 +35,7 @@
 #include "encode_tc.cuh"
 #include "attn_mse4.cuh"
 #include "search_mma.cuh"
+#include "search_mma4.cuh"
 
 struct tq_handle {
   int d = 0, bits = 0, m = 0, norm_dtype = TQ_F32;
@@ -352,11 +353,12 @@ int sm_count(int device) {
   return c;
 }
 
-// Split of the int8 tensor-core search (one CTA per SM, 16 queries per CTA): the number of
-// database chunks makes chunks x query tiles a whole number of waves where it can, chunks a
-// multiple of 256 vectors.
-void search_mma_split(int nq, int64_t n, int sms, int* nchunks, int64_t* chunk) {
-  const int64_t qt = (nq + tqk::sm2::kQT - 1) / tqk::sm2::kQT;
+// Split of the int8 tensor-core searches (one CTA per SM, qtile queries per CTA): the number
+// of database chunks makes chunks x query tiles a whole number of waves where it can, chunks
+// a multiple of 256 vectors.
+void search_mma_split(int nq, int qtile, int64_t n, int sms, int* nchunks, int64_t* chunk) {
+  static_assert(tqk::sm2::kVB == tqk::sm4::kVB, "one block size for both searches");
+  const int64_t qt = (nq + qtile - 1) / qtile;
   int64_t a = sms, bq = qt;   // nc0 = sms / gcd(sms, qt): the fewest chunks giving whole waves
   while (bq) { const int64_t r = a % bq; a = bq; bq = r; }
   const int64_t nc0 = sms / a;
@@ -454,12 +456,13 @@ size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, i
   return off;
 }
 
+// mma: 0 for the SIMT kernel, else the queries per CTA of the tensor-core kernel.
 size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base, float** qr, float** cs,
-                        int64_t** ci, int* nchunks, int64_t* chunk, bool mma) {
+                        int64_t** ci, int* nchunks, int64_t* chunk, int mma) {
   int nc;
   int64_t ch;
   if (mma)
-    search_mma_split(nq, n, sm_count(h->device), &nc, &ch);
+    search_mma_split(nq, mma, n, sm_count(h->device), &nc, &ch);
   else
     search_split(nq, n, &nc, &ch);
   if (nchunks) *nchunks = nc;
@@ -540,6 +543,22 @@ PFN_cuTensorMapEncodeTiled tensor_map_encoder() {
       fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled>(p);
   });
   return fn;
+}
+
+// Code rows as a 2-D byte tensor {row_bytes, rows} for tile loads of box_rows rows and
+// box_bytes (128) bytes with the 128-byte swizzle; bytes and rows past the tensor load as zeros.
+int codes_map_2d(const uint8_t* codes, int64_t rows, int row_bytes, int box_bytes, int box_rows, CUtensorMap* map) {
+  PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+  if (!enc) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const cuuint64_t dims[2] = {(cuuint64_t)row_bytes, (cuuint64_t)rows};
+  const cuuint64_t strides[1] = {(cuuint64_t)row_bytes};
+  const cuuint32_t box[2] = {(cuuint32_t)box_bytes, (cuuint32_t)box_rows};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(map, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  return TQ_OK;
 }
 
 bool tc_encode_ok(const tq_handle* h, const tqk::EncodeArgs& a) {
@@ -793,8 +812,10 @@ size_t tq_attn_workspace_bytes(const tq_handle* hk, const tq_handle* hv, int B, 
 
 size_t tq_search_workspace_bytes(const tq_handle* h, int nq, int64_t n, int k) {
   if (!h || nq < 0 || n < 1 || k < 1) return 0;
-  return std::max(search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, false),
-                  search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, true));
+  size_t b = 0;
+  for (int mode : {0, tqk::sm2::kQT, tqk::sm4::kQT})
+    b = std::max(b, search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, mode));
+  return b;
 }
 
 int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const tq_cache* k, const int32_t* len,
@@ -1065,31 +1086,48 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
   int64_t* ci;
   int nchunks;
   int64_t chunk;
-  // 2-bit codes, d % 128 == 0, d <= 1536, k <= 32: int8 tensor-core bit-plane scores
-  const bool mma = !std::getenv("TQ_SIMT") && h->bits == 2 && h->d % 128 == 0 && h->d <= tqk::sm2::kMaxD &&
-                   k <= tqk::sm2::kMaxK && n < (int64_t(1) << 31) &&
-                   std::fabs(h->cent[3] - h->cent[2] - h->cent[1] + h->cent[0]) < 1e-12;
-  search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk, mma);
+  // int8 tensor-core bit-plane scores: 2-bit codes with d % 128 == 0, or 4-bit codes (symmetric
+  // codebook, Walsh planes) with d % 64 == 0; d <= 1536, k <= 32
+  const bool tc_ok = !std::getenv("TQ_SIMT") && h->d <= 1536 && k <= tqk::sm2::kMaxK && n < (int64_t(1) << 31);
+  const bool mma2 = tc_ok && h->bits == 2 && h->d % 128 == 0 &&
+                    std::fabs(h->cent[3] - h->cent[2] - h->cent[1] + h->cent[0]) < 1e-12;
+  float w4[8], c04 = 0.f;
+  const bool mma4 = tc_ok && h->bits == 4 && h->d % 64 == 0 && plane_coeffs4(h->cent, &c04, w4);
+  search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk,
+                   mma2 ? tqk::sm2::kQT : mma4 ? tqk::sm4::kQT : 0);
   int st = launch_qprep(h, q, TQ_F32, nq, qr, nullptr, s);
   if (st) return st;
-  if (mma) {
+  if (mma4) {
+    tqk::sm4::Args m{};
+    m.qr = qr; m.nq = nq; m.d = h->d; m.codes_B = h->codes_B; m.k = k; m.norm_dtype = h->norm_dtype;
+    m.norms = norms; m.n = n; m.chunk = chunk; m.c0 = c04;
+    for (int i = 0; i < 8; ++i) m.w[i] = w4[i];
+    m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
+    CUtensorMap cmap;
+    if ((st = codes_map_2d(codes, n, h->codes_B, tqk::sm4::kSlice, tqk::sm4::kVB, &cmap))) return st;
+    const size_t msmem = tqk::sm4::smem_bytes();
+    if (once_per_device(13, h->device))
+      cudaFuncSetAttribute(tqk::sm4::search_mma4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+    {
+      KernelScope ks("search", s);
+      const cudaError_t e = launch_pdl(tqk::sm4::search_mma4_kernel,
+                                       dim3((unsigned)nchunks, (unsigned)((nq + tqk::sm4::kQT - 1) / tqk::sm4::kQT)),
+                                       dim3(tqk::sm4::kThreads), msmem, s, cmap, m);
+      if (e != cudaSuccess) return cuda_fail(e, "search_mma4_kernel");
+    }
+    if ((st = launch_check("search_mma4_kernel"))) return st;
+    KernelScope ks("topk_merge", s);
+    tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
+    return launch_check("topk_merge_kernel");
+  }
+  if (mma2) {
     tqk::sm2::Args m{};
     m.qr = qr; m.nq = nq; m.d = h->d; m.codes_B = h->codes_B; m.k = k; m.norm_dtype = h->norm_dtype;
     m.codes = codes; m.norms = norms; m.n = n; m.chunk = chunk;
     m.c0 = (float)h->cent[0]; m.w0 = (float)(h->cent[1] - h->cent[0]); m.w1 = (float)(h->cent[2] - h->cent[0]);
     m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
-    // the codes as a 2-D byte tensor {codes_B, n}: 128-byte x 256-row boxes, 128-byte swizzle
-    PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
-    if (!enc) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
     CUtensorMap cmap;
-    const cuuint64_t dims[2] = {(cuuint64_t)h->codes_B, (cuuint64_t)n};
-    const cuuint64_t strides[1] = {(cuuint64_t)h->codes_B};
-    const cuuint32_t box[2] = {(cuuint32_t)tqk::sm2::kSlice, (cuuint32_t)tqk::sm2::kVB};
-    const cuuint32_t estr[2] = {1, 1};
-    const CUresult r = enc(&cmap, CU_TENSOR_MAP_DATA_TYPE_UINT8, 2, const_cast<uint8_t*>(codes), dims, strides, box,
-                           estr, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
-                           CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
-    if (r != CUDA_SUCCESS) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+    if ((st = codes_map_2d(codes, n, h->codes_B, tqk::sm2::kSlice, tqk::sm2::kVB, &cmap))) return st;
     const size_t msmem = tqk::sm2::smem_bytes();
     if (once_per_device(12, h->device))
       cudaFuncSetAttribute(tqk::sm2::search_mma2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);

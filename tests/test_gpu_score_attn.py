@@ -310,10 +310,13 @@ def test_attention_mse4_tensor_core_path_matches_simt_and_oracle(tq, B, Hkv, L, 
     assert hk.status() == tq.TQ_OK
 
 
-@pytest.mark.parametrize("d,n,nq,k", [(512, 50000, 40, 32), (1536, 9000, 17, 1), (128, 700, 3, 10)])
+@pytest.mark.parametrize("d,n,nq,k", [(512, 50000, 40, 32), (1536, 9000, 17, 1), (128, 700, 3, 10),
+                                     (640, 3000, 16, 10), (1024, 300, 64, 5), (256, 100, 5, 7)])
 def test_search_tensor_core_path_matches_simt_and_oracle(tq, d, n, nq, k):
-    """2-bit codes: the int8 tensor-core search (several 128-vector blocks and chunks, a
-    partial query tile, k = 1 and 32) and the SIMT kernel (TQ_SIMT=1) against the oracle.
+    """2-bit codes: the int8 tensor-core search (several 256-vector blocks and chunks, code
+    rows of one, two and three 128-byte slices and a partial last slice (d = 640), a
+    database shorter than one block, partial query tiles, k = 1 and 32) and the SIMT kernel
+    (TQ_SIMT=1) against the oracle.
     Exact duplicate database rows score identically on either path, so the lower index
     must be returned first."""
     import os
@@ -330,6 +333,49 @@ def test_search_tensor_core_path_matches_simt_and_oracle(tq, d, n, nq, k):
             db[j] = db[best]
     e = oh.encode(db, "f32")
     codes = torch.from_numpy(quant.pack(e["idx"], 2)).cuda()
+    norms = torch.from_numpy(e["n_stored"]).cuda()
+    qg = torch.from_numpy(Q).float().cuda()
+    fast = [x.cpu().numpy() for x in h.search_topk(qg, codes, norms, k)]
+    os.environ["TQ_SIMT"] = "1"
+    try:
+        simt = [x.cpu().numpy() for x in h.search_topk(qg, codes, norms, k)]
+    finally:
+        del os.environ["TQ_SIMT"]
+    S = ops.search_scores(Q.astype(np.float32).astype(np.float64), e["idx"], e["n_stored"], oh.Pi, oh.c)
+    ri, rsc = ops.topk(S, k)
+    for idx, sc in (fast, simt):
+        for i in range(nq):
+            tol = score_tolerance(S[i], np.linalg.norm(Q[i]), 1.0, d)
+            assert len(set(idx[i].tolist())) == k and idx[i].min() >= 0
+            assert np.all(S[i, idx[i]] >= rsc[i, -1] - tol[idx[i]])
+            assert np.all(np.abs(sc[i] - S[i, idx[i]]) <= tol[idx[i]])
+            assert np.all(np.diff(sc[i]) <= 0)
+            for a in range(k - 1):   # equal scores: lower index first
+                if sc[i, a] == sc[i, a + 1]:
+                    assert idx[i, a] < idx[i, a + 1]
+    assert h.status() == tq.TQ_OK
+
+
+@pytest.mark.parametrize("d,n,nq,k", [(1536, 6000, 9, 10), (320, 3000, 13, 32), (128, 200, 4, 1), (512, 20000, 70, 10)])
+def test_search_4bit_tensor_core_path_matches_simt_and_oracle(tq, d, n, nq, k):
+    """4-bit codes: the int8 tensor-core search over the eight Walsh planes of the symmetric
+    codebook (code rows of one to six 128-byte slices, a partial last slice at d = 320, a
+    database shorter than one 256-vector block, partial query tiles of 4, k = 1 and 32) and
+    the SIMT kernel (TQ_SIMT=1) against the oracle; planted duplicates of a best vector must
+    come back lower index first."""
+    import os
+    h = tq.Handle(d, 4, 11)
+    oh = OracleHandle(d, 4, 11)
+    rs = np.random.default_rng(d * 7 + n)
+    db = rs.standard_normal((n, d))
+    db /= np.linalg.norm(db, axis=1, keepdims=True)
+    Q = rs.standard_normal((nq, d))
+    best = int(np.argmax(db @ Q[0]))
+    for j in (n - 1, n // 3 + 1):
+        if j != best:
+            db[j] = db[best]
+    e = oh.encode(db, "f32")
+    codes = torch.from_numpy(quant.pack(e["idx"], 4)).cuda()
     norms = torch.from_numpy(e["n_stored"]).cuda()
     qg = torch.from_numpy(Q).float().cuda()
     fast = [x.cpu().numpy() for x in h.search_topk(qg, codes, norms, k)]
