@@ -56,10 +56,11 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["tq", "reference"], default="tq")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--workload", choices=["decode", "score", "encode", "attn4", "search", "search4"],
+    p.add_argument("--workload", choices=["decode", "score", "encode", "attn4", "search", "search4", "compare"],
                    default="decode",
                    help="decode: the headline decode step (default); the others measure the remaining hot-path "
-                        "rows on their own workloads, one JSON line each (search: 2-bit codes, search4: 4-bit)")
+                        "rows on their own workloads, one JSON line each (search: 2-bit codes, search4: 4-bit; "
+                        "compare: the cfg-2 attention against uncompressed bf16 / fp32 K/V)")
     p.add_argument("--small", action="store_true",
                    help="row workloads only: a reduced size (still above the 126 MB L2, a few hundred MB in "
                         "all) for profiler captures; the numbers of such a run are not bench values")
