@@ -19,7 +19,8 @@ from ._lib import (  # noqa: F401  (the C ABI, same names)
     TQError, make_cache, tq_append, tq_attn_decode, tq_attn_decode_noalloc, tq_decode_step, tq_attn_workspace_bytes, tq_code_bytes, tq_codebook_host,
     tq_create, tq_create_prod, tq_destroy, tq_encode, tq_get_codebook, tq_get_info, tq_get_rotation,
     tq_last_error, tq_last_status, tq_pack_indices, tq_rotation_host, tq_score, tq_score_workspace_bytes,
-    tq_search_topk, tq_search_workspace_bytes, tq_set_norm_dtype, tq_timer_enable, tq_timer_read,
+    tq_search_topk, tq_search_workspace_bytes, tq_selftest_wait_timeout, tq_set_norm_dtype, tq_timer_enable,
+    tq_timer_read,
 )
 
 

@@ -69,6 +69,7 @@ _SIGS = {
     "tq_timer_enable": (_i, [_i]),
     "tq_timer_read": (_i, [ctypes.c_char_p, ctypes.POINTER(ctypes.c_double), _ip, _i]),
     "tq_last_status": (_i, [_vp, _vp]),
+    "tq_selftest_wait_timeout": (_i, [_vp, _i, _vp]),
     "tq_last_error": (ctypes.c_char_p, []),
 }
 for _name, (_res, _args) in _SIGS.items():
@@ -253,6 +254,11 @@ def tq_timer_read(name=None, forget=True):
     check(lib.tq_timer_read(name.encode() if name else None, ctypes.byref(ms), ctypes.byref(n), int(bool(forget))),
           "tq_timer_read")
     return ms.value, n.value
+
+
+def tq_selftest_wait_timeout(h, limit, stream=None):
+    """Makes one bounded device wait run out on purpose; the handle's next status is TQ_ETIMEOUT."""
+    check(lib.tq_selftest_wait_timeout(h, int(limit), _stream(stream)), "tq_selftest_wait_timeout")
 
 
 def tq_last_status(h, stream=None):

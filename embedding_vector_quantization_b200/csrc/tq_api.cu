@@ -645,6 +645,19 @@ int tq_internal_fail(int code, const char* fmt, ...) {
   return code;
 }
 
+namespace tqk {
+// The failure path of every bounded wait, on its own: thread 0 waits for phase 0 of a
+// barrier that expects one arrival and never gets it, gives up after `limit` polls and
+// records kErrTimeout, as a kernel does when a copy or a release never completes.
+__global__ void selftest_wait_kernel(int* err, int limit) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    bar_init(&bar, 1);
+    if (!bar_wait(&bar, 0, limit)) report_error(err, kErrTimeout);
+  }
+}
+}  // namespace tqk
+
 // ============================================================================
 extern "C" {
 
@@ -1204,6 +1217,13 @@ int tq_timer_read(const char* name, double* ms, int* launches, int forget) {
   if (ms) *ms += total;
   if (launches) *launches += count;
   return ok();
+}
+
+int tq_selftest_wait_timeout(const tq_handle* h, int limit, void* stream) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (limit < 1 || limit > (1 << 16)) return fail(TQ_EINVAL, "limit=%d outside 1..65536", limit);
+  tqk::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(h->derr, limit);
+  return launch_check("selftest_wait_kernel");
 }
 
 int tq_last_status(const tq_handle* h, void* stream) {

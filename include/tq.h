@@ -254,6 +254,14 @@ int tq_timer_read(const char* name, double* ms, int* launches, int forget);
  * (TQ_OK if nothing was recorded), or TQ_ECUDA if the stream reported an error. */
 int tq_last_status(const tq_handle* h, void* stream);
 
+/* Self-test of the device-side failure path. One thread of one CTA waits on a shared-memory
+ * barrier that no thread and no copy will complete, giving up after `limit` polls (each poll
+ * may suspend for at most about 20 us), and then records a wait timeout in h's device error
+ * word exactly as the kernels do when a copy or a release never arrives. The next
+ * tq_last_status(h) returns TQ_ETIMEOUT and clears the word; the CUDA context stays usable.
+ *  limit  1 .. 65536 (TQ_EINVAL otherwise). Asynchronous on `stream`. */
+int tq_selftest_wait_timeout(const tq_handle* h, int limit, void* stream);
+
 /* Message for the last failed call on this host thread ("" if none). */
 const char* tq_last_error(void);
 
