@@ -40,8 +40,10 @@ using amma::smem_u32;
 using amma::tma_bulk_g2s;
 
 constexpr int kQT = 16;          // queries per CTA (4 MMA column tiles of 4 queries x hi/lo)
-constexpr int kVB = 256;         // vectors per block (two 16-row MMA tiles per warp)
-constexpr int kStages = 3;       // slice stages
+constexpr int kRT = 3;           // 16-row MMA tiles per warp
+constexpr int kVB = 8 * 16 * kRT;  // vectors per block (384)
+constexpr int kBoxRows = 128;    // rows per TMA box (a box dimension is at most 256)
+constexpr int kStages = 2;       // slice stages
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kMaxD = 1536;      // codes_B = d / 4 <= 384
@@ -50,7 +52,7 @@ constexpr int kMaxK = 32;        // one list entry per lane
 constexpr int kMaxSteps = kMaxCodesB / 32 * 8;   // k-steps: 32-byte chunks x (4 shifts x 2 masks)
 constexpr int kSlice = 128;                       // bytes of a code row per TMA slice (the swizzle span)
 constexpr int kMaxSlices = kMaxCodesB / kSlice;
-constexpr int kSliceBytes = kVB * kSlice;         // 32 KB
+constexpr int kSliceBytes = kVB * kSlice;         // 48 KB
 
 struct Args {
   const float* qr;       // [nq][d] rotated queries
@@ -140,7 +142,8 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_c
     const int sl = J % nsl;
     uint64_t* bar = &sm.full[J % kStages];
     mbar_expect_tx(bar, (uint32_t)kSliceBytes);
-    tma_tile_2d(sm.stage[J % kStages], &cmap, sl * kSlice, (int)v0, bar);   // box {128 bytes, 256 rows}
+    for (int bx = 0; bx < kVB / kBoxRows; ++bx)   // boxes of {128 bytes, 128 rows}
+      tma_tile_2d(sm.stage[J % kStages] + bx * kBoxRows * kSlice, &cmap, sl * kSlice, (int)v0 + bx * kBoxRows, bar);
     issued = J + 1;
   };
   if (tid == 0)
@@ -187,14 +190,14 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_c
   }
   __syncthreads();
 
-  // this lane's rows of ldmatrix: row tile 0 at vr0, row tile 1 at vr0 + 16 (same row mod 8)
-  const int mat = lane >> 3, vr0 = 32 * warp + (lane & 7) + 8 * (mat >> 1);
+  // this lane's rows of ldmatrix: row tile r at vr0 + 16 r (the same row mod 8)
+  const int mat = lane >> 3, vr0 = 16 * kRT * warp + (lane & 7) + 8 * (mat >> 1);
   float ls[2] = {-INFINITY, -INFINITY};   // running top-k of queries 2w, 2w+1: lane j holds entry j
   int64_t li[2] = {-1, -1};
   for (int j = 0; j < nblk; ++j) {
     const int64_t v0 = c0 + (int64_t)j * kVB;
     const int nv = (int)min((int64_t)kVB, c1 - v0);
-    int acc1[2][4][4] = {}, acc16[2][4][4] = {};   // [row tile][column tile]
+    int acc1[kRT][4][4] = {}, acc16[kRT][4][4] = {};   // [row tile][column tile]
     for (int sl = 0; sl < nsl; ++sl) {
       const int J = j * nsl + sl;
       // warp-uniform (the guarded code is warp-collective)
@@ -212,14 +215,14 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_c
           // cw[m][0] = vector g word t, [1] = vector g word 4+t, [2] = vector g+8 word t, [3] = g+8 word 4+t
           // (16-byte unit u of a slice row sits at unit u ^ (row % 8))
           const int unit = ((c4 << 1) | (mat & 1)) ^ (vr0 & 7);
-          uint32_t cw[2][4];
-          ldsm_x4(cw[0], st + vr0 * kSlice + 16 * unit);
-          ldsm_x4(cw[1], st + (vr0 + 16) * kSlice + 16 * unit);
+          uint32_t cw[kRT][4];
+#pragma unroll
+          for (int m = 0; m < kRT; ++m) ldsm_x4(cw[m], st + (vr0 + 16 * m) * kSlice + 16 * unit);
 #pragma unroll
           for (int s = 0; s < 4; ++s) {
-            uint32_t x[2][4];
+            uint32_t x[kRT][4];
 #pragma unroll
-            for (int m = 0; m < 2; ++m)
+            for (int m = 0; m < kRT; ++m)
 #pragma unroll
               for (int i = 0; i < 4; ++i) x[m][i] = cw[m][i] >> s;
 #pragma unroll
@@ -230,7 +233,7 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_c
               for (int nt = 0; nt < 4; ++nt) {
                 const uint2 b = *reinterpret_cast<const uint2*>(&sm.qfrag[kk][nt][g][t][0]);
 #pragma unroll
-                for (int m = 0; m < 2; ++m) {
+                for (int m = 0; m < kRT; ++m) {
                   int(&acc)[4] = fam ? acc16[m][nt] : acc1[m][nt];
                   mma_s8(acc, x[m][0] & mk, x[m][2] & mk, x[m][1] & mk, x[m][3] & mk, b.x, b.y);
                 }
@@ -245,7 +248,7 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_c
     const bool aborted = __any_sync(0xffffffffu, *(volatile int*)&sm.abort_flag != 0);
     __syncthreads();   // the previous block's top-k pass is done with sm.sc
 #pragma unroll
-    for (int m = 0; m < 2; ++m)
+    for (int m = 0; m < kRT; ++m)
 #pragma unroll
       for (int nt = 0; nt < 4; ++nt) {
         const int ql = 4 * nt + t;
@@ -253,7 +256,7 @@ __global__ void __launch_bounds__(kThreads, 1) search_mma2_kernel(const __grid_c
         for (int r = 0; r < 2; ++r) {
           const int hi = 2 * r, lo = 2 * r + 1;
           const int dot = 128 * (acc1[m][nt][hi] + (acc16[m][nt][hi] >> 4)) + (acc1[m][nt][lo] + (acc16[m][nt][lo] >> 4));
-          const int vi = 32 * warp + 16 * m + g + 8 * r;
+          const int vi = 16 * kRT * warp + 16 * m + g + 8 * r;
           const float nrm = vi < nv ? load_norm(a.norms, a.norm_dtype, v0 + vi) : 0.f;
           sm.sc[ql][vi] = nrm * (sm.qc0[ql] + sm.qstep[ql] * (float)dot);
         }

@@ -356,16 +356,15 @@ int sm_count(int device) {
 // Split of the int8 tensor-core searches (one CTA per SM, qtile queries per CTA): the number
 // of database chunks makes chunks x query tiles a whole number of waves where it can, chunks
 // a multiple of 256 vectors.
-void search_mma_split(int nq, int qtile, int64_t n, int sms, int* nchunks, int64_t* chunk) {
-  static_assert(tqk::sm2::kVB == tqk::sm4::kVB, "one block size for both searches");
+void search_mma_split(int nq, int qtile, int vb, int64_t n, int sms, int* nchunks, int64_t* chunk) {
   const int64_t qt = (nq + qtile - 1) / qtile;
   int64_t a = sms, bq = qt;   // nc0 = sms / gcd(sms, qt): the fewest chunks giving whole waves
   while (bq) { const int64_t r = a % bq; a = bq; bq = r; }
   const int64_t nc0 = sms / a;
   int64_t nc = nc0 * std::max<int64_t>(1, (8 * (int64_t)sms + nc0 * qt / 2) / (nc0 * qt));
-  nc = std::max<int64_t>(1, std::min<int64_t>(nc, (n + tqk::sm2::kVB - 1) / tqk::sm2::kVB));
+  nc = std::max<int64_t>(1, std::min<int64_t>(nc, (n + vb - 1) / vb));
   int64_t ch = (n + nc - 1) / nc;
-  ch = (ch + tqk::sm2::kVB - 1) / tqk::sm2::kVB * tqk::sm2::kVB;
+  ch = (ch + vb - 1) / vb * vb;
   *chunk = ch;
   *nchunks = (int)((n + ch - 1) / ch);
 }
@@ -462,7 +461,7 @@ size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base
   int nc;
   int64_t ch;
   if (mma)
-    search_mma_split(nq, mma, n, sm_count(h->device), &nc, &ch);
+    search_mma_split(nq, mma, mma == tqk::sm2::kQT ? tqk::sm2::kVB : tqk::sm4::kVB, n, sm_count(h->device), &nc, &ch);
   else
     search_split(nq, n, &nc, &ch);
   if (nchunks) *nchunks = nc;
@@ -1140,7 +1139,7 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
     m.c0 = (float)h->cent[0]; m.w0 = (float)(h->cent[1] - h->cent[0]); m.w1 = (float)(h->cent[2] - h->cent[0]);
     m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
     CUtensorMap cmap;
-    if ((st = codes_map_2d(codes, n, h->codes_B, tqk::sm2::kSlice, tqk::sm2::kVB, &cmap))) return st;
+    if ((st = codes_map_2d(codes, n, h->codes_B, tqk::sm2::kSlice, tqk::sm2::kBoxRows, &cmap))) return st;
     const size_t msmem = tqk::sm2::smem_bytes();
     if (once_per_device(12, h->device))
       cudaFuncSetAttribute(tqk::sm2::search_mma2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
