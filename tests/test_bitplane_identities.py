@@ -1,0 +1,124 @@
+"""The arithmetic the int8 tensor-core kernels rely on, pinned on the CPU against the oracle's
+codebooks and its LSB-first packer ("Google TurboQuant: 6x KV-cache compression", "Stage 1":
+Lloyd-Max codebooks of the coordinate law; the cache layout packs index j at bits
+[j b, (j + 1) b) of a vector's little-endian bit stream):
+
+  * a 2-bit Lloyd-Max codebook is symmetric, hence affine in its two index bits:
+    c[idx] = c0 + (c1 - c0) b0 + (c2 - c0) b1;
+  * a 16-level one has only odd-degree Walsh terms in the +-1 variables of its index bits, so
+    c[idx] = c[0] + sum_S w_S beta_S(idx) over the four bits and the four three-bit parities;
+  * the word-level extraction of those 0/1 planes from packed code words ((w >> s) & 0x01010101
+    and & 0x10101010; for 4-bit nibbles the shifted copies combined by XOR) picks exactly the
+    planes of the right coordinates;
+  * a value rounded to a 15-bit integer splits exactly into int8 pieces hi * 128 + lo.
+"""
+
+import itertools
+
+import numpy as np
+import pytest
+
+from oracle import codebook, quant
+
+PLANES4 = [(0,), (1,), (2,), (3,), (0, 1, 2), (0, 1, 3), (0, 2, 3), (1, 2, 3)]
+
+
+def _bits(idx, k):
+    return (idx >> k) & 1
+
+
+def _beta(idx, plane):
+    v = 0
+    for k in plane:
+        v ^= _bits(idx, k)
+    return v
+
+
+@pytest.mark.parametrize("d", [64, 128, 256, 1536])
+def test_two_bit_codebook_is_affine_in_its_index_bits(d):
+    c, _ = codebook.lloyd_max(d, 2)
+    assert abs(c[3] - c[2] - c[1] + c[0]) <= 1e-15 * np.max(np.abs(c))
+    for idx in range(4):
+        rec = c[0] + (c[1] - c[0]) * _bits(idx, 0) + (c[2] - c[0]) * _bits(idx, 1)
+        assert abs(rec - c[idx]) <= 1e-15 * np.max(np.abs(c))
+
+
+@pytest.mark.parametrize("d", [64, 128, 256, 1536])
+def test_four_bit_codebook_has_only_odd_walsh_terms(d):
+    c, _ = codebook.lloyd_max(d, 4)
+    cmax = np.max(np.abs(c))
+    # Walsh coefficients a_T = 1/16 sum_idx c[idx] prod_{i in T} (2 b_i - 1)
+    a = {}
+    for T in range(16):
+        sgn = [np.prod([2 * _bits(idx, i) - 1 for i in range(4) if T >> i & 1]) for idx in range(16)]
+        a[T] = float(np.dot(c, sgn)) / 16.0
+        if bin(T).count("1") % 2 == 0:
+            assert abs(a[T]) <= 1e-14 * cmax, (T, a[T])
+    # the plane form: c[idx] = c[0] + sum_S w_S beta_S(idx), w_S = 2 a_{mask(S)} (from
+    # prod (2 b_i - 1) over an odd set = 1 - 2 beta for the four bits and the three-bit parities)
+    masks = [sum(1 << i for i in p) for p in PLANES4]
+    w = [2.0 * a[m] for m in masks]
+    assert abs(a[15]) <= 1e-14 * cmax   # the 4-bit term is even: it vanishes as well
+    for idx in range(16):
+        rec = c[0] + sum(ws * _beta(idx, p) for ws, p in zip(w, PLANES4))
+        assert abs(rec - c[idx]) <= 1e-13 * cmax, (idx, rec, c[idx])
+
+
+def _plane_words(w, S):
+    """The kernels' plane S of every nibble of a 32-bit word (bit 0: low nibble, bit 4: high)."""
+    x1, x2, x3 = w >> 1, w >> 2, w >> 3
+    return [w, x1, x2, x3, w ^ x1 ^ x2, w ^ x1 ^ x3, w ^ x2 ^ x3, x1 ^ x2 ^ x3][S]
+
+
+def test_four_bit_plane_extraction_matches_the_packed_layout():
+    rs = np.random.default_rng(0)
+    idx = rs.integers(0, 16, size=(5, 128))
+    words = quant.pack(idx, 4).view("<u4")          # 32 B per vector = 8 words of 8 nibbles
+    for v in range(idx.shape[0]):
+        for wi, w in enumerate(words[v].tolist()):
+            for S, plane in enumerate(PLANES4):
+                p = _plane_words(w, S)
+                for byte in range(4):
+                    coord = 8 * wi + 2 * byte          # byte k of a word holds coordinates 2k (low), 2k + 1
+                    lo = (p & (0x01010101)) >> (8 * byte) & 0xFF
+                    hi = (p & (0x10101010)) >> (8 * byte) & 0xFF
+                    assert lo == _beta(idx[v, coord], plane)
+                    assert hi == 16 * _beta(idx[v, coord + 1], plane)
+
+
+def test_two_bit_plane_extraction_matches_the_packed_layout():
+    rs = np.random.default_rng(1)
+    idx = rs.integers(0, 4, size=(5, 128))
+    words = quant.pack(idx, 2).view("<u4")          # 32 B per vector = 8 words of 16 codes
+    for v in range(idx.shape[0]):
+        for wi, w in enumerate(words[v].tolist()):
+            for s in range(4):
+                x = w >> s
+                for byte in range(4):
+                    # bit s of a byte: code 4 byte-lane + s // 2 of the word's byte, plane s % 2;
+                    # bit s + 4: code + 2, same plane
+                    code_lo = 16 * wi + 4 * byte + s // 2
+                    code_hi = code_lo + 2
+                    lo = (x & 0x01010101) >> (8 * byte) & 0xFF
+                    hi = (x & 0x10101010) >> (8 * byte) & 0xFF
+                    assert lo == _bits(idx[v, code_lo], s % 2)
+                    assert hi == 16 * _bits(idx[v, code_hi], s % 2)
+
+
+def test_fifteen_bit_values_split_exactly_into_int8_pieces():
+    # the kernels round a value to xi in [-16256, 16256], then hi = xi / 128 rounded half away
+    # from zero and lo = xi - 128 hi
+    for xi in range(-16256, 16257):
+        hi = (xi + 64) >> 7 if xi >= 0 else -((-xi + 64) >> 7)
+        lo = xi - 128 * hi
+        assert -127 <= hi <= 127 and -64 <= lo <= 64
+        assert 128 * hi + lo == xi
+
+
+def test_int32_accumulation_cannot_overflow_at_the_largest_shapes():
+    # 4-bit search at d = 1536: 8 planes x d coordinates of 0/1 (or 16) bytes against |piece| <= 127
+    worst = 16 * 127 * 8 * 1536
+    assert worst < 2 ** 31
+    # the x16 family's sums are multiples of 16, so the exact division by 16 loses nothing
+    for parts in itertools.product([0, 16, 32, 48], repeat=3):
+        assert sum(parts) % 16 == 0
