@@ -44,7 +44,7 @@ WORKLOAD_NAME = ("GQA decode step, TurboQuant prod 3-bit (2-bit Lloyd-Max + 1-bi
                  "and 2 outlier channels")
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) of one attn_prod2_kernel launch on this workload, from
-# `ncu --set full` (profiles/attn_prod2_decode_prod3_ctx32768.md); set to None whenever
+# `ncu --set full` (the attention kernel's profile summary in the repository); set to None whenever
 # that kernel changes until it is captured again.
 ATTN_TRAFFIC_BYTES = 27350272
 
