@@ -30,6 +30,8 @@ that implements it. Modules:
 * :mod:`oracle.codebook` -- Lloyd-Max codebook on the sphere-coordinate density.
 * :mod:`oracle.quant`    -- encode (norm, rotate, bucketize, pack), QJL sketch, dequantize.
 * :mod:`oracle.ops`      -- inner-product scores, decode attention, top-k search.
+* :mod:`oracle.polar`    -- PolarQuant's recursive polar transform and its angle codebooks
+  ("PolarQuant explainer" (aibr.jp); the next row after the TurboQuant path: oracle only so far).
 """
 
-from . import rng, rotation, codebook, quant, ops  # noqa: F401
+from . import rng, rotation, codebook, quant, ops, polar  # noqa: F401
