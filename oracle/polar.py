@@ -170,6 +170,20 @@ def decode(idx, n, Pi, books):
     return np.asarray(n, dtype=np.float64)[:, None] * (y_hat @ np.asarray(Pi))
 
 
+def score(q, idx, n, Pi, books):
+    """<q, x_hat> for each encoded row without reconstructing it: with q' = Pi q, pair i of level 1
+    contributes S_i = q'_2i cos(theta_i) + q'_2i+1 sin(theta_i) per unit radius, and each further
+    level folds two partial scores as S = S_a cos(psi) + S_b sin(psi); the score is ||x|| times the
+    top value. q [d], idx per-level index arrays [n, d / 2^l]."""
+    qp = np.asarray(Pi) @ np.asarray(q, dtype=np.float64)
+    c0 = books[0][0][idx[0]]
+    s = qp[0::2][None, :] * np.cos(c0) + qp[1::2][None, :] * np.sin(c0)
+    for lv in range(1, len(idx)):
+        psi = books[lv][0][idx[lv]]
+        s = s[:, 0::2] * np.cos(psi) + s[:, 1::2] * np.sin(psi)
+    return np.asarray(n, dtype=np.float64) * s[:, 0]
+
+
 def bits_per_vector(d: int, bits) -> int:
     nl = n_levels(d)
     bits = [bits] * nl if np.isscalar(bits) else list(bits)

@@ -104,3 +104,16 @@ def test_encode_decode_distortion_falls_with_bits_and_vanishes_at_high_precision
     xh = polar.decode(e["idx"], e["n_exact"], Pi, books)
     assert np.mean(np.sum((xh - x) ** 2, 1) / np.sum(x ** 2, 1)) < 1e-3
     assert polar.bits_per_vector(d, [4, 2, 2, 2, 2, 2]) == 32 * 4 + 31 * 2
+
+
+@pytest.mark.parametrize("d,bits", [(8, 2), (128, [4, 2, 2, 2, 2, 2, 2])])
+def test_score_up_the_tree_equals_the_dot_product_with_the_reconstruction(d, bits):
+    Pi = rotation.rotation(d, 5, 0)[0]
+    rs = np.random.default_rng(d)
+    x = rs.standard_normal((40, d)) * 2.0
+    q = rs.standard_normal(d)
+    books = polar.codebooks(d, bits)
+    e = polar.encode(x, Pi, books)
+    xh = polar.decode(e["idx"], e["n_exact"], Pi, books)
+    got = polar.score(q, e["idx"], e["n_exact"], Pi, books)
+    assert np.allclose(got, xh @ q, rtol=1e-12, atol=1e-12 * np.abs(xh @ q).max())
