@@ -42,11 +42,22 @@ PACKED_BYTES_PER_TOKEN = 2 * (32 + 16 + 2 + 2)   # K and V: 2-bit codes + sign b
 WORKLOAD_NAME = ("GQA decode step, TurboQuant prod 3-bit (2-bit Lloyd-Max + 1-bit QJL m=128), d=128, "
                  "B=1, 8 KV heads / 32 query heads, context 32768, bf16 K/V with lognormal channel scales "
                  "and 2 outlier channels")
+# Arithmetic of the timed path: int8 x int8 -> int32 tensor-core MMAs on 15-bit fixed-point queries
+# and 14-bit fixed-point softmax weights, fp32 softmax, combine and output.
+DTYPE = "s8xs8->s32 MMA (15/14-bit fixed-point operands), f32 softmax/combine"
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) of one attn_prod2_kernel launch on this workload, from
 # `ncu --set full` (the attention kernel's profile summary in the repository); set to None whenever
 # that kernel changes until it is captured again.
 ATTN_TRAFFIC_BYTES = 27350272
+
+
+def decode_config(world):
+    """The `config` object of the decode-step line (identical in both arms)."""
+    return {"workload": WORKLOAD_NAME, "B": W["B"], "Hkv": W["Hkv"], "Hq": W["Hq"], "context": W["L"],
+            "d": W["d"], "bits": "2 MSE + 1 QJL (m=128)", "l2": "flushed between steps (256 MB write)",
+            "step": "tq_decode_step (append K and V, rotate q, attend, advance len), one CUDA graph replay",
+            "parallelism": f"independent replica per GPU x{world}"}
 
 
 def parse_args():
@@ -141,7 +152,7 @@ class OracleSample:
 
     def __init__(self, group_heads=1):
         import numpy as np
-        from embedding_vector_quantization_b200 import synth
+        import workloads as synth
         from oracle import codebook, ops, quant, rotation
         self.np, self.ops, self.quant = np, ops, quant
         d, m, L = W["d"], W["m"], W["L"]
@@ -215,7 +226,7 @@ def run_reference(args):
     line = {"impl": "reference", "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": args.gpus,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * t_total / max(args.steps, 1),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": WORKLOAD_NAME, "sample": sample},
+            "config": decode_config(int(os.environ.get("WORLD_SIZE", "1"))),
             "cpu_baseline": {"value": value, "unit": "GB/s", "cores": threads, "kind": "oracle", "sample": sample},
             "e2e": {"value": value, "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
@@ -228,7 +239,7 @@ def run_tq(args):
     import torch.distributed as dist
     import embedding_vector_quantization_b200 as tq
     from embedding_vector_quantization_b200 import dist as tqdist
-    from embedding_vector_quantization_b200 import synth
+    import workloads as synth
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))
@@ -421,11 +432,8 @@ def run_tq(args):
     line = {
         "metric": METRIC, "value": value, "unit": "GB/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": max_ms / args.steps, "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "f32", "data": "synthetic",
-        "config": {"workload": WORKLOAD_NAME, "B": B, "Hkv": Hkv, "Hq": Hq, "context": L, "d": d,
-                   "bits": "2 MSE + 1 QJL (m=128)", "l2": "flushed between steps (256 MB write)",
-                   "step": "tq_decode_step (append K and V, rotate q, attend, advance len), one CUDA graph replay",
-                   "parallelism": f"independent replica per GPU x{world}"},
+        "vs_baseline": None, "dtype": DTYPE, "data": "synthetic",
+        "config": decode_config(world),
         "keys_scored_per_s": keys_s,
         "query_key_pairs_per_s": keys_s * (Hq // Hkv),
         "vectors_encoded_per_s": enc_vps,

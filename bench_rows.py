@@ -373,7 +373,8 @@ def run_attn4(args):
     ach = bytes_step / (split_ms / max(split_n, 1) / 1e3) / 1e9
     cfg = {"workload": "GQA decode step, TurboQuant MSE 4-bit K and V, d=128, B=4, 8 KV heads / 32 query heads, "
                        "context 131072, bf16 K/V N(0,1) x U(0.5,2) per (sequence, head)",
-           "B": B, "Hkv": Hkv, "Hq": Hq, "context": L, "d": d, "dtype": "f32",
+           "B": B, "Hkv": Hkv, "Hq": Hq, "context": L, "d": d,
+           "dtype": "s8xs8->s32 MMA (15-bit fixed-point queries, 14-bit weights, Walsh planes), f32 softmax/combine",
            "l2": "not flushed: each step reads 553.6 MB of packed K/V (> 126 MB L2)",
            "step": "tq_decode_step, one CUDA graph replay; len reset outside the timed bracket"}
     roof = {"bound": "hbm", "kernel": "attn_mse4_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
@@ -558,7 +559,7 @@ def run_compare(args):
     import torch
     import torch.nn.functional as F
     import embedding_vector_quantization_b200 as tq
-    from embedding_vector_quantization_b200 import synth
+    import workloads as synth
     Wc = bench.W
     B, Hkv, Hq, L, d, m = Wc["B"], Wc["Hkv"], Wc["Hq"], Wc["L"], Wc["d"], Wc["m"]
     dev = torch.device("cuda", 0)

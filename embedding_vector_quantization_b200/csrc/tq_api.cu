@@ -321,6 +321,22 @@ int check_cache(const tq_handle* h, const tq_cache* c, const char* name) {
   return TQ_OK;
 }
 
+// TQ_SPLITK=<n> (tests and tuning): forces the context chunk of the split kernels to n
+// tokens (attention, scores) or vectors (search), rounded up to the kernel's block and
+// clamped to its limits; 0 or unset keeps the built-in policy. The workspace size
+// functions see the same value, so set it before sizing a workspace.
+int64_t splitk_override() {
+  const char* e = std::getenv("TQ_SPLITK");
+  if (!e || !*e) return 0;
+  const long long v = std::atoll(e);
+  return v > 0 ? (int64_t)v : 0;
+}
+
+int64_t round_chunk(int64_t v, int64_t blk, int64_t lo, int64_t hi) {
+  v = (v + blk - 1) / blk * blk;
+  return std::min<int64_t>(hi, std::max<int64_t>(lo, v));
+}
+
 // Attention split policy (shared by every attention kernel): about two CTAs per
 // SM, chunks a multiple of 128 tokens and at most 1024 tokens long.
 void attn_split(int B, int Hkv, int64_t L_cap, int* nsplit, int64_t* chunk) {
@@ -328,6 +344,7 @@ void attn_split(int B, int Hkv, int64_t L_cap, int* nsplit, int64_t* chunk) {
   const int64_t ns = std::max<int64_t>(1, (2 * 148 + units - 1) / units);
   int64_t ch = (L_cap + ns - 1) / ns;
   ch = std::min<int64_t>(1024, std::max<int64_t>(128, (ch + 127) / 128 * 128));
+  if (const int64_t f = splitk_override()) ch = round_chunk(f, 128, 128, 1024);
   *chunk = ch;
   *nsplit = (int)((L_cap + ch - 1) / ch);
 }
@@ -338,6 +355,7 @@ void search_split(int nq, int64_t n, int* nchunks, int64_t* chunk) {
   nc = std::max<int64_t>(1, std::min<int64_t>(nc, (n + tqk::kSK - 1) / tqk::kSK));
   int64_t ch = (n + nc - 1) / nc;
   ch = (ch + tqk::kSK - 1) / tqk::kSK * tqk::kSK;
+  if (const int64_t f = splitk_override()) ch = round_chunk(f, tqk::kSK, tqk::kSK, (n + tqk::kSK - 1) / tqk::kSK * tqk::kSK);
   *chunk = ch;
   *nchunks = (int)((n + ch - 1) / ch);
 }
@@ -365,6 +383,7 @@ void search_mma_split(int nq, int qtile, int vb, int64_t n, int sms, int* nchunk
   nc = std::max<int64_t>(1, std::min<int64_t>(nc, (n + vb - 1) / vb));
   int64_t ch = (n + nc - 1) / nc;
   ch = (ch + vb - 1) / vb * vb;
+  if (const int64_t f = splitk_override()) ch = round_chunk(f, vb, vb, (n + vb - 1) / vb * vb);
   *chunk = ch;
   *nchunks = (int)((n + ch - 1) / ch);
 }
@@ -855,6 +874,7 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const 
     const int64_t target = 8 * 3 * (int64_t)sm_count(hk->device);
     int64_t chunk = ((units * k->L_cap + target - 1) / target + 255) / 256 * 256;
     chunk = std::max<int64_t>(256, std::min<int64_t>(chunk, (k->L_cap + 255) / 256 * 256));
+    if (const int64_t f = splitk_override()) chunk = round_chunk(f, 256, 256, (k->L_cap + 255) / 256 * 256);
     const int64_t nsp = (k->L_cap + chunk - 1) / chunk;
     tqk::amma::ScoreArgs m{};
     m.qr = w.qr; m.qs = w.qs; m.B = B; m.Hq = Hq; m.Hkv = Hkv;
@@ -877,6 +897,7 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const 
   a.L_cap = k->L_cap; a.len = len; a.logits = logits;
   int64_t ns = std::max<int64_t>(1, std::min<int64_t>((8 * 148 + units - 1) / units, (k->L_cap + 127) / 128));
   a.chunk = ((k->L_cap + ns - 1) / ns + 127) / 128 * 128;
+  if (const int64_t f = splitk_override()) a.chunk = round_chunk(f, 128, 128, (k->L_cap + 127) / 128 * 128);
   ns = (k->L_cap + a.chunk - 1) / a.chunk;
   const int G = Hq / Hkv;
   const size_t smem = ((size_t)G * (hk->d + hk->m) + 16) * 4;

@@ -11,7 +11,10 @@
 //
 // The array's address is a device address that host code cannot name
 // directly; it is looked up once per device with cudaGetSymbolAddress while
-// that device is current, on the first call made on that device.
+// that device is current, on the first call made on that device. The address
+// belongs to the device's context: after cudaDeviceReset (or anything else that
+// destroys and re-creates the primary context) it is stale, as are all handles
+// created before; the library must not be used again in that process.
 
 #include <cuda_runtime.h>
 
@@ -36,8 +39,10 @@ extern "C" int tq_attn_decode_noalloc(const tq_handle* hk, const tq_handle* hv, 
                                       int B, int Hq, int Hkv, const tq_cache* k, const tq_cache* v,
                                       const int32_t* len, float scale, float* out, void* stream) {
   if (!hk || !hv) return tq_internal_fail(TQ_EINVAL, "tq_attn_decode_noalloc: handle is NULL");
-  if (!k) return tq_internal_fail(TQ_EINVAL, "tq_attn_decode_noalloc: key cache is NULL");
   if (B < 0 || Hq < 1 || Hkv < 1) return tq_internal_fail(TQ_EINVAL, "tq_attn_decode_noalloc: bad B/Hq/Hkv");
+  // nothing to attend: tq_attn_decode checks the rest and returns without touching any buffer
+  if (B == 0) return tq_attn_decode(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, len, scale, out, nullptr, 0, stream);
+  if (!k) return tq_internal_fail(TQ_EINVAL, "tq_attn_decode_noalloc: key cache is NULL");
   const size_t need = tq_attn_workspace_bytes(hk, hv, B, Hq, Hkv, k->L_cap);
   if (need == 0) return tq_internal_fail(TQ_EINVAL, "tq_attn_decode_noalloc: invalid shape");
   if (need > kNoAllocScratchBytes)

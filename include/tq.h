@@ -194,8 +194,12 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
  * the library holds it until the process exits); nothing is allocated.
  *  - A shape whose tq_attn_workspace_bytes exceeds 4 MiB is rejected with
  *    TQ_EINVAL (e.g. B*Hq*nsplit*(d+m+2)*4 bytes of partial sums too large).
+ *  - B == 0 returns TQ_OK without touching any buffer, as tq_attn_decode does.
  *  - The first call on a device looks up the array's device address with that
- *    device current; make that first call before any stream capture.
+ *    device current; make that first call before any stream capture. The
+ *    address belongs to the device's primary context: after cudaDeviceReset
+ *    it is stale (as is every handle), so the library must not be used again
+ *    in that process.
  *  - All calls share the one array and nothing in it needs to start at zero
  *    (every call rewrites what it reads). Calls that overlap on the GPU (other
  *    streams, other host threads) race on it: serialise them. */

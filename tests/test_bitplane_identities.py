@@ -122,3 +122,10 @@ def test_int32_accumulation_cannot_overflow_at_the_largest_shapes():
     # the x16 family's sums are multiples of 16, so the exact division by 16 loses nothing
     for parts in itertools.product([0, 16, 32, 48], repeat=3):
         assert sum(parts) % 16 == 0
+
+
+@pytest.mark.parametrize("bits,d", [(1, 128), (2, 128), (2, 1536), (4, 128), (4, 96)])
+def test_fast_layout_decoder_of_the_tests_matches_the_oracle_unpack(bits, d):
+    from gpu_util import unpack_fast
+    rows = np.random.default_rng(bits * 1000 + d).integers(0, 256, size=(300, (d * bits + 7) // 8), dtype=np.uint8)
+    assert np.array_equal(unpack_fast(rows, d, bits).astype(np.int64), quant.unpack(rows, d, bits))

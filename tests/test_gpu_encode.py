@@ -109,7 +109,7 @@ def test_pack_indices_bit_exact(tq):
 
 def test_config1_encode_full(tq):
     """MSE-only d=128, b=3, 4096 fp32 N(0,1) keys (seed 0): parity and empirical distortion."""
-    from embedding_vector_quantization_b200 import synth
+    import workloads as synth
     x = synth.mse_keys()
     frac, _ = _encode_and_check(tq, x, 128, 3, seed=0)
     assert frac < 1e-4

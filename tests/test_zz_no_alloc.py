@@ -15,8 +15,6 @@ import numpy as np
 import pytest
 import torch
 
-from gpu_util import ATTN_RTOL
-
 pytestmark = pytest.mark.gpu
 
 
@@ -49,9 +47,9 @@ def _both(tq, hk, hv, kc, vc, q, lens):
 
 
 def _close(ref, got):
-    for b in range(ref.shape[0]):
-        for h in range(ref.shape[1]):
-            assert np.linalg.norm(got[b, h] - ref[b, h]) <= ATTN_RTOL * max(np.linalg.norm(ref[b, h]), 1e-30)
+    # the same kernels with the same split run on both paths (the split depends on the shape only),
+    # so the outputs must agree bit for bit; a stale or misplaced partial would show here
+    assert np.array_equal(ref, got)
 
 
 def test_noalloc_matches_workspace_entry_point_twice(tq):
@@ -68,6 +66,15 @@ def test_noalloc_matches_workspace_entry_point_twice(tq):
     ref2, got2 = _both(tq, hk2, hv2, kc2, vc2, q2, lens2)
     _close(ref2, got2)
     assert hk.status() == tq.TQ_OK and hk2.status() == tq.TQ_OK
+
+
+def test_noalloc_empty_batch_is_a_no_op(tq):
+    # B == 0: TQ_OK without touching anything, like tq_attn_decode (whose caches may then be NULL)
+    hk = tq.Handle(128, 3, 0, qjl_m=128)
+    hv = tq.Handle(128, 3, 1, qjl_m=128)
+    status = tq._lib.lib.tq_attn_decode_noalloc(hk.ptr, hv.ptr, None, tq.TQ_F32, 0, 8, 2, None, None, None,
+                                                ctypes.c_float(0.1), None, None)
+    assert status == tq.TQ_OK
 
 
 def test_noalloc_rejects_shapes_beyond_its_scratch(tq):

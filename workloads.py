@@ -1,4 +1,4 @@
-"""Seeded synthetic inputs for the five workloads (shared by tests, bench and the oracle checks).
+"""Seeded synthetic inputs for the five workloads (shared by the tests, the bench and the oracle checks).
 
 This module draws inputs only; it holds none of the method's arithmetic.
 Every tensor comes from ``torch.Generator('cpu').manual_seed(seed)`` so the
@@ -70,3 +70,21 @@ def stream_step(t, B=64, Hkv=8, Hq=32, d=128, seed0=11):
     tok = torch.randn(B, Hkv, d, generator=g).to(torch.bfloat16)
     q = torch.randn(B, Hq, d, generator=g)
     return tok, q
+
+
+def random_rows(shape, row_bytes, seed):
+    """Packed rows [*shape, row_bytes] of uniformly random bytes (numpy uint8). Every bit
+    pattern is a valid row of codes or sign bits, so such rows stand in for an encoded cache
+    where a test needs full-size caches faster than an fp64 encode can produce them."""
+    import numpy as np
+    return np.random.default_rng(seed).integers(0, 256, size=tuple(shape) + (row_bytes,), dtype=np.uint8)
+
+
+def random_norms(shape, d, seed, scale=None, dtype="float16"):
+    """Norms [*shape] of Gaussian vectors in R^d: sqrt(chi^2_d) times an optional per-row scale
+    (numpy array broadcast to shape), stored in `dtype` (numpy)."""
+    import numpy as np
+    n = np.sqrt(np.random.default_rng(seed).chisquare(d, size=tuple(shape)))
+    if scale is not None:
+        n = n * scale
+    return n.astype(dtype)
