@@ -28,7 +28,8 @@ that implements it. Modules:
 * :mod:`oracle.rng`      -- SplitMix64 + Box-Muller Gaussian stream (spec).
 * :mod:`oracle.rotation` -- seeded Haar rotation Pi (QR of a Gaussian) and QJL matrix S.
 * :mod:`oracle.codebook` -- Lloyd-Max codebook on the sphere-coordinate density.
-* :mod:`oracle.quant`    -- encode (norm, rotate, bucketize, pack), QJL sketch, dequantize.
+* :mod:`oracle.quant`    -- encode (norm, rotate, bucketize, pack), QJL sketch, dequantize;
+  the QJL-only 1-bit encode (sign sketch of the whole vector plus its norm).
 * :mod:`oracle.ops`      -- inner-product scores, decode attention, top-k search.
 * :mod:`oracle.polar`    -- PolarQuant's recursive polar transform and its angle codebooks
   ("PolarQuant explainer" (aibr.jp); the next row after the TurboQuant path: oracle only so far).

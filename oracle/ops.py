@@ -6,7 +6,9 @@
   efficiency" (hakusoku.com), section "QJL": a full-precision query is
   combined with low-precision data). MSE stage: s = n <Pi q, c[idx]>, which is
   <q, x_hat> rewritten with Pi orthogonal. Prod adds the QJL term of
-  :func:`oracle.quant.qjl_estimate` with the stored residual norm.
+  :func:`oracle.quant.qjl_estimate` with the stored residual norm. QJL-only
+  rows (no MSE bits) score with that term alone, the norm in place of the
+  residual norm.
 * Decode attention: softmax(q K^T / sqrt(d_k)) V over the cached keys and
   values (gemilab.net, sections "Scaled dot-product attention" and "Why the
   KV cache exists"). Reading taken: grouped-query attention maps query head h
@@ -21,7 +23,7 @@ Everything is fp64. Test infrastructure only; see the package docstring.
 
 import numpy as np
 
-from .quant import QJL_SCALE, dequantize
+from .quant import QJL_SCALE, dequantize, dequantize_qjl, qjl_estimate
 
 
 def score_mse(q, idx, n_stored, Pi, centroids):
@@ -40,6 +42,23 @@ def score_prod(q, idx, n_stored, sigma, rnorm_stored, Pi, S, centroids):
     return score_mse(q, idx, n_stored, Pi, centroids) + qjl
 
 
+def score_qjl(q, sigma, n_stored, S):
+    """QJL-only scores (sign sketch of the whole key plus its norm): n sqrt(pi/2)/m <S q, 2 sigma - 1>
+    ("TurboQuant: redefining AI efficiency" (hakusoku.com), section "QJL")."""
+    q = np.asarray(q, dtype=np.float64)
+    return qjl_estimate(q, np.asarray(S) @ q, sigma, n_stored, np.asarray(S).shape[0])
+
+
+def _scores(q, kq, b, hk, L):
+    """Scores of one query against rows 0 .. L-1 of cache (b, hk): MSE, prod or QJL-only."""
+    if "idx" not in kq:
+        return score_qjl(q, kq["sigma"][b, hk, :L], kq["n"][b, hk, :L], kq["S"])
+    if "sigma" in kq:
+        return score_prod(q, kq["idx"][b, hk, :L], kq["n"][b, hk, :L], kq["sigma"][b, hk, :L],
+                          kq["rnorm"][b, hk, :L], kq["Pi"], kq["S"], kq["c"])
+    return score_mse(q, kq["idx"][b, hk, :L], kq["n"][b, hk, :L], kq["Pi"], kq["c"])
+
+
 def softmax_attention(q, K, V, scale):
     """Textbook softmax(scale * q K^T) V for one query q [d]; K, V are [L, d] (fp64)."""
     logits = scale * (np.asarray(K, dtype=np.float64) @ np.asarray(q, dtype=np.float64))
@@ -53,12 +72,13 @@ def decode_attention(q, kq, vq, lens, scale):
 
     q: [B, Hq, d]. kq / vq: dicts describing one quantized cache each, with keys
     ``idx`` [B, Hkv, L, d], ``n`` [B, Hkv, L] (stored norms), ``Pi``, ``c`` and,
-    for prod caches, ``sigma`` [B, Hkv, L, m], ``rnorm`` [B, Hkv, L], ``S``.
+    for prod caches, ``sigma`` [B, Hkv, L, m], ``rnorm`` [B, Hkv, L], ``S``. A
+    QJL-only cache has no ``idx``: ``sigma``, ``n`` and ``S`` only.
     Returns o [B, Hq, d].
     """
     q = np.asarray(q, dtype=np.float64)
     B, Hq, d = q.shape
-    Hkv = kq["idx"].shape[1]
+    Hkv = kq["n"].shape[1]
     group = Hq // Hkv
     out = np.zeros((B, Hq, d))
     for b in range(B):
@@ -73,6 +93,8 @@ def decode_attention(q, kq, vq, lens, scale):
 
 
 def _dequant_rows(cq, b, hk, L):
+    if "idx" not in cq:
+        return dequantize_qjl(cq["sigma"][b, hk, :L], cq["n"][b, hk, :L], cq["S"])
     sig = cq.get("sigma")
     return dequantize(cq["idx"][b, hk, :L], cq["n"][b, hk, :L], cq["Pi"], cq["c"],
                       None if sig is None else sig[b, hk, :L],
@@ -91,21 +113,16 @@ def decode_attention_streaming(q, kq, vq, lens, scale, chunk=1000):
     """
     q = np.asarray(q, dtype=np.float64)
     B, Hq, d = q.shape
-    Hkv = kq["idx"].shape[1]
+    Hkv = kq["n"].shape[1]
     group = Hq // Hkv
     out = np.zeros((B, Hq, d))
-    cv = np.asarray(vq["c"], dtype=np.float64)
+    v_qjl_only = "idx" not in vq
+    cv = None if v_qjl_only else np.asarray(vq["c"], dtype=np.float64)
     for b in range(B):
         L = int(lens[b])
         for h in range(Hq):
             hk = h // group
-            if "sigma" in kq:
-                s_all = score_prod(q[b, h], kq["idx"][b, hk, :L], kq["n"][b, hk, :L],
-                                   kq["sigma"][b, hk, :L], kq["rnorm"][b, hk, :L],
-                                   kq["Pi"], kq["S"], kq["c"])
-            else:
-                s_all = score_mse(q[b, h], kq["idx"][b, hk, :L], kq["n"][b, hk, :L],
-                                  kq["Pi"], kq["c"])
+            s_all = _scores(q[b, h], kq, b, hk, L)
             parts = []
             for lo in range(0, L, chunk):
                 hi = min(L, lo + chunk)
@@ -113,16 +130,18 @@ def decode_attention_streaming(q, kq, vq, lens, scale, chunk=1000):
                 mx = np.max(lg)
                 p = np.exp(lg - mx)
                 w = p * np.asarray(vq["n"][b, hk, lo:hi], dtype=np.float64)
-                acc = w @ cv[vq["idx"][b, hk, lo:hi]]
+                acc = np.zeros(d) if v_qjl_only else w @ cv[vq["idx"][b, hk, lo:hi]]
                 acc_s = None
                 if "sigma" in vq:
-                    ws = p * np.asarray(vq["rnorm"][b, hk, lo:hi], dtype=np.float64)
+                    # QJL-only values: the norm is the projected vector's own norm
+                    rn = vq["n"] if v_qjl_only else vq["rnorm"]
+                    ws = p * np.asarray(rn[b, hk, lo:hi], dtype=np.float64)
                     acc_s = ws @ (2.0 * np.asarray(vq["sigma"][b, hk, lo:hi], dtype=np.float64) - 1.0)
                 parts.append((mx, np.sum(p), acc, acc_s))
             M = max(pt[0] for pt in parts)
             den = sum(pt[1] * np.exp(pt[0] - M) for pt in parts)
             acc = sum(pt[2] * np.exp(pt[0] - M) for pt in parts)
-            o = vq["Pi"].T @ acc
+            o = np.zeros(d) if v_qjl_only else vq["Pi"].T @ acc
             if "sigma" in vq:
                 acc_s = sum(pt[3] * np.exp(pt[0] - M) for pt in parts)
                 m = vq["S"].shape[0]

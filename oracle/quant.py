@@ -134,3 +134,31 @@ def dequantize(idx, n, Pi, centroids, sigma=None, rnorm=None, S=None):
     m = S.shape[0]
     pm = 2.0 * np.asarray(sigma, dtype=np.float64) - 1.0
     return xh + (np.asarray(rnorm, dtype=np.float64) * QJL_SCALE / m)[:, None] * (pm @ S)
+
+
+def encode_qjl(x, S, norm_dtype="f16"):
+    """QJL-only encode: one sign bit per Gaussian projection of the whole vector, plus its norm.
+
+    "TurboQuant: redefining AI efficiency" (hakusoku.com), section "QJL: zero-overhead
+    1-bit compression": a random Johnson-Lindenstrauss projection keeps only each
+    coordinate's sign, with no per-block constants; "TurboQuant / PolarQuant / QJL
+    technical deep dive" (gemilab.net), section "QJL".
+
+    Readings taken: the sketch is the prod stage with no MSE bits, i.e. the residual of a
+    zero reconstruction, r = x; sigma_j = 1 iff (S x)_j >= 0 (sign(0) = +1, so a zero
+    vector has every bit set); the one stored scalar is ||x|| in the handle's norm dtype,
+    which plays the role of the residual norm in the estimator. Returns dict(sigma, z,
+    n_exact, n_stored).
+    """
+    x = np.asarray(x, dtype=np.float64)
+    z = x @ np.asarray(S, dtype=np.float64).T
+    n = norms(x)
+    return {"sigma": (z >= 0).astype(np.int64), "z": z, "n_exact": n, "n_stored": n.astype(_DTYPES[norm_dtype])}
+
+
+def dequantize_qjl(sigma, n, S):
+    """Vector estimate of a QJL-only row: x_tilde = n sqrt(pi/2)/m S^T (2 sigma - 1) (unbiased over S)."""
+    S = np.asarray(S, dtype=np.float64)
+    m = S.shape[0]
+    pm = 2.0 * np.asarray(sigma, dtype=np.float64) - 1.0
+    return (np.asarray(n, dtype=np.float64) * QJL_SCALE / m)[:, None] * (pm @ S)
