@@ -188,3 +188,49 @@ def bits_per_vector(d: int, bits) -> int:
     nl = n_levels(d)
     bits = [bits] * nl if np.isscalar(bits) else list(bits)
     return sum((d >> lv) * b for lv, b in zip(range(1, nl + 1), bits))
+
+
+# ---------------------------------------------------------------- packed layout
+
+def row_bytes(d: int, bits) -> int:
+    """Bytes of one packed row: the level fields concatenated, rounded up to 16 bytes."""
+    return 16 * ((bits_per_vector(d, bits) + 127) // 128)
+
+
+def pack(idx, d: int, bits) -> np.ndarray:
+    """Packs per-level indices (list over levels of [n, d / 2^l]) into rows of row_bytes(d, bits).
+
+    Reading taken (the pages give no bit layout): level 1's indices first, then level 2's, and
+    so on; inside the row's little-endian bitstream every index occupies its level's width,
+    least significant bit first, one after the other with no gaps; the pad bits up to the
+    16-byte row boundary are zero. This pair of functions is the only place the oracle states
+    the layout.
+    """
+    nl = n_levels(d)
+    bits = [bits] * nl if np.isscalar(bits) else list(bits)
+    n = np.asarray(idx[0]).shape[0]
+    streams = []
+    for lv in range(nl):
+        a = np.asarray(idx[lv], dtype=np.uint64)
+        planes = (a[:, :, None] >> np.arange(bits[lv], dtype=np.uint64)) & np.uint64(1)
+        streams.append(planes.reshape(n, -1).astype(np.uint8))
+    stream = np.concatenate(streams, axis=1)
+    out = np.zeros((n, row_bytes(d, bits)), dtype=np.uint8)
+    packed = np.packbits(stream, axis=1, bitorder="little")
+    out[:, :packed.shape[1]] = packed
+    return out
+
+
+def unpack(codes, d: int, bits):
+    """Inverse of :func:`pack`: rows -> list over levels of [n, d / 2^l] int64 indices."""
+    nl = n_levels(d)
+    bits = [bits] * nl if np.isscalar(bits) else list(bits)
+    codes = np.asarray(codes, dtype=np.uint8)
+    stream = np.unpackbits(codes, axis=1, bitorder="little").astype(np.int64)
+    out, pos = [], 0
+    for lv in range(nl):
+        cnt, b = d >> (lv + 1), bits[lv]
+        f = stream[:, pos:pos + cnt * b].reshape(-1, cnt, b)
+        out.append(np.sum(f << np.arange(b, dtype=np.int64), axis=2))
+        pos += cnt * b
+    return out

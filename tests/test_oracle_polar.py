@@ -117,3 +117,41 @@ def test_score_up_the_tree_equals_the_dot_product_with_the_reconstruction(d, bit
     xh = polar.decode(e["idx"], e["n_exact"], Pi, books)
     got = polar.score(q, e["idx"], e["n_exact"], Pi, books)
     assert np.allclose(got, xh @ q, rtol=1e-12, atol=1e-12 * np.abs(xh @ q).max())
+
+
+def _read_golden(name):
+    import os
+    vals = {}
+    with open(os.path.join(os.path.dirname(__file__), "golden", name)) as fh:
+        for line in fh:
+            if line.startswith("#") or not line.strip():
+                continue
+            key, *rest = line.split()
+            vals[key] = rest
+    return vals
+
+
+def test_pack_hand_worked_example():
+    g = _read_golden("polar_pack_d8.txt")
+    d = int(g["d"][0])
+    bits = [int(v) for v in g["bits"]]
+    idx = [np.array([[int(v) for v in g[f"level{lv}"]]]) for lv in (1, 2, 3)]
+    want = np.array([[int(v, 16) for v in g["bytes"]]], dtype=np.uint8)
+    assert polar.row_bytes(d, bits) == 16
+    assert np.array_equal(polar.pack(idx, d, bits), want)
+    got = polar.unpack(want, d, bits)
+    assert all(np.array_equal(a, b) for a, b in zip(got, idx))
+
+
+@pytest.mark.parametrize("d,bits", [(128, [4, 2, 2, 2, 2, 2, 2]), (32, 3), (64, [1, 4, 3, 2, 1, 1]), (256, 2)])
+def test_pack_round_trip_and_zero_pad(d, bits):
+    nl = polar.n_levels(d)
+    bl = [bits] * nl if np.isscalar(bits) else bits
+    rs = np.random.default_rng(d)
+    idx = [rs.integers(0, 1 << bl[lv], size=(9, d >> (lv + 1))) for lv in range(nl)]
+    codes = polar.pack(idx, d, bits)
+    assert codes.shape == (9, polar.row_bytes(d, bits)) and codes.shape[1] % 16 == 0
+    assert all(np.array_equal(a, b) for a, b in zip(polar.unpack(codes, d, bits), idx))
+    total = polar.bits_per_vector(d, bits)
+    tail = np.unpackbits(codes, axis=1, bitorder="little")[:, total:]
+    assert not tail.any()
