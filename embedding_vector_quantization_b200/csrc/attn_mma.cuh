@@ -18,13 +18,19 @@
 //    every MMA uses one of the two mask families, so its accumulator is exact
 //    after a final division by 16 (kept in separate accumulators for keys).
 //  * Query side (keys as the MMA rows): queries are rotated once, scaled by the
-//    codebook slopes, rounded to 15-bit integers and split into two int8 pieces
-//    (hi * 128 + lo), which fill the 8 MMA columns (4 heads x 2 pieces).
+//    codebook slopes, rounded to 22-bit integers and split into three int8 pieces
+//    (hi * 2^14 + mid * 2^7 + lo): one n8 tile holds the hi and mid pieces of the
+//    4 heads, a second n8 tile the lo pieces (columns 2h; the odd columns are 0).
 //  * Value side (bit rows of the value codes as the MMA rows, tokens as the
 //    reduction): softmax weights p * ||v|| (and p * rnorm for the QJL part) are
-//    rounded to 14-bit integers against the chunk maximum and split into two
-//    int8 pieces; ldmatrix .trans.b8 gathers "byte j of 4 consecutive tokens"
-//    into one register.
+//    rounded to 16-bit integers against the chunk maximum and split into two
+//    unsigned 8-bit pieces (hi * 256 + lo; u8 x u8 MMAs, since bits and weights
+//    are non-negative); ldmatrix .trans.b8 gathers "byte j of 4 consecutive
+//    tokens" into one register.
+//  * Precision: a query piece is off by at most half a step of max|q| / 2^21, a
+//    weight by half a step of max ||v|| / 65535; on keys and values with 10x
+//    outlier channels this keeps the attention output within a few 1e-4 of the
+//    exact result (the 15-bit queries and 14-bit weights used before reached 1.3e-3).
 //  * Two passes per context chunk: all key scores first (kept in shared memory,
 //    giving the exact chunk maximum), then all values with one fixed weight
 //    scale, so the value sums accumulate in int32 across the whole chunk.
@@ -81,13 +87,15 @@ struct Args {
 struct __align__(16) Smem {
   unsigned char stage[kStages][kStageBytes];
   float logits[kG][kMaxChunk];  // key pass output: scaled logits in log2 units [head][token]
-  uint32_t qfrag[12][2][4][8];  // key-side B fragments: [k-step][register][quad index t][column g]
-  int8_t pw[2][2][8][kBlk];     // integer softmax weights of a value block, double buffered:
+  uint32_t qfrag[2][12][2][4][8];  // key-side B fragments: [n tile][k-step][register][quad index t][column g]
+  uint8_t pw[2][2][8][kBlk];    // integer softmax weights of a value block, double buffered:
                                 // [buffer][0: value weights, 1: QJL weights][col = head*2+piece][token]
   float qconst[kG][4];        // c0*sum(q'), delta_mse, delta_qjl, sum(qs)
   float red_f[kWarps][kG];
   float hmax[kG];
-  float nmax[2];
+  float dv[2][kG];            // weight steps per head: max_t p_t ||v_t|| / 65535 (0: values, 1: QJL)
+  float inv[2][kG];
+  float red_w[kWarps][2][kG]; // per warp: max_t (logit + log2 ||v_t||), max_t (logit + log2 rnorm_t)
   int red_i[kWarps][2 * kG];
   float vacc[3][kG][128];     // value-side sums of the two token halves (rows of each byte group)
   __half vnorm[kMaxChunk];    // value norms and residual norms of the chunk (copied with the key blocks)
@@ -124,6 +132,15 @@ __device__ __forceinline__ void tma_bulk_g2s(void* dst, const void* src, uint32_
 __device__ __forceinline__ void mma_s8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
                                        uint32_t b0, uint32_t b1) {
   asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.s8.s8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
+               "{%0,%1,%2,%3};\n"
+               : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
+               : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
+}
+
+// Unsigned variant (0/1 bit planes times non-negative weight pieces).
+__device__ __forceinline__ void mma_u8(int (&d)[4], uint32_t a0, uint32_t a1, uint32_t a2, uint32_t a3,
+                                       uint32_t b0, uint32_t b1) {
+  asm volatile("mma.sync.aligned.m16n8k32.row.col.s32.u8.u8.s32 {%0,%1,%2,%3}, {%4,%5,%6,%7}, {%8,%9}, "
                "{%0,%1,%2,%3};\n"
                : "+r"(d[0]), "+r"(d[1]), "+r"(d[2]), "+r"(d[3])
                : "r"(a0), "r"(a1), "r"(a2), "r"(a3), "r"(b0), "r"(b1));
@@ -181,10 +198,13 @@ __device__ __forceinline__ int qfrag_sign_offset(int i) {
 
 // Query side of the key MMAs for the kG heads h0 .. h0 + 3 of sequence b (one warp per
 // head, warps 0..3): rotated queries scaled by the codebook slopes and S q, rounded to
-// 15-bit integers against their maxima and split into int8 hi/lo pieces in B-fragment
-// order; qconst[h] = {c0 sum(q'), step of the code pieces, step of the sign pieces, sum(S q)}.
+// 22-bit integers against their maxima and split into int8 pieces hi * 2^14 + mid * 2^7 + lo
+// in B-fragment order (n tile 0: column 2h = hi, 2h + 1 = mid; n tile 1: column 2h = lo);
+// qconst[h] = {c0 sum(q'), step of the code pieces, step of the sign pieces, sum(S q)}.
+constexpr float kQMax = 2080768.f;   // 127 * 2^14: the largest |integer| a query value maps to
 __device__ __forceinline__ void prepare_query(const float* qr_rows, const float* qs_rows, float kb0, float kb1,
-                                              float kc0, uint32_t (&qfrag)[12][2][4][8], float (&qconst)[kG][4]) {
+                                              float kc0, uint32_t (&qfrag)[2][12][2][4][8],
+                                              float (&qconst)[kG][4]) {
   const int lane = threadIdx.x & 31, h = threadIdx.x >> 5;
   if (h >= kG) return;
   const float* qr = qr_rows + (size_t)h * kD;
@@ -209,20 +229,25 @@ __device__ __forceinline__ void prepare_query(const float* qr_rows, const float*
     mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
     ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
   }
-  const float dm = mx > 0.f ? mx / 16256.f : 1.f;
-  const float ds = ms > 0.f ? ms / 16256.f : 1.f;
-  int8_t* qf = reinterpret_cast<int8_t*>(&qfrag[0][0][0][0]);
+  const float dm = mx > 0.f ? mx / kQMax : 1.f;
+  const float ds = ms > 0.f ? ms / kQMax : 1.f;
+  int8_t* qf0 = reinterpret_cast<int8_t*>(&qfrag[0][0][0][0][0]);
+  int8_t* qf1 = reinterpret_cast<int8_t*>(&qfrag[1][0][0][0][0]);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int j = lane + 32 * i;
     const float v[3] = {x0[i] / dm, x1[i] / dm, xs[i] / ds};
 #pragma unroll
     for (int c = 0; c < 3; ++c) {
-      const int xi = __float2int_rn(v[c]);
-      const int hi = (xi >= 0) ? (xi + 64) >> 7 : -((-xi + 64) >> 7);
+      const int xi = __float2int_rn(v[c]);                                   // |xi| <= 127 * 2^14
+      const int hi = (xi >= 0) ? (xi + 8192) >> 14 : -((-xi + 8192) >> 14);  // |hi| <= 127
+      const int r = xi - (hi << 14);                                         // |r| <= 2^13
+      const int mid = (r >= 0) ? (r + 64) >> 7 : -((-r + 64) >> 7);         // |mid| <= 64
       const int off = (c < 2) ? qfrag_code_offset(c, j) : qfrag_sign_offset(j);
-      qf[off + (2 * h) * 4] = (int8_t)hi;                   // column g = 2h (hi piece)
-      qf[off + (2 * h + 1) * 4] = (int8_t)(xi - 128 * hi);  // column g = 2h + 1 (lo piece)
+      qf0[off + (2 * h) * 4] = (int8_t)hi;
+      qf0[off + (2 * h + 1) * 4] = (int8_t)mid;
+      qf1[off + (2 * h) * 4] = (int8_t)(r - (mid << 7));                     // |lo| <= 64
+      qf1[off + (2 * h + 1) * 4] = 0;
     }
   }
   if (lane == 0) {
@@ -234,10 +259,12 @@ __device__ __forceinline__ void prepare_query(const float* qr_rows, const float*
 }
 
 // Raw scores (tq_score's formula) of keys kbase + g and kbase + g + 8 of a staged key block
-// for query head t = lane % 4: twelve int8 MMAs over the code and sign bit planes.
+// for query head t = lane % 4: the code and sign bit planes against the query pieces, n tile 0
+// (hi and mid pieces, fragments qb held in registers) and n tile 1 (lo pieces, read from
+// shared memory: qlo = &qfrag[1][0][0][t][g]).
 __device__ __forceinline__ void mtile_scores(const unsigned char* st, const __half* nrm, const __half* rnm, int kbase,
-                                             const uint32_t (&qb)[12][2], float c0h, float dmh, float dsh, float ssh,
-                                             float (&sc)[2]) {
+                                             const uint32_t (&qb)[12][2], const uint32_t* qlo, float c0h, float dmh,
+                                             float dsh, float ssh, float (&sc)[2]) {
   const int lane = threadIdx.x & 31, g = lane >> 2;
   uint32_t cw[4], sw[2];
   {
@@ -247,32 +274,43 @@ __device__ __forceinline__ void mtile_scores(const unsigned char* st, const __ha
     const int skey = kbase + r + 8 * (mat & 1);
     ldsm_x2(sw, st + kStageCodes + skey * kSignsB);
   }
-  // six independent accumulator chains of length two (even / odd shifts)
+  // tile 0: six independent accumulator chains of length two (even / odd shifts); tile 1: four chains
   int dm1[2][4] = {}, dm16[2][4] = {}, ds1[4] = {}, ds16[4] = {};
+  int lm1[4] = {}, lm16[4] = {}, ls1[4] = {}, ls16[4] = {};
+  // lo-piece fragments: word (kk, slot) of this thread at qlo[(kk * 2 + slot) * 32]
+  auto lo = [&](int kk, int slot) { return qlo[(kk * 2 + slot) * 32]; };
   // code words: cw[0] = key g word t, cw[1] = key g word 4+t, cw[2] = key g+8 word t, cw[3] = key g+8 word 4+t
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
     const uint32_t x0 = cw[0] >> s, x1 = cw[1] >> s, x2 = cw[2] >> s, x3 = cw[3] >> s;
-    mma_s8(dm1[s & 1], x0 & 0x01010101u, x2 & 0x01010101u, x1 & 0x01010101u, x3 & 0x01010101u, qb[s][0], qb[s][1]);
-    mma_s8(dm16[s & 1], x0 & 0x10101010u, x2 & 0x10101010u, x1 & 0x10101010u, x3 & 0x10101010u, qb[4 + s][0],
-           qb[4 + s][1]);
+    const uint32_t a0 = x0 & 0x01010101u, a1 = x2 & 0x01010101u, a2 = x1 & 0x01010101u, a3 = x3 & 0x01010101u;
+    const uint32_t b0 = x0 & 0x10101010u, b1 = x2 & 0x10101010u, b2 = x1 & 0x10101010u, b3 = x3 & 0x10101010u;
+    mma_s8(dm1[s & 1], a0, a1, a2, a3, qb[s][0], qb[s][1]);
+    mma_s8(dm16[s & 1], b0, b1, b2, b3, qb[4 + s][0], qb[4 + s][1]);
+    mma_s8(lm1, a0, a1, a2, a3, lo(s, 0), lo(s, 1));
+    mma_s8(lm16, b0, b1, b2, b3, lo(4 + s, 0), lo(4 + s, 1));
   }
   // sign words: sw[0] = key g word t, sw[1] = key g+8 word t
 #pragma unroll
   for (int s = 0; s < 2; ++s) {
     const uint32_t y0 = sw[0] >> s, y1 = sw[1] >> s, z0 = sw[0] >> (s + 2), z1 = sw[1] >> (s + 2);
-    mma_s8(ds1, y0 & 0x01010101u, y1 & 0x01010101u, z0 & 0x01010101u, z1 & 0x01010101u, qb[8 + s][0], qb[8 + s][1]);
-    mma_s8(ds16, y0 & 0x10101010u, y1 & 0x10101010u, z0 & 0x10101010u, z1 & 0x10101010u, qb[10 + s][0],
-           qb[10 + s][1]);
+    const uint32_t a0 = y0 & 0x01010101u, a1 = y1 & 0x01010101u, a2 = z0 & 0x01010101u, a3 = z1 & 0x01010101u;
+    const uint32_t b0 = y0 & 0x10101010u, b1 = y1 & 0x10101010u, b2 = z0 & 0x10101010u, b3 = z1 & 0x10101010u;
+    mma_s8(ds1, a0, a1, a2, a3, qb[8 + s][0], qb[8 + s][1]);
+    mma_s8(ds16, b0, b1, b2, b3, qb[10 + s][0], qb[10 + s][1]);
+    mma_s8(ls1, a0, a1, a2, a3, lo(8 + s, 0), lo(8 + s, 1));
+    mma_s8(ls16, b0, b1, b2, b3, lo(10 + s, 0), lo(10 + s, 1));
   }
   const float kqjl = kQjlScale / (float)kM;
 #pragma unroll
   for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
     const int key = kbase + g + 8 * r;
-    const int hi = 2 * r, lo = 2 * r + 1;
-    const int mse = 128 * (dm1[0][hi] + dm1[1][hi] + ((dm16[0][hi] + dm16[1][hi]) >> 4)) +
-                    (dm1[0][lo] + dm1[1][lo] + ((dm16[0][lo] + dm16[1][lo]) >> 4));
-    const int qjl = 128 * (ds1[hi] + (ds16[hi] >> 4)) + (ds1[lo] + (ds16[lo] >> 4));
+    const int hi = 2 * r, md = 2 * r + 1;   // tile 0: columns 2t (hi) and 2t + 1 (mid); tile 1: column 2t (lo)
+    // exact in int32: at most 256 code (128 sign) positions of |piece| <= 127 each, times 2^14
+    const int mse = (dm1[0][hi] + dm1[1][hi] + ((dm16[0][hi] + dm16[1][hi]) >> 4)) * 16384 +
+                    (dm1[0][md] + dm1[1][md] + ((dm16[0][md] + dm16[1][md]) >> 4)) * 128 + lm1[hi] + (lm16[hi] >> 4);
+    const int qjl = (ds1[hi] + (ds16[hi] >> 4)) * 16384 + (ds1[md] + (ds16[md] >> 4)) * 128 + ls1[hi] +
+                    (ls16[hi] >> 4);
     const float n = __half2float(nrm[key]), rn = __half2float(rnm[key]);
     sc[r] = n * (c0h + dmh * (float)mse) + rn * kqjl * (2.f * dsh * (float)qjl - ssh);
   }
@@ -302,6 +340,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
+  if (tid < 2 * kG) (&sm.dv[0][0])[tid] = 1.f;   // an empty chunk keeps unit steps (its sums are 0)
   __syncthreads();
 
   auto issue = [&](int j) {  // block j: K block (j < nblk) or V block j - nblk
@@ -348,12 +387,12 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 #pragma unroll
   for (int kk = 0; kk < 12; ++kk)
 #pragma unroll
-    for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[kk][slot][t][g];
+    for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[0][kk][slot][t][g];
 
   const float scale2 = a.scale * 1.4426950408889634f;
   float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
   float run_max = -INFINITY;   // this thread's max logit of head t
-  float vn_max = 0.f, vr_max = 0.f;
+  float wv_max = -INFINITY, wr_max = -INFINITY;   // log2 of this thread's largest p ||v|| and p rnorm (head t)
 
   // value-side accumulators: 8 m-tiles (bit rows 0..7 of bytes g, g+8 of this warp's byte group)
   int vacc[8][4];
@@ -363,16 +402,16 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
   int wsum[2] = {0, 0};        // sum of integer weights (value, QJL) for head (P-warps)
 
   const int bg = warp % 3, half = warp / 3;   // value side: byte group and token half (warps 0..5)
-  float dv1 = 1.f, dv2 = 1.f, inv1 = 1.f, inv2 = 1.f;
 
   // Integer weights of value block jj into pw[jj & 1]: thread -> (head, 4 consecutive tokens)
-  // per round; w1 = round(p * ||v|| / dv1), w2 = round(p * rnorm / dv2) with p = exp2(logit - max),
-  // each split into 7-bit pieces (hi * 128 + lo). Also accumulates sum p and the integer sums.
+  // per round; w1 = round(p * ||v|| / dv[0][h]), w2 = round(p * rnorm / dv[1][h]) with
+  // p = exp2(logit - max), each split into 8-bit pieces (hi * 256 + lo). Also accumulates sum p
+  // and the integer sums.
   auto prepare_weights = [&](int jj, int tix, int nthreads) {
     const int tb = jj * kBlk;
     const int nval = min(kBlk, ntok - tb);
     const int h = tix & 3;
-    const float hm = sm.hmax[h];
+    const float hm = sm.hmax[h], inv1 = sm.inv[0][h], inv2 = sm.inv[1][h];
     for (int q4 = (tix >> 2) * 4; q4 < kBlk; q4 += (nthreads >> 2) * 4) {
       const float4 l4 = *reinterpret_cast<const float4*>(&sm.logits[h][tb + q4]);
       const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
@@ -382,18 +421,18 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
         const int tok = q4 + q;
         if (tok < nval) {
           const float p = exp2_approx(lv[q] - hm);
-          const int w1 = __float2int_rn(p * __half2float(sm.vnorm[tb + tok]) * inv1);
-          const int w2 = __float2int_rn(p * __half2float(sm.vrn[tb + tok]) * inv2);
-          w1h |= (uint32_t)(w1 >> 7) << (8 * q);
-          w1l |= (uint32_t)(w1 & 127) << (8 * q);
-          w2h |= (uint32_t)(w2 >> 7) << (8 * q);
-          w2l |= (uint32_t)(w2 & 127) << (8 * q);
+          const int w1 = min(__float2int_rn(p * __half2float(sm.vnorm[tb + tok]) * inv1), 65535);
+          const int w2 = min(__float2int_rn(p * __half2float(sm.vrn[tb + tok]) * inv2), 65535);
+          w1h |= (uint32_t)(w1 >> 8) << (8 * q);
+          w1l |= (uint32_t)(w1 & 255) << (8 * q);
+          w2h |= (uint32_t)(w2 >> 8) << (8 * q);
+          w2l |= (uint32_t)(w2 & 255) << (8 * q);
           lsum += p;
           wsum[0] += w1;
           wsum[1] += w2;
         }
       }
-      int8_t* blk = &sm.pw[jj & 1][0][0][0];
+      uint8_t* blk = &sm.pw[jj & 1][0][0][0];
       *reinterpret_cast<uint32_t*>(blk + (2 * h) * kBlk + q4) = w1h;
       *reinterpret_cast<uint32_t*>(blk + (2 * h + 1) * kBlk + q4) = w1l;
       *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h) * kBlk + q4) = w2h;
@@ -437,33 +476,32 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 #pragma unroll
       for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
       if (g == 0) sm.red_f[warp][t] = m;
-      float vn = vn_max, vr = vr_max;
+      float wv = wv_max, wr = wr_max;
 #pragma unroll
-      for (int o = 1; o < 32; o <<= 1) {
-        vn = fmaxf(vn, __shfl_xor_sync(0xffffffffu, vn, o));
-        vr = fmaxf(vr, __shfl_xor_sync(0xffffffffu, vr, o));
+      for (int o = 4; o < 32; o <<= 1) {
+        wv = fmaxf(wv, __shfl_xor_sync(0xffffffffu, wv, o));
+        wr = fmaxf(wr, __shfl_xor_sync(0xffffffffu, wr, o));
       }
-      if (lane == 0) sm.red_i[warp][0] = __float_as_int(vn), sm.red_i[warp][1] = __float_as_int(vr);
+      if (g == 0) sm.red_w[warp][0][t] = wv, sm.red_w[warp][1][t] = wr;
       __syncthreads();
       if (tid < kG) {
-        float mm = -INFINITY;
-        for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.red_f[w][tid]);
-        sm.hmax[tid] = mm;
-      }
-      if (tid == 0) {
-        float n1 = 0.f, n2 = 0.f;
+        float mm = -INFINITY, mv = -INFINITY, mr = -INFINITY;
         for (int w = 0; w < kWarps; ++w) {
-          n1 = fmaxf(n1, __int_as_float(sm.red_i[w][0]));
-          n2 = fmaxf(n2, __int_as_float(sm.red_i[w][1]));
+          mm = fmaxf(mm, sm.red_f[w][tid]);
+          mv = fmaxf(mv, sm.red_w[w][0][tid]);
+          mr = fmaxf(mr, sm.red_w[w][1][tid]);
         }
-        sm.nmax[0] = n1;
-        sm.nmax[1] = n2;
+        sm.hmax[tid] = mm;
+        // 16-bit weights per head against the head's largest weight of the chunk (a hair above it,
+        // so that the approximate exp2 / log2 cannot push the largest weight past 65535)
+        const float s1 = exp2_approx(mv - mm) * (1.f + 1.f / 4096.f) / 65535.f;
+        const float s2 = exp2_approx(mr - mm) * (1.f + 1.f / 4096.f) / 65535.f;
+        sm.dv[0][tid] = (s1 > 0.f && s1 < INFINITY) ? s1 : 1.f;
+        sm.dv[1][tid] = (s2 > 0.f && s2 < INFINITY) ? s2 : 1.f;
+        sm.inv[0][tid] = 1.f / sm.dv[0][tid];
+        sm.inv[1][tid] = 1.f / sm.dv[1][tid];
       }
       __syncthreads();
-      dv1 = sm.nmax[0] > 0.f ? sm.nmax[0] / 16383.f : 1.f;
-      dv2 = sm.nmax[1] > 0.f ? sm.nmax[1] / 16383.f : 1.f;
-      inv1 = 1.f / dv1;
-      inv2 = 1.f / dv2;
       // integer weights of the first value block (all threads); later blocks are prepared
       // by warps 6 and 7 while warps 0..5 run the value MMAs of the block before
       prepare_weights(0, tid, kThreads);
@@ -476,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
       for (int mt = 0; mt < 2; ++mt) {
         const int kbase = 128 * mt + 16 * warp;
         float sc[2];
-        mtile_scores(st, nrm, rnm, kbase, qb, c0h, dmh, dsh, ssh, sc);
+        mtile_scores(st, nrm, rnm, kbase, qb, &sm.qfrag[1][0][0][t][g], c0h, dmh, dsh, ssh, sc);
 #pragma unroll
         for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
           const int key = kbase + g + 8 * r;
@@ -484,22 +522,21 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
           const float v = (key < nvalid) ? sc[r] * scale2 : -INFINITY;
           sm.logits[t][tok_base + key] = v;
           run_max = fmaxf(run_max, v);
+          // the token's weights will be exp2(v - max) ||v|| and exp2(v - max) rnorm (value norms
+          // arrived with the key block): track their largest logarithms for the weight steps
+          wv_max = fmaxf(wv_max, v + __log2f(__half2float(nrm[2 * kBlk + key])));
+          wr_max = fmaxf(wr_max, v + __log2f(__half2float(nrm[3 * kBlk + key])));
         }
       }
-      // value norms of these tokens (they arrived with the key block): keep for the value pass
+      // value norms of these tokens: keep for the value pass
       if (tid < kBlk) {
-        const __half vn = nrm[2 * kBlk + tid], vr = nrm[3 * kBlk + tid];
-        sm.vnorm[tok_base + tid] = vn;
-        sm.vrn[tok_base + tid] = vr;
-        if (tid < nvalid) {
-          vn_max = fmaxf(vn_max, __half2float(vn));
-          vr_max = fmaxf(vr_max, __half2float(vr));
-        }
+        sm.vnorm[tok_base + tid] = nrm[2 * kBlk + tid];
+        sm.vrn[tok_base + tid] = nrm[3 * kBlk + tid];
       }
     } else {
       // ---------------- value pass (warps 0..5: byte group bg, token half)
       if (warp < 6) {
-        const int8_t* pw = &sm.pw[jj & 1][bg == 2 ? 1 : 0][0][0];
+        const uint8_t* pw = &sm.pw[jj & 1][bg == 2 ? 1 : 0][0][0];
 #pragma unroll
         for (int kq = 0; kq < 4; ++kq) {
           const int tk = 128 * half + 32 * kq;  // first token of this 32-token k-step
@@ -512,8 +549,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 #pragma unroll
           for (int s = 0; s < 4; ++s) {
             const uint32_t x0 = r[0] >> s, x1 = r[1] >> s, x2 = r[2] >> s, x3 = r[3] >> s;
-            mma_s8(vacc[s], x0 & 0x01010101u, x1 & 0x01010101u, x2 & 0x01010101u, x3 & 0x01010101u, b0, b1);
-            mma_s8(vacc[4 + s], x0 & 0x10101010u, x1 & 0x10101010u, x2 & 0x10101010u, x3 & 0x10101010u, b0, b1);
+            mma_u8(vacc[s], x0 & 0x01010101u, x1 & 0x01010101u, x2 & 0x01010101u, x3 & 0x01010101u, b0, b1);
+            mma_u8(vacc[4 + s], x0 & 0x10101010u, x1 & 0x10101010u, x2 & 0x10101010u, x3 & 0x10101010u, b0, b1);
           }
         }
       } else if (jj + 1 < nblk) {
@@ -560,8 +597,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int f = (u < 4) ? 0 : 4;
-      const float v0 = 128.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
-      const float v1 = 128.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
+      const float v0 = 256.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
+      const float v1 = 256.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
       sm.vacc[bg][t][g * 8 + u] = v0;          // byte g, bit u
       sm.vacc[bg][t][64 + g * 8 + u] = v1;     // byte g + 8, bit u
     }
@@ -571,8 +608,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 #pragma unroll
     for (int u = 0; u < 8; ++u) {
       const int f = (u < 4) ? 0 : 4;
-      const float v0 = 128.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
-      const float v1 = 128.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
+      const float v0 = 256.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
+      const float v1 = 256.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
       sm.vacc[bg][t][g * 8 + u] += v0;
       sm.vacc[bg][t][64 + g * 8 + u] += v1;
     }
@@ -596,11 +633,11 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
       const int byte = j >> 2, grp = byte >> 4, bl = byte & 15, u0 = 2 * (j & 3);
       const int idx = (bl < 8) ? bl * 8 : 64 + (bl - 8) * 8;
       const float d0 = sm.vacc[grp][h][idx + u0], d1 = sm.vacc[grp][h][idx + u0 + 1];
-      v = dv1 * (a.vc0 * (float)W1 + a.vb0 * d0 + a.vb1 * d1);
+      v = sm.dv[0][h] * (a.vc0 * (float)W1 + a.vb0 * d0 + a.vb1 * d1);
     } else {
       const int p = j - kD, byte = p >> 3, u = p & 7;
       const int idx = (byte < 8) ? byte * 8 + u : 64 + (byte - 8) * 8 + u;
-      v = dv2 * (2.f * sm.vacc[2][h][idx] - (float)W2);
+      v = sm.dv[1][h] * (2.f * sm.vacc[2][h][idx] - (float)W2);
     }
     a.part[(((size_t)b * a.Hq + h0 + h) * a.nsplit + split) * stride + j] = v;
   }
@@ -642,7 +679,7 @@ struct ScoreArgs {
 
 struct __align__(16) ScoreSmem {
   unsigned char stage[kSStages][kSStageBytes];
-  uint32_t qfrag[12][2][4][8];
+  uint32_t qfrag[2][12][2][4][8];
   float qconst[kG][4];
   uint64_t full[kSStages];
   uint64_t empty[kSStages];
@@ -698,7 +735,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
 #pragma unroll
   for (int kk = 0; kk < 12; ++kk)
 #pragma unroll
-    for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[kk][slot][t][g];
+    for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[0][kk][slot][t][g];
   const float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
   float* lrow = a.logits + ((size_t)b * a.Hq + h0 + t) * a.L_cap + start;   // head t's scores of the chunk
 
@@ -724,7 +761,8 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
     float sc[2][2];
     if (!aborted) {
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) mtile_scores(st, nrm, rnm, 128 * mt + 16 * warp, qb, c0h, dmh, dsh, ssh, sc[mt]);
+      for (int mt = 0; mt < 2; ++mt)
+        mtile_scores(st, nrm, rnm, 128 * mt + 16 * warp, qb, &sm.qfrag[1][0][0][t][g], c0h, dmh, dsh, ssh, sc[mt]);
     }
     __syncwarp();
     if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[j % kSStages])) : "memory");

@@ -12,12 +12,13 @@
 //    b_i ^ b_j ^ b_k. A packed 4-bit word gives every plane of its 8 coordinates with
 //    shifts and one 3-input XOR; (plane >> 0) & 0x01010101 holds the low-nibble
 //    coordinates of 4 bytes, & 0x10101010 the high-nibble ones (value 16).
-//  * Keys (MMA rows): sum_S w_S <q', beta_S> with w_S q' rounded to 15-bit integers
-//    against one step per head and split into int8 hi/lo pieces, so all planes
-//    accumulate exactly into one int32 (a second for the x16 family).
+//  * Keys (MMA rows): sum_S w_S <q', beta_S> with w_S q' rounded to 22-bit integers
+//    against one step per head and split into int8 pieces hi * 2^14 + mid * 2^7 + lo
+//    (n tile 0: hi and mid of the 4 heads; n tile 1: lo at columns 2h), so all planes
+//    accumulate exactly into int32 sums per piece.
 //  * Values (bit rows of the codes as MMA rows, tokens as the reduction): per-plane
-//    integer sums of the softmax weights p n_v rounded to 14 bits against the chunk
-//    maximum, combined with w_S once per chunk.
+//    integer sums of the softmax weights p n_v rounded to 16 bits against the chunk
+//    maximum (unsigned 8-bit hi/lo pieces, u8 x u8 MMAs), combined with w_S once per chunk.
 //  * Two passes per chunk as in attn_mma.cuh: all key blocks (exact chunk maximum), then
 //    all value blocks with one weight scale.
 //
@@ -37,6 +38,7 @@ using amma::mbar_expect_tx;
 using amma::mbar_init;
 using amma::mbar_wait;
 using amma::mma_s8;
+using amma::mma_u8;
 using amma::smem_u32;
 using amma::tma_bulk_g2s;
 
@@ -73,13 +75,14 @@ struct Args {
 struct __align__(16) Smem {
   unsigned char stage[kStages][kStageBytes];
   float logits[kG][kMaxChunk];     // key pass output: scaled logits in log2 units [head][token]
-  uint32_t qfrag[32][4][8][2];     // key-side B fragments [k-step][quad index t][column g][register]
-  int8_t pw[2][8][kBlk];           // integer weights of a value block, double buffered [buf][col][token]
+  uint32_t qfrag[2][32][4][8][2];  // key-side B fragments [n tile][k-step][quad index t][column g][register]
+  uint8_t pw[2][8][kBlk];          // integer weights of a value block, double buffered [buf][col][token]
   float acc[kG][kD];               // value sums by coordinate (rotated domain), before the scale
   float qconst[kG][2];             // c0 sum(q'), integer step of the query pieces
   float red_f[kWarps][kG];
   float hmax[kG];
-  float nmax;
+  float dv[kG];                    // weight step per head: max_t p_t ||v_t|| / 65535
+  float red_w[kWarps][kG];         // per warp: max_t (logit + log2 ||v_t||)
   int red_i[kWarps][kG];
   __half vnorm[kMaxChunk];
   uint64_t full[kStages];
@@ -110,9 +113,10 @@ __device__ __forceinline__ int qfrag_offset(int S, int c) {
 }
 
 // Query pieces of heads h0 .. h0 + 3 (warps 0..3, one head each): w_S q'_c rounded to
-// 15-bit integers against max |w_S q'_c| and split into int8 hi/lo in B-fragment order.
+// 22-bit integers against max |w_S q'_c| and split into int8 pieces hi * 2^14 + mid * 2^7 + lo
+// in B-fragment order (n tile 0: column 2h = hi, 2h + 1 = mid; n tile 1: column 2h = lo).
 __device__ __forceinline__ void prepare_query4(const float* qr_rows, const float* kw, float kc0,
-                                               uint32_t (&qfrag)[32][4][8][2], float (&qconst)[kG][2]) {
+                                               uint32_t (&qfrag)[2][32][4][8][2], float (&qconst)[kG][2]) {
   const int lane = threadIdx.x & 31, h = threadIdx.x >> 5;
   if (h >= kG) return;
   const float* qr = qr_rows + (size_t)h * kD;
@@ -131,18 +135,23 @@ __device__ __forceinline__ void prepare_query4(const float* qr_rows, const float
     mq = fmaxf(mq, __shfl_xor_sync(0xffffffffu, mq, o));
   }
   const float mx = mq * mw;
-  const float dq = mx > 0.f ? mx / 16256.f : 1.f;
-  int8_t* qf = reinterpret_cast<int8_t*>(&qfrag[0][0][0][0]);
+  const float dq = mx > 0.f ? mx / amma::kQMax : 1.f;
+  int8_t* qf0 = reinterpret_cast<int8_t*>(&qfrag[0][0][0][0][0]);
+  int8_t* qf1 = reinterpret_cast<int8_t*>(&qfrag[1][0][0][0][0]);
 #pragma unroll
   for (int i = 0; i < 4; ++i) {
     const int c = lane + 32 * i;
 #pragma unroll
     for (int S = 0; S < kPlanes; ++S) {
-      const int xi = __float2int_rn(kw[S] * q[i] / dq);
-      const int hi = (xi >= 0) ? (xi + 64) >> 7 : -((-xi + 64) >> 7);
+      const int xi = __float2int_rn(kw[S] * q[i] / dq);                      // |xi| <= 127 * 2^14
+      const int hi = (xi >= 0) ? (xi + 8192) >> 14 : -((-xi + 8192) >> 14);  // |hi| <= 127
+      const int r = xi - hi * 16384;                                         // |r| <= 2^13
+      const int mid = (r >= 0) ? (r + 64) >> 7 : -((-r + 64) >> 7);         // |mid| <= 64
       const int off = qfrag_offset(S, c);
-      qf[off + (2 * h) * 8] = (int8_t)hi;                   // column g = 2h (hi piece)
-      qf[off + (2 * h + 1) * 8] = (int8_t)(xi - 128 * hi);  // column g = 2h + 1 (lo piece)
+      qf0[off + (2 * h) * 8] = (int8_t)hi;
+      qf0[off + (2 * h + 1) * 8] = (int8_t)mid;
+      qf1[off + (2 * h) * 8] = (int8_t)(r - 128 * mid);                      // |lo| <= 64
+      qf1[off + (2 * h + 1) * 8] = 0;
     }
   }
   if (lane == 0) {
@@ -154,8 +163,8 @@ __device__ __forceinline__ void prepare_query4(const float* qr_rows, const float
 // Raw scores n_k <q', c[idx]> of keys kbase + g, kbase + g + 8 (m-tile 0) and kbase + 128 + g,
 // kbase + 136 + g (m-tile 1) of a staged key block, for query head t = lane % 4.
 template <int S>
-__device__ __forceinline__ void key_plane(const uint32_t (&cw)[2][8], const uint32_t (&qfrag)[32][4][8][2],
-                                          int (&a1)[2][4], int (&a16)[2][4]) {
+__device__ __forceinline__ void key_plane(const uint32_t (&cw)[2][8], const uint32_t (&qfrag)[2][32][4][8][2],
+                                          int (&a1)[2][4], int (&a16)[2][4], int (&l1)[2][4], int (&l16)[2][4]) {
   const int lane = threadIdx.x & 31, g = lane >> 2, t = lane & 3;
 #pragma unroll
   for (int h = 0; h < 2; ++h) {
@@ -167,20 +176,24 @@ __device__ __forceinline__ void key_plane(const uint32_t (&cw)[2][8], const uint
 #pragma unroll
     for (int nu = 0; nu < 2; ++nu) {
       const int kk = (S * 2 + nu) * 2 + h;
-      const uint2 b = *reinterpret_cast<const uint2*>(&qfrag[kk][t][g][0]);
+      const uint2 b = *reinterpret_cast<const uint2*>(&qfrag[0][kk][t][g][0]);
+      const uint2 bl = *reinterpret_cast<const uint2*>(&qfrag[1][kk][t][g][0]);
       const uint32_t m = nu ? 0x10101010u : 0x01010101u;
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt) {
         // words: p[0] = key g word t, p[1] = key g word 4+t, p[2] = key g+8 word t, p[3] = key g+8 word 4+t
         int(&acc)[4] = nu ? a16[mt] : a1[mt];
-        mma_s8(acc, p[mt][0] & m, p[mt][2] & m, p[mt][1] & m, p[mt][3] & m, b.x, b.y);
+        int(&accl)[4] = nu ? l16[mt] : l1[mt];
+        const uint32_t x0 = p[mt][0] & m, x1 = p[mt][2] & m, x2 = p[mt][1] & m, x3 = p[mt][3] & m;
+        mma_s8(acc, x0, x1, x2, x3, b.x, b.y);
+        mma_s8(accl, x0, x1, x2, x3, bl.x, bl.y);
       }
     }
   }
 }
 
 __device__ __forceinline__ void key_scores4(const unsigned char* st, const __half* nrm, int kbase,
-                                            const uint32_t (&qfrag)[32][4][8][2], float c0h, float dqh,
+                                            const uint32_t (&qfrag)[2][32][4][8][2], float c0h, float dqh,
                                             float (&sc)[2][2]) {
   const int lane = threadIdx.x & 31, g = lane >> 2;
   uint32_t cw[2][8];
@@ -196,23 +209,27 @@ __device__ __forceinline__ void key_scores4(const unsigned char* st, const __hal
       cw[mt][4] = w4[0]; cw[mt][5] = w4[1]; cw[mt][6] = w4[2]; cw[mt][7] = w4[3];
     }
   }
-  int a1[2][4] = {}, a16[2][4] = {};   // per m-tile: the x1 and the x16 families
-  key_plane<0>(cw, qfrag, a1, a16);
-  key_plane<1>(cw, qfrag, a1, a16);
-  key_plane<2>(cw, qfrag, a1, a16);
-  key_plane<3>(cw, qfrag, a1, a16);
-  key_plane<4>(cw, qfrag, a1, a16);
-  key_plane<5>(cw, qfrag, a1, a16);
-  key_plane<6>(cw, qfrag, a1, a16);
-  key_plane<7>(cw, qfrag, a1, a16);
+  // per m-tile: the x1 and the x16 families of n tile 0 (hi, mid) and n tile 1 (lo)
+  int a1[2][4] = {}, a16[2][4] = {}, l1[2][4] = {}, l16[2][4] = {};
+  key_plane<0>(cw, qfrag, a1, a16, l1, l16);
+  key_plane<1>(cw, qfrag, a1, a16, l1, l16);
+  key_plane<2>(cw, qfrag, a1, a16, l1, l16);
+  key_plane<3>(cw, qfrag, a1, a16, l1, l16);
+  key_plane<4>(cw, qfrag, a1, a16, l1, l16);
+  key_plane<5>(cw, qfrag, a1, a16, l1, l16);
+  key_plane<6>(cw, qfrag, a1, a16, l1, l16);
+  key_plane<7>(cw, qfrag, a1, a16, l1, l16);
 #pragma unroll
   for (int mt = 0; mt < 2; ++mt)
 #pragma unroll
     for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
       const int key = kbase + 128 * mt + g + 8 * r;
-      const int hi = 2 * r, lo = 2 * r + 1;
-      const int dot = 128 * (a1[mt][hi] + (a16[mt][hi] >> 4)) + (a1[mt][lo] + (a16[mt][lo] >> 4));
-      sc[mt][r] = __half2float(nrm[key]) * (c0h + dqh * (float)dot);
+      const int hi = 2 * r, md = 2 * r + 1;
+      // the hi sum times 2^14 is formed in float (exact: |sum| < 2^17); the rest is exact in int32
+      const int phi = a1[mt][hi] + (a16[mt][hi] >> 4);
+      const int rest = 128 * (a1[mt][md] + (a16[mt][md] >> 4)) + l1[mt][hi] + (l16[mt][hi] >> 4);
+      const float dot = 16384.f * (float)phi + (float)rest;
+      sc[mt][r] = __half2float(nrm[key]) * (c0h + dqh * dot);
     }
 }
 
@@ -221,8 +238,8 @@ __device__ __forceinline__ void key_scores4(const unsigned char* st, const __hal
 template <int S>
 __device__ __forceinline__ void value_plane(const uint32_t (&r)[4], uint32_t b0, uint32_t b1, int (&vacc)[kPlanes][2][4]) {
   const uint32_t p0 = plane<S>(r[0]), p1 = plane<S>(r[1]), p2 = plane<S>(r[2]), p3 = plane<S>(r[3]);
-  mma_s8(vacc[S][0], p0 & 0x01010101u, p1 & 0x01010101u, p2 & 0x01010101u, p3 & 0x01010101u, b0, b1);
-  mma_s8(vacc[S][1], p0 & 0x10101010u, p1 & 0x10101010u, p2 & 0x10101010u, p3 & 0x10101010u, b0, b1);
+  mma_u8(vacc[S][0], p0 & 0x01010101u, p1 & 0x01010101u, p2 & 0x01010101u, p3 & 0x01010101u, b0, b1);
+  mma_u8(vacc[S][1], p0 & 0x10101010u, p1 & 0x10101010u, p2 & 0x10101010u, p3 & 0x10101010u, b0, b1);
 }
 
 __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
@@ -249,6 +266,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   for (int i = tid; i < kG * kD; i += kThreads) (&sm.acc[0][0])[i] = 0.f;
+  if (tid < kG) sm.dv[tid] = 1.f;   // an empty chunk keeps unit steps (its sums are 0)
   __syncthreads();
 
   auto issue = [&](int j) {  // job j: key block j (j < nblk) or value block j - nblk
@@ -281,10 +299,9 @@ __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
   __syncthreads();
   const float c0h = sm.qconst[t][0], dqh = sm.qconst[t][1];
   const float scale2 = a.scale * 1.4426950408889634f;
-  float run_max = -INFINITY, vn_max = 0.f;
+  float run_max = -INFINITY, wv_max = -INFINITY;   // wv_max: log2 of the largest p ||v|| of head t
   float lsum = 0.f;
   int wsum = 0;
-  float inv1 = 1.f, dv1 = 1.f;
   const int bg = warp & 3, half = warp >> 2;   // value side: 16-byte group of the code rows, token half
   int issued = min(kAhead, njobs);
   // start of job j: refill the stage of job j - 2 once every warp has released it, then wait
@@ -325,13 +342,10 @@ __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
         const float v = (key < nvalid) ? sc[mt][r] * scale2 : -INFINITY;   // log2 units
         sm.logits[t][tok_base + key] = v;
         run_max = fmaxf(run_max, v);
+        wv_max = fmaxf(wv_max, v + __log2f(__half2float(nrm[kBlk + key])));   // its weight exp2(v - max) ||v||
       }
     // value norms of these tokens came with the key block: keep them for the value pass
-    if (tid < kBlk) {
-      const __half vn = nrm[kBlk + tid];
-      sm.vnorm[tok_base + tid] = vn;
-      if (tid < nvalid) vn_max = fmaxf(vn_max, __half2float(vn));
-    }
+    if (tid < kBlk) sm.vnorm[tok_base + tid] = nrm[kBlk + tid];
     end_job(j);
   }
 
@@ -342,24 +356,24 @@ __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
 #pragma unroll
     for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
     if (g == 0) sm.red_f[warp][t] = m;
-    float vn = vn_max;
+    float wv = wv_max;
 #pragma unroll
-    for (int o = 1; o < 32; o <<= 1) vn = fmaxf(vn, __shfl_xor_sync(0xffffffffu, vn, o));
-    if (lane == 0) sm.red_i[warp][0] = __float_as_int(vn);
+    for (int o = 4; o < 32; o <<= 1) wv = fmaxf(wv, __shfl_xor_sync(0xffffffffu, wv, o));
+    if (g == 0) sm.red_w[warp][t] = wv;
     __syncthreads();
     if (tid < kG) {
-      float mm = -INFINITY;
-      for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.red_f[w][tid]);
+      float mm = -INFINITY, mv = -INFINITY;
+      for (int w = 0; w < kWarps; ++w) {
+        mm = fmaxf(mm, sm.red_f[w][tid]);
+        mv = fmaxf(mv, sm.red_w[w][tid]);
+      }
       sm.hmax[tid] = mm;
-    }
-    if (tid == 0) {
-      float n1 = 0.f;
-      for (int w = 0; w < kWarps; ++w) n1 = fmaxf(n1, __int_as_float(sm.red_i[w][0]));
-      sm.nmax = n1;
+      // 16-bit weights per head against the head's largest weight (a hair above it, so that the
+      // approximate exp2 / log2 cannot push the largest weight past 65535)
+      const float s1 = exp2_approx(mv - mm) * (1.f + 1.f / 4096.f) / 65535.f;
+      sm.dv[tid] = (s1 > 0.f && s1 < INFINITY) ? s1 : 1.f;
     }
     __syncthreads();
-    dv1 = sm.nmax > 0.f ? sm.nmax / 16383.f : 1.f;
-    inv1 = 1.f / dv1;
   }
 
   // ---------------- value pass: integer weights of each block (all threads), then MMAs
@@ -377,7 +391,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
     {
       {
         const int h = tid & 3, q4 = (tid >> 2) * 4;
-        const float hm = sm.hmax[h];
+        const float hm = sm.hmax[h], inv1 = 1.f / sm.dv[h];
         const float4 l4 = *reinterpret_cast<const float4*>(&sm.logits[h][tok_base + q4]);
         const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
         uint32_t w1h = 0, w1l = 0;
@@ -385,19 +399,19 @@ __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
         for (int q = 0; q < 4; ++q) {
           if (q4 + q < nvalid) {
             const float p = exp2_approx(lv[q] - hm);
-            const int w1 = __float2int_rn(p * __half2float(sm.vnorm[tok_base + q4 + q]) * inv1);
-            w1h |= (uint32_t)(w1 >> 7) << (8 * q);
-            w1l |= (uint32_t)(w1 & 127) << (8 * q);
+            const int w1 = min(__float2int_rn(p * __half2float(sm.vnorm[tok_base + q4 + q]) * inv1), 65535);
+            w1h |= (uint32_t)(w1 >> 8) << (8 * q);
+            w1l |= (uint32_t)(w1 & 255) << (8 * q);
             lsum += p;
             wsum += w1;
           }
         }
-        int8_t* blk = &sm.pw[jj & 1][0][0];
+        uint8_t* blk = &sm.pw[jj & 1][0][0];
         *reinterpret_cast<uint32_t*>(blk + (2 * h) * kBlk + q4) = w1h;
         *reinterpret_cast<uint32_t*>(blk + (2 * h + 1) * kBlk + q4) = w1l;
       }
       __syncthreads();
-      const int8_t* pw = &sm.pw[jj & 1][0][0];
+      const uint8_t* pw = &sm.pw[jj & 1][0][0];
 #pragma unroll
       for (int kq = 0; kq < 4; ++kq) {
         const int tk = 128 * half + 32 * kq;   // first token of this 32-token k-step
@@ -451,8 +465,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
 #pragma unroll
       for (int nu = 0; nu < 2; ++nu) {
         const int f = nu ? 4 : 0;
-        const float v0 = 128.f * (float)(vacc[S][nu][0] >> f) + (float)(vacc[S][nu][1] >> f);
-        const float v1 = 128.f * (float)(vacc[S][nu][2] >> f) + (float)(vacc[S][nu][3] >> f);
+        const float v0 = 256.f * (float)(vacc[S][nu][0] >> f) + (float)(vacc[S][nu][1] >> f);
+        const float v1 = 256.f * (float)(vacc[S][nu][2] >> f) + (float)(vacc[S][nu][3] >> f);
         cs[0][nu] = fmaf(a.vw[S], v0, cs[0][nu]);
         cs[1][nu] = fmaf(a.vw[S], v1, cs[1][nu]);
       }
@@ -467,7 +481,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
     const int h = i / kD, c = i % kD;
     int W = 0;
     for (int w = 0; w < kWarps; ++w) W += sm.red_i[w][h];
-    a.part[(((size_t)b * a.Hq + h0 + h) * a.nsplit + split) * stride + c] = dv1 * (a.vc0 * (float)W + sm.acc[h][c]);
+    a.part[(((size_t)b * a.Hq + h0 + h) * a.nsplit + split) * stride + c] = sm.dv[h] * (a.vc0 * (float)W + sm.acc[h][c]);
   }
   if (tid < kG) {
     float l = 0.f;

@@ -115,7 +115,41 @@ def test_fifteen_bit_values_split_exactly_into_int8_pieces():
         assert 128 * hi + lo == xi
 
 
+def test_twenty_two_bit_query_values_split_exactly_into_three_int8_pieces():
+    # the attention and score kernels round a query value to xi in [-127 * 2^14, 127 * 2^14], then
+    # hi = xi / 2^14 and mid = (xi - 2^14 hi) / 2^7, each rounded half away from zero, and
+    # lo = xi - 2^14 hi - 2^7 mid; every piece fits an int8 and they rebuild xi exactly
+    def split(xi):
+        hi = (xi + 8192) >> 14 if xi >= 0 else -((-xi + 8192) >> 14)
+        r = xi - hi * 16384
+        mid = (r + 64) >> 7 if r >= 0 else -((-r + 64) >> 7)
+        return hi, mid, r - 128 * mid
+    top = 127 * 16384
+    rs = np.random.default_rng(0)
+    values = list(range(-20000, 20001)) + [top - k for k in range(20000)] + [-top + k for k in range(20000)]
+    values += rs.integers(-top, top + 1, size=50000).tolist()
+    for xi in values:
+        hi, mid, lo = split(int(xi))
+        assert -127 <= hi <= 127 and -64 <= mid <= 64 and -64 <= lo <= 64
+        assert hi * 16384 + mid * 128 + lo == xi
+
+
+def test_sixteen_bit_weights_split_exactly_into_u8_pieces():
+    # softmax weights are rounded to w in [0, 65535] and split into hi = w >> 8, lo = w & 255
+    for w in range(0, 65536):
+        hi, lo = w >> 8, w & 255
+        assert 0 <= hi <= 255 and 0 <= lo <= 255 and 256 * hi + lo == w
+
+
 def test_int32_accumulation_cannot_overflow_at_the_largest_shapes():
+    # 3-bit prod attention, key side: 256 code (and 128 sign) positions of |piece| <= 127, the hi
+    # sum scaled by 2^14 and added to the mid sum scaled by 2^7 and the lo sum
+    assert 256 * 127 * 16384 + 256 * 64 * 128 + 256 * 64 < 2 ** 31
+    # value side: 1024 tokens (the largest chunk) of u8 pieces <= 255 times a 0/16 plane value,
+    # and the chunk sum of 16-bit weights
+    assert 1024 * 255 * 16 < 2 ** 31 and 1024 * 65535 < 2 ** 31
+    # the 4-bit kernel's hi sum over 8 planes x 128 coordinates is formed in float (exact below 2^24)
+    assert 8 * 128 * 127 < 2 ** 24
     # 4-bit search at d = 1536: 8 planes x d coordinates of 0/1 (or 16) bytes against |piece| <= 127
     worst = 16 * 127 * 8 * 1536
     assert worst < 2 ** 31
