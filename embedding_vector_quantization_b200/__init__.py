@@ -17,7 +17,8 @@ from . import _lib
 from ._lib import (  # noqa: F401  (the C ABI, same names)
     TQ_BF16, TQ_EINVAL, TQ_ECAPACITY, TQ_ECUDA, TQ_ENOMEM, TQ_ETIMEOUT, TQ_EUNSUPPORTED, TQ_F16, TQ_F32, TQ_OK,
     TQError, make_cache, tq_append, tq_attn_decode, tq_attn_decode_noalloc, tq_decode_step, tq_attn_workspace_bytes, tq_code_bytes, tq_codebook_host,
-    tq_create, tq_create_prod, tq_destroy, tq_encode, tq_get_codebook, tq_get_info, tq_get_rotation,
+    tq_create, tq_create_polar, tq_create_prod, tq_destroy, tq_get_polar_codebook, tq_polar_codebook_host,
+    tq_polar_info, tq_encode, tq_get_codebook, tq_get_info, tq_get_rotation,
     tq_last_error, tq_last_status, tq_pack_indices, tq_rotation_host, tq_score, tq_score_workspace_bytes,
     tq_search_topk, tq_search_workspace_bytes, tq_selftest_wait_timeout, tq_set_norm_dtype, tq_timer_enable,
     tq_timer_read,
@@ -33,7 +34,8 @@ class Handle:
     """Owns one library handle: Pi, S, S Pi^T and the codebook on the current device.
 
     ``bits`` is the total bits per coordinate; with ``qjl_m > 0`` it splits into
-    ``bits - 1`` MSE bits plus one QJL sign per projection.
+    ``bits - 1`` MSE bits plus one QJL sign per projection. ``bits = 1`` with
+    ``qjl_m > 0`` gives QJL-only rows: the signs and the norm, no codes.
     """
 
     def __init__(self, d, bits, seed=0, qjl_m=0, norm_dtype=None):
@@ -47,6 +49,10 @@ class Handle:
     @property
     def prod(self):
         return self.m > 0
+
+    @property
+    def qjl_only(self):
+        return self.m > 0 and self.bits_mse == 0
 
     @property
     def ptr(self):
@@ -77,11 +83,13 @@ class Handle:
         """Empty packed storage for vectors of leading shape ``shape``."""
         torch = _torch()
         shape = tuple(shape) if isinstance(shape, (tuple, list)) else (shape,)
-        out = {"codes": torch.empty(shape + (self.codes_B,), dtype=torch.uint8, device=device),
-               "norms": torch.empty(shape, dtype=self.norm_torch_dtype(), device=device),
+        out = {"codes": None, "norms": torch.empty(shape, dtype=self.norm_torch_dtype(), device=device),
                "signs": None, "rnorms": None}
+        if self.codes_B:
+            out["codes"] = torch.empty(shape + (self.codes_B,), dtype=torch.uint8, device=device)
         if self.prod:
             out["signs"] = torch.empty(shape + (self.signs_B,), dtype=torch.uint8, device=device)
+        if self.prod and not self.qjl_only:
             out["rnorms"] = torch.empty(shape, dtype=torch.float16, device=device)
         return out
 
@@ -118,6 +126,26 @@ class Handle:
         return idx, score
 
 
+class PolarHandle(Handle):
+    """Recursive polar transform handle ("PolarQuant explainer", sections 1 and 3): log2(d)
+    levels of angles, ``bits_level1`` bits at level 1 and ``bits_upper`` at the others."""
+
+    def __init__(self, d, bits_level1, bits_upper, seed=0, norm_dtype=None):
+        self._h = tq_create_polar(d, bits_level1, bits_upper, seed)
+        if norm_dtype is not None:
+            tq_set_norm_dtype(self._h, norm_dtype)
+        self.d, self.bits_mse, self.m, self.norm_dtype = tq_get_info(self._h)
+        self.codes_B, self.signs_B = tq_code_bytes(self._h)
+        self.levels, self.bits_level1, self.bits_upper = tq_polar_info(self._h)
+        self.seed = seed
+
+    def level_bits(self):
+        return [self.bits_level1] + [self.bits_upper] * (self.levels - 1)
+
+    def codebook(self, level=1):
+        return tq_get_polar_codebook(self._h, level, self.level_bits()[level - 1])
+
+
 class Cache:
     """A quantized K or V cache [B][Hkv][L_cap] for one handle (tensors + ABI struct)."""
 
@@ -136,11 +164,9 @@ class Cache:
                       self.rnorms, stream)
             return
         tmp = self.handle.encode(x.contiguous(), stream=stream)
-        self.codes[:, :, :L].copy_(tmp["codes"])
-        self.norms[:, :, :L].copy_(tmp["norms"])
-        if self.handle.prod:
-            self.signs[:, :, :L].copy_(tmp["signs"])
-            self.rnorms[:, :, :L].copy_(tmp["rnorms"])
+        for name in ("codes", "norms", "signs", "rnorms"):
+            if tmp[name] is not None:
+                getattr(self, name)[:, :, :L].copy_(tmp[name])
 
     def append(self, x_new, len_, advance=True, stream=None):
         tq_append(self.handle.ptr, x_new.contiguous(), self.B, self.Hkv, self.struct, len_, advance, stream)

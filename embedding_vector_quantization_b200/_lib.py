@@ -49,6 +49,10 @@ _SIGS = {
     "tq_rotation_host": (_i, [_i, _i, _u64, _dp, _dp]),
     "tq_create": (_i, [_i, _i, _u64, ctypes.POINTER(_vp)]),
     "tq_create_prod": (_i, [_i, _i, _i, _u64, ctypes.POINTER(_vp)]),
+    "tq_create_polar": (_i, [_i, _i, _i, _u64, ctypes.POINTER(_vp)]),
+    "tq_polar_info": (_i, [_vp, _ip, _ip, _ip]),
+    "tq_get_polar_codebook": (_i, [_vp, _i, _dp, _dp]),
+    "tq_polar_codebook_host": (_i, [_i, _i, _dp, _dp]),
     "tq_set_norm_dtype": (_i, [_vp, _i]),
     "tq_destroy": (None, [_vp]),
     "tq_get_info": (_i, [_vp, _ip, _ip, _ip, _ip]),
@@ -148,6 +152,32 @@ def tq_create_prod(d, bits, qjl_m, seed):
     h = _vp()
     check(lib.tq_create_prod(d, bits, qjl_m, seed, ctypes.byref(h)), "tq_create_prod")
     return h
+
+
+def tq_create_polar(d, bits_level1, bits_upper, seed):
+    h = _vp()
+    check(lib.tq_create_polar(d, bits_level1, bits_upper, seed, ctypes.byref(h)), "tq_create_polar")
+    return h
+
+
+def tq_polar_info(h):
+    n, b1, bu = ctypes.c_int(), ctypes.c_int(), ctypes.c_int()
+    check(lib.tq_polar_info(h, ctypes.byref(n), ctypes.byref(b1), ctypes.byref(bu)), "tq_polar_info")
+    return n.value, b1.value, bu.value
+
+
+def tq_get_polar_codebook(h, level, bits):
+    c = np.zeros(1 << bits)
+    b = np.zeros((1 << bits) - 1)
+    check(lib.tq_get_polar_codebook(h, level, _dptr(c), _dptr(b)), "tq_get_polar_codebook")
+    return c, b
+
+
+def tq_polar_codebook_host(level, bits):
+    c = np.zeros(1 << bits)
+    b = np.zeros((1 << bits) - 1)
+    check(lib.tq_polar_codebook_host(level, bits, _dptr(c), _dptr(b)), "tq_polar_codebook_host")
+    return c, b
 
 
 def tq_set_norm_dtype(h, dtype):

@@ -130,7 +130,8 @@ __global__ void __launch_bounds__(kRowsThreads) encode_rows_kernel(EncodeArgs a,
   const int ngroups = d / 32;
   for (int w = tid; w < R * ngroups; w += blockDim.x) {
     const int r = w / ngroups, grp = w % ngroups;
-    uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + out_row(r) * (int64_t)a.codes_B) + grp * bits;
+    // QJL-only rows (0 MSE bits): no codes; idx stays 0 (centroid 0) and nothing is written
+    uint32_t* dst = bits ? reinterpret_cast<uint32_t*>(a.codes + out_row(r) * (int64_t)a.codes_B) + grp * bits : nullptr;
     uint64_t win = 0;
     int nb = 0, wout = 0;
     float e2 = 0.f;
@@ -153,7 +154,8 @@ __global__ void __launch_bounds__(kRowsThreads) encode_rows_kernel(EncodeArgs a,
   __syncthreads();
   if (m > 0) {
     // rnorm = ||x|| * ||e||; z = (S Pi^T) e, one thread per projection i and a stride of rows
-    if (tid < R) a.rnorms[out_row(tid)] = __double2half(nrm[tid] > 0.0 ? nrm[tid] * sqrt((double)esq[tid]) : 0.0);
+    if (tid < R && a.rnorms)   // QJL-only rows keep the norm alone
+      a.rnorms[out_row(tid)] = __double2half(nrm[tid] > 0.0 ? nrm[tid] * sqrt((double)esq[tid]) : 0.0);
     const int pgroups = max(1, (int)blockDim.x / m);
     for (int base = tid; base < m * pgroups; base += blockDim.x) {
       const int i = base % m, rg = base / m;

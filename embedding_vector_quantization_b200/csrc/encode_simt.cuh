@@ -167,7 +167,9 @@ __global__ void __launch_bounds__(kEncThreads) encode_simt_kernel(EncodeArgs a) 
     const int64_t orow = (r < a.rows) ? encode_out_row(a, r) : -1;
     float e2 = 0.f;
     if (orow >= 0 && jg < d) {
-      uint32_t* dst = reinterpret_cast<uint32_t*>(a.codes + orow * (int64_t)a.codes_B) + (jg >> 5) * a.bits;
+      // QJL-only rows (0 MSE bits) have no codes: idx stays 0 (centroid 0) and nothing is written
+      uint32_t* dst = a.bits ? reinterpret_cast<uint32_t*>(a.codes + orow * (int64_t)a.codes_B) + (jg >> 5) * a.bits
+                             : nullptr;
       uint64_t win = 0;
       int nb = 0, wout = 0;
       for (int t = 0; t < 32; ++t) {
@@ -199,7 +201,7 @@ __global__ void __launch_bounds__(kEncThreads) encode_simt_kernel(EncodeArgs a) 
     const int64_t r = v0 + tid;
     if (r < a.rows) {
       const int64_t orow = encode_out_row(a, r);
-      if (orow >= 0) {
+      if (orow >= 0 && a.rnorms) {   // QJL-only rows keep the norm alone
         const double nn = nsq[tid];
         a.rnorms[orow] = __double2half(nn > 0.0 ? nn * sqrt((double)esq[tid]) : 0.0);
       }

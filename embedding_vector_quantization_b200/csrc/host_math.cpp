@@ -19,6 +19,10 @@
 //    closed form of int t (1 - t^2)^k dt;
 //  * Lloyd start at the quantiles (i + 1/2) / L, stop when no centroid moves by
 //    1e-15 (or 1e5 iterations), then force exact odd symmetry.
+//
+// The angle codebooks of the recursive polar transform ("PolarQuant explainer"
+// (aibr.jp), sections 1 and 3: angles quantized with codebooks designed from their
+// analytic distribution) follow the same Lloyd iteration on each level's law.
 
 #include "host_math.h"
 
@@ -258,6 +262,91 @@ int codebook(int d, int bits, double* centroids, double* bounds) {
     if (step < 1e-15) break;
   }
   for (int i = 0; i < L; ++i) centroids[i] = 0.5 * (c[i] - c[L - 1 - i]);
+  for (int i = 0; i + 1 < L; ++i) bounds[i] = 0.5 * (centroids[i] + centroids[i + 1]);
+  return 0;
+}
+
+// ---------------------------------------------------------------- polar angle codebooks
+
+namespace {
+
+// Law of a level-l angle of the recursive polar transform of a uniform direction, l >= 2:
+// density proportional to (sin psi cos psi)^(k-1) = (sin(2 psi) / 2)^(k-1) on [0, pi/2],
+// k = 2^(l-1). Masses and first moments by composite Gauss-Legendre quadrature of the
+// integrand scaled to 1 at its peak, sin(2 psi)^(k-1).
+struct AngleLaw {
+  double p;      // exponent k - 1
+  double panel;  // quadrature panel width
+  double Z;      // total mass of the scaled integrand
+
+  explicit AngleLaw(int k) : p(k - 1.0) {
+    panel = std::min(0.05, 0.3 / std::sqrt(static_cast<double>(k)));
+    Z = raw(0.0, 0.5 * M_PI, false);
+  }
+  double integrand(double psi) const {
+    const double s = std::sin(2.0 * psi);
+    if (p == 0.0) return 1.0;
+    if (s <= 0.0) return 0.0;
+    return std::exp(p * std::log(s));
+  }
+  double raw(double lo, double hi, bool first_moment) const {
+    if (hi <= lo) return 0.0;
+    const int panels = std::max(1, static_cast<int>(std::ceil((hi - lo) / panel)));
+    const double h = (hi - lo) / panels;
+    const GaussLegendre& g = gl();
+    double sum = 0.0;
+    for (int pi = 0; pi < panels; ++pi) {
+      const double mid = lo + (pi + 0.5) * h;
+      double acc = 0.0;
+      for (int i = 0; i < GaussLegendre::kN; ++i) {
+        const double t = mid + 0.5 * h * g.x[i];
+        acc += g.w[i] * integrand(t) * (first_moment ? t : 1.0);
+      }
+      sum += 0.5 * h * acc;
+    }
+    return sum;
+  }
+  double mass(double a, double b) const { return raw(a, b, false) / Z; }
+  double moment(double a, double b) const { return raw(a, b, true) / Z; }
+};
+
+}  // namespace
+
+int polar_codebook(int level, int bits, double* centroids, double* bounds) {
+  if (level < 1 || level > 16 || bits < 1 || bits > 8) return -1;
+  const int L = 1 << bits;
+  if (level == 1) {
+    // uniform on (-pi, pi]: the Lloyd fixed point is the uniform grid of L cells
+    for (int i = 0; i < L; ++i) centroids[i] = -M_PI + (2.0 * i + 1.0) * M_PI / L;
+    for (int i = 0; i + 1 < L; ++i) bounds[i] = -M_PI + 2.0 * (i + 1) * M_PI / L;
+    return 0;
+  }
+  const AngleLaw law(1 << (level - 1));
+  const double top = 0.5 * M_PI;
+  std::vector<double> c(L), nc(L), edge(L + 1);
+  for (int i = 0; i < L; ++i) {   // start at the quantiles (i + 1/2) / L
+    const double target = (i + 0.5) / L;
+    double lo = 0.0, hi = top;
+    for (int it = 0; it < 200 && hi - lo > 1e-16; ++it) {
+      const double mid = 0.5 * (lo + hi);
+      (law.mass(0.0, mid) < target ? lo : hi) = mid;
+    }
+    c[i] = 0.5 * (lo + hi);
+  }
+  for (int it = 0; it < 100000; ++it) {
+    edge[0] = 0.0;
+    edge[L] = top;
+    for (int i = 0; i + 1 < L; ++i) edge[i + 1] = 0.5 * (c[i] + c[i + 1]);
+    double step = 0.0;
+    for (int i = 0; i < L; ++i) {
+      nc[i] = law.moment(edge[i], edge[i + 1]) / law.mass(edge[i], edge[i + 1]);
+      step = std::max(step, std::fabs(nc[i] - c[i]));
+    }
+    c.swap(nc);
+    if (step < 1e-15) break;
+  }
+  // the law is symmetric about pi/4
+  for (int i = 0; i < L; ++i) centroids[i] = 0.5 * (c[i] + (top - c[L - 1 - i]));
   for (int i = 0; i + 1 < L; ++i) bounds[i] = 0.5 * (centroids[i] + centroids[i + 1]);
   return 0;
 }

@@ -18,4 +18,10 @@ void rotation(int d, int m, uint64_t seed, double* Pi, double* S);
 // Returns 0, or -1 for d < 3 or bits outside 1..8.
 int codebook(int d, int bits, double* centroids, double* bounds);
 
+// Lloyd-Max codebook of the level-`level` angle of the recursive polar transform of a
+// uniform direction: level 1 is uniform on (-pi, pi] (uniform grid); level l >= 2 has
+// density proportional to (sin psi cos psi)^(2^(l-1) - 1) on [0, pi/2].
+// Returns 0, or -1 for level outside 1..16 or bits outside 1..8.
+int polar_codebook(int level, int bits, double* centroids, double* bounds);
+
 }  // namespace tqhost

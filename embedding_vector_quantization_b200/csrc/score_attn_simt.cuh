@@ -92,23 +92,29 @@ __global__ void __launch_bounds__(256) qprep_kernel(const void* q, int q_dtype, 
 // ---------------------------------------------------------------- cache view
 
 struct CacheView {
-  const uint8_t* codes;
+  const uint8_t* codes;   // NULL for QJL-only rows (bits == 0)
   const uint8_t* signs;
   const void* norms;
-  const __half* rnorms;
+  const __half* rnorms;   // NULL for QJL-only rows: the norm weighs the signs
   int bits, m, norm_dtype, codes_B, signs_B;
   const float* cent;
 };
+
+// Weight of a row's sign sum: the residual norm (prod), or the norm itself (QJL-only rows,
+// whose sketch is of the whole vector: "TurboQuant: redefining AI efficiency", "QJL").
+__device__ __forceinline__ float qjl_norm(const CacheView& c, int64_t row) {
+  return c.rnorms ? __half2float(c.rnorms[row]) : load_norm(c.norms, c.norm_dtype, row);
+}
 
 // MSE and QJL parts of G query scores for one key row (thread-serial over d).
 __device__ __forceinline__ void key_scores(const CacheView& c, int64_t row, int d, int G,
                                            const float* qr_s, const float* qs_s, const float* cen,
                                            float* out) {
-  const uint32_t* cw = reinterpret_cast<const uint32_t*>(c.codes + row * (int64_t)c.codes_B);
   float am[kMaxGroup];
 #pragma unroll
   for (int g = 0; g < kMaxGroup; ++g) am[g] = 0.f;
-  for (int j = 0; j < d; ++j) {
+  const uint32_t* cw = c.bits ? reinterpret_cast<const uint32_t*>(c.codes + row * (int64_t)c.codes_B) : nullptr;
+  for (int j = 0; c.bits && j < d; ++j) {
     const float cv = cen[packed_field(cw, j, c.bits)];
 #pragma unroll
     for (int g = 0; g < kMaxGroup; ++g)
@@ -128,7 +134,7 @@ __device__ __forceinline__ void key_scores(const CacheView& c, int64_t row, int 
       for (int g = 0; g < kMaxGroup; ++g)
         if (g < G) as[g] = fmaf(qs_s[g * c.m + j], pm, as[g]);
     }
-    const float w = __half2float(c.rnorms[row]) * (kQjlScale / (float)c.m);
+    const float w = qjl_norm(c, row) * (kQjlScale / (float)c.m);
 #pragma unroll
     for (int g = 0; g < kMaxGroup; ++g) out[g] = fmaf(w, as[g], out[g]);
   }
@@ -231,7 +237,7 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_simt_kernel(AttnArgs 
     if (i < end) {
       key_scores(a.k, base + i, d, G, qr_s, qs_s, kcen, s);
       wv_s[tid] = load_norm(a.v.norms, a.v.norm_dtype, base + i);
-      wr_s[tid] = (mv > 0) ? __half2float(a.v.rnorms[base + i]) : 0.f;  // sqrt(pi/2)/m applied in combine
+      wr_s[tid] = (mv > 0) ? qjl_norm(a.v, base + i) : 0.f;  // sqrt(pi/2)/m applied in combine
     } else {
 #pragma unroll
       for (int g = 0; g < kMaxGroup; ++g) s[g] = -INFINITY;
@@ -277,12 +283,12 @@ __global__ void __launch_bounds__(kAttnThreads) attn_split_simt_kernel(AttnArgs 
     const int nk = (int)min((int64_t)kAttnThreads, end - sb);
     for (int t = 0; t < nk; ++t) {
       const int64_t row = base + sb + t;
-      const uint32_t* vw = reinterpret_cast<const uint32_t*>(a.v.codes + row * (int64_t)a.v.codes_B);
+      const uint32_t* vw = a.v.bits ? reinterpret_cast<const uint32_t*>(a.v.codes + row * (int64_t)a.v.codes_B) : nullptr;
       const float wn = wv_s[t];
 #pragma unroll
       for (int r = 0; r < 2; ++r) {
         const int j = tid + r * kAttnThreads;
-        if (j < d) {
+        if (j < d && a.v.bits) {   // QJL-only values have no MSE part
           const float cv = vcen[packed_field(vw, j, a.v.bits)] * wn;
 #pragma unroll
           for (int g = 0; g < kMaxGroup; ++g)

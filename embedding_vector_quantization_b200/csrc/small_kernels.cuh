@@ -102,7 +102,7 @@ __device__ __forceinline__ int32_t append_vector(const EncodeArgs& a, int b, int
         for (int o = 16; o > 0; o >>= 1) e2 += __shfl_xor_sync(0xffffffffu, e2, o);
         if (lane == 0) red[warp] = e2;
         __syncthreads();
-        if (tid == 0) {
+        if (tid == 0 && a.rnorms) {   // QJL-only rows keep the norm alone
           float t = 0.f;
           for (int w = 0; w < kSmallThreads / 32; ++w) t += red[w];
           a.rnorms[orow] = __double2half(nn > 0.0 ? nn * sqrt((double)t) : 0.0);

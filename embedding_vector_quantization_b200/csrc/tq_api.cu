@@ -36,6 +36,7 @@
 #include "attn_mse4.cuh"
 #include "search_mma.cuh"
 #include "search_mma4.cuh"
+#include "polar.cuh"
 
 struct tq_handle {
   int d = 0, bits = 0, m = 0, norm_dtype = TQ_F32;
@@ -52,6 +53,11 @@ struct tq_handle {
   float* dbnd = nullptr;  // [2^bits - 1]
   int* derr = nullptr;    // device error word
   uint8_t* dOps = nullptr; // d = 128: pre-swizzled 16-bit hi/lo operands of the tensor-core encode
+  // recursive polar transform handles (tq_create_polar): per-level angle codebooks
+  int polar = 0;
+  tqk::polar::Layout play{};
+  std::vector<std::vector<double>> pcent, pbnd;
+  tqk::polar::Table* dTab = nullptr;
 };
 
 namespace {
@@ -165,9 +171,11 @@ void free_device(tq_handle* h) {
   cudaFree(h->dbnd);
   cudaFree(h->derr);
   cudaFree(h->dOps);
+  cudaFree(h->dTab);
   h->dPi = h->dPiT = h->dS = h->dST = h->dMT = h->dcent = h->dbnd = nullptr;
   h->derr = nullptr;
   h->dOps = nullptr;
+  h->dTab = nullptr;
 }
 
 template <typename T>
@@ -231,7 +239,7 @@ int create_common(int d, int bits_mse, int m, uint64_t seed, int norm_dtype, tq_
   *out = nullptr;
   if (d < 32 || d > 4096) return fail(TQ_EUNSUPPORTED, "d=%d outside 32..4096", d);
   if (d % 32 != 0) return fail(TQ_EUNSUPPORTED, "d=%d is not a multiple of 32", d);
-  if (bits_mse < 1 || bits_mse > 4) return fail(TQ_EUNSUPPORTED, "MSE bits=%d outside 1..4", bits_mse);
+  if (bits_mse < (m > 0 ? 0 : 1) || bits_mse > 4) return fail(TQ_EUNSUPPORTED, "MSE bits=%d outside 1..4", bits_mse);
   if (m < 0 || m % 32 != 0 || m > 1024) return fail(TQ_EUNSUPPORTED, "qjl_m=%d (needs m %% 32 == 0, m <= 1024)", m);
   if (m > 0 && d > tqk::kEncBN) return fail(TQ_EUNSUPPORTED, "prod handles need d <= %d", tqk::kEncBN);
   if (fault_is("alloc")) return fail(TQ_ENOMEM, "injected allocation failure (TQ_FAULT=alloc)");
@@ -254,7 +262,10 @@ int create_common(int d, int bits_mse, int m, uint64_t seed, int norm_dtype, tq_
   h->cent.resize(L);
   h->bnd.resize(L - 1);
   tqhost::rotation(d, m, seed, h->Pi.data(), m ? h->S.data() : nullptr);
-  if (tqhost::codebook(d, bits_mse, h->cent.data(), h->bnd.data()) != 0) {
+  if (bits_mse == 0) {
+    // QJL-only rows: no MSE stage; its one-cell codebook is the coordinate law's mean, 0
+    h->cent[0] = 0.0;
+  } else if (tqhost::codebook(d, bits_mse, h->cent.data(), h->bnd.data()) != 0) {
     delete h;
     return fail(TQ_EINVAL, "codebook(d=%d, bits=%d) failed", d, bits_mse);
   }
@@ -295,12 +306,114 @@ int create_common(int d, int bits_mse, int m, uint64_t seed, int norm_dtype, tq_
   return ok();
 }
 
+// Recursive polar transform handle: d a power of two (32 .. 256), log2 d levels, bits1 at
+// level 1 and bits_up at every further level (each 1..4); Pi as for the MSE path (seed).
+int create_polar(int d, int bits1, int bits_up, uint64_t seed, tq_handle** out) {
+  if (!out) return fail(TQ_EINVAL, "out is NULL");
+  *out = nullptr;
+  if (d < 32 || d > 256 || (d & (d - 1)) != 0)
+    return fail(TQ_EUNSUPPORTED, "polar handles need d a power of two in 32..256 (d=%d)", d);
+  if (bits1 < 1 || bits1 > 4 || bits_up < 1 || bits_up > 4)
+    return fail(TQ_EUNSUPPORTED, "polar level bits %d/%d outside 1..4", bits1, bits_up);
+  if (fault_is("alloc")) return fail(TQ_ENOMEM, "injected allocation failure (TQ_FAULT=alloc)");
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return cuda_fail(e, "cudaGetDevice");
+  tq_handle* h = new tq_handle();
+  h->d = d;
+  h->bits = 0;
+  h->m = 0;
+  h->seed = seed;
+  h->norm_dtype = TQ_F32;
+  h->device = dev;
+  h->polar = 1;
+  int nlev = 0;
+  while ((1 << nlev) < d) ++nlev;
+  h->play.d = d;
+  h->play.nlev = nlev;
+  int off = 0;
+  tqk::polar::Table tab{};
+  h->pcent.resize(nlev);
+  h->pbnd.resize(nlev);
+  for (int l = 0; l < nlev; ++l) {
+    const int b = l == 0 ? bits1 : bits_up, L = 1 << b;
+    h->play.bits[l] = b;
+    h->play.off[l] = off;
+    off += (d >> (l + 1)) * b;
+    h->pcent[l].resize(L);
+    h->pbnd[l].resize(L - 1);
+    if (tqhost::polar_codebook(l + 1, b, h->pcent[l].data(), h->pbnd[l].data()) != 0) {
+      delete h;
+      return fail(TQ_EINVAL, "polar codebook (level %d, %d bits) failed", l + 1, b);
+    }
+    for (int i = 0; i < 16; ++i) tab.bnd[l][i] = i < L - 1 ? (float)h->pbnd[l][i] : INFINITY;
+    for (int i = 0; i < L; ++i) {
+      tab.cs[l][i] = (float)std::cos(h->pcent[l][i]);
+      tab.sn[l][i] = (float)std::sin(h->pcent[l][i]);
+    }
+  }
+  h->codes_B = 16 * ((off + 127) / 128);
+  h->signs_B = 0;
+  h->Pi.resize((size_t)d * d);
+  tqhost::rotation(d, 0, seed, h->Pi.data(), nullptr);
+  std::vector<float> Pi(h->Pi.begin(), h->Pi.end()), PiT((size_t)d * d);
+  for (int i = 0; i < d; ++i)
+    for (int j = 0; j < d; ++j) PiT[(size_t)j * d + i] = (float)h->Pi[(size_t)i * d + j];
+  std::vector<uint8_t> tb(sizeof(tab));
+  std::memcpy(tb.data(), &tab, sizeof(tab));
+  int st = TQ_OK;
+  if ((st = upload(&h->dPi, Pi, "Pi")) || (st = upload(&h->dPiT, PiT, "PiT")) ||
+      (st = upload(reinterpret_cast<uint8_t**>(&h->dTab), tb, "polar tables"))) {
+    free_device(h);
+    delete h;
+    return st;
+  }
+  e = cudaMalloc(&h->derr, sizeof(int));
+  if (e == cudaSuccess) e = cudaMemset(h->derr, 0, sizeof(int));
+  if (e != cudaSuccess) {
+    free_device(h);
+    delete h;
+    return fail(TQ_ENOMEM, "cudaMalloc(error word): %s", cudaGetErrorString(e));
+  }
+  *out = h;
+  return ok();
+}
+
+int polar_encode_launch(const tq_handle* h, const void* x, int x_dtype, int64_t n, uint8_t* codes, void* norms,
+                        int32_t* len, int Hkv, int64_t L_cap, cudaStream_t s) {
+  tqk::polar::EncodeArgs a{};
+  a.x = x; a.x_dtype = x_dtype; a.rows = n; a.lay = h->play; a.norm_dtype = h->norm_dtype; a.PiT = h->dPiT;
+  a.tab = h->dTab; a.codes = codes; a.codes_B = h->codes_B; a.norms = norms; a.len = len; a.Hkv = Hkv;
+  a.L_cap = L_cap; a.err = h->derr;
+  const size_t smem = tqk::polar::encode_smem_bytes(h->d);
+  if (once_per_device(14, h->device))
+    cudaFuncSetAttribute(tqk::polar::polar_encode_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  KernelScope ks(len ? "append" : "encode", s);
+  tqk::polar::polar_encode_kernel<<<(unsigned)((n + tqk::polar::kBM - 1) / tqk::polar::kBM), tqk::polar::kThreads,
+                                    smem, s>>>(a);
+  return launch_check("polar_encode_kernel");
+}
+
+template <int D>
+int polar_score_launch_d(const tq_handle* h, const tqk::polar::ScoreArgs& a, dim3 grid, size_t smem, cudaStream_t s) {
+  static std::atomic<uint64_t> attr_done{0};
+  const uint64_t bit = 1ull << (h->device & 63);
+  if ((attr_done.fetch_or(bit) & bit) == 0)
+    cudaFuncSetAttribute(tqk::polar::polar_score_kernel<D>, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
+  KernelScope ks("score", s);
+  tqk::polar::polar_score_kernel<D><<<grid, tqk::polar::kSThreads, smem, s>>>(a);
+  return launch_check("polar_score_kernel");
+}
+
+// QJL-only handles (prod with no MSE bits) store signs and the norm only: no codes, no rnorms.
+bool qjl_only(const tq_handle* h) { return h->m > 0 && h->bits == 0; }
+
 tqk::CacheView view_of(const tq_handle* h, const tq_cache* c) {
   tqk::CacheView v;
   v.codes = c->codes;
   v.signs = c->signs;
   v.norms = c->norms;
-  v.rnorms = static_cast<const __half*>(c->rnorms);
+  v.rnorms = qjl_only(h) ? nullptr : static_cast<const __half*>(c->rnorms);
   v.bits = h->bits;
   v.m = h->m;
   v.norm_dtype = h->norm_dtype;
@@ -312,10 +425,11 @@ tqk::CacheView view_of(const tq_handle* h, const tq_cache* c) {
 
 int check_cache(const tq_handle* h, const tq_cache* c, const char* name) {
   if (!c) return fail(TQ_EINVAL, "%s cache is NULL", name);
-  if (!c->codes || !c->norms) return fail(TQ_EINVAL, "%s cache: codes/norms NULL", name);
-  if (h->m > 0 && (!c->signs || !c->rnorms)) return fail(TQ_EINVAL, "%s cache: prod handle needs signs and rnorms", name);
+  if ((!c->codes && h->codes_B > 0) || !c->norms) return fail(TQ_EINVAL, "%s cache: codes/norms NULL", name);
+  if (h->m > 0 && !c->signs) return fail(TQ_EINVAL, "%s cache: prod handle needs signs", name);
+  if (h->m > 0 && !qjl_only(h) && !c->rnorms) return fail(TQ_EINVAL, "%s cache: prod handle needs rnorms", name);
   if (c->L_cap < 1) return fail(TQ_EINVAL, "%s cache: L_cap=%lld", name, (long long)c->L_cap);
-  if (!aligned(c->codes, 16) || (c->signs && !aligned(c->signs, 16)) || !aligned(c->norms, 4) ||
+  if ((c->codes && !aligned(c->codes, 16)) || (c->signs && !aligned(c->signs, 16)) || !aligned(c->norms, 4) ||
       (c->rnorms && !aligned(c->rnorms, 2)))
     return fail(TQ_EINVAL, "%s cache: misaligned pointer", name);
   return TQ_OK;
@@ -581,7 +695,7 @@ int codes_map_2d(const uint8_t* codes, int64_t rows, int row_bytes, int box_byte
 
 bool tc_encode_ok(const tq_handle* h, const tqk::EncodeArgs& a) {
   if (std::getenv("TQ_SIMT")) return false;
-  return h->dOps && a.len == nullptr && (a.x_dtype == TQ_BF16 || a.x_dtype == TQ_F16) && a.rows >= 1024 &&
+  return h->dOps && h->bits > 0 && a.len == nullptr && (a.x_dtype == TQ_BF16 || a.x_dtype == TQ_F16) && a.rows >= 1024 &&
          a.rows < (int64_t)1 << 31;
 }
 
@@ -699,9 +813,38 @@ int tq_create(int d, int bits, uint64_t seed, tq_handle** out) {
 }
 
 int tq_create_prod(int d, int bits, int qjl_m, uint64_t seed, tq_handle** out) {
-  if (bits < 2 || bits > 5) return fail(TQ_EUNSUPPORTED, "prod bits=%d outside 2..5", bits);
+  if (bits < 1 || bits > 5) return fail(TQ_EUNSUPPORTED, "prod bits=%d outside 1..5", bits);
   if (qjl_m < 32) return fail(TQ_EUNSUPPORTED, "qjl_m=%d < 32", qjl_m);
   return create_common(d, bits - 1, qjl_m, seed, TQ_F16, out);
+}
+
+int tq_create_polar(int d, int bits_level1, int bits_upper, uint64_t seed, tq_handle** out) {
+  return create_polar(d, bits_level1, bits_upper, seed, out);
+}
+
+int tq_polar_info(const tq_handle* h, int* nlevels, int* bits_level1, int* bits_upper) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (!h->polar) return fail(TQ_EINVAL, "not a polar handle");
+  if (nlevels) *nlevels = h->play.nlev;
+  if (bits_level1) *bits_level1 = h->play.bits[0];
+  if (bits_upper) *bits_upper = h->play.bits[1];
+  return ok();
+}
+
+int tq_get_polar_codebook(const tq_handle* h, int level, double* centroids, double* bounds) {
+  if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (!h->polar) return fail(TQ_EINVAL, "not a polar handle");
+  if (level < 1 || level > h->play.nlev) return fail(TQ_EINVAL, "level %d outside 1..%d", level, h->play.nlev);
+  if (centroids) std::memcpy(centroids, h->pcent[level - 1].data(), h->pcent[level - 1].size() * sizeof(double));
+  if (bounds) std::memcpy(bounds, h->pbnd[level - 1].data(), h->pbnd[level - 1].size() * sizeof(double));
+  return ok();
+}
+
+int tq_polar_codebook_host(int level, int bits, double* centroids, double* bounds) {
+  if (!centroids || !bounds) return fail(TQ_EINVAL, "NULL output");
+  if (level < 1 || level > 16 || bits < 1 || bits > 8) return fail(TQ_EINVAL, "level=%d bits=%d out of range", level, bits);
+  if (tqhost::polar_codebook(level, bits, centroids, bounds) != 0) return fail(TQ_EINVAL, "polar codebook failed");
+  return ok();
 }
 
 int tq_set_norm_dtype(tq_handle* h, int dtype) {
@@ -735,6 +878,7 @@ int tq_code_bytes(const tq_handle* h, int* codes_B, int* signs_B) {
 
 int tq_get_codebook(const tq_handle* h, double* centroids, double* bounds) {
   if (!h) return fail(TQ_EINVAL, "handle is NULL");
+  if (h->polar) return fail(TQ_EINVAL, "polar handles have one codebook per level (tq_get_polar_codebook)");
   if (centroids) std::memcpy(centroids, h->cent.data(), h->cent.size() * sizeof(double));
   if (bounds) std::memcpy(bounds, h->bnd.data(), h->bnd.size() * sizeof(double));
   return ok();
@@ -753,11 +897,13 @@ int tq_encode(const tq_handle* h, const void* x, int x_dtype, int64_t n, uint8_t
   if (n < 0) return fail(TQ_EINVAL, "n=%lld", (long long)n);
   if (!valid_dtype(x_dtype)) return fail(TQ_EINVAL, "x dtype %d", x_dtype);
   if (n == 0) return ok();
-  if (!x || !codes || !norms) return fail(TQ_EINVAL, "x/codes/norms NULL");
-  if (h->m > 0 && (!signs || !rnorms)) return fail(TQ_EINVAL, "prod handle needs signs and rnorms");
-  if (!aligned(x, 16) || !aligned(codes, 16) || (signs && !aligned(signs, 16)) || !aligned(norms, 4))
+  if (!x || (!codes && h->codes_B > 0) || !norms) return fail(TQ_EINVAL, "x/codes/norms NULL");
+  if (h->m > 0 && (!signs || (!rnorms && !qjl_only(h)))) return fail(TQ_EINVAL, "prod handle needs signs and rnorms");
+  if (qjl_only(h)) codes = nullptr, rnorms = nullptr;   // QJL-only rows: signs and the norm
+  if (!aligned(x, 16) || (codes && !aligned(codes, 16)) || (signs && !aligned(signs, 16)) || !aligned(norms, 4))
     return fail(TQ_EINVAL, "misaligned pointer");
   if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
+  if (h->polar) return polar_encode_launch(h, x, x_dtype, n, codes, norms, nullptr, 0, 0, static_cast<cudaStream_t>(stream));
   tqk::EncodeArgs a{};
   a.x = x; a.x_dtype = x_dtype; a.rows = n; a.d = h->d; a.bits = h->bits; a.m = h->m;
   a.norm_dtype = h->norm_dtype; a.PiT = h->dPiT; a.MT = h->dMT; a.cent = h->dcent; a.bnd = h->dbnd;
@@ -770,6 +916,7 @@ int tq_pack_indices(const tq_handle* h, const uint8_t* idx, int64_t n, uint8_t* 
   if (!h) return fail(TQ_EINVAL, "handle is NULL");
   if (n < 0) return fail(TQ_EINVAL, "n=%lld", (long long)n);
   if (n == 0) return ok();
+  if (h->bits == 0) return fail(TQ_EINVAL, "QJL-only and polar handles have no MSE codes to pack");
   if (!idx || !codes) return fail(TQ_EINVAL, "NULL pointer");
   if (!aligned(codes, 4)) return fail(TQ_EINVAL, "codes misaligned");
   const int64_t work = n * (h->d / 32);
@@ -791,12 +938,22 @@ int tq_append(const tq_handle* h, const void* x_new, int x_dtype, int B, int Hkv
   if (!aligned(x_new, 16)) return fail(TQ_EINVAL, "x_new misaligned");
   if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (h->polar) {
+    if ((st = polar_encode_launch(h, x_new, x_dtype, (int64_t)B * Hkv, cache->codes, cache->norms, len, Hkv,
+                                  cache->L_cap, s)))
+      return st;
+    if (!advance) return ok();
+    KernelScope ks("advance_len", s);
+    tqk::advance_len_kernel<<<(B + 255) / 256, 256, 0, s>>>(len, B, cache->L_cap);
+    return launch_check("advance_len_kernel");
+  }
   tqk::EncodeArgs a{};
   a.x = x_new; a.x_dtype = x_dtype; a.rows = (int64_t)B * Hkv; a.d = h->d; a.bits = h->bits; a.m = h->m;
   a.norm_dtype = h->norm_dtype; a.PiT = h->dPiT; a.MT = h->dMT; a.cent = h->dcent; a.bnd = h->dbnd;
   a.codes = cache->codes; a.codes_B = h->codes_B; a.signs = cache->signs; a.signs_B = h->signs_B;
-  a.norms = cache->norms; a.rnorms = static_cast<__half*>(cache->rnorms);
+  a.norms = cache->norms; a.rnorms = qjl_only(h) ? nullptr : static_cast<__half*>(cache->rnorms);
   a.len = len; a.Hkv = Hkv; a.L_cap = cache->L_cap; a.err = h->derr;
+  if (qjl_only(h)) a.codes = nullptr;
   if (h->d <= tqk::kSmallMaxD && h->m <= tqk::kSmallMaxD && Hkv <= 8) {
     // one CTA per (sequence, head); the Hkv CTAs of a sequence form a cluster
     const size_t smem = tqk::append_cluster_smem_bytes(h->d, h->m);
@@ -869,6 +1026,25 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const 
   st = launch_qprep(hk, q, TQ_F32, B * Hq, w.qr, w.qs, s);
   if (st) return st;
   const int64_t units = (int64_t)B * Hkv;
+  if (hk->polar) {
+    if (Hq / Hkv > tqk::polar::kMaxG) return fail(TQ_EUNSUPPORTED, "polar scores need Hq/Hkv <= %d", tqk::polar::kMaxG);
+    tqk::polar::ScoreArgs pa{};
+    pa.qr = w.qr; pa.B = B; pa.Hq = Hq; pa.Hkv = Hkv; pa.lay = hk->play; pa.codes = k->codes; pa.codes_B = hk->codes_B;
+    pa.norms = k->norms; pa.norm_dtype = hk->norm_dtype; pa.tab = hk->dTab; pa.L_cap = k->L_cap; pa.len = len;
+    pa.logits = logits;
+    int64_t ns = std::max<int64_t>(1, std::min<int64_t>((8 * 148 + units - 1) / units, (k->L_cap + 127) / 128));
+    pa.chunk = ((k->L_cap + ns - 1) / ns + 127) / 128 * 128;
+    if (const int64_t f = splitk_override()) pa.chunk = round_chunk(f, 128, 128, (k->L_cap + 127) / 128 * 128);
+    ns = (k->L_cap + pa.chunk - 1) / pa.chunk;
+    const dim3 grid((unsigned)units, (unsigned)ns);
+    const size_t smem = tqk::polar::score_smem_bytes(hk->d, hk->play.bits[0], Hq / Hkv, hk->codes_B);
+    switch (hk->d) {
+      case 32: return polar_score_launch_d<32>(hk, pa, grid, smem, s);
+      case 64: return polar_score_launch_d<64>(hk, pa, grid, smem, s);
+      case 128: return polar_score_launch_d<128>(hk, pa, grid, smem, s);
+      default: return polar_score_launch_d<256>(hk, pa, grid, smem, s);
+    }
+  }
   if (score_prod2_fast_path(hk, Hq / Hkv, k)) {
     // about eight waves of 3 CTAs per SM; chunks are whole 256-key blocks
     const int64_t target = 8 * 3 * (int64_t)sm_count(hk->device);
@@ -915,6 +1091,7 @@ int attn_check(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dt
                const tq_cache* k, const tq_cache* v, const int32_t* len, float scale, float* out, void* workspace,
                size_t ws_bytes) {
   if (!hk || !hv) return fail(TQ_EINVAL, "handle is NULL");
+  if (hk->polar || hv->polar) return fail(TQ_EUNSUPPORTED, "decode attention takes MSE, prod or QJL-only handles");
   if (hk->d != hv->d) return fail(TQ_EINVAL, "K and V handles differ in d (%d vs %d)", hk->d, hv->d);
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return fail(TQ_EINVAL, "B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
   if (Hq / Hkv > tqk::kMaxGroup) return fail(TQ_EUNSUPPORTED, "group Hq/Hkv=%d > %d", Hq / Hkv, tqk::kMaxGroup);
@@ -1075,8 +1252,9 @@ int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int 
     a.x = x; a.x_dtype = x_dtype; a.rows = (int64_t)B * Hkv; a.d = h->d; a.bits = h->bits; a.m = h->m;
     a.norm_dtype = h->norm_dtype; a.PiT = h->dPiT; a.MT = h->dMT; a.cent = h->dcent; a.bnd = h->dbnd;
     a.codes = c->codes; a.codes_B = h->codes_B; a.signs = c->signs; a.signs_B = h->signs_B;
-    a.norms = c->norms; a.rnorms = static_cast<__half*>(c->rnorms);
+    a.norms = c->norms; a.rnorms = qjl_only(h) ? nullptr : static_cast<__half*>(c->rnorms);
     a.len = len; a.Hkv = Hkv; a.L_cap = c->L_cap; a.err = h->derr;
+    if (qjl_only(h)) a.codes = nullptr;
     return a;
   };
   tqk::PrologueArgs p{};
@@ -1105,7 +1283,7 @@ int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int 
 int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* codes, const void* norms, int64_t n,
                    int k, int64_t* idx, float* score, void* workspace, size_t ws_bytes, void* stream) {
   if (!h) return fail(TQ_EINVAL, "handle is NULL");
-  if (h->m > 0) return fail(TQ_EUNSUPPORTED, "search takes MSE handles");
+  if (h->m > 0 || h->polar) return fail(TQ_EUNSUPPORTED, "search takes MSE handles");
   if (nq < 0 || n < 1 || k < 1 || k > tqk::kMaxTopK || k > n)
     return fail(TQ_EINVAL, "nq=%d n=%lld k=%d", nq, (long long)n, k);
   if (nq == 0) return ok();

@@ -10,8 +10,10 @@
  *          sections "KV cache basics", "PolarQuant: Cartesian to polar", "QJL",
  *          "GPU kernel optimisation".
  *  [HAKU]  "TurboQuant: redefining AI efficiency with extreme compression"
- *          (hakusoku.com), sections "PolarQuant", "QJL", "Impact on
- *          high-dimensional vector search".
+ *          (hakusoku.com), sections "PolarQuant", "QJL: zero-overhead 1-bit
+ *          compression", "Impact on high-dimensional vector search".
+ *  [POLAR] "PolarQuant explainer" (aibr.jp), sections 1 and 3 (the recursive
+ *          polar transform and its angle codebooks).
  *  [FRAC]  "Fractal KV-cache archive" (gist.science), section "Problem
  *          statement" (amortised O(1) append to a growing cache).
  *
@@ -26,7 +28,8 @@
  *    enqueued asynchronously; no hot call synchronises. Errors the GPU detects
  *    (cache overflow, bounded-wait timeouts) are OR-ed into a per-handle
  *    device error word that tq_last_status() reads.
- *  - Sizes: d % 32 == 0, 32 <= d <= 4096; MSE bits in 1..4; QJL m % 32 == 0.
+ *  - Sizes: d % 32 == 0, 32 <= d <= 4096; MSE bits in 1..4 (0 for QJL-only
+ *    rows); QJL m % 32 == 0.
  *
  * Packed layout (one row per vector, caller-allocated, rows contiguous):
  *  - codes: ceil(d * b / 8) bytes, b = MSE bits. LSB-first contiguous: bit t of
@@ -35,6 +38,8 @@
  *  - signs (prod handles): m / 8 bytes, bit j = 1 iff projection j of the
  *    residual is >= 0.
  *  - norms: one per row, fp32 or fp16 (tq_set_norm_dtype); rnorms: fp16.
+ *  - QJL-only rows (tq_create_prod with bits = 1): no codes (codes_B = 0) and
+ *    no rnorms; signs of the projections of the whole vector, and its norm.
  */
 #ifndef TQ_H
 #define TQ_H
@@ -66,7 +71,8 @@ typedef struct tq_handle tq_handle; /* opaque; owns Pi, S, S Pi^T and the codebo
  * All pointers are device pointers, row-major in the order [B][Hkv][L_cap]
  * (then the packed row). codes/signs rows must start on 16-byte boundaries
  * (base pointers 16-byte aligned); norms/rnorms 4-byte aligned.
- * signs and rnorms are NULL for MSE-only handles. */
+ * signs and rnorms are NULL for MSE-only handles; codes and rnorms may be NULL
+ * for QJL-only handles (they are not read). */
 typedef struct tq_cache {
   uint8_t* codes;   /* [B][Hkv][L_cap][codes_B]                  */
   uint8_t* signs;   /* [B][Hkv][L_cap][signs_B] or NULL           */
@@ -84,6 +90,13 @@ typedef struct tq_cache {
  * [-1, 1] [TQ6x Stage 1]. Writes 2^bits ascending centroids and 2^bits - 1
  * boundaries (midpoints) to host arrays. 3 <= d <= 65536, 1 <= bits <= 8. */
 int tq_codebook_host(int d, int bits, double* centroids, double* bounds);
+
+/* Lloyd-Max codebook of the level-`level` angle of the recursive polar transform of
+ * a uniform direction [POLAR sections 1, 3]: level 1 is uniform on (-pi, pi] (the
+ * uniform grid); level l >= 2 has density proportional to
+ * (sin psi cos psi)^(2^(l-1) - 1) on [0, pi/2]. 2^bits ascending centroids and
+ * 2^bits - 1 midpoint boundaries (host arrays). 1 <= level <= 16, 1 <= bits <= 8. */
+int tq_polar_codebook_host(int level, int bits, double* centroids, double* bounds);
 
 /* Seeded rotation Pi (d x d, row-major, y = Pi u) = Q of a Householder QR of a
  * Gaussian matrix G with diag(R) > 0 [TQ6x Stage 1], and the QJL matrix S
@@ -103,8 +116,31 @@ int tq_create(int d, int bits, uint64_t seed, tq_handle** out);
 
 /* Prod handle [TQ6x Stage 2]: `bits` total per coordinate = (bits - 1) MSE bits
  * + one QJL sign per projection, qjl_m projections (m % 32 == 0, m <= 1024).
- * Norms default to fp16; residual norms are always fp16. 2 <= bits <= 5. */
+ * Norms default to fp16; residual norms are always fp16. 1 <= bits <= 5; d <= 128.
+ * bits = 1 makes QJL-only rows [HAKU "QJL: zero-overhead 1-bit compression"]:
+ * no MSE stage, the signs of S x (sign(0) = +1) and ||x||, which weighs the
+ * signs where a prod row uses its residual norm. */
 int tq_create_prod(int d, int bits, int qjl_m, uint64_t seed, tq_handle** out);
+
+/* Recursive polar transform handle [POLAR sections 1 and 3; HAKU "PolarQuant"]:
+ * y = Pi x / ||x|| (Pi as tq_create's for `seed`), then log2(d) levels: level 1
+ * pairs (y_2i, y_2i+1) into a radius and an angle atan2(y_2i+1, y_2i) in (-pi, pi],
+ * each further level pairs the previous radii (angle in [0, pi/2]); every angle
+ * is bucketized against its level's Lloyd-Max codebook (tq_polar_codebook_host),
+ * bits_level1 bits at level 1 and bits_upper at every other level (each 1..4).
+ * d a power of two, 32 <= d <= 256. Norms fp32 by default.
+ * Row layout: the level fields one after the other, level 1 first, each index
+ * LSB-first in its level's width; codes_B = 16 * ceil(total bits / 128), pad
+ * bits 0. Works with tq_encode, tq_append and tq_score (s = ||x|| <Pi q, y_hat>,
+ * y_hat the unit vector rebuilt from the centroids); other hot calls return
+ * TQ_EUNSUPPORTED for polar handles. */
+int tq_create_polar(int d, int bits_level1, int bits_upper, uint64_t seed, tq_handle** out);
+
+/* Levels and widths of a polar handle (TQ_EINVAL for other handles). */
+int tq_polar_info(const tq_handle* h, int* nlevels, int* bits_level1, int* bits_upper);
+
+/* Host copies (fp64) of level `level`'s (1-based) centroids and boundaries. */
+int tq_get_polar_codebook(const tq_handle* h, int level, double* centroids, double* bounds);
 
 /* Storage type of the per-vector norm: TQ_F32 or TQ_F16. */
 int tq_set_norm_dtype(tq_handle* h, int dtype);
@@ -121,7 +157,8 @@ int tq_get_info(const tq_handle* h, int* d, int* bits_mse, int* qjl_m, int* norm
  * MSE-only handles). */
 int tq_code_bytes(const tq_handle* h, int* codes_B, int* signs_B);
 
-/* Host copies (fp64) of the codebook: 2^b centroids and 2^b - 1 boundaries. */
+/* Host copies (fp64) of the codebook: 2^b centroids and 2^b - 1 boundaries
+ * (TQ_EINVAL for polar handles: tq_get_polar_codebook). */
 int tq_get_codebook(const tq_handle* h, double* centroids, double* bounds);
 
 /* Host copies (fp64) of Pi (d*d) and, if S != NULL and the handle is prod, S (m*d). */
@@ -133,7 +170,8 @@ int tq_get_rotation(const tq_handle* h, double* Pi, double* S);
 
 /* Encode n vectors [TQ6x Stage 1 and 2; DEEP "PolarQuant", "QJL"]:
  * norm = ||x||, y = Pi x / norm, index_j = #{i : bound_i < y_j}, bit-pack;
- * prod handles also write signs of S r, r = x - norm * Pi^T c[index], and ||r||.
+ * prod handles also write signs of S r, r = x - norm * Pi^T c[index], and ||r||
+ * (QJL-only handles: signs of S x and the norm; codes and rnorms may be NULL).
  *  x      device [n][d] of x_dtype (TQ_F32 / TQ_F16 / TQ_BF16), 16-byte aligned
  *  codes  device [n][codes_B];  signs device [n][signs_B] (prod) or NULL
  *  norms  device [n] of the handle's norm dtype;  rnorms device [n] fp16 (prod) or NULL
@@ -142,7 +180,7 @@ int tq_encode(const tq_handle* h, const void* x, int x_dtype, int64_t n,
               uint8_t* codes, uint8_t* signs, void* norms, void* rnorms, void* stream);
 
 /* Test hook: packs indices idx (device uint8 [n][d], each < 2^b) into codes
- * (device [n][codes_B]) with the layout above. */
+ * (device [n][codes_B]) with the layout above. TQ_EINVAL for QJL-only handles. */
 int tq_pack_indices(const tq_handle* h, const uint8_t* idx, int64_t n, uint8_t* codes, void* stream);
 
 /* Streaming append of one token per (sequence, head) [TQ6x Stage 1: online
@@ -163,7 +201,9 @@ size_t tq_search_workspace_bytes(const tq_handle* h, int nq, int64_t n, int k);
 
 /* Inner-product scores of full-precision queries against a quantized key cache
  * [HAKU "QJL": precise query vs low-bit data; TQ6x Stage 2]:
- *   s = norm * <Pi q, c[index]>  (+ rnorm * sqrt(pi/2)/m * <S q, 2 sigma - 1> for prod).
+ *   s = norm * <Pi q, c[index]>  (+ rnorm * sqrt(pi/2)/m * <S q, 2 sigma - 1> for prod;
+ *   QJL-only keys: s = norm * sqrt(pi/2)/m * <S q, 2 sigma - 1>; polar keys:
+ *   s = norm * <Pi q, y_hat> folded up the transform tree [POLAR section 3], Hq/Hkv <= 8).
  *  q        device fp32 [B][Hq][d];  Hq % Hkv == 0; query head h reads KV head h / (Hq/Hkv)
  *  k, len   key cache and device int32 [B] lengths (0 <= len[b] <= L_cap)
  *  logits   device fp32 [B][Hq][L_cap]; entries i < len[b] are written, the rest untouched
@@ -175,7 +215,8 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv,
 /* Fused GQA decode attention over quantized K and V [DEEP "Scaled dot-product
  * attention"; TQ6x Stage 1 and 2]: out = softmax(scale * s) V_hat per query
  * head, s from tq_score's formula with hk, V_hat the dequantized values of hv
- * (prod V adds the QJL back-projection rnorm sqrt(pi/2)/m S^T (2 sigma - 1)).
+ * (prod V adds the QJL back-projection rnorm sqrt(pi/2)/m S^T (2 sigma - 1);
+ * QJL-only V is that back-projection alone, with the norm in place of rnorm).
  *  q        device [B][Hq][d] fp32 (q_dtype TQ_F32) or bf16 (TQ_BF16)
  *  k, v     caches of hk and hv (same d; any bits/prod mix)
  *  out      device fp32 [B][Hq][d]; a sequence with len[b] == 0 gets zeros

@@ -50,6 +50,19 @@ def test_host_codebook_matches_oracle(tq, d, bits):
     assert np.array_equal(c, -c[::-1])
 
 
+@pytest.mark.parametrize("level,bits", [(1, 4), (1, 3), (2, 1), (2, 2), (3, 2), (4, 3), (5, 4), (7, 2), (8, 2)])
+def test_host_polar_codebook_matches_oracle(tq, level, bits):
+    from oracle import polar
+    c, b = tq.tq_polar_codebook_host(level, bits)
+    co, bo = polar.lloyd_max(level, bits)
+    # the oracle's cell moments come from a cumulative table (about 1e-12 relative); the library
+    # integrates each cell by Gauss-Legendre quadrature
+    assert np.allclose(c, co, rtol=0, atol=2e-10)
+    assert np.allclose(b, bo, rtol=0, atol=2e-10)
+    if level > 1:   # symmetric about pi/4
+        assert np.allclose(c + c[::-1], np.pi / 2, atol=1e-15)
+
+
 @pytest.mark.parametrize("d,m,seed", [(32, 32, 0), (128, 128, 2), (128, 0, 3), (256, 64, 9)])
 def test_host_rotation_matches_oracle(tq, d, m, seed):
     Pi, S = tq.tq_rotation_host(d, m, seed)
