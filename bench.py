@@ -19,6 +19,10 @@ e2e     = same metric through the C ABI with host buffers: per step one CUDA
           staging buffer, runs the step and copies the attention output back to
           pinned memory, all inside the timed bracket; the host fills the
           staging buffer between steps.
+rows    = (N = 1, unless --no-rows) every other hot-path row measured after the headline's
+          timed region with a few steps each and folded into the same line: the cfg-1 encode
+          + score record, the streaming score step, the prefill encode, the 4-bit decode step,
+          the 3-bit decode step over an HBM-sized cache, and the 2- and 4-bit searches.
 Multi-GPU (--gpus N under torchrun): every rank runs its own independent
 instance of the workload (weak scaling, no collective on the data path); the
 reported time is the max over ranks.
@@ -67,11 +71,15 @@ def parse_args():
     p.add_argument("--warmup", type=int, default=10)
     p.add_argument("--impl", choices=["tq", "reference"], default="tq")
     p.add_argument("--no-cpu-baseline", action="store_true")
-    p.add_argument("--workload", choices=["decode", "score", "encode", "attn4", "search", "search4", "compare"],
+    p.add_argument("--workload", choices=["decode", "score", "encode", "attn4", "attn3big", "search", "search4",
+                                          "compare", "cfg1"],
                    default="decode",
                    help="decode: the headline decode step (default); the others measure the remaining hot-path "
-                        "rows on their own workloads, one JSON line each (search: 2-bit codes, search4: 4-bit; "
+                        "rows on their own workloads, one JSON line each (attn3big: the 3-bit decode step over a "
+                        "64 x 8 x 16384-token cache; search: 2-bit codes, search4: 4-bit; "
                         "compare: the cfg-2 attention against uncompressed bf16 / fp32 K/V)")
+    p.add_argument("--no-rows", action="store_true",
+                   help="decode only: skip the other hot-path rows that the default run folds into its line")
     p.add_argument("--small", action="store_true",
                    help="row workloads only: a reduced size (still above the 126 MB L2, a few hundred MB in "
                         "all) for profiler captures; the numbers of such a run are not bench values")
@@ -450,6 +458,10 @@ def run_tq(args):
         "kernels_per_step": kernels_per_step,
         "clocks": clocks,
     }
+    if world == 1 and not args.no_rows:
+        # every other hot-path row, a few steps each, after the headline's timed region
+        import bench_rows
+        line["rows"] = bench_rows.collect_rows(args)
     if world == 1 and not args.no_cpu_baseline:
         gbs, el, reps_c, threads = oracle_decode_sample()
         line["cpu_baseline"] = {"value": gbs, "unit": "GB/s", "cores": threads, "kind": "oracle",

@@ -1,5 +1,5 @@
 """Measurement of the hot-path rows other than the headline decode step (`bench.py
---workload score|encode|attn4|search`): one JSON line each, same keys as the headline
+--workload score|encode|attn4|attn3big|search|search4|compare`): one JSON line each, same keys as the headline
 line (metric, value, roofline of the row's dominant kernel, clocks, launches) plus the CPU
 oracle timed on a bounded sample of the same workload.
 
@@ -10,6 +10,8 @@ Workloads (all synthetic, seeded; the big inputs are drawn on the GPU):
   encode  the prefill of that cache: 8,388,608 bf16 vectors, prod 2+1, d = 128.
   attn4   4 sequences x 8 KV heads x context 131072, K and V 4-bit MSE, fp16 norms, bf16
           K/V with a per-(sequence, head) scale ~ U(0.5, 2); one tq_decode_step per step.
+  attn3big  the 3-bit prod decode step (2-bit codes + 128 QJL signs, fp16 norms) over 64
+          sequences x 8 KV heads x context 16384 (872 MB of packed K/V: HBM-bound).
   search  1,000,000 x 1536 L2-normalised fp32 database vectors, 2-bit MSE codes, 1024
           queries, top-10.
 """
@@ -20,6 +22,10 @@ import time
 import bench
 
 ROWS = ("score", "encode", "attn4", "search")
+
+# When a list, _line appends each row's line here instead of printing it (the default bench run
+# folds every row into the headline line, see collect_rows).
+COLLECT = None
 
 
 def _events(torch):
@@ -42,6 +48,9 @@ def _line(args, metric, value, unit, ms_per_step, config, roofline, launches, cl
         line.update(extra)
     if cpu:
         line["cpu_baseline"] = cpu
+    if COLLECT is not None:
+        COLLECT.append(line)
+        return
     print(json.dumps(line), flush=True)
 
 
@@ -288,6 +297,9 @@ def oracle_encode_sample(budget_s=12.0, rows=16384):
 # ------------------------------------------------------------------ attention, 4-bit MSE (cfg 3)
 
 S3 = dict(B=4, Hkv=8, Hq=32, L=131072, d=128, bits=4, seed_k=5, seed_v=6, seed_q=7)
+# the 3-bit prod decode step over a cache of the streaming workload's size: 64 sequences x 8 KV
+# heads x 16384 tokens (872 MB of packed K/V), an HBM-bound read
+S5A = dict(B=64, Hkv=8, Hq=32, L=16384, d=128, bits=3, m=128, seed_k=10, seed_v=12, seed_q=13)
 
 
 def run_attn4(args):
@@ -295,17 +307,48 @@ def run_attn4(args):
     import embedding_vector_quantization_b200 as tq
     if args.small:
         S3["B"] = 1         # 138 MB of packed K/V
-    B, Hkv, Hq, L, d = S3["B"], S3["Hkv"], S3["Hq"], S3["L"], S3["d"]
-    hk = tq.Handle(d, S3["bits"], 0, norm_dtype=tq.TQ_F16)
-    hv = tq.Handle(d, S3["bits"], 1, norm_dtype=tq.TQ_F16)
+    hk = tq.Handle(S3["d"], S3["bits"], 0, norm_dtype=tq.TQ_F16)
+    hv = tq.Handle(S3["d"], S3["bits"], 1, norm_dtype=tq.TQ_F16)
+    spec = dict(S3, bytes_per_token=2 * (64 + 2), kernel="attn_mse4_kernel", scaled=True,
+                workload="GQA decode step, TurboQuant MSE 4-bit K and V, d=128, B=%d, 8 KV heads / 32 query heads, "
+                         "context 131072, bf16 K/V N(0,1) x U(0.5,2) per (sequence, head)" % S3["B"],
+                dtype="s8xs8->s32 MMA (22-bit fixed-point queries, Walsh planes), u8xu8->s32 MMA (16-bit "
+                      "weights), f32 softmax/combine",
+                metric="packed-KV GB/s (cfg 3 decode step, 4-bit MSE)")
+    cpu = None if args.no_cpu_baseline else oracle_attn4_sample()
+    _run_decode_row(args, tq, torch, hk, hv, spec, cpu)
+
+
+def run_attn3big(args):
+    import torch
+    import embedding_vector_quantization_b200 as tq
+    if args.small:
+        S5A["B"] = 8        # 109 MB of packed K/V
+    hk = tq.Handle(S5A["d"], S5A["bits"], 0, qjl_m=S5A["m"])
+    hv = tq.Handle(S5A["d"], S5A["bits"], 1, qjl_m=S5A["m"])
+    spec = dict(S5A, bytes_per_token=2 * (32 + 16 + 2 + 2), kernel="attn_prod2_kernel", scaled=False,
+                workload="GQA decode step, TurboQuant prod 3-bit (2-bit Lloyd-Max + 1-bit QJL m=128), d=128, "
+                         "B=%d, 8 KV heads / 32 query heads, context 16384, bf16 K/V N(0,1)" % S5A["B"],
+                dtype="s8xs8->s32 MMA (22-bit fixed-point queries), u8xu8->s32 MMA (16-bit weights), "
+                      "f32 softmax/combine",
+                metric="packed-KV GB/s (3-bit decode step over an HBM-sized cache)")
+    _run_decode_row(args, tq, torch, hk, hv, spec, None)
+
+
+def _run_decode_row(args, tq, torch, hk, hv, spec, cpu):
+    """One decode step (tq_decode_step in a CUDA graph) over a cache larger than L2, timed per step."""
+    B, Hkv, Hq, L, d = spec["B"], spec["Hkv"], spec["Hq"], spec["L"], spec["d"]
     kc, vc = tq.Cache(hk, B, Hkv, L), tq.Cache(hv, B, Hkv, L)
     enc_ms = 0.0
-    for h, cache, seed in ((hk, kc, S3["seed_k"]), (hv, vc, S3["seed_v"])):
+    for h, cache, seed in ((hk, kc, spec["seed_k"]), (hv, vc, spec["seed_v"])):
         g = torch.Generator(device="cuda").manual_seed(seed)
-        scl = (0.5 + 1.5 * torch.rand(B, Hkv, 1, 1, generator=g, device="cuda"))      # U(0.5, 2) per (b, head)
+        if spec["scaled"]:
+            scl = (0.5 + 1.5 * torch.rand(B, Hkv, 1, 1, generator=g, device="cuda"))      # U(0.5, 2) per (b, head)
+        else:
+            scl = torch.ones(B, Hkv, 1, 1, device="cuda")
         enc_ms += _encode_into(tq, h, cache, lambda l0, n: (torch.randn(B, Hkv, n, d, generator=g, device="cuda")
                                                            * scl).to(torch.bfloat16), L, 8192, torch)
-    gq = torch.Generator(device="cuda").manual_seed(S3["seed_q"])
+    gq = torch.Generator(device="cuda").manual_seed(spec["seed_q"])
     W, T = args.warmup, args.steps
     qs = torch.randn(T + W, B, Hq, d, generator=gq, device="cuda")
     kn = torch.randn(T + W, B, Hkv, d, generator=gq, device="cuda").to(torch.bfloat16)
@@ -360,35 +403,35 @@ def run_attn4(args):
     clocks = sampler.stop()
     total_ms = sum(a.elapsed_time(b) for a, b in evs)
     split_ms, split_n = 0.0, 0
+    kern = {}
     for t in range(T):
         set_inputs(W + t)
         graph_k.replay()
         torch.cuda.synchronize()
-        ms_k, n_k = tq.tq_timer_read("attn_split", forget=False)
-        split_ms += ms_k
-        split_n += n_k
+        for name in ("prologue", "attn_split", "attn_combine"):
+            ms_k, n_k = tq.tq_timer_read(name, forget=False)
+            kern[name] = kern.get(name, 0.0) + ms_k
+            if name == "attn_split":
+                split_ms += ms_k
+                split_n += n_k
     _, kernels_per_step = tq.tq_timer_read(None, forget=False)
-    bytes_step = B * Hkv * L * 2 * (64 + 2)        # K and V: 4-bit codes (64 B) + fp16 norm per token
+    bytes_step = B * Hkv * L * spec["bytes_per_token"]
     peak, src = _peak("hbm")
     ach = bytes_step / (split_ms / max(split_n, 1) / 1e3) / 1e9
-    cfg = {"workload": "GQA decode step, TurboQuant MSE 4-bit K and V, d=128, B=4, 8 KV heads / 32 query heads, "
-                       "context 131072, bf16 K/V N(0,1) x U(0.5,2) per (sequence, head)",
-           "B": B, "Hkv": Hkv, "Hq": Hq, "context": L, "d": d,
-           "dtype": "s8xs8->s32 MMA (15-bit fixed-point queries, 14-bit weights, Walsh planes), f32 softmax/combine",
-           "l2": "not flushed: each step reads 553.6 MB of packed K/V (> 126 MB L2)",
+    cfg = {"workload": spec["workload"], "B": B, "Hkv": Hkv, "Hq": Hq, "context": L, "d": d, "dtype": spec["dtype"],
+           "l2": "not flushed: each step reads %.1f MB of packed K/V (> 126 MB L2)" % (bytes_step / 1e6),
            "step": "tq_decode_step, one CUDA graph replay; len reset outside the timed bracket"}
-    roof = {"bound": "hbm", "kernel": "attn_mse4_kernel", "achieved": ach, "peak": peak, "unit": "GB/s",
+    roof = {"bound": "hbm", "kernel": spec["kernel"], "achieved": ach, "peak": peak, "unit": "GB/s",
             "frac": ach / peak, "traffic": None, "peak_source": src, "launch_ms": split_ms / max(split_n, 1),
             "algorithmic_bytes_per_launch": bytes_step}
     value = bytes_step * T / (total_ms / 1e3) / 1e9
     extra = {"tokens_per_s": B * Hkv * L * T / (total_ms / 1e3),
+             "kernel_us_per_step": {k: round(1e3 * v / T, 2) for k, v in kern.items()},
              "prefill_encode": {"vectors": 2 * B * Hkv * L, "ms": enc_ms,
                                 "vectors_per_s": 2 * B * Hkv * L / (enc_ms / 1e3)}}
-    cpu = None if args.no_cpu_baseline else oracle_attn4_sample()
     if args.small:
-        cfg["workload"] += " [reduced for profiling: 1 sequence]"
-    _line(args, "packed-KV GB/s (cfg 3 decode step, 4-bit MSE)", value, "GB/s", total_ms / T, cfg, roof,
-          kernels_per_step * T, clocks, extra, cpu)
+        cfg["workload"] += " [reduced for profiling]"
+    _line(args, spec["metric"], value, "GB/s", total_ms / T, cfg, roof, kernels_per_step * T, clocks, extra, cpu)
 
 
 def oracle_attn4_sample(budget_s=12.0, L=32768):
@@ -634,6 +677,115 @@ def run_compare(args):
           extra["speedup_vs_bf16"], "x", us["turboquant_3bit"] / 1e3, cfg, roof, 3 * reps, clocks, extra)
 
 
+# ------------------------------------------------------------------ the small MSE workload (cfg 1)
+
+def _unpack_rows(codes, d, bits):
+    """Indices of LSB-first packed rows (uint8 [n, B] numpy) -> int64 [n, d]."""
+    import numpy as np
+    stream = np.unpackbits(codes, axis=1, bitorder="little")[:, : d * bits].reshape(codes.shape[0], d, bits)
+    return (stream.astype(np.int64) << np.arange(bits)).sum(axis=2)
+
+
+def run_cfg1(args):
+    """MSE-only 3-bit TurboQuant, d = 128: 4096 fp32 N(0,1) keys (seed 0) encoded, one N(0,1) query
+    (seed 1) scored against all of them. Reports the index usage, norms, scores and the empirical
+    distortion mean ||x - x_hat||^2 / ||x||^2 (x_hat rebuilt on the host from the GPU's codes with
+    the handle's Pi and codebook); the CPU leg (the oracle) adds the near-boundary index mismatch
+    fraction and the largest score difference."""
+    import numpy as np
+    import torch
+    import embedding_vector_quantization_b200 as tq
+    import workloads
+    d, bits, n = 128, 3, 4096
+    h = tq.Handle(d, bits, 0)
+    x = workloads.mse_keys(n, d, seed=0)
+    q = workloads.queries((1, 1, d), 1)
+    xg = x.cuda()
+    cache = tq.Cache(h, 1, 1, n)
+    lens = torch.full((1,), n, dtype=torch.int32, device="cuda")
+    ws = torch.empty(tq.tq_score_workspace_bytes(h.ptr, 1, 1), dtype=torch.uint8, device="cuda")
+    logits = torch.zeros(1, 1, n, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        cache.fill(xg.view(1, 1, n, d))
+        tq.score(h, q.cuda(), cache, lens, logits=logits, workspace=ws)
+    torch.cuda.synchronize()
+    reps = 20
+    e_ms = s_ms = 0.0
+    for _ in range(reps):
+        a, b = _events(torch)
+        a.record()
+        cache.fill(xg.view(1, 1, n, d))
+        b.record()
+        c, e = _events(torch)
+        c.record()
+        tq.score(h, q.cuda(), cache, lens, logits=logits, workspace=ws)
+        e.record()
+        torch.cuda.synchronize()
+        e_ms += a.elapsed_time(b)
+        s_ms += c.elapsed_time(e)
+    codes = cache.codes.cpu().numpy().reshape(n, -1)
+    norms = cache.norms.cpu().numpy().reshape(n)
+    scores = logits.cpu().numpy().reshape(n)
+    idx = _unpack_rows(codes, d, bits)
+    cent, _ = h.codebook()
+    Pi, _ = h.rotation()
+    xh = norms.astype(np.float64)[:, None] * (cent[idx] @ Pi)
+    xd = x.double().numpy()
+    dist = float(np.mean(np.sum((xd - xh) ** 2, axis=1) / np.sum(xd * xd, axis=1)))
+    rec = {"workload": "MSE-only TurboQuant, d=128, b=3: 4096 fp32 N(0,1) keys (seed 0), 1 N(0,1) query (seed 1)",
+           "encode_us": 1e3 * e_ms / reps, "score_us": 1e3 * s_ms / reps,
+           "index_histogram": np.bincount(idx.ravel(), minlength=8).tolist(),
+           "norms": {"mean": float(norms.mean()), "min": float(norms.min()), "max": float(norms.max())},
+           "scores": {"first": [float(v) for v in scores[:4]], "mean": float(scores.mean()),
+                      "std": float(scores.std())},
+           "empirical_mse_distortion": dist,
+           "expected_mse_distortion": "d * MSE(3 bits, d = 128) = 0.0340 (the Lloyd-Max codebook's own MSE)"}
+    if not args.no_cpu_baseline:
+        from oracle import codebook, ops, quant, rotation
+        t0 = time.perf_counter()
+        Pio, _ = rotation.rotation(d, 0)
+        co, bo = codebook.lloyd_max(d, bits)
+        eo = quant.encode_mse(xd, Pio, co, bo, "f32")
+        so = ops.score_mse(q.double().numpy().reshape(d), eo["idx"], eo["n_stored"], Pio, co)
+        el = time.perf_counter() - t0
+        mism = idx != eo["idx"]
+        near = np.abs(eo["y"][mism] - bo[np.minimum(idx[mism], eo["idx"][mism])]) if mism.any() else np.zeros(0)
+        rec["oracle"] = {"index_mismatch_fraction": float(mism.mean()),
+                         "mismatches_within_1e-5_of_a_boundary": bool(np.all(near < 1e-5)),
+                         "max_abs_score_difference": float(np.max(np.abs(scores - so))),
+                         "oracle_seconds": el, "kind": "oracle", "cores": bench.blas_threads()}
+    if COLLECT is not None:
+        COLLECT.append({"metric": "cfg1", "record": rec})
+    else:
+        print(json.dumps({"metric": "MSE-only 3-bit encode + score record (cfg 1)", "record": rec}), flush=True)
+
+
+def collect_rows(args, rows=("cfg1", "score", "encode", "attn4", "attn3big", "search", "search4")):
+    """Runs every other hot-path row with a few steps and returns {row: its line}. The rows'
+    own CPU baselines are skipped (the cfg-1 record keeps its oracle check)."""
+    import copy
+    global COLLECT
+    out = {}
+    fns = {"cfg1": run_cfg1, "score": run_score, "encode": run_encode, "attn4": run_attn4, "attn3big": run_attn3big,
+           "search": lambda a: run_search(a, bits=2), "search4": lambda a: run_search(a, bits=4)}
+    for name in rows:
+        a = copy.copy(args)
+        a.steps, a.warmup, a.small = 10, 3, False
+        a.no_cpu_baseline = name != "cfg1" or args.no_cpu_baseline
+        COLLECT = []
+        try:
+            fns[name](a)
+            line = COLLECT[-1] if COLLECT else {"error": "no line"}
+        except Exception as exc:   # a row that fails is reported, the headline line still prints
+            line = {"error": f"{type(exc).__name__}: {exc}"}
+        finally:
+            COLLECT = None
+        out[name] = line
+        import torch
+        torch.cuda.empty_cache()
+    return out
+
+
 def run(args):
     if args.workload == "compare":
         run_compare(args)
@@ -641,4 +793,5 @@ def run(args):
     if args.workload == "search4":
         run_search(args, bits=4)
         return
-    {"score": run_score, "encode": run_encode, "attn4": run_attn4, "search": run_search}[args.workload](args)
+    {"score": run_score, "encode": run_encode, "attn4": run_attn4, "attn3big": run_attn3big,
+     "search": run_search, "cfg1": run_cfg1}[args.workload](args)

@@ -21,6 +21,8 @@
 //    codebook slopes, rounded to 22-bit integers and split into three int8 pieces
 //    (hi * 2^14 + mid * 2^7 + lo): one n8 tile holds the hi and mid pieces of the
 //    4 heads, a second n8 tile the lo pieces (columns 2h; the odd columns are 0).
+//    The QJL projections S q (weighed by the small residual norms) are rounded to
+//    15-bit integers, two pieces hi * 2^7 + lo in the first tile only.
 //  * Value side (bit rows of the value codes as the MMA rows, tokens as the
 //    reduction): softmax weights p * ||v|| (and p * rnorm for the QJL part) are
 //    rounded to 16-bit integers against the chunk maximum and split into two
@@ -34,6 +36,11 @@
 //  * Two passes per context chunk: all key scores first (kept in shared memory,
 //    giving the exact chunk maximum), then all values with one fixed weight
 //    scale, so the value sums accumulate in int32 across the whole chunk.
+//  * The whole chunk (at most 896 tokens: 93 KB of keys and values) is staged in
+//    shared memory: every TMA copy of the chunk is issued at launch, one mbarrier
+//    per 256-token block of keys and of values, so the cold read of the cache has
+//    all of its bytes requested at once and the key pass starts on the first block
+//    while the rest arrive.
 //
 // Partial results use the layout of the split kernel in score_attn_simt.cuh
 // ([B*Hq][nsplit][d + m + 2]: rotated-domain value sum, QJL sum, max, sum of
@@ -49,17 +56,18 @@ namespace amma {
 constexpr int kD = 128;
 constexpr int kM = 128;
 constexpr int kG = 4;
-constexpr int kBlk = 256;                     // tokens per pipeline block
-constexpr int kStages = 5;
+constexpr int kBlk = 256;                     // tokens per block (one mbarrier each)
 constexpr int kWarps = 8;
 constexpr int kThreads = kWarps * 32;
 constexpr int kCodesB = 32, kSignsB = 16;
 constexpr int kStageCodes = kBlk * kCodesB;   // 8192
 constexpr int kStageSigns = kBlk * kSignsB;   // 4096
-// key block: codes, signs, norms, rnorms + the value norms and rnorms of the same tokens;
-// value block: codes and signs only (its norms came with the key block)
-constexpr int kStageBytes = kStageCodes + kStageSigns + 4 * kBlk * 2;  // 14336
-constexpr int kMaxChunk = 1024;
+constexpr int kMaxChunk = 896;                // the chunk's keys and values fit shared memory twice per SM
+constexpr int kMaxBlk = (kMaxChunk + kBlk - 1) / kBlk;   // 4
+// padded row strides against shared-memory bank conflicts: the 4 heads' logit rows start 8 banks
+// apart, and the rows of a weight block 4 banks apart
+constexpr int kLogitStride = kMaxChunk + 8;
+constexpr int kPwRow = kBlk + 16;
 
 struct Args {
   const float* qr;  // [B*Hq][128] Pi_K q
@@ -84,24 +92,39 @@ struct Args {
   int* err;
 };
 
+// Key-pass data of the chunk; after the key pass its codes and signs are dead and hold the
+// value pass's integer weights and sums instead.
+struct __align__(16) KeyArea {
+  union {
+    unsigned char codes[kMaxChunk * kCodesB];
+    uint8_t pw[kMaxBlk][2][8][kPwRow];  // integer softmax weights of the chunk's value blocks:
+                                        // [block][0: value weights, 1: QJL weights][col = head*2+piece][token]
+  };
+  union {
+    unsigned char signs[kMaxChunk * kSignsB];
+    float vacc[3][kG][128];     // value-side sums of the two token halves (rows of each byte group)
+  };
+  __half kn[kMaxChunk];         // key norms, residual norms, and the value norms and residual norms
+  __half krn[kMaxChunk];        // (these arrive with the keys: the weight steps need them)
+  __half vn[kMaxChunk];
+  __half vrn[kMaxChunk];
+};
+
 struct __align__(16) Smem {
-  unsigned char stage[kStages][kStageBytes];
-  float logits[kG][kMaxChunk];  // key pass output: scaled logits in log2 units [head][token]
+  KeyArea k;
+  unsigned char vcodes[kMaxChunk * kCodesB];
+  unsigned char vsigns[kMaxChunk * kSignsB];
+  float logits[kG][kLogitStride];  // key pass output: scaled logits in log2 units [head][token]
   uint32_t qfrag[2][12][2][4][8];  // key-side B fragments: [n tile][k-step][register][quad index t][column g]
-  uint8_t pw[2][2][8][kBlk];    // integer softmax weights of a value block, double buffered:
-                                // [buffer][0: value weights, 1: QJL weights][col = head*2+piece][token]
   float qconst[kG][4];        // c0*sum(q'), delta_mse, delta_qjl, sum(qs)
   float red_f[kWarps][kG];
   float hmax[kG];
   float dv[2][kG];            // weight steps per head: max_t p_t ||v_t|| / 65535 (0: values, 1: QJL)
   float inv[2][kG];
-  float red_w[kWarps][2][kG]; // per warp: max_t (logit + log2 ||v_t||), max_t (logit + log2 rnorm_t)
+  float red_w[kWarps][2][kG]; // per warp and head: the largest p ||v|| and p rnorm
   int red_i[kWarps][2 * kG];
-  float vacc[3][kG][128];     // value-side sums of the two token halves (rows of each byte group)
-  __half vnorm[kMaxChunk];    // value norms and residual norms of the chunk (copied with the key blocks)
-  __half vrn[kMaxChunk];
-  uint64_t full[kStages];
-  uint64_t empty[kStages];    // one arrival per warp when it is done with the stage
+  uint64_t kfull[kMaxBlk];    // key block j has arrived
+  uint64_t vfull[kMaxBlk];    // value block j has arrived
   int W[2][kG];               // chunk sums of the integer value / QJL weights per head
   int abort_flag;
 };
@@ -197,11 +220,13 @@ __device__ __forceinline__ int qfrag_sign_offset(int i) {
 }
 
 // Query side of the key MMAs for the kG heads h0 .. h0 + 3 of sequence b (one warp per
-// head, warps 0..3): rotated queries scaled by the codebook slopes and S q, rounded to
-// 22-bit integers against their maxima and split into int8 pieces hi * 2^14 + mid * 2^7 + lo
-// in B-fragment order (n tile 0: column 2h = hi, 2h + 1 = mid; n tile 1: column 2h = lo);
+// head, warps 0..3): rotated queries scaled by the codebook slopes, rounded to 22-bit
+// integers against their maximum and split into int8 pieces hi * 2^14 + mid * 2^7 + lo in
+// B-fragment order (n tile 0: column 2h = hi, 2h + 1 = mid; n tile 1: column 2h = lo); S q
+// rounded to 15-bit integers, hi * 2^7 + lo in n tile 0 (columns 2h, 2h + 1).
 // qconst[h] = {c0 sum(q'), step of the code pieces, step of the sign pieces, sum(S q)}.
 constexpr float kQMax = 2080768.f;   // 127 * 2^14: the largest |integer| a query value maps to
+constexpr float kSMax = 16256.f;     // 127 * 2^7: the same for the QJL projections
 __device__ __forceinline__ void prepare_query(const float* qr_rows, const float* qs_rows, float kb0, float kb1,
                                               float kc0, uint32_t (&qfrag)[2][12][2][4][8],
                                               float (&qconst)[kG][4]) {
@@ -230,7 +255,7 @@ __device__ __forceinline__ void prepare_query(const float* qr_rows, const float*
     ms = fmaxf(ms, __shfl_xor_sync(0xffffffffu, ms, o));
   }
   const float dm = mx > 0.f ? mx / kQMax : 1.f;
-  const float ds = ms > 0.f ? ms / kQMax : 1.f;
+  const float ds = ms > 0.f ? ms / kSMax : 1.f;
   int8_t* qf0 = reinterpret_cast<int8_t*>(&qfrag[0][0][0][0][0]);
   int8_t* qf1 = reinterpret_cast<int8_t*>(&qfrag[1][0][0][0][0]);
 #pragma unroll
@@ -238,16 +263,23 @@ __device__ __forceinline__ void prepare_query(const float* qr_rows, const float*
     const int j = lane + 32 * i;
     const float v[3] = {x0[i] / dm, x1[i] / dm, xs[i] / ds};
 #pragma unroll
-    for (int c = 0; c < 3; ++c) {
+    for (int c = 0; c < 2; ++c) {
       const int xi = __float2int_rn(v[c]);                                   // |xi| <= 127 * 2^14
       const int hi = (xi >= 0) ? (xi + 8192) >> 14 : -((-xi + 8192) >> 14);  // |hi| <= 127
-      const int r = xi - (hi << 14);                                         // |r| <= 2^13
+      const int r = xi - hi * 16384;                                         // |r| <= 2^13
       const int mid = (r >= 0) ? (r + 64) >> 7 : -((-r + 64) >> 7);         // |mid| <= 64
-      const int off = (c < 2) ? qfrag_code_offset(c, j) : qfrag_sign_offset(j);
+      const int off = qfrag_code_offset(c, j);
       qf0[off + (2 * h) * 4] = (int8_t)hi;
       qf0[off + (2 * h + 1) * 4] = (int8_t)mid;
-      qf1[off + (2 * h) * 4] = (int8_t)(r - (mid << 7));                     // |lo| <= 64
+      qf1[off + (2 * h) * 4] = (int8_t)(r - mid * 128);                      // |lo| <= 64
       qf1[off + (2 * h + 1) * 4] = 0;
+    }
+    {
+      const int xi = __float2int_rn(v[2]);                                   // |xi| <= 127 * 2^7
+      const int hi = (xi >= 0) ? (xi + 64) >> 7 : -((-xi + 64) >> 7);        // |hi| <= 127
+      const int off = qfrag_sign_offset(j);
+      qf0[off + (2 * h) * 4] = (int8_t)hi;
+      qf0[off + (2 * h + 1) * 4] = (int8_t)(xi - 128 * hi);                  // |lo| <= 64
     }
   }
   if (lane == 0) {
@@ -259,26 +291,26 @@ __device__ __forceinline__ void prepare_query(const float* qr_rows, const float*
 }
 
 // Raw scores (tq_score's formula) of keys kbase + g and kbase + g + 8 of a staged key block
-// for query head t = lane % 4: the code and sign bit planes against the query pieces, n tile 0
-// (hi and mid pieces, fragments qb held in registers) and n tile 1 (lo pieces, read from
-// shared memory: qlo = &qfrag[1][0][0][t][g]).
-__device__ __forceinline__ void mtile_scores(const unsigned char* st, const __half* nrm, const __half* rnm, int kbase,
-                                             const uint32_t (&qb)[12][2], const uint32_t* qlo, float c0h, float dmh,
-                                             float dsh, float ssh, float (&sc)[2]) {
+// for query head t = lane % 4: the code bit planes against the query pieces of n tile 0 (hi and
+// mid, fragments qb held in registers) and n tile 1 (lo: lo(k-step, register) returns this
+// thread's fragment word, from registers or shared memory), the sign bit planes against the
+// two pieces of S q in n tile 0.
+template <typename LoFn>
+__device__ __forceinline__ void mtile_scores(const unsigned char* codes, const unsigned char* signs, const __half* nrm,
+                                             const __half* rnm, int kbase, const uint32_t (&qb)[12][2], LoFn lo,
+                                             float c0h, float dmh, float dsh, float ssh, float (&sc)[2]) {
   const int lane = threadIdx.x & 31, g = lane >> 2;
   uint32_t cw[4], sw[2];
   {
     const int mat = lane >> 3, r = lane & 7;
     const int key = kbase + r + 8 * (mat >> 1);
-    ldsm_x4(cw, st + key * kCodesB + 16 * (mat & 1));
+    ldsm_x4(cw, codes + key * kCodesB + 16 * (mat & 1));
     const int skey = kbase + r + 8 * (mat & 1);
-    ldsm_x2(sw, st + kStageCodes + skey * kSignsB);
+    ldsm_x2(sw, signs + skey * kSignsB);
   }
-  // tile 0: six independent accumulator chains of length two (even / odd shifts); tile 1: four chains
+  // tile 0: six independent accumulator chains (codes: even / odd shifts); tile 1: two chains
   int dm1[2][4] = {}, dm16[2][4] = {}, ds1[4] = {}, ds16[4] = {};
-  int lm1[4] = {}, lm16[4] = {}, ls1[4] = {}, ls16[4] = {};
-  // lo-piece fragments: word (kk, slot) of this thread at qlo[(kk * 2 + slot) * 32]
-  auto lo = [&](int kk, int slot) { return qlo[(kk * 2 + slot) * 32]; };
+  int lm1[4] = {}, lm16[4] = {};
   // code words: cw[0] = key g word t, cw[1] = key g word 4+t, cw[2] = key g+8 word t, cw[3] = key g+8 word 4+t
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
@@ -298,19 +330,17 @@ __device__ __forceinline__ void mtile_scores(const unsigned char* st, const __ha
     const uint32_t b0 = y0 & 0x10101010u, b1 = y1 & 0x10101010u, b2 = z0 & 0x10101010u, b3 = z1 & 0x10101010u;
     mma_s8(ds1, a0, a1, a2, a3, qb[8 + s][0], qb[8 + s][1]);
     mma_s8(ds16, b0, b1, b2, b3, qb[10 + s][0], qb[10 + s][1]);
-    mma_s8(ls1, a0, a1, a2, a3, lo(8 + s, 0), lo(8 + s, 1));
-    mma_s8(ls16, b0, b1, b2, b3, lo(10 + s, 0), lo(10 + s, 1));
   }
   const float kqjl = kQjlScale / (float)kM;
 #pragma unroll
   for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
     const int key = kbase + g + 8 * r;
     const int hi = 2 * r, md = 2 * r + 1;   // tile 0: columns 2t (hi) and 2t + 1 (mid); tile 1: column 2t (lo)
-    // exact in int32: at most 256 code (128 sign) positions of |piece| <= 127 each, times 2^14
+    // exact in int32: at most 256 code positions of |piece| <= 127 each, times 2^14
     const int mse = (dm1[0][hi] + dm1[1][hi] + ((dm16[0][hi] + dm16[1][hi]) >> 4)) * 16384 +
                     (dm1[0][md] + dm1[1][md] + ((dm16[0][md] + dm16[1][md]) >> 4)) * 128 + lm1[hi] + (lm16[hi] >> 4);
-    const int qjl = (ds1[hi] + (ds16[hi] >> 4)) * 16384 + (ds1[md] + (ds16[md] >> 4)) * 128 + ls1[hi] +
-                    (ls16[hi] >> 4);
+    // column 2t + 1 holds the lo piece of S q here
+    const int qjl = (ds1[hi] + (ds16[hi] >> 4)) * 128 + ds1[md] + (ds16[md] >> 4);
     const float n = __half2float(nrm[key]), rn = __half2float(rnm[key]);
     sc[r] = n * (c0h + dmh * (float)mse) + rn * kqjl * (2.f * dsh * (float)qjl - ssh);
   }
@@ -328,14 +358,14 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
   const int64_t start = (int64_t)split * a.chunk;
   const int64_t end = min(L, start + a.chunk);
   const int ntok = (int)max((int64_t)0, end - start);
-  const int nblk = (ntok + kBlk - 1) / kBlk;
+  const int nblk = (ntok + kBlk - 1) / kBlk;           // <= kMaxBlk (chunk <= kMaxChunk)
   const int64_t row0 = (int64_t)bh * a.L_cap + start;  // cache row of the chunk's first token
 
-  // ---------------- setup: barriers, query pieces
+  // ---------------- setup: barriers
   if (tid == 0) {
-    for (int s = 0; s < kStages; ++s) {
-      mbar_init(&sm.full[s], 1);
-      mbar_init(&sm.empty[s], kWarps);
+    for (int j = 0; j < kMaxBlk; ++j) {
+      mbar_init(&sm.kfull[j], 1);
+      mbar_init(&sm.vfull[j], 1);
     }
     sm.abort_flag = 0;
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
@@ -343,233 +373,276 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
   if (tid < 2 * kG) (&sm.dv[0][0])[tid] = 1.f;   // an empty chunk keeps unit steps (its sums are 0)
   __syncthreads();
 
-  auto issue = [&](int j) {  // block j: K block (j < nblk) or V block j - nblk
-    const bool kside = j < nblk;
-    const int jj = kside ? j : j - nblk;
-    const int64_t tok0 = (int64_t)jj * kBlk;
-    const int64_t left = a.L_cap - (start + tok0);
-    const int ncopy = (int)min((int64_t)kBlk, left);   // multiple of 8 (L_cap % 8 == 0)
-    const int64_t r = row0 + tok0;
-    unsigned char* st = sm.stage[j % kStages];
-    uint64_t* bar = &sm.full[j % kStages];
-    const uint32_t bytes = (uint32_t)ncopy * (kCodesB + kSignsB + (kside ? 8 : 0));
-    mbar_expect_tx(bar, bytes);
-    tma_bulk_g2s(st, (kside ? a.kcodes : a.vcodes) + r * kCodesB, ncopy * kCodesB, bar);
-    tma_bulk_g2s(st + kStageCodes, (kside ? a.ksigns : a.vsigns) + r * kSignsB, ncopy * kSignsB, bar);
-    if (kside) {
-      unsigned char* nb = st + kStageCodes + kStageSigns;
-      tma_bulk_g2s(nb, a.knorm + r, ncopy * 2, bar);
-      tma_bulk_g2s(nb + 2 * kBlk, a.krn + r, ncopy * 2, bar);
-      tma_bulk_g2s(nb + 4 * kBlk, a.vnorm + r, ncopy * 2, bar);
-      tma_bulk_g2s(nb + 6 * kBlk, a.vrn + r, ncopy * 2, bar);
+  // Every copy of the chunk, issued at once by warp 0: key blocks first (codes, signs, the key
+  // norms and residual norms and the value norms and residual norms), then value blocks
+  // (codes, signs). Rows up to L_cap are copied (whole 8-token groups, L_cap % 8 == 0), at
+  // most the chunk's kMaxChunk slots.
+  auto issue_all = [&]() {
+    if (warp != 0) return;
+    auto ncopy_of = [&](int j) {
+      return (int)min(min((int64_t)kBlk, a.L_cap - (start + (int64_t)j * kBlk)), (int64_t)(kMaxChunk - j * kBlk));
+    };
+    if (lane < nblk) {
+      const uint32_t nc = (uint32_t)ncopy_of(lane);
+      mbar_expect_tx(&sm.kfull[lane], nc * (kCodesB + kSignsB + 8));
+      mbar_expect_tx(&sm.vfull[lane], nc * (kCodesB + kSignsB));
+    }
+    __syncwarp();
+    // copy c of block j: lane c handles copy c of every block (8 copies per block pair)
+    if (lane < 8) {
+      for (int j = 0; j < nblk; ++j) {
+        const int nc = ncopy_of(j);
+        const int64_t r = row0 + (int64_t)j * kBlk;
+        const int tk = j * kBlk;
+        switch (lane) {
+          case 0: tma_bulk_g2s(sm.k.codes + tk * kCodesB, a.kcodes + r * kCodesB, nc * kCodesB, &sm.kfull[j]); break;
+          case 1: tma_bulk_g2s(sm.k.signs + tk * kSignsB, a.ksigns + r * kSignsB, nc * kSignsB, &sm.kfull[j]); break;
+          case 2: tma_bulk_g2s(sm.k.kn + tk, a.knorm + r, nc * 2, &sm.kfull[j]); break;
+          case 3: tma_bulk_g2s(sm.k.krn + tk, a.krn + r, nc * 2, &sm.kfull[j]); break;
+          case 4: tma_bulk_g2s(sm.k.vn + tk, a.vnorm + r, nc * 2, &sm.kfull[j]); break;
+          case 5: tma_bulk_g2s(sm.k.vrn + tk, a.vrn + r, nc * 2, &sm.kfull[j]); break;
+          default: break;
+        }
+      }
+      for (int j = 0; j < nblk; ++j) {
+        const int nc = ncopy_of(j);
+        const int64_t r = row0 + (int64_t)j * kBlk;
+        const int tk = j * kBlk;
+        if (lane == 6) tma_bulk_g2s(sm.vcodes + tk * kCodesB, a.vcodes + r * kCodesB, nc * kCodesB, &sm.vfull[j]);
+        if (lane == 7) tma_bulk_g2s(sm.vsigns + tk * kSignsB, a.vsigns + r * kSignsB, nc * kSignsB, &sm.vfull[j]);
+      }
     }
   };
-  const int njobs = 2 * nblk;
-  constexpr int kAhead = kStages - 2;   // jobs in flight ahead of the one being consumed (3)
   grid_dep_launch();
   // The kernel before this one in a decode step (append + query rotation) writes only the
-  // slot len[b] and the rotated queries: a chunk that does not hold the slot may start
-  // streaming its cache blocks before waiting for it.
+  // slot len[b] and the rotated queries, so every CTA streams its chunk before waiting for it;
+  // the one chunk per sequence that holds the slot copies that token's rows again after the
+  // wait (patch_slot), once the block that holds it has arrived.
   const int64_t slot = (int64_t)max(a.len[b], 0);
-  const bool holds_new = a.len_extra && slot >= start && slot < start + a.chunk;
-  if (holds_new) grid_dep_wait();
-  if (tid == 0)
-    for (int j = 0; j < min(kAhead, njobs); ++j) issue(j);
-  if (!holds_new) grid_dep_wait();
+  const bool holds_new = a.len_extra && slot >= start && slot < end;
+  const int s_loc = holds_new ? (int)(slot - start) : -1, s_blk = holds_new ? s_loc / kBlk : -1;
+  issue_all();
+  grid_dep_wait();
+  // this token's rows as the previous kernel wrote them (key side: codes, signs, the four norms;
+  // value side: codes, signs); called with the block's data resident, followed by a CTA barrier
+  auto patch_slot = [&](bool key_side) {
+    const int64_t r = row0 + s_loc;
+    if (key_side) {
+      if (tid < 8) reinterpret_cast<uint32_t*>(sm.k.codes + s_loc * kCodesB)[tid] =
+          reinterpret_cast<const uint32_t*>(a.kcodes + r * kCodesB)[tid];
+      else if (tid < 12) reinterpret_cast<uint32_t*>(sm.k.signs + s_loc * kSignsB)[tid - 8] =
+          reinterpret_cast<const uint32_t*>(a.ksigns + r * kSignsB)[tid - 8];
+      else if (tid == 12) sm.k.kn[s_loc] = a.knorm[r];
+      else if (tid == 13) sm.k.krn[s_loc] = a.krn[r];
+      else if (tid == 14) sm.k.vn[s_loc] = a.vnorm[r];
+      else if (tid == 15) sm.k.vrn[s_loc] = a.vrn[r];
+    } else {
+      if (tid < 8) reinterpret_cast<uint32_t*>(sm.vcodes + s_loc * kCodesB)[tid] =
+          reinterpret_cast<const uint32_t*>(a.vcodes + r * kCodesB)[tid];
+      else if (tid < 12) reinterpret_cast<uint32_t*>(sm.vsigns + s_loc * kSignsB)[tid - 8] =
+          reinterpret_cast<const uint32_t*>(a.vsigns + r * kSignsB)[tid - 8];
+    }
+  };
 
   // query constants and int8 pieces (one warp per head)
   prepare_query(a.qr + ((size_t)b * a.Hq + h0) * kD, a.qs + ((size_t)b * a.Hq + h0) * kM, a.kb0, a.kb1, a.kc0,
                 sm.qfrag, sm.qconst);
   __syncthreads();
 
-  // B fragments of the key-side MMAs (constant for the CTA): 12 k-steps x 2 registers
-  uint32_t qb[12][2];
+  // B fragments of the key-side MMAs, n tile 0 (constant for the CTA): 12 k-steps x 2 registers
+  uint32_t qb[12][2], ql[8][2];   // n tile 0 (all k-steps) and n tile 1 (lo pieces: the code k-steps)
 #pragma unroll
   for (int kk = 0; kk < 12; ++kk)
 #pragma unroll
-    for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[0][kk][slot][t][g];
+    for (int sl = 0; sl < 2; ++sl) {
+      qb[kk][sl] = sm.qfrag[0][kk][sl][t][g];
+      if (kk < 8) ql[kk][sl] = sm.qfrag[1][kk][sl][t][g];
+    }
+  auto lo_reg = [&](int kk, int sl) { return ql[kk][sl]; };
 
   const float scale2 = a.scale * 1.4426950408889634f;
-  float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
+  const float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
   float run_max = -INFINITY;   // this thread's max logit of head t
-  float wv_max = -INFINITY, wr_max = -INFINITY;   // log2 of this thread's largest p ||v|| and p rnorm (head t)
 
+  // No warp ever leaves early: a wait that runs out sets abort_flag, after which no further
+  // waits happen, so every warp still meets the same CTA barriers; the results are discarded.
+  auto wait_full = [&](uint64_t* bar) {
+    if (*(volatile int*)&sm.abort_flag) return;
+    if (!mbar_wait(bar, 0)) sm.abort_flag = 1;
+  };
+
+  // ---------------- key pass: warp w scores keys 16w .. 16w+15 and 128+16w .. of every block
+  for (int j = 0; j < nblk; ++j) {
+    wait_full(&sm.kfull[j]);
+    if (j == s_blk) {   // uniform in the CTA
+      patch_slot(true);
+      __syncthreads();
+    }
+    const int tok_base = j * kBlk;
+    const int nvalid = min(kBlk, ntok - tok_base);
+    const unsigned char* kc = sm.k.codes + tok_base * kCodesB;
+    const unsigned char* ks = sm.k.signs + tok_base * kSignsB;
+    const __half* nrm = sm.k.kn + tok_base;
+    const __half* rnm = sm.k.krn + tok_base;
+#pragma unroll
+    for (int mt = 0; mt < 2; ++mt) {
+      const int kbase = 128 * mt + 16 * warp;
+      float sc[2];
+      mtile_scores(kc, ks, nrm, rnm, kbase, qb, lo_reg, c0h, dmh, dsh, ssh, sc);
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
+        const int key = kbase + g + 8 * r;
+        // softmax scale * log2(e): the weights are exp2(logit - max)
+        // (the last block of a chunk may be partial: nothing past its valid keys is stored, the
+        // logits rows hold kMaxChunk tokens)
+        if (key < nvalid) {
+          const float v = sc[r] * scale2;
+          sm.logits[t][tok_base + key] = v;
+          run_max = fmaxf(run_max, v);
+        }
+      }
+    }
+  }
+
+  // Integer softmax weights of the chunk, all value blocks at once (all threads): thread ->
+  // (head h = tid & 3, 4 consecutive tokens q4 .. q4 + 3 of every block). With
+  // p = exp2(logit - max): w1 = round(p ||v|| / dv[0][h]), w2 = round(p rnorm / dv[1][h]), the
+  // steps being each head's largest p ||v|| and p rnorm of the chunk over 65535 (16-bit
+  // weights), split into 8-bit pieces (hi * 256 + lo). Also the sums of p and of the weights.
+  float lsum = 0.f;
+  int wsum[2] = {0, 0};
+  if (nblk > 0) {
+    __syncthreads();   // the key area's codes and signs are dead from here on
+    if (lane == 0) {
+      for (int h = 0; h < kG; ++h) sm.red_f[warp][h] = -INFINITY;
+    }
+    __syncwarp();
+    float m = run_max;
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+    if (g == 0) sm.red_f[warp][t] = m;
+    __syncthreads();
+    if (tid < kG) {
+      float mm = -INFINITY;
+      for (int w = 0; w < kWarps; ++w) mm = fmaxf(mm, sm.red_f[w][tid]);
+      sm.hmax[tid] = mm;
+    }
+    __syncthreads();
+    const int h = tid & 3, q4 = (tid >> 2) * 4;
+    const float hm = sm.hmax[h];
+    float pv[kMaxBlk][4], pr[kMaxBlk][4];   // p ||v|| and p rnorm of this thread's tokens
+    float mv = 0.f, mr = 0.f;
+#pragma unroll
+    for (int jj = 0; jj < kMaxBlk; ++jj) {
+      const int tb = jj * kBlk, nval = min(kBlk, ntok - tb);
+      const float4 l4 = (q4 < nval) ? *reinterpret_cast<const float4*>(&sm.logits[h][tb + q4])
+                                    : make_float4(0.f, 0.f, 0.f, 0.f);
+      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
+      const __half2 n01 = *reinterpret_cast<const __half2*>(&sm.k.vn[tb + q4]);
+      const __half2 n23 = *reinterpret_cast<const __half2*>(&sm.k.vn[tb + q4 + 2]);
+      const __half2 r01 = *reinterpret_cast<const __half2*>(&sm.k.vrn[tb + q4]);
+      const __half2 r23 = *reinterpret_cast<const __half2*>(&sm.k.vrn[tb + q4 + 2]);
+      const float2 fn01 = __half22float2(n01), fn23 = __half22float2(n23);
+      const float2 fr01 = __half22float2(r01), fr23 = __half22float2(r23);
+      const float vn[4] = {fn01.x, fn01.y, fn23.x, fn23.y}, vr[4] = {fr01.x, fr01.y, fr23.x, fr23.y};
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const bool ok = q4 + q < nval;   // tokens past the chunk's end get zero weight
+        const float pp = ok ? exp2_approx(lv[q] - hm) : 0.f;
+        lsum += pp;
+        pv[jj][q] = ok ? pp * vn[q] : 0.f;   // (norm slots past the copied rows hold stale data)
+        pr[jj][q] = ok ? pp * vr[q] : 0.f;
+        mv = fmaxf(mv, pv[jj][q]);
+        mr = fmaxf(mr, pr[jj][q]);
+      }
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      mv = fmaxf(mv, __shfl_xor_sync(0xffffffffu, mv, o));
+      mr = fmaxf(mr, __shfl_xor_sync(0xffffffffu, mr, o));
+    }
+    if (g == 0) sm.red_w[warp][0][t] = mv, sm.red_w[warp][1][t] = mr;
+    __syncthreads();
+    if (tid < 2 * kG) {
+      float mx = 0.f;
+      for (int w = 0; w < kWarps; ++w) mx = fmaxf(mx, sm.red_w[w][tid / kG][tid % kG]);
+      const float st = mx / 65535.f;
+      sm.dv[tid / kG][tid % kG] = st > 0.f ? st : 1.f;
+      sm.inv[tid / kG][tid % kG] = st > 0.f ? 1.f / st : 0.f;
+    }
+    __syncthreads();
+    const float inv1 = sm.inv[0][h], inv2 = sm.inv[1][h];
+    // round to nearest (even) through the float adder: x + 1.5 * 2^23 leaves the integer in the low
+    // mantissa bits for 0 <= x < 2^22 (here x <= 65535 * (1 + 2^-23))
+    auto to_int = [](float x) { return __float_as_int(x + 12582912.f) - 0x4B400000; };
+#pragma unroll
+    for (int jj = 0; jj < kMaxBlk; ++jj) {
+      if (jj >= nblk) break;
+      uint32_t w1h = 0, w1l = 0, w2h = 0, w2l = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int w1 = min(to_int(pv[jj][q] * inv1), 65535), w2 = min(to_int(pr[jj][q] * inv2), 65535);
+        w1h |= (uint32_t)(w1 >> 8) << (8 * q);
+        w1l |= (uint32_t)(w1 & 255) << (8 * q);
+        w2h |= (uint32_t)(w2 >> 8) << (8 * q);
+        w2l |= (uint32_t)(w2 & 255) << (8 * q);
+        wsum[0] += w1;
+        wsum[1] += w2;
+      }
+      uint8_t* blk = &sm.k.pw[jj][0][0][0];
+      *reinterpret_cast<uint32_t*>(blk + (2 * h) * kPwRow + q4) = w1h;
+      *reinterpret_cast<uint32_t*>(blk + (2 * h + 1) * kPwRow + q4) = w1l;
+      *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h) * kPwRow + q4) = w2h;
+      *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h + 1) * kPwRow + q4) = w2l;
+    }
+    __syncthreads();
+  }
+
+  // ---------------- value pass (warps 0..5: byte group bg, token half)
   // value-side accumulators: 8 m-tiles (bit rows 0..7 of bytes g, g+8 of this warp's byte group)
   int vacc[8][4];
 #pragma unroll
   for (int u = 0; u < 8; ++u) vacc[u][0] = vacc[u][1] = vacc[u][2] = vacc[u][3] = 0;
-  float lsum = 0.f;            // sum of p for head (P-warps)
-  int wsum[2] = {0, 0};        // sum of integer weights (value, QJL) for head (P-warps)
-
-  const int bg = warp % 3, half = warp / 3;   // value side: byte group and token half (warps 0..5)
-
-  // Integer weights of value block jj into pw[jj & 1]: thread -> (head, 4 consecutive tokens)
-  // per round; w1 = round(p * ||v|| / dv[0][h]), w2 = round(p * rnorm / dv[1][h]) with
-  // p = exp2(logit - max), each split into 8-bit pieces (hi * 256 + lo). Also accumulates sum p
-  // and the integer sums.
-  auto prepare_weights = [&](int jj, int tix, int nthreads) {
-    const int tb = jj * kBlk;
-    const int nval = min(kBlk, ntok - tb);
-    const int h = tix & 3;
-    const float hm = sm.hmax[h], inv1 = sm.inv[0][h], inv2 = sm.inv[1][h];
-    for (int q4 = (tix >> 2) * 4; q4 < kBlk; q4 += (nthreads >> 2) * 4) {
-      const float4 l4 = *reinterpret_cast<const float4*>(&sm.logits[h][tb + q4]);
-      const float lv[4] = {l4.x, l4.y, l4.z, l4.w};
-      uint32_t w1h = 0, w1l = 0, w2h = 0, w2l = 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        const int tok = q4 + q;
-        if (tok < nval) {
-          const float p = exp2_approx(lv[q] - hm);
-          const int w1 = min(__float2int_rn(p * __half2float(sm.vnorm[tb + tok]) * inv1), 65535);
-          const int w2 = min(__float2int_rn(p * __half2float(sm.vrn[tb + tok]) * inv2), 65535);
-          w1h |= (uint32_t)(w1 >> 8) << (8 * q);
-          w1l |= (uint32_t)(w1 & 255) << (8 * q);
-          w2h |= (uint32_t)(w2 >> 8) << (8 * q);
-          w2l |= (uint32_t)(w2 & 255) << (8 * q);
-          lsum += p;
-          wsum[0] += w1;
-          wsum[1] += w2;
-        }
-      }
-      uint8_t* blk = &sm.pw[jj & 1][0][0][0];
-      *reinterpret_cast<uint32_t*>(blk + (2 * h) * kBlk + q4) = w1h;
-      *reinterpret_cast<uint32_t*>(blk + (2 * h + 1) * kBlk + q4) = w1l;
-      *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h) * kBlk + q4) = w2h;
-      *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h + 1) * kBlk + q4) = w2l;
-    }
-  };
-
-  // No warp ever leaves this loop early: a wait that runs out sets abort_flag, after
-  // which nothing new is issued and no further waits happen, so every warp still
-  // meets the same CTA barriers; the results are then discarded.
-  int issued = min(kAhead, njobs);
-  for (int j = 0; j < njobs; ++j) {
-    const bool aborted = *(volatile int*)&sm.abort_flag != 0;
-    if (tid == 0 && !aborted && j + kAhead < njobs) {
-      // refill the stage of job j + kAhead - kStages (= j - 2) once every warp has released it
-      const int jo = j + kAhead - kStages;   // = j - 2
-      if (jo >= 0 && !mbar_wait(&sm.empty[jo % kStages], (jo / kStages) & 1)) {
-        sm.abort_flag = 1;
-      } else {
-        issue(j + kAhead);
-        issued = j + kAhead + 1;
-      }
-    }
-    if (!aborted && !mbar_wait(&sm.full[j % kStages], (j / kStages) & 1)) sm.abort_flag = 1;
-    const bool kside = j < nblk;
-    const int jj = kside ? j : j - nblk;
-    const unsigned char* st = sm.stage[j % kStages];
-    const __half* nrm = reinterpret_cast<const __half*>(st + kStageCodes + kStageSigns);
-    const __half* rnm = nrm + kBlk;
-    const int tok_base = jj * kBlk;
-    const int nvalid = min(kBlk, ntok - tok_base);
-
-    if (j == nblk) {
-      // ------------ between the passes: chunk maxima, weight scales, first P block
-      __syncthreads();
-      if (lane == 0) {
-        for (int h = 0; h < kG; ++h) sm.red_f[warp][h] = -INFINITY;
-      }
-      __syncwarp();
-      float m = run_max;
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
-      if (g == 0) sm.red_f[warp][t] = m;
-      float wv = wv_max, wr = wr_max;
-#pragma unroll
-      for (int o = 4; o < 32; o <<= 1) {
-        wv = fmaxf(wv, __shfl_xor_sync(0xffffffffu, wv, o));
-        wr = fmaxf(wr, __shfl_xor_sync(0xffffffffu, wr, o));
-      }
-      if (g == 0) sm.red_w[warp][0][t] = wv, sm.red_w[warp][1][t] = wr;
-      __syncthreads();
-      if (tid < kG) {
-        float mm = -INFINITY, mv = -INFINITY, mr = -INFINITY;
-        for (int w = 0; w < kWarps; ++w) {
-          mm = fmaxf(mm, sm.red_f[w][tid]);
-          mv = fmaxf(mv, sm.red_w[w][0][tid]);
-          mr = fmaxf(mr, sm.red_w[w][1][tid]);
-        }
-        sm.hmax[tid] = mm;
-        // 16-bit weights per head against the head's largest weight of the chunk (a hair above it,
-        // so that the approximate exp2 / log2 cannot push the largest weight past 65535)
-        const float s1 = exp2_approx(mv - mm) * (1.f + 1.f / 4096.f) / 65535.f;
-        const float s2 = exp2_approx(mr - mm) * (1.f + 1.f / 4096.f) / 65535.f;
-        sm.dv[0][tid] = (s1 > 0.f && s1 < INFINITY) ? s1 : 1.f;
-        sm.dv[1][tid] = (s2 > 0.f && s2 < INFINITY) ? s2 : 1.f;
-        sm.inv[0][tid] = 1.f / sm.dv[0][tid];
-        sm.inv[1][tid] = 1.f / sm.dv[1][tid];
-      }
-      __syncthreads();
-      // integer weights of the first value block (all threads); later blocks are prepared
-      // by warps 6 and 7 while warps 0..5 run the value MMAs of the block before
-      prepare_weights(0, tid, kThreads);
+  const int bg = warp % 3, half = warp / 3;
+  for (int jj = 0; jj < nblk; ++jj) {
+    wait_full(&sm.vfull[jj]);
+    if (jj == s_blk) {   // uniform in the CTA
+      patch_slot(false);
       __syncthreads();
     }
-
-    if (kside) {
-      // ---------------- key pass: warp w scores keys 16w .. 16w+15 and 128+16w .. of the block
+    if (warp < 6) {
+      const uint8_t* pw = &sm.k.pw[jj][bg == 2 ? 1 : 0][0][0];
+      const unsigned char* vc = sm.vcodes + jj * kStageCodes;
+      const unsigned char* vs = sm.vsigns + jj * kStageSigns;
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt) {
-        const int kbase = 128 * mt + 16 * warp;
-        float sc[2];
-        mtile_scores(st, nrm, rnm, kbase, qb, &sm.qfrag[1][0][0][t][g], c0h, dmh, dsh, ssh, sc);
+      for (int kq = 0; kq < 4; ++kq) {
+        const int tk = 128 * half + 32 * kq;  // first token of this 32-token k-step
+        uint32_t r[4];
+        const int tok = tk + (lane & 15) + 16 * (lane >> 4);
+        const unsigned char* rowp = (bg < 2) ? vc + tok * kCodesB + 16 * bg : vs + tok * kSignsB;
+        ldsm_t8_x2(r, rowp);
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(pw + g * kPwRow + tk + 4 * t);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(pw + g * kPwRow + tk + 16 + 4 * t);
 #pragma unroll
-        for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
-          const int key = kbase + g + 8 * r;
-          // softmax scale * log2(e): the weights are exp2(logit - max)
-          const float v = (key < nvalid) ? sc[r] * scale2 : -INFINITY;
-          sm.logits[t][tok_base + key] = v;
-          run_max = fmaxf(run_max, v);
-          // the token's weights will be exp2(v - max) ||v|| and exp2(v - max) rnorm (value norms
-          // arrived with the key block): track their largest logarithms for the weight steps
-          wv_max = fmaxf(wv_max, v + __log2f(__half2float(nrm[2 * kBlk + key])));
-          wr_max = fmaxf(wr_max, v + __log2f(__half2float(nrm[3 * kBlk + key])));
+        for (int s = 0; s < 4; ++s) {
+          const uint32_t x0 = r[0] >> s, x1 = r[1] >> s, x2 = r[2] >> s, x3 = r[3] >> s;
+          mma_u8(vacc[s], x0 & 0x01010101u, x1 & 0x01010101u, x2 & 0x01010101u, x3 & 0x01010101u, b0, b1);
+          mma_u8(vacc[4 + s], x0 & 0x10101010u, x1 & 0x10101010u, x2 & 0x10101010u, x3 & 0x10101010u, b0, b1);
         }
       }
-      // value norms of these tokens: keep for the value pass
-      if (tid < kBlk) {
-        sm.vnorm[tok_base + tid] = nrm[2 * kBlk + tid];
-        sm.vrn[tok_base + tid] = nrm[3 * kBlk + tid];
-      }
-    } else {
-      // ---------------- value pass (warps 0..5: byte group bg, token half)
-      if (warp < 6) {
-        const uint8_t* pw = &sm.pw[jj & 1][bg == 2 ? 1 : 0][0][0];
-#pragma unroll
-        for (int kq = 0; kq < 4; ++kq) {
-          const int tk = 128 * half + 32 * kq;  // first token of this 32-token k-step
-          uint32_t r[4];
-          const int tok = tk + (lane & 15) + 16 * (lane >> 4);
-          const unsigned char* rowp = (bg < 2) ? st + tok * kCodesB + 16 * bg : st + kStageCodes + tok * kSignsB;
-          ldsm_t8_x2(r, rowp);
-          const uint32_t b0 = *reinterpret_cast<const uint32_t*>(pw + g * kBlk + tk + 4 * t);
-          const uint32_t b1 = *reinterpret_cast<const uint32_t*>(pw + g * kBlk + tk + 16 + 4 * t);
-#pragma unroll
-          for (int s = 0; s < 4; ++s) {
-            const uint32_t x0 = r[0] >> s, x1 = r[1] >> s, x2 = r[2] >> s, x3 = r[3] >> s;
-            mma_u8(vacc[s], x0 & 0x01010101u, x1 & 0x01010101u, x2 & 0x01010101u, x3 & 0x01010101u, b0, b1);
-            mma_u8(vacc[4 + s], x0 & 0x10101010u, x1 & 0x10101010u, x2 & 0x10101010u, x3 & 0x10101010u, b0, b1);
-          }
-        }
-      } else if (jj + 1 < nblk) {
-        prepare_weights(jj + 1, tid - 6 * 32, 64);
-      }
-      __syncthreads();   // the next block's weights are ready; this block's are no longer read
     }
-    __syncwarp();
-    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[j % kStages])) : "memory");
   }
 
   __syncthreads();
   if (sm.abort_flag) {
-    // a copy or a release never completed: record it, then wait (bounded) for the
-    // copies that may still be in flight into this CTA's shared memory before leaving
+    // a copy never completed: record it, then wait (bounded) for the copies that may still be in
+    // flight into this CTA's shared memory before leaving
     if (tid == 0) {
       report_error(a.err, kErrTimeout);
-      for (int jx = max(0, issued - kStages); jx < issued; ++jx)
-        (void)mbar_wait(&sm.full[jx % kStages], (jx / kStages) & 1);
+      for (int j = 0; j < nblk; ++j) {
+        (void)mbar_wait(&sm.kfull[j], 0);
+        (void)mbar_wait(&sm.vfull[j], 0);
+      }
     }
     __syncthreads();
     return;
@@ -599,8 +672,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
       const int f = (u < 4) ? 0 : 4;
       const float v0 = 256.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
       const float v1 = 256.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
-      sm.vacc[bg][t][g * 8 + u] = v0;          // byte g, bit u
-      sm.vacc[bg][t][64 + g * 8 + u] = v1;     // byte g + 8, bit u
+      sm.k.vacc[bg][t][g * 8 + u] = v0;          // byte g, bit u
+      sm.k.vacc[bg][t][64 + g * 8 + u] = v1;     // byte g + 8, bit u
     }
   }
   __syncthreads();
@@ -610,8 +683,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
       const int f = (u < 4) ? 0 : 4;
       const float v0 = 256.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
       const float v1 = 256.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
-      sm.vacc[bg][t][g * 8 + u] += v0;
-      sm.vacc[bg][t][64 + g * 8 + u] += v1;
+      sm.k.vacc[bg][t][g * 8 + u] += v0;
+      sm.k.vacc[bg][t][64 + g * 8 + u] += v1;
     }
   }
   __syncthreads();
@@ -632,12 +705,12 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
       // code c = j: byte c / 4 (group c / 64), bits 2(c % 4) (plane 0) and 2(c % 4) + 1 (plane 1)
       const int byte = j >> 2, grp = byte >> 4, bl = byte & 15, u0 = 2 * (j & 3);
       const int idx = (bl < 8) ? bl * 8 : 64 + (bl - 8) * 8;
-      const float d0 = sm.vacc[grp][h][idx + u0], d1 = sm.vacc[grp][h][idx + u0 + 1];
+      const float d0 = sm.k.vacc[grp][h][idx + u0], d1 = sm.k.vacc[grp][h][idx + u0 + 1];
       v = sm.dv[0][h] * (a.vc0 * (float)W1 + a.vb0 * d0 + a.vb1 * d1);
     } else {
       const int p = j - kD, byte = p >> 3, u = p & 7;
       const int idx = (byte < 8) ? byte * 8 + u : 64 + (byte - 8) * 8 + u;
-      v = sm.dv[1][h] * (2.f * sm.vacc[2][h][idx] - (float)W2);
+      v = sm.dv[1][h] * (2.f * sm.k.vacc[2][h][idx] - (float)W2);
     }
     a.part[(((size_t)b * a.Hq + h0 + h) * a.nsplit + split) * stride + j] = v;
   }
@@ -736,6 +809,9 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
   for (int kk = 0; kk < 12; ++kk)
 #pragma unroll
     for (int slot = 0; slot < 2; ++slot) qb[kk][slot] = sm.qfrag[0][kk][slot][t][g];
+  // lo-piece fragments stay in shared memory here (three CTAs per SM leave no room in registers)
+  const uint32_t* qlo = &sm.qfrag[1][0][0][t][g];
+  auto lo_smem = [&](int kk, int sl) { return qlo[(kk * 2 + sl) * 32]; };
   const float c0h = sm.qconst[t][0], dmh = sm.qconst[t][1], dsh = sm.qconst[t][2], ssh = sm.qconst[t][3];
   float* lrow = a.logits + ((size_t)b * a.Hq + h0 + t) * a.L_cap + start;   // head t's scores of the chunk
 
@@ -762,7 +838,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
     if (!aborted) {
 #pragma unroll
       for (int mt = 0; mt < 2; ++mt)
-        mtile_scores(st, nrm, rnm, 128 * mt + 16 * warp, qb, &sm.qfrag[1][0][0][t][g], c0h, dmh, dsh, ssh, sc[mt]);
+        mtile_scores(st, st + kStageCodes, nrm, rnm, 128 * mt + 16 * warp, qb, lo_smem, c0h, dmh, dsh, ssh, sc[mt]);
     }
     __syncwarp();
     if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[j % kSStages])) : "memory");

@@ -16,6 +16,7 @@ constexpr float kQjlScale = 1.2533141373155002512f;  // sqrt(pi / 2)
 constexpr int kErrCapacity = 1;
 constexpr int kErrTimeout = 2;
 constexpr int kErrInternal = 4;   // a kernel found its own launch state unusable (e.g. shared memory alignment)
+constexpr int kErrBounds = 8;     // TQ_CHECK=1: a device-resident argument (a length) was out of range
 
 __device__ __forceinline__ void report_error(int* err, int bit) {
   if (err) atomicOr(err, bit);

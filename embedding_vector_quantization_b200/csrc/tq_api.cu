@@ -5,10 +5,17 @@
 // Fault injection for tests (host side only; no GPU fault is ever caused):
 //   TQ_FAULT=alloc   -> tq_create* fails with TQ_ENOMEM before allocating
 //   TQ_FAULT=launch  -> hot calls fail with TQ_ECUDA before launching
+//   TQ_FAULT=timeout -> hot calls record a wait timeout in the handle's error word (no wait
+//                       happens), as a kernel does when a copy never arrives
+// Checks: TQ_CHECK=1 makes the hot calls that read device lengths first validate every
+// len[b] against 0 .. L_cap on the device, recording an out-of-range length in the handle's
+// error word (tq_last_status: TQ_EINVAL) instead of clamping it silently.
+// Tracing: every hot call is an NVTX range named after the entry point.
 
 #include <cuda.h>
 #include <cudaTypedefs.h>
 #include <cuda_runtime.h>
+#include <nvtx3/nvToolsExt.h>
 
 #include <algorithm>
 #include <atomic>
@@ -93,6 +100,17 @@ int cuda_fail(cudaError_t e, const char* where) {
     cudaError_t e_ = (call);                            \
     if (e_ != cudaSuccess) return cuda_fail(e_, #call); \
   } while (0)
+
+// One NVTX range per hot call (free when no profiler is attached).
+struct NvtxRange {
+  explicit NvtxRange(const char* name) { nvtxRangePushA(name); }
+  ~NvtxRange() { nvtxRangePop(); }
+};
+
+bool check_mode() {
+  const char* c = std::getenv("TQ_CHECK");
+  return c && std::strcmp(c, "1") == 0;
+}
 
 int launch_check(const char* what) {
   cudaError_t e = cudaGetLastError();
@@ -452,13 +470,14 @@ int64_t round_chunk(int64_t v, int64_t blk, int64_t lo, int64_t hi) {
 }
 
 // Attention split policy (shared by every attention kernel): about two CTAs per
-// SM, chunks a multiple of 128 tokens and at most 1024 tokens long.
+// SM, chunks a multiple of 128 tokens and at most 896 tokens long (the 3-bit kernel
+// stages a whole chunk of keys and values in shared memory).
 void attn_split(int B, int Hkv, int64_t L_cap, int* nsplit, int64_t* chunk) {
   const int64_t units = std::max<int64_t>(1, (int64_t)B * Hkv);
   const int64_t ns = std::max<int64_t>(1, (2 * 148 + units - 1) / units);
   int64_t ch = (L_cap + ns - 1) / ns;
-  ch = std::min<int64_t>(1024, std::max<int64_t>(128, (ch + 127) / 128 * 128));
-  if (const int64_t f = splitk_override()) ch = round_chunk(f, 128, 128, 1024);
+  ch = std::min<int64_t>(tqk::amma::kMaxChunk, std::max<int64_t>(128, (ch + 127) / 128 * 128));
+  if (const int64_t f = splitk_override()) ch = round_chunk(f, 128, 128, tqk::amma::kMaxChunk);
   *chunk = ch;
   *nsplit = (int)((L_cap + ch - 1) / ch);
 }
@@ -778,6 +797,17 @@ int tq_internal_fail(int code, const char* fmt, ...) {
 }
 
 namespace tqk {
+// TQ_CHECK=1: every len[b] must lie in 0 .. L_cap.
+__global__ void check_lens_kernel(const int32_t* len, int B, int64_t L_cap, int* err) {
+  const int b = blockIdx.x * blockDim.x + threadIdx.x;
+  if (b < B && (len[b] < 0 || (int64_t)len[b] > L_cap)) report_error(err, kErrBounds);
+}
+
+// TQ_FAULT=timeout: the error a timed-out wait records, without any wait.
+__global__ void inject_error_kernel(int* err, int bit) {
+  if (threadIdx.x == 0) report_error(err, bit);
+}
+
 // The failure path of every bounded wait, on its own: thread 0 waits for phase 0 of a
 // barrier that expects one arrival and never gets it, gives up after `limit` polls and
 // records kErrTimeout, as a kernel does when a copy or a release never completes.
@@ -789,6 +819,22 @@ __global__ void selftest_wait_kernel(int* err, int limit) {
   }
 }
 }  // namespace tqk
+
+namespace {
+// TQ_CHECK and TQ_FAULT=timeout work that precedes a hot call's kernels (len may be NULL).
+int pre_launch(const tq_handle* h, const int32_t* len, int B, int64_t L_cap, cudaStream_t s) {
+  if (len && B > 0 && check_mode()) {
+    tqk::check_lens_kernel<<<(B + 255) / 256, 256, 0, s>>>(len, B, L_cap, h->derr);
+    if (int st = launch_check("check_lens_kernel")) return st;
+  }
+  if (fault_is("timeout")) {
+    tqk::inject_error_kernel<<<1, 32, 0, s>>>(h->derr, tqk::kErrTimeout);
+    return launch_check("inject_error_kernel");
+  }
+  return TQ_OK;
+}
+
+}  // namespace
 
 // ============================================================================
 extern "C" {
@@ -893,6 +939,7 @@ int tq_get_rotation(const tq_handle* h, double* Pi, double* S) {
 
 int tq_encode(const tq_handle* h, const void* x, int x_dtype, int64_t n, uint8_t* codes, uint8_t* signs,
               void* norms, void* rnorms, void* stream) {
+  NvtxRange nvtx("tq_encode");
   if (!h) return fail(TQ_EINVAL, "handle is NULL");
   if (n < 0) return fail(TQ_EINVAL, "n=%lld", (long long)n);
   if (!valid_dtype(x_dtype)) return fail(TQ_EINVAL, "x dtype %d", x_dtype);
@@ -903,6 +950,7 @@ int tq_encode(const tq_handle* h, const void* x, int x_dtype, int64_t n, uint8_t
   if (!aligned(x, 16) || (codes && !aligned(codes, 16)) || (signs && !aligned(signs, 16)) || !aligned(norms, 4))
     return fail(TQ_EINVAL, "misaligned pointer");
   if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
+  if (int st = pre_launch(h, nullptr, 0, 0, static_cast<cudaStream_t>(stream))) return st;
   if (h->polar) return polar_encode_launch(h, x, x_dtype, n, codes, norms, nullptr, 0, 0, static_cast<cudaStream_t>(stream));
   tqk::EncodeArgs a{};
   a.x = x; a.x_dtype = x_dtype; a.rows = n; a.d = h->d; a.bits = h->bits; a.m = h->m;
@@ -913,6 +961,7 @@ int tq_encode(const tq_handle* h, const void* x, int x_dtype, int64_t n, uint8_t
 }
 
 int tq_pack_indices(const tq_handle* h, const uint8_t* idx, int64_t n, uint8_t* codes, void* stream) {
+  NvtxRange nvtx("tq_pack_indices");
   if (!h) return fail(TQ_EINVAL, "handle is NULL");
   if (n < 0) return fail(TQ_EINVAL, "n=%lld", (long long)n);
   if (n == 0) return ok();
@@ -928,6 +977,7 @@ int tq_pack_indices(const tq_handle* h, const uint8_t* idx, int64_t n, uint8_t* 
 
 int tq_append(const tq_handle* h, const void* x_new, int x_dtype, int B, int Hkv, const tq_cache* cache,
               int32_t* len, int advance, void* stream) {
+  NvtxRange nvtx("tq_append");
   if (!h) return fail(TQ_EINVAL, "handle is NULL");
   if (B < 0 || Hkv < 1) return fail(TQ_EINVAL, "B=%d Hkv=%d", B, Hkv);
   if (!valid_dtype(x_dtype)) return fail(TQ_EINVAL, "x dtype %d", x_dtype);
@@ -938,6 +988,7 @@ int tq_append(const tq_handle* h, const void* x_new, int x_dtype, int B, int Hkv
   if (!aligned(x_new, 16)) return fail(TQ_EINVAL, "x_new misaligned");
   if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = pre_launch(h, len, B, cache->L_cap, s))) return st;
   if (h->polar) {
     if ((st = polar_encode_launch(h, x_new, x_dtype, (int64_t)B * Hkv, cache->codes, cache->norms, len, Hkv,
                                   cache->L_cap, s)))
@@ -1008,6 +1059,7 @@ size_t tq_search_workspace_bytes(const tq_handle* h, int nq, int64_t n, int k) {
 
 int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const tq_cache* k, const int32_t* len,
              float* logits, void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("tq_score");
   if (!hk) return fail(TQ_EINVAL, "handle is NULL");
   if (B < 0 || Hq < 1 || Hkv < 1 || Hq % Hkv != 0) return fail(TQ_EINVAL, "B=%d Hq=%d Hkv=%d", B, Hq, Hkv);
   if (Hq / Hkv > tqk::kMaxGroup) return fail(TQ_EUNSUPPORTED, "group Hq/Hkv=%d > %d", Hq / Hkv, tqk::kMaxGroup);
@@ -1021,6 +1073,7 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const 
   if (!aligned(workspace, 16)) return fail(TQ_EINVAL, "workspace misaligned");
   if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = pre_launch(hk, len, B, k->L_cap, s))) return st;
   ScoreWs w;
   score_ws_layout(hk, B * Hq, static_cast<char*>(workspace), &w);
   st = launch_qprep(hk, q, TQ_F32, B * Hq, w.qr, w.qs, s);
@@ -1225,8 +1278,10 @@ extern "C" {
 int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
                    const tq_cache* k, const tq_cache* v, const int32_t* len, float scale, float* out,
                    void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("tq_attn_decode");
   int st = attn_check(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, len, scale, out, workspace, ws_bytes);
   if (st || B == 0) return st;
+  if ((st = pre_launch(hk, len, B, k->L_cap, static_cast<cudaStream_t>(stream)))) return st;
   return attn_impl(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, const_cast<int32_t*>(len), scale, out, workspace,
                    static_cast<cudaStream_t>(stream), false);
 }
@@ -1234,6 +1289,7 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
 int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, const void* k_new,
                    const void* v_new, int x_dtype, int B, int Hq, int Hkv, const tq_cache* k, const tq_cache* v,
                    int32_t* len, float scale, float* out, void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("tq_decode_step");
   int st = attn_check(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, len, scale, out, workspace, ws_bytes);
   if (st || B == 0) return st;
   if (!valid_dtype(x_dtype)) return fail(TQ_EINVAL, "x dtype %d", x_dtype);
@@ -1242,6 +1298,7 @@ int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int 
   if (hk->d > tqk::kSmallMaxD || hk->m > tqk::kSmallMaxD || hv->m > tqk::kSmallMaxD || hk->d > tqk::kWideMaxD)
     return fail(TQ_EUNSUPPORTED, "tq_decode_step needs d <= %d and m <= %d", tqk::kSmallMaxD, tqk::kSmallMaxD);
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if ((st = pre_launch(hk, len, B, k->L_cap, s))) return st;
   ScoreWs w;
   float* part;
   int nsplit;
@@ -1282,6 +1339,7 @@ int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int 
 
 int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* codes, const void* norms, int64_t n,
                    int k, int64_t* idx, float* score, void* workspace, size_t ws_bytes, void* stream) {
+  NvtxRange nvtx("tq_search_topk");
   if (!h) return fail(TQ_EINVAL, "handle is NULL");
   if (h->m > 0 || h->polar) return fail(TQ_EUNSUPPORTED, "search takes MSE handles");
   if (nq < 0 || n < 1 || k < 1 || k > tqk::kMaxTopK || k > n)
@@ -1293,6 +1351,7 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
   if (ws_bytes < need) return fail(TQ_EINVAL, "workspace %zu < %zu bytes", ws_bytes, need);
   if (fault_is("launch")) return fail(TQ_ECUDA, "injected launch failure (TQ_FAULT=launch)");
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (int st0 = pre_launch(h, nullptr, 0, 0, s)) return st0;
   float *qr, *cs;
   int64_t* ci;
   int nchunks;
@@ -1437,6 +1496,7 @@ int tq_last_status(const tq_handle* h, void* stream) {
     if (e != cudaSuccess) return cuda_fail(e, "clear error word");
   }
   if (word & tqk::kErrInternal) return fail(TQ_ECUDA, "a kernel found its shared memory misaligned");
+  if (word & tqk::kErrBounds) return fail(TQ_EINVAL, "a length len[b] outside 0 .. L_cap (found by TQ_CHECK=1)");
   if (word & tqk::kErrTimeout) return fail(TQ_ETIMEOUT, "a bounded device wait timed out");
   if (word & tqk::kErrCapacity) return fail(TQ_ECAPACITY, "append skipped a full sequence (len == L_cap)");
   return ok();

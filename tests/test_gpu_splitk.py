@@ -5,9 +5,9 @@ ring of TMA stages. At the small shapes of the other parity tests a chunk holds 
 two blocks, so the ring never wraps. Here every kernel runs chunks of several blocks:
 
 * attn_prod2_kernel at the exact decode-step workload (1 sequence, 8 KV / 32 query
-  heads, context 32768: 37 chunks of 896 tokens = 4 key + 4 value blocks on a 5-stage
-  ring), plus a ragged length and forced 1024-token chunks;
-* attn_mse4_kernel with 1024-token chunks (4 + 4 blocks on a 4-stage ring);
+  heads, context 32768: 37 chunks of 896 tokens, each staged whole as 4 key and 4 value
+  blocks with one barrier each), plus a ragged length and forced 512-token chunks;
+* attn_mse4_kernel with 896-token chunks (4 + 4 blocks on its 4-stage ring);
 * score_prod2_kernel with 5- and 10-block chunks on its 4-stage ring (TQ_SPLITK);
 * search_mma2_kernel / search_mma4_kernel with 3 to 6 blocks per chunk.
 
@@ -101,11 +101,11 @@ def decode_workload(tq):
     return dict(hk=hk, hv=hv, ohk=ohk, ohv=ohv, K=K, V=V, kc=kc, vc=vc, kod=kod, vod=vod, q=q, L=L)
 
 
-@pytest.mark.parametrize("length,force", [(32768, None), (30001, None), (32768, 1024)])
+@pytest.mark.parametrize("length,force", [(32768, None), (30001, None), (32768, 512)])
 def test_attn_prod2_decode_workload_matches_oracle(tq, decode_workload, length, force):
     """attn_prod2_kernel at the decode-step workload's own split (896-token chunks of 3.5
-    blocks: 4 key and 4 value jobs per chunk through the 5-stage ring), at a ragged length
-    and with forced 1024-token chunks."""
+    blocks: 4 key and 4 value blocks per chunk, a partial last block), at a ragged length
+    and with forced 512-token chunks."""
     w = decode_workload
     lens = torch.tensor([length], dtype=torch.int32).cuda()
     scale = 1.0 / np.sqrt(128)
@@ -151,11 +151,11 @@ def test_decode_step_decode_workload_matches_oracle(tq, decode_workload):
     print(f"decode step at the decode workload: max relative attention error {worst:.2e}")
 
 
-@pytest.mark.parametrize("lens,force", [([10240, 10239, 9000, 5121], None), ([2048, 1, 0, 1500], 1024)])
-def test_attn_mse4_1024_token_chunks_match_oracle(tq, lens, force):
-    """attn_mse4_kernel with 1024-token chunks (4 key + 4 value jobs through its 4-stage ring):
-    4 sequences x 8 KV heads x 10240 tokens (the 4-bit workload's own split policy gives 10
-    chunks of 1024), ragged and empty lengths."""
+@pytest.mark.parametrize("lens,force", [([10240, 10239, 9000, 5121], None), ([2048, 1, 0, 1500], 640)])
+def test_attn_mse4_multiblock_chunks_match_oracle(tq, lens, force):
+    """attn_mse4_kernel with 896-token chunks (4 key + 4 value jobs through its 4-stage ring):
+    4 sequences x 8 KV heads x 10240 tokens (the split policy gives 12 chunks of 896, the last
+    one partial), ragged and empty lengths; and forced 640-token chunks."""
     B, Hkv, G, d = 4, 8, 4, 128
     L = max(max(lens), 128)
     L = (L + 7) // 8 * 8
@@ -175,7 +175,7 @@ def test_attn_mse4_1024_token_chunks_match_oracle(tq, lens, force):
     assert hk.status() == tq.TQ_OK
     ref = ops.decode_attention(q.double().numpy(), kod, vod, [max(1, x) for x in lens], scale)
     worst = _check_attention(o, ref, lens)
-    print(f"4-bit attention, chunk {force or 1024}: max relative attention error {worst:.2e}")
+    print(f"4-bit attention, chunk {force or 896}: max relative attention error {worst:.2e}")
 
 
 @pytest.mark.parametrize("force,lens", [(2560, [8192, 6001]), (1280, [8192, 2561]), (1024, [8192, 7937])])
