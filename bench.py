@@ -22,7 +22,8 @@ e2e     = same metric through the C ABI with host buffers: per step one CUDA
 rows    = (N = 1, unless --no-rows) every other hot-path row measured after the headline's
           timed region with a few steps each and folded into the same line: the cfg-1 encode
           + score record, the streaming score step, the prefill encode, the 4-bit decode step,
-          the 3-bit decode step over an HBM-sized cache, and the 2- and 4-bit searches.
+          the 3-bit decode step over an HBM-sized cache, the 2- and 4-bit searches, and the
+          scores over polar-transform and QJL-only keys.
 Multi-GPU (--gpus N under torchrun): every rank runs its own independent
 instance of the workload (weak scaling, no collective on the data path); the
 reported time is the max over ranks.
@@ -53,7 +54,7 @@ FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) of one attn_prod2_kernel launch on this workload, from
 # `ncu --set full` (the attention kernel's profile summary in the repository); set to None whenever
 # that kernel changes until it is captured again.
-ATTN_TRAFFIC_BYTES = 27350272
+ATTN_TRAFFIC_BYTES = None
 
 
 def decode_config(world):
@@ -72,7 +73,7 @@ def parse_args():
     p.add_argument("--impl", choices=["tq", "reference"], default="tq")
     p.add_argument("--no-cpu-baseline", action="store_true")
     p.add_argument("--workload", choices=["decode", "score", "encode", "attn4", "attn3big", "search", "search4",
-                                          "compare", "cfg1"],
+                                          "compare", "cfg1", "polar", "qjl"],
                    default="decode",
                    help="decode: the headline decode step (default); the others measure the remaining hot-path "
                         "rows on their own workloads, one JSON line each (attn3big: the 3-bit decode step over a "

@@ -67,11 +67,9 @@ def _encode_into(tq, h, cache, x_of, L, slice_len, torch):
         b.record()
         torch.cuda.synchronize()
         ms += a.elapsed_time(b)
-        cache.codes[:, :, l0:l0 + n].copy_(out["codes"])
-        cache.norms[:, :, l0:l0 + n].copy_(out["norms"])
-        if h.m:
-            cache.signs[:, :, l0:l0 + n].copy_(out["signs"])
-            cache.rnorms[:, :, l0:l0 + n].copy_(out["rnorms"])
+        for name in ("codes", "signs", "norms", "rnorms"):   # (QJL-only rows have no codes or rnorms)
+            if out[name] is not None:
+                getattr(cache, name)[:, :, l0:l0 + n].copy_(out[name])
         del x, out
     return ms
 
@@ -677,6 +675,108 @@ def run_compare(args):
           extra["speedup_vs_bf16"], "x", us["turboquant_3bit"] / 1e3, cfg, roof, 3 * reps, clocks, extra)
 
 
+# ------------------------------------------------------------------ polar and QJL-only scores (next rows)
+
+def run_score_kind(args, kind):
+    """Scores of 32 query heads (4 per KV head) over a cache of the next rows' formats, d = 128:
+    kind "polar" (recursive polar transform, 4 bits at level 1, 2 bits above: 48-byte rows,
+    fp32 norms; 32 sequences x 8 KV heads x 16384 keys) or "qjl" (QJL-only 1-bit rows: 128 sign
+    bits and an fp16 norm; 64 x 8 x 16384). One tq_score per step in a CUDA graph; the prefill
+    encode is timed too. Both score kernels run on the CUDA cores (table lookups and fp32 FMAs
+    for polar, sign-weighted sums for QJL-only), so the roofline is the fp32 SIMT peak."""
+    import torch
+    import embedding_vector_quantization_b200 as tq
+    d, Hkv, G, L = 128, 8, 4, 16384
+    B = 32 if kind == "polar" else 64
+    if args.small:
+        B = 4
+    Hq = Hkv * G
+    h = tq.PolarHandle(d, 4, 2, seed=0) if kind == "polar" else tq.Handle(d, 1, 0, qjl_m=128)
+    cache = tq.Cache(h, B, Hkv, L)
+    g = torch.Generator(device="cuda").manual_seed(10)
+    enc_ms = _encode_into(tq, h, cache, lambda l0, n: torch.randn(B, Hkv, n, d, generator=g, device="cuda")
+                          .to(torch.bfloat16), L, 2048, torch)
+    gq = torch.Generator(device="cuda").manual_seed(11)
+    W, T = args.warmup, args.steps
+    qs = torch.randn(T + W, B, Hq, d, generator=gq, device="cuda")
+    q_in = qs[0].clone()
+    lens = torch.full((B,), L, dtype=torch.int32, device="cuda")
+    logits = torch.empty(B, Hq, L, dtype=torch.float32, device="cuda")
+    ws = torch.empty(tq.tq_score_workspace_bytes(h.ptr, B, Hq), dtype=torch.uint8, device="cuda")
+
+    def step():
+        tq.tq_score(h.ptr, q_in, B, Hq, Hkv, cache.struct, lens, logits, ws)
+
+    s_ = torch.cuda.Stream()
+    s_.wait_stream(torch.cuda.current_stream())
+    with torch.cuda.stream(s_):
+        step()
+    torch.cuda.current_stream().wait_stream(s_)
+    torch.cuda.synchronize()
+    graph = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph):
+        step()
+    tq.tq_timer_read(None, forget=True)
+    tq.tq_timer_enable(True)
+    graph_k = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(graph_k):
+        step()
+    tq.tq_timer_enable(False)
+    for t in range(W):
+        q_in.copy_(qs[t])
+        graph.replay()
+    torch.cuda.synchronize()
+    sampler = bench.ClockSampler("GPU-" + str(torch.cuda.get_device_properties(0).uuid))
+    sampler.start()
+    evs = []
+    for t in range(T):
+        q_in.copy_(qs[W + t])
+        ev = _events(torch)
+        ev[0].record()
+        graph.replay()
+        ev[1].record()
+        evs.append(ev)
+    torch.cuda.synchronize()
+    clocks = sampler.stop()
+    total_ms = sum(a.elapsed_time(b) for a, b in evs)
+    sc_ms, sc_n = 0.0, 0
+    for t in range(T):
+        q_in.copy_(qs[W + t])
+        graph_k.replay()
+        torch.cuda.synchronize()
+        ms_k, n_k = tq.tq_timer_read("score", forget=False)
+        sc_ms += ms_k
+        sc_n += n_k
+    _, kernels_per_step = tq.tq_timer_read(None, forget=False)
+    keys = B * Hkv * L
+    row = h.codes_B + h.signs_B + (4 if h.norm_dtype == tq.TQ_F32 else 2)
+    # fp32 flops the kernel's arithmetic needs per (key, query head): polar, a product and an FMA
+    # per fold of the d - 1 tree nodes above the level-1 table lookups; QJL-only, an FMA per sign
+    flops_per = (4 * (d // 2 - 1) + 2) if kind == "polar" else 2 * 128
+    flops = keys * G * flops_per
+    sm_mhz = clocks.get("sm_mhz") or 1965.0
+    peak = torch.cuda.get_device_properties(0).multi_processor_count * FP32_LANES_PER_SM * 2 * sm_mhz * 1e6 / 1e12
+    launch_ms = sc_ms / max(sc_n, 1)
+    ach = flops / (launch_ms / 1e3) / 1e12
+    name = {"polar": "recursive polar transform (PolarQuant), d=128, 4 bits at level 1 and 2 bits at levels 2-7 "
+                     "(2.98 bits per coordinate)",
+            "qjl": "QJL-only 1-bit keys (128 sign bits + fp16 norm), d=128"}[kind]
+    cfg = {"workload": f"scores of 4 query heads per KV head over {name}; {B} sequences x 8 KV heads x 16384 keys",
+           "B": B, "Hkv": Hkv, "Hq": Hq, "context": L, "d": d,
+           "dtype": "f32 SIMT (per-query tables)" if kind == "polar" else "f32 SIMT",
+           "l2": "not flushed: each step reads %.0f MB of packed keys and writes %.0f MB of logits"
+                 % (keys * row / 1e6, keys * G * 4 / 1e6)}
+    roof = {"bound": "alu", "kernel": "polar_score_kernel" if kind == "polar" else "score_simt_kernel",
+            "achieved": ach, "peak": peak, "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+            "peak_source": "derived: SMs x 128 fp32 lanes x 2 flop x median sampled SM clock",
+            "launch_ms": launch_ms, "algorithmic_flops_per_launch": flops,
+            "hbm_gbs_of_the_same_launch": (keys * row + keys * G * 4) / (launch_ms / 1e3) / 1e9}
+    extra = {"keys_scored_per_s": keys * T / (total_ms / 1e3),
+             "prefill_encode": {"vectors": keys, "ms": enc_ms, "vectors_per_s": keys / (enc_ms / 1e3)}}
+    _line(args, f"keys scored/sec ({kind} keys)", extra["keys_scored_per_s"], "keys/s", total_ms / T, cfg, roof,
+          kernels_per_step * T, clocks, extra, None)
+
+
 # ------------------------------------------------------------------ the small MSE workload (cfg 1)
 
 def _unpack_rows(codes, d, bits):
@@ -750,9 +850,14 @@ def run_cfg1(args):
         el = time.perf_counter() - t0
         mism = idx != eo["idx"]
         near = np.abs(eo["y"][mism] - bo[np.minimum(idx[mism], eo["idx"][mism])]) if mism.any() else np.zeros(0)
+        # scores against the oracle scoring the GPU's own codes (the parity rule), and end to end
+        # against the oracle's own encode (a code inside the 1e-5 band moves its key's score a step)
+        sg = ops.score_mse(q.double().numpy().reshape(d), idx, norms.astype(np.float64), Pio, co)
+        floor = np.linalg.norm(q.double().numpy()) * norms.astype(np.float64) / np.sqrt(d)
         rec["oracle"] = {"index_mismatch_fraction": float(mism.mean()),
                          "mismatches_within_1e-5_of_a_boundary": bool(np.all(near < 1e-5)),
-                         "max_abs_score_difference": float(np.max(np.abs(scores - so))),
+                         "max_score_error_on_gpu_codes_rel_to_floor": float(np.max(np.abs(scores - sg) / floor)),
+                         "max_abs_score_difference_end_to_end": float(np.max(np.abs(scores - so))),
                          "oracle_seconds": el, "kind": "oracle", "cores": bench.blas_threads()}
     if COLLECT is not None:
         COLLECT.append({"metric": "cfg1", "record": rec})
@@ -760,14 +865,15 @@ def run_cfg1(args):
         print(json.dumps({"metric": "MSE-only 3-bit encode + score record (cfg 1)", "record": rec}), flush=True)
 
 
-def collect_rows(args, rows=("cfg1", "score", "encode", "attn4", "attn3big", "search", "search4")):
+def collect_rows(args, rows=("cfg1", "score", "encode", "attn4", "attn3big", "search", "search4", "polar", "qjl")):
     """Runs every other hot-path row with a few steps and returns {row: its line}. The rows'
     own CPU baselines are skipped (the cfg-1 record keeps its oracle check)."""
     import copy
     global COLLECT
     out = {}
     fns = {"cfg1": run_cfg1, "score": run_score, "encode": run_encode, "attn4": run_attn4, "attn3big": run_attn3big,
-           "search": lambda a: run_search(a, bits=2), "search4": lambda a: run_search(a, bits=4)}
+           "search": lambda a: run_search(a, bits=2), "search4": lambda a: run_search(a, bits=4),
+           "polar": lambda a: run_score_kind(a, "polar"), "qjl": lambda a: run_score_kind(a, "qjl")}
     for name in rows:
         a = copy.copy(args)
         a.steps, a.warmup, a.small = 10, 3, False
@@ -794,4 +900,5 @@ def run(args):
         run_search(args, bits=4)
         return
     {"score": run_score, "encode": run_encode, "attn4": run_attn4, "attn3big": run_attn3big,
-     "search": run_search, "cfg1": run_cfg1}[args.workload](args)
+     "search": run_search, "cfg1": run_cfg1, "polar": lambda a: run_score_kind(a, "polar"),
+     "qjl": lambda a: run_score_kind(a, "qjl")}[args.workload](args)

@@ -290,60 +290,69 @@ __device__ __forceinline__ void prepare_query(const float* qr_rows, const float*
   }
 }
 
-// Raw scores (tq_score's formula) of keys kbase + g and kbase + g + 8 of a staged key block
-// for query head t = lane % 4: the code bit planes against the query pieces of n tile 0 (hi and
-// mid, fragments qb held in registers) and n tile 1 (lo: lo(k-step, register) returns this
-// thread's fragment word, from registers or shared memory), the sign bit planes against the
-// two pieces of S q in n tile 0.
-template <typename LoFn>
+// Raw scores (tq_score's formula) of keys kbase[i] + g and kbase[i] + g + 8 of a staged key
+// block (NT m-tiles of 16 keys, their MMAs interleaved for independent accumulator chains) for
+// query head t = lane % 4: the code bit planes against the query pieces of n tile 0 (hi and mid,
+// fragments qb held in registers) and n tile 1 (lo: lo(k-step, register) returns this thread's
+// fragment word, from registers or shared memory), the sign bit planes against the two pieces of
+// S q in n tile 0.
+template <int NT, typename LoFn>
 __device__ __forceinline__ void mtile_scores(const unsigned char* codes, const unsigned char* signs, const __half* nrm,
-                                             const __half* rnm, int kbase, const uint32_t (&qb)[12][2], LoFn lo,
-                                             float c0h, float dmh, float dsh, float ssh, float (&sc)[2]) {
+                                             const __half* rnm, const int (&kbase)[NT], const uint32_t (&qb)[12][2],
+                                             LoFn lo, float c0h, float dmh, float dsh, float ssh, float (&sc)[NT][2]) {
   const int lane = threadIdx.x & 31, g = lane >> 2;
-  uint32_t cw[4], sw[2];
-  {
+  uint32_t cw[NT][4], sw[NT][2];
+#pragma unroll
+  for (int i = 0; i < NT; ++i) {
     const int mat = lane >> 3, r = lane & 7;
-    const int key = kbase + r + 8 * (mat >> 1);
-    ldsm_x4(cw, codes + key * kCodesB + 16 * (mat & 1));
-    const int skey = kbase + r + 8 * (mat & 1);
-    ldsm_x2(sw, signs + skey * kSignsB);
+    const int key = kbase[i] + r + 8 * (mat >> 1);
+    ldsm_x4(cw[i], codes + key * kCodesB + 16 * (mat & 1));
+    const int skey = kbase[i] + r + 8 * (mat & 1);
+    ldsm_x2(sw[i], signs + skey * kSignsB);
   }
-  // tile 0: six independent accumulator chains (codes: even / odd shifts); tile 1: two chains
-  int dm1[2][4] = {}, dm16[2][4] = {}, ds1[4] = {}, ds16[4] = {};
-  int lm1[4] = {}, lm16[4] = {};
+  // per m-tile: codes (x1 and x16 families, n tiles 0 and 1) and signs (n tile 0)
+  int dm1[NT][4] = {}, dm16[NT][4] = {}, lm1[NT][4] = {}, lm16[NT][4] = {}, ds1[NT][4] = {}, ds16[NT][4] = {};
   // code words: cw[0] = key g word t, cw[1] = key g word 4+t, cw[2] = key g+8 word t, cw[3] = key g+8 word 4+t
 #pragma unroll
   for (int s = 0; s < 4; ++s) {
-    const uint32_t x0 = cw[0] >> s, x1 = cw[1] >> s, x2 = cw[2] >> s, x3 = cw[3] >> s;
-    const uint32_t a0 = x0 & 0x01010101u, a1 = x2 & 0x01010101u, a2 = x1 & 0x01010101u, a3 = x3 & 0x01010101u;
-    const uint32_t b0 = x0 & 0x10101010u, b1 = x2 & 0x10101010u, b2 = x1 & 0x10101010u, b3 = x3 & 0x10101010u;
-    mma_s8(dm1[s & 1], a0, a1, a2, a3, qb[s][0], qb[s][1]);
-    mma_s8(dm16[s & 1], b0, b1, b2, b3, qb[4 + s][0], qb[4 + s][1]);
-    mma_s8(lm1, a0, a1, a2, a3, lo(s, 0), lo(s, 1));
-    mma_s8(lm16, b0, b1, b2, b3, lo(4 + s, 0), lo(4 + s, 1));
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const uint32_t x0 = cw[i][0] >> s, x1 = cw[i][1] >> s, x2 = cw[i][2] >> s, x3 = cw[i][3] >> s;
+      const uint32_t a0 = x0 & 0x01010101u, a1 = x2 & 0x01010101u, a2 = x1 & 0x01010101u, a3 = x3 & 0x01010101u;
+      const uint32_t b0 = x0 & 0x10101010u, b1 = x2 & 0x10101010u, b2 = x1 & 0x10101010u, b3 = x3 & 0x10101010u;
+      mma_s8(dm1[i], a0, a1, a2, a3, qb[s][0], qb[s][1]);
+      mma_s8(dm16[i], b0, b1, b2, b3, qb[4 + s][0], qb[4 + s][1]);
+      mma_s8(lm1[i], a0, a1, a2, a3, lo(s, 0), lo(s, 1));
+      mma_s8(lm16[i], b0, b1, b2, b3, lo(4 + s, 0), lo(4 + s, 1));
+    }
   }
   // sign words: sw[0] = key g word t, sw[1] = key g+8 word t
 #pragma unroll
   for (int s = 0; s < 2; ++s) {
-    const uint32_t y0 = sw[0] >> s, y1 = sw[1] >> s, z0 = sw[0] >> (s + 2), z1 = sw[1] >> (s + 2);
-    const uint32_t a0 = y0 & 0x01010101u, a1 = y1 & 0x01010101u, a2 = z0 & 0x01010101u, a3 = z1 & 0x01010101u;
-    const uint32_t b0 = y0 & 0x10101010u, b1 = y1 & 0x10101010u, b2 = z0 & 0x10101010u, b3 = z1 & 0x10101010u;
-    mma_s8(ds1, a0, a1, a2, a3, qb[8 + s][0], qb[8 + s][1]);
-    mma_s8(ds16, b0, b1, b2, b3, qb[10 + s][0], qb[10 + s][1]);
+#pragma unroll
+    for (int i = 0; i < NT; ++i) {
+      const uint32_t y0 = sw[i][0] >> s, y1 = sw[i][1] >> s, z0 = sw[i][0] >> (s + 2), z1 = sw[i][1] >> (s + 2);
+      const uint32_t a0 = y0 & 0x01010101u, a1 = y1 & 0x01010101u, a2 = z0 & 0x01010101u, a3 = z1 & 0x01010101u;
+      const uint32_t b0 = y0 & 0x10101010u, b1 = y1 & 0x10101010u, b2 = z0 & 0x10101010u, b3 = z1 & 0x10101010u;
+      mma_s8(ds1[i], a0, a1, a2, a3, qb[8 + s][0], qb[8 + s][1]);
+      mma_s8(ds16[i], b0, b1, b2, b3, qb[10 + s][0], qb[10 + s][1]);
+    }
   }
   const float kqjl = kQjlScale / (float)kM;
 #pragma unroll
-  for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
-    const int key = kbase + g + 8 * r;
-    const int hi = 2 * r, md = 2 * r + 1;   // tile 0: columns 2t (hi) and 2t + 1 (mid); tile 1: column 2t (lo)
-    // exact in int32: at most 256 code positions of |piece| <= 127 each, times 2^14
-    const int mse = (dm1[0][hi] + dm1[1][hi] + ((dm16[0][hi] + dm16[1][hi]) >> 4)) * 16384 +
-                    (dm1[0][md] + dm1[1][md] + ((dm16[0][md] + dm16[1][md]) >> 4)) * 128 + lm1[hi] + (lm16[hi] >> 4);
-    // column 2t + 1 holds the lo piece of S q here
-    const int qjl = (ds1[hi] + (ds16[hi] >> 4)) * 128 + ds1[md] + (ds16[md] >> 4);
-    const float n = __half2float(nrm[key]), rn = __half2float(rnm[key]);
-    sc[r] = n * (c0h + dmh * (float)mse) + rn * kqjl * (2.f * dsh * (float)qjl - ssh);
-  }
+  for (int i = 0; i < NT; ++i)
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
+      const int key = kbase[i] + g + 8 * r;
+      const int hi = 2 * r, md = 2 * r + 1;   // tile 0: columns 2t (hi) and 2t + 1 (mid); tile 1: column 2t (lo)
+      // exact in int32: at most 256 code positions of |piece| <= 127 each, times 2^14
+      const int mse = (dm1[i][hi] + (dm16[i][hi] >> 4)) * 16384 + (dm1[i][md] + (dm16[i][md] >> 4)) * 128 +
+                      lm1[i][hi] + (lm16[i][hi] >> 4);
+      // column 2t + 1 holds the lo piece of S q here
+      const int qjl = (ds1[i][hi] + (ds16[i][hi] >> 4)) * 128 + ds1[i][md] + (ds16[i][md] >> 4);
+      const float n = __half2float(nrm[key]), rn = __half2float(rnm[key]);
+      sc[i][r] = n * (c0h + dmh * (float)mse) + rn * kqjl * (2.f * dsh * (float)qjl - ssh);
+    }
 }
 
 __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
@@ -484,11 +493,21 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
     const unsigned char* ks = sm.k.signs + tok_base * kSignsB;
     const __half* nrm = sm.k.kn + tok_base;
     const __half* rnm = sm.k.krn + tok_base;
+    // warp w: keys 16w .. 16w+15 and 128+16w .. 128+16w+15 (both m-tiles at once, or the first
+    // alone when the block's valid keys end before the second; warp-uniform)
+    float sc[2][2];
+    if (16 * warp + 128 < nvalid) {
+      const int kb2[2] = {16 * warp, 128 + 16 * warp};
+      mtile_scores<2>(kc, ks, nrm, rnm, kb2, qb, lo_reg, c0h, dmh, dsh, ssh, sc);
+    } else if (16 * warp < nvalid) {
+      const int kb1[1] = {16 * warp};
+      float sc1[1][2];
+      mtile_scores<1>(kc, ks, nrm, rnm, kb1, qb, lo_reg, c0h, dmh, dsh, ssh, sc1);
+      sc[0][0] = sc1[0][0], sc[0][1] = sc1[0][1], sc[1][0] = sc[1][1] = 0.f;
+    }
 #pragma unroll
     for (int mt = 0; mt < 2; ++mt) {
       const int kbase = 128 * mt + 16 * warp;
-      float sc[2];
-      mtile_scores(kc, ks, nrm, rnm, kbase, qb, lo_reg, c0h, dmh, dsh, ssh, sc);
 #pragma unroll
       for (int r = 0; r < 2; ++r) {  // r = 0: key g, r = 1: key g + 8
         const int key = kbase + g + 8 * r;
@@ -496,7 +515,7 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
         // (the last block of a chunk may be partial: nothing past its valid keys is stored, the
         // logits rows hold kMaxChunk tokens)
         if (key < nvalid) {
-          const float v = sc[r] * scale2;
+          const float v = sc[mt][r] * scale2;
           sm.logits[t][tok_base + key] = v;
           run_max = fmaxf(run_max, v);
         }
@@ -614,9 +633,11 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
       const uint8_t* pw = &sm.k.pw[jj][bg == 2 ? 1 : 0][0][0];
       const unsigned char* vc = sm.vcodes + jj * kStageCodes;
       const unsigned char* vs = sm.vsigns + jj * kStageSigns;
+      const int nvalv = min(kBlk, ntok - jj * kBlk);
 #pragma unroll
       for (int kq = 0; kq < 4; ++kq) {
         const int tk = 128 * half + 32 * kq;  // first token of this 32-token k-step
+        if (tk >= nvalv) break;               // past the chunk's end (weights 0; warp-uniform)
         uint32_t r[4];
         const int tok = tk + (lane & 15) + 16 * (lane >> 4);
         const unsigned char* rowp = (bg < 2) ? vc + tok * kCodesB + 16 * bg : vs + tok * kSignsB;
@@ -837,8 +858,12 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
     float sc[2][2];
     if (!aborted) {
 #pragma unroll
-      for (int mt = 0; mt < 2; ++mt)
-        mtile_scores(st, st + kStageCodes, nrm, rnm, 128 * mt + 16 * warp, qb, lo_smem, c0h, dmh, dsh, ssh, sc[mt]);
+      for (int mt = 0; mt < 2; ++mt) {
+        const int kb1[1] = {128 * mt + 16 * warp};
+        float sc1[1][2];
+        mtile_scores<1>(st, st + kStageCodes, nrm, rnm, kb1, qb, lo_smem, c0h, dmh, dsh, ssh, sc1);
+        sc[mt][0] = sc1[0][0], sc[mt][1] = sc1[0][1];
+      }
     }
     __syncwarp();
     if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[j % kSStages])) : "memory");
