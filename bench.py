@@ -47,14 +47,15 @@ PACKED_BYTES_PER_TOKEN = 2 * (32 + 16 + 2 + 2)   # K and V: 2-bit codes + sign b
 WORKLOAD_NAME = ("GQA decode step, TurboQuant prod 3-bit (2-bit Lloyd-Max + 1-bit QJL m=128), d=128, "
                  "B=1, 8 KV heads / 32 query heads, context 32768, bf16 K/V with lognormal channel scales "
                  "and 2 outlier channels")
-# Arithmetic of the timed path: int8 x int8 -> int32 tensor-core MMAs on 15-bit fixed-point queries
-# and 14-bit fixed-point softmax weights, fp32 softmax, combine and output.
-DTYPE = "s8xs8->s32 MMA (15/14-bit fixed-point operands), f32 softmax/combine"
+# Arithmetic of the timed path: int8 x int8 -> int32 tensor-core MMAs on fixed-point queries (22-bit
+# against the codes, 15-bit against the QJL signs) and 16-bit fixed-point softmax weights, fp32
+# softmax, combine and output.
+DTYPE = "s8xs8->s32 MMA (22/15-bit fixed-point queries, 16-bit weights), f32 softmax/combine"
 FALLBACK_HBM_GBS = 6650.0
 # DRAM bytes (read + write) of one attn_prod2_kernel launch on this workload, from
 # `ncu --set full` (the attention kernel's profile summary in the repository); set to None whenever
 # that kernel changes until it is captured again.
-ATTN_TRAFFIC_BYTES = None
+ATTN_TRAFFIC_BYTES = 27_368_192
 
 
 def decode_config(world):

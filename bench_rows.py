@@ -17,6 +17,7 @@ Workloads (all synthetic, seeded; the big inputs are drawn on the GPU):
 """
 
 import json
+import os
 import time
 
 import bench
@@ -468,7 +469,7 @@ FP32_LANES_PER_SM = 128   # fp32 FMA lanes per B200 SM (4 partitions x 32)
 
 
 def run_search(args, bits=None):
-    """cfg-4 search at 2 bits (int8 tensor-core kernel) or 4 bits (SIMT kernel with the centroid table)."""
+    """cfg-4 search at 2 or 4 bits on the tcgen05 kernel (TQ_SEARCH_MMA=1: the legacy int8 kernels)."""
     import torch
     import embedding_vector_quantization_b200 as tq
     bits = S4["bits"] if bits is None else bits
@@ -529,7 +530,20 @@ def run_search(args, bits=None):
                        "N(0,I) database vectors, 1024 queries (stands in for the pages' vector-search benchmarks)",
            "n": n, "nq": nq, "d": d, "k": k,
            "l2": f"not flushed: the {n * d * bits // 8 // 1000000} MB of codes exceed the 126 MB L2"}
-    if bits in (2, 4):
+    if not os.environ.get("TQ_SEARCH_MMA") and d % 128 == 0:
+        # tcgen05 int8 contractions into tensor memory: the measured bf16 dense peak x 2 (the
+        # nominal int8 : bf16 ratio, 4.5 : 2.25 PFLOP/s)
+        bf16, src = _peak("tensor")
+        peak = 2.0 * bf16
+        cfg["dtype"] = ("int8 tcgen05 mma (15-bit centroid and query pieces: three contractions into two "
+                        "int32 accumulators in tensor memory)")
+        roof = {"bound": "tensor", "kernel": "search_tc_kernel", "achieved": ach, "peak": peak,
+                "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
+                "peak_source": f"{src} x 2 (int8 : bf16 nominal ratio)",
+                "launch_ms": s_ms / max(s_n, 1), "algorithmic_flops_per_launch": flops,
+                "note": "algorithmic 2d flops per (query, vector); the kernel executes 3x that in int8 MMA "
+                        "operations (C_h Q_h, C_h Q_l, C_l Q_h), so its tensor-bound ceiling is 1/3 of the peak"}
+    elif bits in (2, 4):
         # int8 tensor-core contraction: the measured bf16 dense peak x 2 (the nominal int8 : bf16
         # ratio, 4.5 : 2.25 PFLOP/s)
         bf16, src = _peak("tensor")

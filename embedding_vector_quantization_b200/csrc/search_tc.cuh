@@ -1,0 +1,490 @@
+// Top-k inner-product search over MSE codes of 1 to 4 bits on the 5th-generation tensor cores
+// (tcgen05.mma kind::i8, accumulators in tensor memory, query operand staged by TMA).
+//
+// "TurboQuant: redefining AI efficiency" (hakusoku.com), "Impact on high-dimensional vector
+// search": s = ||x|| <Pi q, c[idx]> over the compressed database, ranked by score (equal scores:
+// lower index first).
+//
+// Fixed point. The centroids and each rotated query are rounded to integers against one step
+// each, c_i ~ step_c C_i and q'_j ~ step_q Q_j with |C|, |Q| <= 16319, and split into int8 pieces
+// C = 128 C_h + C_l, Q = 128 Q_h + Q_l (C_l, Q_l in [-64, 63], C_h, Q_h in [-127, 127]). Then
+//   <Q, C[idx]> = 16384 <Q_h, C_h[idx]> + 128 (<Q_l, C_h[idx]> + <Q_h, C_l[idx]>) + <Q_l, C_l[idx]>;
+// the kernel forms the first two terms exactly in int32 (two accumulators, three int8
+// contractions of depth d) and drops the last, which is below 2^-16 of |Q_j C_j| per coordinate.
+// Any codebook works (no symmetry or affine structure is assumed): a coordinate's two operand
+// bytes C_h[idx], C_l[idx] come from 16-entry tables by byte permutes.
+//
+// Tiles. Queries are the MMA rows (M = 128 per CTA, one per tensor-memory lane), database vectors
+// the columns (N = 256 per tile). A CTA holds one query tile and walks a contiguous chunk of the
+// database, 256 vectors per tile; a tile is a loop over K-chunks of 128 coordinates (one 128-byte
+// swizzle atom of int8):
+//   warp 0, lane 0   TMA: Q_h and Q_l of the K-chunk (two 16 KB boxes, 128-byte swizzle), 3 stages
+//   warp 1           tensor-memory allocation (512 columns: acc_hi, acc_mid); lane 0 issues
+//                    4 K-steps x 3 MMAs per K-chunk, then commits the stages and the accumulator
+//   warps 2-5        expansion: thread p owns vector rows p and p + 128 of the tile, keeps their
+//                    packed codes of the next K-chunk in flight in registers, and writes C_h and C_l
+//                    of all 128 coordinates into the swizzled B tiles of a 2-stage ring
+//   warps 6-9        epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31, so thread t owns
+//                    query 32 (w % 4) + lane: it turns the row's 2 x 256 accumulators into scores and
+//                    keeps the query's running top-k (k <= 32) as a sorted list in registers.
+// Per query and chunk the list goes to the candidate arrays, which topk_merge_kernel reduces.
+// Every wait is bounded; a wait that runs out sets an abort flag (checked by every loop) and the
+// error word's kErrTimeout bit; the kernel then waits (bounded) for its own copies and MMAs and
+// frees its tensor memory.
+#pragma once
+
+#include <cuda.h>
+
+#include "common.cuh"
+#include "encode_tc.cuh"
+
+namespace tqk {
+namespace stc {
+
+using etc::bar_arrive;
+using etc::expect_tx;
+using etc::mma_commit;
+using etc::sts128;
+using etc::sw128_desc;
+using etc::tc_fence_after;
+using etc::tc_fence_before;
+using etc::tma_load_2d;
+using etc::wait_bar;
+
+constexpr int kQ = 128;          // queries per CTA (MMA M, tensor-memory lanes)
+constexpr int kV = 256;          // vectors per tile (MMA N)
+constexpr int kKC = 128;         // coordinates per K-chunk
+constexpr int kQS = 3;           // query-operand stages
+constexpr int kVS = 2;           // vector-operand stages
+constexpr int kMaxK = 32;        // list entries per query
+constexpr int kMaxBits = 4;
+constexpr int kCMax = 16319;     // |C|, |Q| bound: 128 * 127 + 63
+constexpr int kThreads = 320;    // 10 warps
+constexpr int kExpandWarp0 = 2, kEpiWarp0 = 6;
+constexpr uint32_t kTmemCols = 512;
+
+constexpr uint32_t kQStage = 2u * kQ * kKC;              // 32 KB: Q_h box, then Q_l box
+constexpr uint32_t kVStage = 2u * kV * kKC;              // 64 KB: C_h tile, then C_l tile
+constexpr uint32_t kOffQ = 0;
+constexpr uint32_t kOffV = kOffQ + kQS * kQStage;         // 96 KB
+constexpr uint32_t kOffNorm = kOffV + kVS * kVStage;      // 224 KB: float [2][kV]
+constexpr uint32_t kOffBars = kOffNorm + 2 * kV * 4;
+// q_full[kQS], q_empty[kQS], v_full[kVS], v_empty[kVS], acc_full, acc_empty
+constexpr int kNumBars = 2 * kQS + 2 * kVS + 2;
+constexpr uint32_t kOffTmemSlot = kOffBars + 8 * kNumBars;
+constexpr uint32_t kOffAbort = kOffTmemSlot + 4;
+constexpr uint32_t kSmemBytes = kOffAbort + 4;
+static_assert(kSmemBytes <= 232448, "search_tc layout exceeds the shared memory of one CTA");
+
+struct Args {
+  int nq, nq_pad, d, k, norm_dtype, codes_B;
+  const uint8_t* codes;    // [n][codes_B]
+  const void* norms;       // [n]
+  const float* qscale;     // [nq]: step_q * step_c
+  int64_t n, chunk;        // database rows, rows per CTA chunk (a multiple of kV)
+  uint32_t th[4], tl[4];   // C_h[idx], C_l[idx] as bytes, idx = 0 .. 15
+  float* cand_s;           // [nchunks][nq][k]
+  int64_t* cand_i;
+  int* err;
+};
+
+// 16-entry table lookup of four 4-bit indices (nibbles 0..3 of x) -> four bytes: two 8-entry
+// permutes, then a permute that takes byte j from the second when bit 3 of nibble j is set.
+__device__ __forceinline__ uint32_t lut16(uint32_t x, uint32_t t0, uint32_t t1, uint32_t t2, uint32_t t3) {
+  const uint32_t sel = x & 0x7777u;
+  const uint32_t lo = __byte_perm(t0, t1, sel), hi = __byte_perm(t2, t3, sel);
+  return __byte_perm(lo, hi, 0x3210u | ((x >> 1) & 0x4444u));
+}
+
+// Four fields of BITS bits (bits 0 .. 4 BITS - 1 of x) -> selector nibbles 0..3 (BITS = 1, 3).
+template <int BITS>
+__device__ __forceinline__ uint32_t nibbles4(uint32_t x) {
+  constexpr uint32_t m = (1u << BITS) - 1;
+  return (x & m) | ((x >> BITS & m) << 4) | ((x >> (2 * BITS) & m) << 8) | ((x >> (3 * BITS) & m) << 12);
+}
+
+// Eight 2-bit fields (bits 0..15 of x) -> nibbles 0..7.
+__device__ __forceinline__ uint32_t nibbles8_2bit(uint32_t x) {
+  uint32_t t = x & 0xFFFFu;
+  t = (t | (t << 8)) & 0x00FF00FFu;
+  t = (t | (t << 4)) & 0x0F0F0F0Fu;
+  t = (t | (t << 2)) & 0x33333333u;
+  return t;
+}
+
+// Operand bytes of 16 coordinates (unit u of a 128-coordinate code chunk w[]) -> h[4], l[4].
+template <int BITS>
+__device__ __forceinline__ void expand_unit(const uint32_t (&w)[4 * BITS], int u, const uint32_t (&th)[4],
+                                            const uint32_t (&tl)[4], uint32_t (&h)[4], uint32_t (&l)[4]) {
+  if constexpr (BITS == 4) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t x = w[2 * u + half];
+      h[2 * half] = lut16(x, th[0], th[1], th[2], th[3]);
+      l[2 * half] = lut16(x, tl[0], tl[1], tl[2], tl[3]);
+      h[2 * half + 1] = lut16(x >> 16, th[0], th[1], th[2], th[3]);
+      l[2 * half + 1] = lut16(x >> 16, tl[0], tl[1], tl[2], tl[3]);
+    }
+  } else if constexpr (BITS == 2) {
+#pragma unroll
+    for (int half = 0; half < 2; ++half) {
+      const uint32_t t = nibbles8_2bit(w[u] >> (16 * half));
+      h[2 * half] = __byte_perm(th[0], 0u, t);
+      l[2 * half] = __byte_perm(tl[0], 0u, t);
+      h[2 * half + 1] = __byte_perm(th[0], 0u, t >> 16);
+      l[2 * half + 1] = __byte_perm(tl[0], 0u, t >> 16);
+    }
+  } else if constexpr (BITS == 1) {
+    const uint32_t x = w[u >> 1] >> (16 * (u & 1));
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t s = nibbles4<1>(x >> (4 * j));
+      h[j] = __byte_perm(th[0], th[1], s);
+      l[j] = __byte_perm(tl[0], tl[1], s);
+    }
+  } else {   // BITS == 3: unit u is the 48 bits at bit 48 u of the chunk
+    const int wi = (3 * u) >> 1, sh = 16 * (u & 1);
+    const uint32_t w0 = w[wi], w1 = w[wi + 1], w2 = (wi + 2 < 12) ? w[wi + 2 < 12 ? wi + 2 : 0] : 0u;
+    const uint64_t win = (uint64_t)__funnelshift_r(w0, w1, sh) | ((uint64_t)(__funnelshift_r(w1, w2, sh) & 0xFFFFu) << 32);
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const uint32_t s = nibbles4<3>((uint32_t)(win >> (12 * j)));
+      h[j] = __byte_perm(th[0], th[1], s);
+      l[j] = __byte_perm(tl[0], tl[1], s);
+    }
+  }
+}
+
+// Packed codes of one row's K-chunk: 16 BITS bytes = 4 BITS words (zeros past the chunk's end).
+template <int BITS>
+__device__ __forceinline__ void load_chunk(const uint8_t* row, bool ok, uint32_t (&w)[4 * BITS]) {
+#pragma unroll
+  for (int i = 0; i < BITS; ++i) {
+    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+    if (ok) v = __ldg(reinterpret_cast<const uint4*>(row) + i);
+    w[4 * i] = v.x;
+    w[4 * i + 1] = v.y;
+    w[4 * i + 2] = v.z;
+    w[4 * i + 3] = v.w;
+  }
+}
+
+// Named barrier over n threads that also ORs a predicate across them.
+__device__ __forceinline__ bool bar_red_or(int id, int n, bool pred) {
+  uint32_t r;
+  asm volatile(
+      "{\n .reg .pred p, q;\n setp.ne.u32 p, %1, 0;\n bar.red.or.pred q, %2, %3, p;\n selp.u32 %0, 1, 0, q;\n}\n"
+      : "=r"(r)
+      : "r"((uint32_t)pred), "r"(id), "r"(n)
+      : "memory");
+  return r != 0;
+}
+
+__device__ __forceinline__ void mma_i8(uint32_t d_tmem, uint64_t a, uint64_t b, uint32_t idesc, uint32_t acc) {
+  asm volatile(
+      "{\n .reg .pred p;\n setp.ne.b32 p, %4, 0;\n tcgen05.mma.cta_group::1.kind::i8 [%0], %1, %2, %3, p;\n}\n" ::"r"(
+          d_tmem),
+      "l"(a), "l"(b), "r"(idesc), "r"(acc));
+}
+
+// Instruction descriptor, kind::i8: int32 accumulate, A and B signed 8-bit, both K-major, M = 128, N = kV.
+__host__ __device__ constexpr uint32_t idesc_i8() {
+  return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kV >> 3) << 17) | ((uint32_t)(kQ >> 4) << 24);
+}
+
+__device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
+      : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7]), "=r"(v[8]),
+        "=r"(v[9]), "=r"(v[10]), "=r"(v[11]), "=r"(v[12]), "=r"(v[13]), "=r"(v[14]), "=r"(v[15])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_wait_ld2(uint32_t (&x)[16], uint32_t (&y)[16]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]), "+r"(x[7]),
+                 "+r"(x[8]), "+r"(x[9]), "+r"(x[10]), "+r"(x[11]), "+r"(x[12]), "+r"(x[13]), "+r"(x[14]), "+r"(x[15]),
+                 "+r"(y[0]), "+r"(y[1]), "+r"(y[2]), "+r"(y[3]), "+r"(y[4]), "+r"(y[5]), "+r"(y[6]), "+r"(y[7]),
+                 "+r"(y[8]), "+r"(y[9]), "+r"(y[10]), "+r"(y[11]), "+r"(y[12]), "+r"(y[13]), "+r"(y[14]), "+r"(y[15])
+               :
+               : "memory");
+}
+
+// qmap: the query pieces as a 2-D int8 tensor {d, 2 nq_pad} (Q_h rows, then Q_l rows), box
+// {128, 128}, 128-byte swizzle. Grid: (chunks, query tiles of 128).
+template <int BITS>
+__global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_constant__ CUtensorMap qmap, Args a) {
+  extern __shared__ __align__(1024) unsigned char smem[];
+  const uint32_t base = smem_addr(smem);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int q0 = blockIdx.y * kQ;
+  const int64_t c0 = (int64_t)blockIdx.x * a.chunk, c1 = min(a.n, c0 + a.chunk);
+  const int ntiles = (int)((max(c1 - c0, (int64_t)0) + kV - 1) / kV);
+  const int nkc = a.d / kKC;
+  const int total = ntiles * nkc;   // K-chunks of this CTA
+
+  const uint32_t bars = base + kOffBars;
+  auto q_full = [&](int s) { return bars + 8u * s; };
+  auto q_empty = [&](int s) { return bars + 8u * (kQS + s); };
+  auto v_full = [&](int s) { return bars + 8u * (2 * kQS + s); };
+  auto v_empty = [&](int s) { return bars + 8u * (2 * kQS + kVS + s); };
+  const uint32_t acc_full = bars + 8u * (2 * kQS + 2 * kVS), acc_empty = acc_full + 8u;
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + kOffAbort);
+  float* nrm_s = reinterpret_cast<float*>(smem + kOffNorm);
+
+  if ((base & 1023u) != 0) {   // the swizzled operand layout needs 1024-byte alignment
+    if (tid == 0) report_error(a.err, kErrInternal);
+    return;
+  }
+  if (tid == 0) {
+    *abort_flag = 0;
+    for (int s = 0; s < kQS; ++s) {
+      bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + s, 1);
+      bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + kQS + s, 1);
+    }
+    for (int s = 0; s < kVS; ++s) {
+      bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + s, 4);   // the four expansion warps
+      bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + kVS + s, 1);
+    }
+    bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + 2 * kVS, 1);       // acc_full: commit
+    bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + 2 * kVS + 1, 4);   // acc_empty: epilogue warps
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  if (warp == 1) {
+    asm volatile("tcgen05.alloc.cta_group::1.sync.aligned.shared::cta.b32 [%0], %1;\n" ::"r"(base + kOffTmemSlot),
+                 "r"(kTmemCols)
+                 : "memory");
+    asm volatile("tcgen05.relinquish_alloc_permit.cta_group::1.sync.aligned;\n" ::: "memory");
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(smem + kOffTmemSlot);
+  int* const err = a.err;
+  auto fail_wait = [&]() {
+    *abort_flag = 1;
+    report_error(err, kErrTimeout);
+  };
+  grid_dep_wait();   // the query pieces come from the kernel before this one
+
+  if (warp == 0) {
+    // ---------------- TMA: query pieces of every K-chunk
+    if (lane == 0) {
+      int issued = 0;
+      for (; issued < total; ++issued) {
+        const int s = issued % kQS, kc = issued % nkc;
+        if (issued >= kQS && !*abort_flag && !wait_bar(q_empty(s), ((issued / kQS) - 1) & 1)) fail_wait();
+        if (*abort_flag) break;
+        expect_tx(q_full(s), kQStage);
+        tma_load_2d(base + kOffQ + s * kQStage, &qmap, kc * kKC, q0, q_full(s));
+        tma_load_2d(base + kOffQ + s * kQStage + kQStage / 2, &qmap, kc * kKC, a.nq_pad + q0, q_full(s));
+      }
+      // never leave with a copy still landing in this CTA's shared memory
+      for (int i = (issued > kQS ? issued - kQS : 0); i < issued; ++i) (void)wait_bar(q_full(i % kQS), (i / kQS) & 1);
+    }
+  } else if (warp == 1) {
+    // ---------------- MMA issue
+    if (lane == 0) {
+      constexpr uint32_t idesc = idesc_i8();
+      const uint32_t acc_hi = tmem, acc_mid = tmem + (uint32_t)kV;
+      int it = 0, committed_tiles = 0;
+      for (int t = 0; t < ntiles && !*abort_flag; ++t) {
+        if (t >= 1 && !wait_bar(acc_empty, (t - 1) & 1)) { fail_wait(); break; }
+        tc_fence_after();
+        for (int kc = 0; kc < nkc; ++kc, ++it) {
+          const int sq = it % kQS, sv = it % kVS;
+          if (!wait_bar(q_full(sq), (it / kQS) & 1) || !wait_bar(v_full(sv), (it / kVS) & 1)) { fail_wait(); break; }
+          tc_fence_after();
+          const uint32_t qa = base + kOffQ + sq * kQStage, vb = base + kOffV + sv * kVStage;
+#pragma unroll
+          for (int kk = 0; kk < kKC / 32; ++kk) {
+            const uint32_t off = kk * 32;
+            const uint64_t ah = sw128_desc(qa + off), al = sw128_desc(qa + kQStage / 2 + off);
+            const uint64_t bh = sw128_desc(vb + off), bl = sw128_desc(vb + kVStage / 2 + off);
+            const uint32_t acc = (kc > 0 || kk > 0) ? 1u : 0u;
+            mma_i8(acc_hi, ah, bh, idesc, acc);
+            mma_i8(acc_mid, al, bh, idesc, acc);
+            mma_i8(acc_mid, ah, bl, idesc, 1u);
+          }
+          mma_commit(q_empty(sq));
+          mma_commit(v_empty(sv));
+        }
+        if (*abort_flag) break;
+        mma_commit(acc_full);
+        committed_tiles = t + 1;
+      }
+      // tensor memory is released below: make sure no MMA still writes it
+      if (committed_tiles > 0) (void)wait_bar(acc_full, (committed_tiles - 1) & 1);
+    }
+  } else if (warp < kEpiWarp0) {
+    // ---------------- expansion: codes -> C_h / C_l operand tiles
+    const int p = tid - 32 * kExpandWarp0;   // 0 .. 127: rows p and p + 128
+    constexpr int W = 4 * BITS;
+    const int cbytes = kKC * BITS / 8;       // code bytes of a row's K-chunk
+    const uint8_t* codes = a.codes;
+    const int64_t codes_B = a.codes_B;
+    uint32_t th[4], tl[4];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      th[i] = a.th[i];
+      tl[i] = a.tl[i];
+    }
+    uint32_t cur[2][W], nxt[2][W];
+    auto fetch = [&](int itx, uint32_t(&w)[2][W]) {
+      const int t = itx / nkc, kc = itx % nkc;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int64_t v = c0 + (int64_t)t * kV + p + 128 * r;
+        const bool ok = itx < total && v < c1;
+        load_chunk<BITS>(codes + (ok ? v : 0) * codes_B + (int64_t)kc * cbytes, ok, w[r]);
+      }
+    };
+    fetch(0, cur);
+    for (int it = 0; it < total; ++it) {
+      fetch(it + 1, nxt);
+      const int s = it % kVS;
+      bool ok = !*abort_flag;
+      if (ok && it >= kVS && !wait_bar(v_empty(s), ((it / kVS) - 1) & 1)) { fail_wait(); ok = false; }
+      if (!__all_sync(0xffffffffu, ok)) break;
+      const uint32_t vb = base + kOffV + s * kVStage;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int row = p + 128 * r;
+        const uint32_t rh = vb + row * 128, rl = rh + kVStage / 2;
+#pragma unroll
+        for (int u = 0; u < 8; ++u) {
+          uint32_t h[4], l[4];
+          expand_unit<BITS>(cur[r], u, th, tl, h, l);
+          const uint32_t o = (uint32_t)((u ^ (row & 7)) << 4);
+          sts128(rh + o, h[0], h[1], h[2], h[3]);
+          sts128(rl + o, l[0], l[1], l[2], l[3]);
+        }
+      }
+      asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor-core reads
+      __syncwarp();
+      if (lane == 0) bar_arrive(v_full(s));
+#pragma unroll
+      for (int r = 0; r < 2; ++r)
+#pragma unroll
+        for (int i = 0; i < W; ++i) cur[r][i] = nxt[r][i];
+    }
+  } else {
+    // ---------------- epilogue: scores and running top-k, one query per thread
+    const int quarter = warp & 3, ql = 32 * quarter + lane, q = q0 + ql;
+    const int e = tid - 32 * kEpiWarp0;   // 0 .. 127
+    const bool qok = q < a.nq;
+    const float qscale = qok ? a.qscale[q] : 0.f;
+    const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
+    // the list, descending: entries kMaxK - k .. kMaxK - 1 are the running top-k (empty: -inf),
+    // the ones before them +inf sentinels that no score displaces, so the k-th best is always
+    // the last entry and an insertion bubbles through fixed register positions
+    const int k = a.k;
+    float ls[kMaxK];
+    int li[kMaxK];
+#pragma unroll
+    for (int j = 0; j < kMaxK; ++j) {
+      ls[j] = j < kMaxK - k ? INFINITY : -INFINITY;
+      li[j] = -1;
+    }
+    float thr = -INFINITY;
+    for (int t = 0; t < ntiles; ++t) {
+      const int64_t v0 = c0 + (int64_t)t * kV;
+      const int nv = (int)min((int64_t)kV, c1 - v0);
+      float* nb = nrm_s + (t & 1) * kV;
+#pragma unroll
+      for (int r = 0; r < 2; ++r) {
+        const int j = e + 128 * r;
+        nb[j] = j < nv ? load_norm(a.norms, a.norm_dtype, v0 + j) : 0.f;
+      }
+      bool ok = !*abort_flag;
+      if (ok && !wait_bar(acc_full, t & 1)) { fail_wait(); ok = false; }
+      // one decision for all four warps (this barrier also publishes the norms): tcgen05.ld is
+      // warp-collective and every epilogue warp must reach the same barriers
+      if (bar_red_or(1, 128, !ok)) break;
+      tc_fence_after();
+#pragma unroll 1
+      for (int cb = 0; cb < kV / 16; ++cb) {
+        uint32_t hi[16], mid[16];
+        tmem_ld16(lane_addr + 16 * cb, hi);
+        tmem_ld16(lane_addr + kV + 16 * cb, mid);
+        tmem_wait_ld2(hi, mid);
+        if (16 * cb >= nv) continue;   // the same for the whole warp
+#pragma unroll
+        for (int j = 0; j < 16; ++j) {
+          const int col = 16 * cb + j;
+          const float v = fmaf(16384.f, (float)(int)hi[j], 128.f * (float)(int)mid[j]);
+          const float s = v * (qscale * nb[col]);
+          if (qok && col < nv && s > thr) {   // visited in index order: an equal score ranks after
+            float cs = s;
+            int ci = (int)(v0 + col);
+#pragma unroll
+            for (int x = 0; x < kMaxK; ++x) {
+              const bool sw = cs > ls[x];
+              const float ts = ls[x];
+              const int ti = li[x];
+              ls[x] = sw ? cs : ts;
+              li[x] = sw ? ci : ti;
+              cs = sw ? ts : cs;
+              ci = sw ? ti : ci;
+            }
+            thr = ls[kMaxK - 1];
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(acc_empty);
+    }
+    if (qok && !*abort_flag) {
+      const size_t o = ((size_t)blockIdx.x * a.nq + q) * k - (kMaxK - k);
+#pragma unroll
+      for (int x = 0; x < kMaxK; ++x)
+        if (x >= kMaxK - k) {
+          a.cand_s[o + x] = ls[x];
+          a.cand_i[o + x] = li[x];
+        }
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) {
+    __syncwarp();
+    asm volatile("tcgen05.dealloc.cta_group::1.sync.aligned.b32 %0, %1;\n" ::"r"(tmem), "r"(kTmemCols) : "memory");
+  }
+}
+
+// Query pieces: row q of qr (rotated queries, fp32) -> Q_h (row q) and Q_l (row nq_pad + q) of
+// `pieces`, Q = rint(q' / step_q) with step_q = max_j |q'_j| / 16319; qscale[q] = step_q * step_c.
+// Rows nq .. nq_pad - 1 are zero. One warp per row.
+__global__ void search_tc_qprep_kernel(const float* qr, int nq, int nq_pad, int d, float step_c, int8_t* pieces,
+                                       float* qscale) {
+  grid_dep_launch();
+  grid_dep_wait();   // qr comes from the rotation kernel before this one
+  const int lane = threadIdx.x & 31;
+  const int q = blockIdx.x * (blockDim.x / 32) + (threadIdx.x >> 5);
+  if (q >= nq_pad) return;
+  int8_t* ph = pieces + (size_t)q * d;
+  int8_t* pl = pieces + (size_t)(nq_pad + q) * d;
+  if (q >= nq) {
+    for (int j = lane; j < d; j += 32) ph[j] = pl[j] = 0;
+    return;
+  }
+  const float* row = qr + (size_t)q * d;
+  float mx = 0.f;
+  for (int j = lane; j < d; j += 32) mx = fmaxf(mx, fabsf(row[j]));
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, o));
+  const float inv = mx > 0.f ? (float)kCMax / mx : 0.f;
+  for (int j = lane; j < d; j += 32) {
+    const int x = max(-kCMax, min(kCMax, __float2int_rn(row[j] * inv)));
+    const int h = (x + 64) >> 7;   // floor: x - 128 h in [-64, 63]
+    ph[j] = (int8_t)h;
+    pl[j] = (int8_t)(x - 128 * h);
+  }
+  if (lane == 0) qscale[q] = mx > 0.f ? (mx / (float)kCMax) * step_c : 0.f;
+}
+
+}  // namespace stc
+}  // namespace tqk

@@ -43,6 +43,7 @@
 #include "attn_mse4.cuh"
 #include "search_mma.cuh"
 #include "search_mma4.cuh"
+#include "search_tc.cuh"
 #include "polar.cuh"
 
 struct tq_handle {
@@ -120,8 +121,8 @@ int launch_check(const char* what) {
 
 // True the first time (kernel slot, device) is seen: per-device one-time kernel attributes.
 bool once_per_device(int slot, int device) {
-  static std::atomic<uint64_t> seen[16];
-  if (slot < 0 || slot >= 16 || device < 0 || device >= 64) return true;
+  static std::atomic<uint64_t> seen[32];
+  if (slot < 0 || slot >= 32 || device < 0 || device >= 64) return true;
   const uint64_t bit = 1ull << device;
   return (seen[slot].fetch_or(bit) & bit) == 0;
 }
@@ -521,6 +522,47 @@ void search_mma_split(int nq, int qtile, int vb, int64_t n, int sms, int* nchunk
   *nchunks = (int)((n + ch - 1) / ch);
 }
 
+// Split of the tcgen05 search (one CTA per SM, 128 queries per CTA): chunks x query tiles is
+// the smallest whole number of waves, chunks a multiple of 256 vectors.
+void search_tc_split(int nq, int64_t n, int sms, int* nchunks, int64_t* chunk) {
+  const int64_t vb = tqk::stc::kV;
+  const int64_t qt = (nq + tqk::stc::kQ - 1) / tqk::stc::kQ;
+  int64_t a = sms, bq = qt;
+  while (bq) { const int64_t r = a % bq; a = bq; bq = r; }
+  int64_t nc = sms / a;
+  nc = std::max<int64_t>(1, std::min<int64_t>(nc, (n + vb - 1) / vb));
+  int64_t ch = (n + nc - 1) / nc;
+  ch = (ch + vb - 1) / vb * vb;
+  if (const int64_t f = splitk_override()) ch = round_chunk(f, vb, vb, (n + vb - 1) / vb * vb);
+  *chunk = ch;
+  *nchunks = (int)((n + ch - 1) / ch);
+}
+
+// The tcgen05 search covers MSE codes of 1 to 4 bits with d a multiple of 128 and k <= 32.
+// TQ_SIMT=1 forces the SIMT kernel; TQ_SEARCH_MMA=1 the legacy int8 kernels (2 and 4 bits).
+bool search_tc_ok(const tq_handle* h, int64_t n, int k) {
+  if (std::getenv("TQ_SIMT") || std::getenv("TQ_SEARCH_MMA")) return false;
+  return h->bits >= 1 && h->bits <= tqk::stc::kMaxBits && h->d % tqk::stc::kKC == 0 && k <= tqk::stc::kMaxK &&
+         n < ((int64_t)1 << 31);
+}
+
+// Centroids as 15-bit integers against one step, split into int8 pieces C = 128 C_h + C_l
+// (C_l in [-64, 63]); the pieces go to the kernel as little-endian byte tables.
+void centroid_pieces(const std::vector<double>& c, float* step_c, uint32_t th[4], uint32_t tl[4]) {
+  double cmax = 0.0;
+  for (double v : c) cmax = std::max(cmax, std::fabs(v));
+  const double step = cmax > 0.0 ? cmax / tqk::stc::kCMax : 1.0;
+  for (int w = 0; w < 4; ++w) th[w] = tl[w] = 0u;
+  for (size_t i = 0; i < c.size() && i < 16; ++i) {
+    long x = std::lround(c[i] / step);
+    x = std::max<long>(-tqk::stc::kCMax, std::min<long>(tqk::stc::kCMax, x));
+    const long hi = (long)std::floor((x + 64) / 128.0), lo = x - 128 * hi;
+    th[i / 4] |= (uint32_t)(uint8_t)(int8_t)hi << (8 * (i % 4));
+    tl[i / 4] |= (uint32_t)(uint8_t)(int8_t)lo << (8 * (i % 4));
+  }
+  *step_c = (float)step;
+}
+
 // The int8 tensor-core attention kernel covers 3-bit prod K and V caches (2-bit
 // codes + 128 QJL signs, fp16 norms) at d = 128 with 4 query heads per KV head.
 // TQ_SIMT=1 forces the SIMT kernels (used by tests to cross-check both paths).
@@ -608,11 +650,17 @@ size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, i
 }
 
 // mma: 0 for the SIMT kernel, else the queries per CTA of the tensor-core kernel.
+// mma == tqk::stc::kQ: the tcgen05 search, which also takes the int8 query pieces
+// [2][nq_pad][d] and their scales [nq_pad] (pieces / qscale, else unused).
 size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base, float** qr, float** cs,
-                        int64_t** ci, int* nchunks, int64_t* chunk, int mma) {
+                        int64_t** ci, int* nchunks, int64_t* chunk, int mma, int8_t** pieces = nullptr,
+                        float** qscale = nullptr) {
   int nc;
   int64_t ch;
-  if (mma)
+  const bool tc = mma == tqk::stc::kQ;
+  if (tc)
+    search_tc_split(nq, n, sm_count(h->device), &nc, &ch);
+  else if (mma)
     search_mma_split(nq, mma, mma == tqk::sm2::kQT ? tqk::sm2::kVB : tqk::sm4::kVB, n, sm_count(h->device), &nc, &ch);
   else
     search_split(nq, n, &nc, &ch);
@@ -621,6 +669,13 @@ size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base
   size_t off = 0;
   if (qr) *qr = reinterpret_cast<float*>(base + off);
   off += round_up((size_t)nq * h->d * 4, 256);
+  if (tc) {
+    const size_t nq_pad = (size_t)(nq + tqk::stc::kQ - 1) / tqk::stc::kQ * tqk::stc::kQ;
+    if (pieces) *pieces = reinterpret_cast<int8_t*>(base + off);
+    off += round_up(2 * nq_pad * h->d, 256);
+    if (qscale) *qscale = reinterpret_cast<float*>(base + off);
+    off += round_up(nq_pad * 4, 256);
+  }
   if (cs) *cs = reinterpret_cast<float*>(base + off);
   off += round_up((size_t)nc * nq * k * 4, 256);
   if (ci) *ci = reinterpret_cast<int64_t*>(base + off);
@@ -1052,7 +1107,7 @@ size_t tq_attn_workspace_bytes(const tq_handle* hk, const tq_handle* hv, int B, 
 size_t tq_search_workspace_bytes(const tq_handle* h, int nq, int64_t n, int k) {
   if (!h || nq < 0 || n < 1 || k < 1) return 0;
   size_t b = 0;
-  for (int mode : {0, tqk::sm2::kQT, tqk::sm4::kQT})
+  for (int mode : {0, tqk::sm2::kQT, tqk::sm4::kQT, tqk::stc::kQ})
     b = std::max(b, search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, mode));
   return b;
 }
@@ -1356,6 +1411,47 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
   int64_t* ci;
   int nchunks;
   int64_t chunk;
+  if (search_tc_ok(h, n, k)) {
+    int8_t* pieces;
+    float* qscale;
+    search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk, tqk::stc::kQ,
+                     &pieces, &qscale);
+    const int nq_pad = (nq + tqk::stc::kQ - 1) / tqk::stc::kQ * tqk::stc::kQ;
+    tqk::stc::Args m{};
+    m.nq = nq; m.nq_pad = nq_pad; m.d = h->d; m.k = k; m.norm_dtype = h->norm_dtype; m.codes_B = h->codes_B;
+    m.codes = codes; m.norms = norms; m.qscale = qscale; m.n = n; m.chunk = chunk;
+    m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
+    float step_c;
+    centroid_pieces(h->cent, &step_c, m.th, m.tl);
+    CUtensorMap qmap;
+    int st = codes_map_2d(reinterpret_cast<const uint8_t*>(pieces), 2 * (int64_t)nq_pad, h->d, tqk::stc::kKC,
+                          tqk::stc::kQ, &qmap);
+    if (st) return st;
+    if ((st = launch_qprep(h, q, TQ_F32, nq, qr, nullptr, s))) return st;
+    {
+      KernelScope ks("search_qprep", s);
+      const cudaError_t e = launch_pdl(tqk::stc::search_tc_qprep_kernel, dim3((unsigned)(nq_pad / 8)), dim3(256), 0,
+                                       s, (const float*)qr, nq, nq_pad, h->d, step_c, pieces, qscale);
+      if (e != cudaSuccess) return cuda_fail(e, "search_tc_qprep_kernel");
+    }
+    if ((st = launch_check("search_tc_qprep_kernel"))) return st;
+    auto kern = h->bits == 1 ? tqk::stc::search_tc_kernel<1>
+              : h->bits == 2 ? tqk::stc::search_tc_kernel<2>
+              : h->bits == 3 ? tqk::stc::search_tc_kernel<3>
+                             : tqk::stc::search_tc_kernel<4>;
+    if (once_per_device(16 + h->bits, h->device))
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tqk::stc::kSmemBytes);
+    {
+      KernelScope ks("search", s);
+      const cudaError_t e = launch_pdl(kern, dim3((unsigned)nchunks, (unsigned)(nq_pad / tqk::stc::kQ)),
+                                       dim3(tqk::stc::kThreads), (size_t)tqk::stc::kSmemBytes, s, qmap, m);
+      if (e != cudaSuccess) return cuda_fail(e, "search_tc_kernel");
+    }
+    if ((st = launch_check("search_tc_kernel"))) return st;
+    KernelScope ks("topk_merge", s);
+    tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
+    return launch_check("topk_merge_kernel");
+  }
   // int8 tensor-core bit-plane scores: 2-bit codes with d % 128 == 0, or 4-bit codes (symmetric
   // codebook, Walsh planes) with d % 64 == 0; d <= 1536, k <= 32
   const bool tc_ok = !std::getenv("TQ_SIMT") && h->d <= 1536 && k <= tqk::sm2::kMaxK && n < (int64_t(1) << 31);
