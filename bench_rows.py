@@ -469,7 +469,7 @@ FP32_LANES_PER_SM = 128   # fp32 FMA lanes per B200 SM (4 partitions x 32)
 
 
 def run_search(args, bits=None):
-    """cfg-4 search at 2 or 4 bits on the tcgen05 kernel (TQ_SEARCH_MMA=1: the legacy int8 kernels)."""
+    """cfg-4 search at 2 or 4 bits on the tcgen05 kernel (TQ_SIMT=1: the SIMT kernel)."""
     import torch
     import embedding_vector_quantization_b200 as tq
     bits = S4["bits"] if bits is None else bits
@@ -530,7 +530,7 @@ def run_search(args, bits=None):
                        "N(0,I) database vectors, 1024 queries (stands in for the pages' vector-search benchmarks)",
            "n": n, "nq": nq, "d": d, "k": k,
            "l2": f"not flushed: the {n * d * bits // 8 // 1000000} MB of codes exceed the 126 MB L2"}
-    if not os.environ.get("TQ_SEARCH_MMA") and d % 128 == 0:
+    if not os.environ.get("TQ_SIMT") and d % 64 == 0 and d >= 128:
         # tcgen05 int8 contractions into tensor memory: the measured bf16 dense peak x 2 (the
         # nominal int8 : bf16 ratio, 4.5 : 2.25 PFLOP/s)
         bf16, src = _peak("tensor")
@@ -543,19 +543,6 @@ def run_search(args, bits=None):
                 "launch_ms": s_ms / max(s_n, 1), "algorithmic_flops_per_launch": flops,
                 "note": "algorithmic 2d flops per (query, vector); the kernel executes 3x that in int8 MMA "
                         "operations (C_h Q_h, C_h Q_l, C_l Q_h), so its tensor-bound ceiling is 1/3 of the peak"}
-    elif bits in (2, 4):
-        # int8 tensor-core contraction: the measured bf16 dense peak x 2 (the nominal int8 : bf16
-        # ratio, 4.5 : 2.25 PFLOP/s)
-        bf16, src = _peak("tensor")
-        peak = 2.0 * bf16
-        planes = 2 if bits == 2 else 8
-        cfg["dtype"] = "int8 mma (bit planes x 15-bit query pieces), s32 accumulate"
-        roof = {"bound": "tensor", "kernel": f"search_mma{bits}_kernel", "achieved": ach, "peak": peak,
-                "unit": "TFLOP/s", "frac": ach / peak, "traffic": None,
-                "peak_source": f"{src} x 2 (int8 : bf16 nominal ratio)",
-                "launch_ms": s_ms / max(s_n, 1), "algorithmic_flops_per_launch": flops,
-                "note": f"algorithmic 2d flops per (query, vector); the int8 bit-plane form executes {2 * planes}x "
-                        f"that in MMA operations ({planes} planes x hi/lo query pieces)"}
     else:
         # fp32 FMAs on the CUDA cores: SMs x 128 lanes x 2 flop x the median sampled SM clock
         sm_mhz = clocks.get("sm_mhz") or 1965.0

@@ -10,9 +10,14 @@
 // C = 128 C_h + C_l, Q = 128 Q_h + Q_l (C_l, Q_l in [-64, 63], C_h, Q_h in [-127, 127]). Then
 //   <Q, C[idx]> = 16384 <Q_h, C_h[idx]> + 128 (<Q_l, C_h[idx]> + <Q_h, C_l[idx]>) + <Q_l, C_l[idx]>;
 // the kernel forms the first two terms exactly in int32 (two accumulators, three int8
-// contractions of depth d) and drops the last, which is below 2^-16 of |Q_j C_j| per coordinate.
+// contractions of depth d) and drops the last, at most 64 * 64 per coordinate: 1.6e-5 of
+// max|c| max|q'|, below the 15-bit rounding of c and q' themselves.
 // Any codebook works (no symmetry or affine structure is assumed): a coordinate's two operand
 // bytes C_h[idx], C_l[idx] come from 16-entry tables by byte permutes.
+//
+// d is a multiple of 64 (at least 128): a last K-chunk of 64 coordinates reads the query pieces
+// past d as zeros (the TMA box's out-of-bounds fill), so whatever the expansion writes there adds
+// nothing.
 //
 // Tiles. Queries are the MMA rows (M = 128 per CTA, one per tensor-memory lane), database vectors
 // the columns (N = 256 per tile). A CTA holds one query tile and walks a contiguous chunk of the
@@ -21,12 +26,12 @@
 //   warp 0, lane 0   TMA: Q_h and Q_l of the K-chunk (two 16 KB boxes, 128-byte swizzle), 3 stages
 //   warp 1           tensor-memory allocation (512 columns: acc_hi, acc_mid); lane 0 issues
 //                    4 K-steps x 3 MMAs per K-chunk, then commits the stages and the accumulator
-//   warps 2-5        expansion: thread p owns vector rows p and p + 128 of the tile, keeps their
-//                    packed codes of the next K-chunk in flight in registers, and writes C_h and C_l
-//                    of all 128 coordinates into the swizzled B tiles of a 2-stage ring
-//   warps 6-9        epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31, so thread t owns
+//   warps 2-9        expansion: thread p owns vector row p of the tile, keeps its packed codes of
+//                    the next K-chunk in flight in registers, and writes C_h and C_l of all 128
+//                    coordinates into the swizzled B tiles of a 2-stage ring
+//   warps 10-13      epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31, so thread t owns
 //                    query 32 (w % 4) + lane: it turns the row's 2 x 256 accumulators into scores and
-//                    keeps the query's running top-k (k <= 32) as a sorted list in registers.
+//                    keeps the query's running top-k (k <= 16 or <= 32) as a sorted list in registers.
 // Per query and chunk the list goes to the candidate arrays, which topk_merge_kernel reduces.
 // Every wait is bounded; a wait that runs out sets an abort flag (checked by every loop) and the
 // error word's kErrTimeout bit; the kernel then waits (bounded) for its own copies and MMAs and
@@ -59,8 +64,8 @@ constexpr int kVS = 2;           // vector-operand stages
 constexpr int kMaxK = 32;        // list entries per query
 constexpr int kMaxBits = 4;
 constexpr int kCMax = 16319;     // |C|, |Q| bound: 128 * 127 + 63
-constexpr int kThreads = 320;    // 10 warps
-constexpr int kExpandWarp0 = 2, kEpiWarp0 = 6;
+constexpr int kThreads = 448;    // 14 warps
+constexpr int kExpandWarp0 = 2, kEpiWarp0 = 10;   // eight expansion warps, four epilogue warps
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kQStage = 2u * kQ * kKC;              // 32 KB: Q_h box, then Q_l box
@@ -155,17 +160,31 @@ __device__ __forceinline__ void expand_unit(const uint32_t (&w)[4 * BITS], int u
   }
 }
 
-// Packed codes of one row's K-chunk: 16 BITS bytes = 4 BITS words (zeros past the chunk's end).
+// Packed codes of one row's K-chunk: 16 BITS bytes = 4 BITS words, of which the first `nbytes`
+// (a multiple of 8) are read and the rest are zero. Rows are 16-byte aligned when d % 128 == 0
+// (a16), else 8-byte aligned (d % 64 == 0).
 template <int BITS>
-__device__ __forceinline__ void load_chunk(const uint8_t* row, bool ok, uint32_t (&w)[4 * BITS]) {
+__device__ __forceinline__ void load_chunk(const uint8_t* row, bool ok, int nbytes, bool a16, uint32_t (&w)[4 * BITS]) {
 #pragma unroll
-  for (int i = 0; i < BITS; ++i) {
-    uint4 v = make_uint4(0u, 0u, 0u, 0u);
-    if (ok) v = __ldg(reinterpret_cast<const uint4*>(row) + i);
-    w[4 * i] = v.x;
-    w[4 * i + 1] = v.y;
-    w[4 * i + 2] = v.z;
-    w[4 * i + 3] = v.w;
+  for (int i = 0; i < 4 * BITS; ++i) w[i] = 0u;
+  if (!ok) return;
+  if (a16 && nbytes == 16 * BITS) {
+#pragma unroll
+    for (int i = 0; i < BITS; ++i) {
+      const uint4 x = __ldg(reinterpret_cast<const uint4*>(row) + i);
+      w[4 * i] = x.x;
+      w[4 * i + 1] = x.y;
+      w[4 * i + 2] = x.z;
+      w[4 * i + 3] = x.w;
+    }
+  } else {
+#pragma unroll
+    for (int i = 0; i < 2 * BITS; ++i)
+      if (8 * i < nbytes) {
+        const uint2 x = __ldg(reinterpret_cast<const uint2*>(row) + i);
+        w[2 * i] = x.x;
+        w[2 * i + 1] = x.y;
+      }
   }
 }
 
@@ -192,6 +211,22 @@ __host__ __device__ constexpr uint32_t idesc_i8() {
   return (2u << 4) | (1u << 7) | (1u << 10) | ((uint32_t)(kV >> 3) << 17) | ((uint32_t)(kQ >> 4) << 24);
 }
 
+__device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
+               : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
+               : "r"(taddr));
+}
+
+// Waits for this thread's tensor-memory loads; the loaded registers are operands, so that no use
+// of them is scheduled before the wait.
+__device__ __forceinline__ void tmem_wait_ld8x2(uint32_t (&x)[8], uint32_t (&y)[8]) {
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n"
+               : "+r"(x[0]), "+r"(x[1]), "+r"(x[2]), "+r"(x[3]), "+r"(x[4]), "+r"(x[5]), "+r"(x[6]), "+r"(x[7]),
+                 "+r"(y[0]), "+r"(y[1]), "+r"(y[2]), "+r"(y[3]), "+r"(y[4]), "+r"(y[5]), "+r"(y[6]), "+r"(y[7])
+               :
+               : "memory");
+}
+
 __device__ __forceinline__ void tmem_ld16(uint32_t taddr, uint32_t (&v)[16]) {
   asm volatile(
       "tcgen05.ld.sync.aligned.32x32b.x16.b32 {%0,%1,%2,%3,%4,%5,%6,%7,%8,%9,%10,%11,%12,%13,%14,%15}, [%16];\n"
@@ -212,7 +247,7 @@ __device__ __forceinline__ void tmem_wait_ld2(uint32_t (&x)[16], uint32_t (&y)[1
 
 // qmap: the query pieces as a 2-D int8 tensor {d, 2 nq_pad} (Q_h rows, then Q_l rows), box
 // {128, 128}, 128-byte swizzle. Grid: (chunks, query tiles of 128).
-template <int BITS>
+template <int BITS, int KMAX>
 __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_constant__ CUtensorMap qmap, Args a) {
   extern __shared__ __align__(1024) unsigned char smem[];
   const uint32_t base = smem_addr(smem);
@@ -220,7 +255,7 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
   const int q0 = blockIdx.y * kQ;
   const int64_t c0 = (int64_t)blockIdx.x * a.chunk, c1 = min(a.n, c0 + a.chunk);
   const int ntiles = (int)((max(c1 - c0, (int64_t)0) + kV - 1) / kV);
-  const int nkc = a.d / kKC;
+  const int nkc = (a.d + kKC - 1) / kKC;   // the last K-chunk may hold 64 coordinates
   const int total = ntiles * nkc;   // K-chunks of this CTA
 
   const uint32_t bars = base + kOffBars;
@@ -243,7 +278,7 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
       bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + kQS + s, 1);
     }
     for (int s = 0; s < kVS; ++s) {
-      bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + s, 4);   // the four expansion warps
+      bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + s, kEpiWarp0 - kExpandWarp0);   // expansion warps
       bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + kVS + s, 1);
     }
     bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + 2 * kVS, 1);       // acc_full: commit
@@ -318,9 +353,11 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
     }
   } else if (warp < kEpiWarp0) {
     // ---------------- expansion: codes -> C_h / C_l operand tiles
-    const int p = tid - 32 * kExpandWarp0;   // 0 .. 127: rows p and p + 128
+    const int p = tid - 32 * kExpandWarp0;   // 0 .. 255: row p
     constexpr int W = 4 * BITS;
     const int cbytes = kKC * BITS / 8;       // code bytes of a row's K-chunk
+    const int last_bytes = (a.d - (nkc - 1) * kKC) * BITS / 8;   // ... of its last K-chunk
+    const bool a16 = (a.codes_B & 15) == 0;
     const uint8_t* codes = a.codes;
     const int64_t codes_B = a.codes_B;
     uint32_t th[4], tl[4];
@@ -329,15 +366,13 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
       th[i] = a.th[i];
       tl[i] = a.tl[i];
     }
-    uint32_t cur[2][W], nxt[2][W];
-    auto fetch = [&](int itx, uint32_t(&w)[2][W]) {
+    uint32_t cur[W], nxt[W];
+    auto fetch = [&](int itx, uint32_t(&w)[W]) {
       const int t = itx / nkc, kc = itx % nkc;
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int64_t v = c0 + (int64_t)t * kV + p + 128 * r;
-        const bool ok = itx < total && v < c1;
-        load_chunk<BITS>(codes + (ok ? v : 0) * codes_B + (int64_t)kc * cbytes, ok, w[r]);
-      }
+      const int64_t v = c0 + (int64_t)t * kV + p;
+      const bool ok = itx < total && v < c1;
+      load_chunk<BITS>(codes + (ok ? v : 0) * codes_B + (int64_t)kc * cbytes, ok, kc == nkc - 1 ? last_bytes : cbytes,
+                       a16, w);
     };
     fetch(0, cur);
     for (int it = 0; it < total; ++it) {
@@ -347,46 +382,69 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
       if (ok && it >= kVS && !wait_bar(v_empty(s), ((it / kVS) - 1) & 1)) { fail_wait(); ok = false; }
       if (!__all_sync(0xffffffffu, ok)) break;
       const uint32_t vb = base + kOffV + s * kVStage;
+      const uint32_t rh = vb + p * 128, rl = rh + kVStage / 2;
 #pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int row = p + 128 * r;
-        const uint32_t rh = vb + row * 128, rl = rh + kVStage / 2;
-#pragma unroll
-        for (int u = 0; u < 8; ++u) {
-          uint32_t h[4], l[4];
-          expand_unit<BITS>(cur[r], u, th, tl, h, l);
-          const uint32_t o = (uint32_t)((u ^ (row & 7)) << 4);
-          sts128(rh + o, h[0], h[1], h[2], h[3]);
-          sts128(rl + o, l[0], l[1], l[2], l[3]);
-        }
+      for (int u = 0; u < 8; ++u) {
+        uint32_t h[4], l[4];
+        expand_unit<BITS>(cur, u, th, tl, h, l);
+        const uint32_t o = (uint32_t)((u ^ (p & 7)) << 4);
+        sts128(rh + o, h[0], h[1], h[2], h[3]);
+        sts128(rl + o, l[0], l[1], l[2], l[3]);
       }
       asm volatile("fence.proxy.async.shared::cta;\n" ::: "memory");   // generic writes -> tensor-core reads
       __syncwarp();
       if (lane == 0) bar_arrive(v_full(s));
 #pragma unroll
-      for (int r = 0; r < 2; ++r)
-#pragma unroll
-        for (int i = 0; i < W; ++i) cur[r][i] = nxt[r][i];
+      for (int i = 0; i < W; ++i) cur[i] = nxt[i];
     }
   } else {
     // ---------------- epilogue: scores and running top-k, one query per thread
     const int quarter = warp & 3, ql = 32 * quarter + lane, q = q0 + ql;
     const int e = tid - 32 * kEpiWarp0;   // 0 .. 127
     const bool qok = q < a.nq;
-    const float qscale = qok ? a.qscale[q] : 0.f;
+    const float qscale128 = qok ? 128.f * a.qscale[q] : 0.f;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
-    // the list, descending: entries kMaxK - k .. kMaxK - 1 are the running top-k (empty: -inf),
+    // the list, descending: entries KMAX - k .. KMAX - 1 are the running top-k (empty: -inf),
     // the ones before them +inf sentinels that no score displaces, so the k-th best is always
     // the last entry and an insertion bubbles through fixed register positions
-    const int k = a.k;
-    float ls[kMaxK];
-    int li[kMaxK];
+    const int k = a.k;   // <= KMAX
+    float ls[KMAX];
+    int li[KMAX];
 #pragma unroll
-    for (int j = 0; j < kMaxK; ++j) {
-      ls[j] = j < kMaxK - k ? INFINITY : -INFINITY;
+    for (int j = 0; j < KMAX; ++j) {
+      ls[j] = j < KMAX - k ? INFINITY : -INFINITY;
       li[j] = -1;
     }
     float thr = -INFINITY;
+    // every position from the old list at once: x keeps its entry if that is >= s, takes s if
+    // entry x - 1 is >= s, else takes entry x - 1 (the last entry falls off)
+    auto insert = [&](float sj, int ci) {
+      bool prev_ge = true;
+      float lp = 0.f;
+      int ip = -1;
+#pragma unroll
+      for (int x = 0; x < KMAX; ++x) {
+        const bool ge = ls[x] >= sj;
+        const float lx = ls[x];
+        const int ix = li[x];
+        ls[x] = ge ? lx : (prev_ge ? sj : lp);
+        li[x] = ge ? ix : (prev_ge ? ci : ip);
+        lp = lx;
+        ip = ix;
+        prev_ge = ge;
+      }
+      thr = ls[KMAX - 1];
+    };
+    // candidates above the threshold wait in a small buffer (in index order) and are inserted
+    // once 8 have gathered, and at the end of each tile (one copy of the insertion code)
+    constexpr int kBuf = 16;
+    float bs[kBuf];
+    int bi[kBuf];
+    int nbuf = 0;
+    auto flush = [&]() {
+      for (int x = 0; x < nbuf; ++x) insert(bs[x], bi[x]);
+      nbuf = 0;
+    };
     for (int t = 0; t < ntiles; ++t) {
       const int64_t v0 = c0 + (int64_t)t * kV;
       const int nv = (int)min((int64_t)kV, c1 - v0);
@@ -402,44 +460,50 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
       // warp-collective and every epilogue warp must reach the same barriers
       if (bar_red_or(1, 128, !ok)) break;
       tc_fence_after();
+      // 8 columns per step; the next step's accumulators load while this step is scored
+      // (tcgen05.wait::ld waits for every load of the thread, so the loaded registers are copied
+      // out before the next loads are issued into them)
+      const int nsteps = (nv + 7) / 8;   // the same for the whole warp
+      uint32_t hA[8], mA[8];
+      if (nsteps > 0) {
+        tmem_ld8(lane_addr, hA);
+        tmem_ld8(lane_addr + kV, mA);
+      }
 #pragma unroll 1
-      for (int cb = 0; cb < kV / 16; ++cb) {
-        uint32_t hi[16], mid[16];
-        tmem_ld16(lane_addr + 16 * cb, hi);
-        tmem_ld16(lane_addr + kV + 16 * cb, mid);
-        tmem_wait_ld2(hi, mid);
-        if (16 * cb >= nv) continue;   // the same for the whole warp
+      for (int st = 0; st < nsteps; ++st) {
+        tmem_wait_ld8x2(hA, mA);
+        uint32_t h[8], mm[8];
 #pragma unroll
-        for (int j = 0; j < 16; ++j) {
-          const int col = 16 * cb + j;
-          const float v = fmaf(16384.f, (float)(int)hi[j], 128.f * (float)(int)mid[j]);
-          const float s = v * (qscale * nb[col]);
-          if (qok && col < nv && s > thr) {   // visited in index order: an equal score ranks after
-            float cs = s;
-            int ci = (int)(v0 + col);
+        for (int j = 0; j < 8; ++j) h[j] = hA[j], mm[j] = mA[j];
+        if (st + 1 < nsteps) {
+          tmem_ld8(lane_addr + 8 * (st + 1), hA);
+          tmem_ld8(lane_addr + kV + 8 * (st + 1), mA);
+        }
+        const int c = 8 * st;
+        const float4 n0 = *reinterpret_cast<const float4*>(nb + c), n1 = *reinterpret_cast<const float4*>(nb + c + 4);
+        const float nr[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
 #pragma unroll
-            for (int x = 0; x < kMaxK; ++x) {
-              const bool sw = cs > ls[x];
-              const float ts = ls[x];
-              const int ti = li[x];
-              ls[x] = sw ? cs : ts;
-              li[x] = sw ? ci : ti;
-              cs = sw ? ts : cs;
-              ci = sw ? ti : ci;
-            }
-            thr = ls[kMaxK - 1];
+        for (int j = 0; j < 8; ++j) {
+          // 16384 acc_hi + 128 acc_mid = 128 (128 acc_hi + acc_mid)
+          const float sj = fmaf(128.f, (float)(int)h[j], (float)(int)mm[j]) * (qscale128 * nr[j]);
+          if (qok && c + j < nv && sj > thr) {   // visited in index order: an equal score ranks after
+            bs[nbuf] = sj;
+            bi[nbuf] = (int)(v0 + c + j);
+            ++nbuf;
           }
         }
+        if (nbuf >= 8) flush();
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(acc_empty);
+      if (__any_sync(0xffffffffu, nbuf > 0)) flush();
     }
     if (qok && !*abort_flag) {
-      const size_t o = ((size_t)blockIdx.x * a.nq + q) * k - (kMaxK - k);
+      const size_t o = ((size_t)blockIdx.x * a.nq + q) * k - (KMAX - k);
 #pragma unroll
-      for (int x = 0; x < kMaxK; ++x)
-        if (x >= kMaxK - k) {
+      for (int x = 0; x < KMAX; ++x)
+        if (x >= KMAX - k) {
           a.cand_s[o + x] = ls[x];
           a.cand_i[o + x] = li[x];
         }

@@ -27,7 +27,7 @@ constexpr int kSmallThreads = 256;
 // ---------------------------------------------------------------- append
 
 __host__ __device__ inline size_t append_cluster_smem_bytes(int d, int m) {
-  return (size_t)d * (d + m) * 4 + (size_t)3 * d * 4 + 64 + 4 * 16 + 64;
+  return (size_t)d * (d + m) * 4 + (size_t)3 * d * 4 + 64 + 4 * 16 + 64 + 32 * 4;
 }
 
 // Encodes input row b * Hkv + h into slot len[b] of KV head h (len itself is not changed);
@@ -43,6 +43,8 @@ __device__ __forceinline__ int32_t append_vector(const EncodeArgs& a, int b, int
   uint64_t* bar = reinterpret_cast<uint64_t*>(words + 16);  // [2]
   float* red = reinterpret_cast<float*>(bar + 2);           // [16]
   double* nrm = reinterpret_cast<double*>(red + 16);        // [2]
+  float* tbnd = reinterpret_cast<float*>(nrm + 2);          // [16] boundaries, then [16] centroids
+  float* tcent = tbnd + 16;
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
 
   const int32_t pos = a.len[b];
@@ -56,6 +58,9 @@ __device__ __forceinline__ int32_t append_vector(const EncodeArgs& a, int b, int
   }
   if (tid < 16) words[tid] = 0u;
   if (tid < d) xs[tid] = load_any(a.x, a.x_dtype, r * d + tid);
+  if (tid < L - 1) tbnd[tid] = a.bnd[tid];
+  if (tid < L) tcent[tid] = a.cent[tid];
+  grid_dep_launch();   // a dependent kernel may start once this CTA's loads are in flight
   __syncthreads();
   if (full) {
     if (tid == 0 && h == 0) report_error(a.err, kErrCapacity);
@@ -87,11 +92,11 @@ __device__ __forceinline__ int32_t append_vector(const EncodeArgs& a, int b, int
         for (int k = 0; k < d; ++k) acc = fmaf(mat[k * d + tid], xs[k], acc);
         const float y = acc * inv;
         uint32_t idx = 0;
-        for (int i = 0; i < L - 1; ++i) idx += (y > a.bnd[i]) ? 1u : 0u;
+        for (int i = 0; i < L - 1; ++i) idx += (y > tbnd[i]) ? 1u : 0u;
         const int bit = tid * bits;
         atomicOr(&words[bit >> 5], idx << (bit & 31));
         if ((bit & 31) + bits > 32) atomicOr(&words[(bit >> 5) + 1], idx >> (32 - (bit & 31)));
-        e = y - a.cent[idx];
+        e = y - tcent[idx];
       }
       __syncthreads();   // all reads of xs are done: it now holds e
       if (tid < d) xs[tid] = e;
@@ -171,6 +176,7 @@ __device__ __forceinline__ void qprep_tile(const void* q, int q_dtype, int rows,
 #pragma unroll 4
     for (int i = tid; i < nr * d; i += blockDim.x) qsh[i] = load_any(q, q_dtype, (int64_t)row0 * d + i);
   }
+  grid_dep_launch();   // a dependent kernel may start once this CTA's loads are in flight
   cp_async_wait_all();
   __syncthreads();
   const int c = tid % kWideCols;
@@ -214,14 +220,16 @@ struct PrologueArgs {
 
 __global__ void __launch_bounds__(kSmallThreads) decode_prologue_kernel(PrologueArgs p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  grid_dep_launch();
+  // each role signals the attention kernel (launched as this one's dependent) once its own
+  // loads are in flight, so that they queue ahead of the attention's streaming reads
   const int bid = blockIdx.x;
   if (bid == 0 && threadIdx.x < 2 && p.pf[threadIdx.x] && p.pf_bytes[threadIdx.x])
     asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p.pf[threadIdx.x]), "r"(p.pf_bytes[threadIdx.x])
                  : "memory");
   if (bid < 2 * p.nvec) {
     const int v = bid % p.nvec;
-    (void)append_vector(bid < p.nvec ? p.k : p.v, v / p.k.Hkv, v % p.k.Hkv, smem_raw);
+    const EncodeArgs& a = bid < p.nvec ? p.k : p.v;
+    (void)append_vector(a, v / a.Hkv, v % a.Hkv, smem_raw);
   } else {
     const int t = bid - 2 * p.nvec;
     qprep_tile(p.q, p.q_dtype, p.rows, p.d, p.PiT, p.ST, p.m, p.qr, p.qs, t / p.qcols, t % p.qcols, kQRows,

@@ -41,8 +41,6 @@
 #include "small_kernels.cuh"
 #include "encode_tc.cuh"
 #include "attn_mse4.cuh"
-#include "search_mma.cuh"
-#include "search_mma4.cuh"
 #include "search_tc.cuh"
 #include "polar.cuh"
 
@@ -505,23 +503,6 @@ int sm_count(int device) {
   return c;
 }
 
-// Split of the int8 tensor-core searches (one CTA per SM, qtile queries per CTA): the number
-// of database chunks makes chunks x query tiles a whole number of waves where it can, chunks
-// a multiple of 256 vectors.
-void search_mma_split(int nq, int qtile, int vb, int64_t n, int sms, int* nchunks, int64_t* chunk) {
-  const int64_t qt = (nq + qtile - 1) / qtile;
-  int64_t a = sms, bq = qt;   // nc0 = sms / gcd(sms, qt): the fewest chunks giving whole waves
-  while (bq) { const int64_t r = a % bq; a = bq; bq = r; }
-  const int64_t nc0 = sms / a;
-  int64_t nc = nc0 * std::max<int64_t>(1, (8 * (int64_t)sms + nc0 * qt / 2) / (nc0 * qt));
-  nc = std::max<int64_t>(1, std::min<int64_t>(nc, (n + vb - 1) / vb));
-  int64_t ch = (n + nc - 1) / nc;
-  ch = (ch + vb - 1) / vb * vb;
-  if (const int64_t f = splitk_override()) ch = round_chunk(f, vb, vb, (n + vb - 1) / vb * vb);
-  *chunk = ch;
-  *nchunks = (int)((n + ch - 1) / ch);
-}
-
 // Split of the tcgen05 search (one CTA per SM, 128 queries per CTA): chunks x query tiles is
 // the smallest whole number of waves, chunks a multiple of 256 vectors.
 void search_tc_split(int nq, int64_t n, int sms, int* nchunks, int64_t* chunk) {
@@ -538,12 +519,12 @@ void search_tc_split(int nq, int64_t n, int sms, int* nchunks, int64_t* chunk) {
   *nchunks = (int)((n + ch - 1) / ch);
 }
 
-// The tcgen05 search covers MSE codes of 1 to 4 bits with d a multiple of 128 and k <= 32.
-// TQ_SIMT=1 forces the SIMT kernel; TQ_SEARCH_MMA=1 the legacy int8 kernels (2 and 4 bits).
+// The tcgen05 search covers MSE codes of 1 to 4 bits with d a multiple of 64 (at least 128) and
+// k <= 32; TQ_SIMT=1 forces the SIMT kernel.
 bool search_tc_ok(const tq_handle* h, int64_t n, int k) {
-  if (std::getenv("TQ_SIMT") || std::getenv("TQ_SEARCH_MMA")) return false;
-  return h->bits >= 1 && h->bits <= tqk::stc::kMaxBits && h->d % tqk::stc::kKC == 0 && k <= tqk::stc::kMaxK &&
-         n < ((int64_t)1 << 31);
+  if (std::getenv("TQ_SIMT")) return false;
+  return h->bits >= 1 && h->bits <= tqk::stc::kMaxBits && h->d % 64 == 0 && h->d >= tqk::stc::kKC &&
+         k <= tqk::stc::kMaxK && n < ((int64_t)1 << 31);
 }
 
 // Centroids as 15-bit integers against one step, split into int8 pieces C = 128 C_h + C_l
@@ -650,18 +631,15 @@ size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, i
 }
 
 // mma: 0 for the SIMT kernel, else the queries per CTA of the tensor-core kernel.
-// mma == tqk::stc::kQ: the tcgen05 search, which also takes the int8 query pieces
-// [2][nq_pad][d] and their scales [nq_pad] (pieces / qscale, else unused).
+// tc: the tcgen05 search, which also takes the int8 query pieces [2][nq_pad][d] and their
+// scales [nq_pad] (pieces / qscale, else unused); otherwise the SIMT search.
 size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base, float** qr, float** cs,
-                        int64_t** ci, int* nchunks, int64_t* chunk, int mma, int8_t** pieces = nullptr,
+                        int64_t** ci, int* nchunks, int64_t* chunk, bool tc, int8_t** pieces = nullptr,
                         float** qscale = nullptr) {
   int nc;
   int64_t ch;
-  const bool tc = mma == tqk::stc::kQ;
   if (tc)
     search_tc_split(nq, n, sm_count(h->device), &nc, &ch);
-  else if (mma)
-    search_mma_split(nq, mma, mma == tqk::sm2::kQT ? tqk::sm2::kVB : tqk::sm4::kVB, n, sm_count(h->device), &nc, &ch);
   else
     search_split(nq, n, &nc, &ch);
   if (nchunks) *nchunks = nc;
@@ -1107,8 +1085,8 @@ size_t tq_attn_workspace_bytes(const tq_handle* hk, const tq_handle* hv, int B, 
 size_t tq_search_workspace_bytes(const tq_handle* h, int nq, int64_t n, int k) {
   if (!h || nq < 0 || n < 1 || k < 1) return 0;
   size_t b = 0;
-  for (int mode : {0, tqk::sm2::kQT, tqk::sm4::kQT, tqk::stc::kQ})
-    b = std::max(b, search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, mode));
+  for (bool tc : {false, true})
+    b = std::max(b, search_ws_layout(h, nq, n, k, nullptr, nullptr, nullptr, nullptr, nullptr, nullptr, tc));
   return b;
 }
 
@@ -1414,8 +1392,8 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
   if (search_tc_ok(h, n, k)) {
     int8_t* pieces;
     float* qscale;
-    search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk, tqk::stc::kQ,
-                     &pieces, &qscale);
+    search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk, true, &pieces,
+                     &qscale);
     const int nq_pad = (nq + tqk::stc::kQ - 1) / tqk::stc::kQ * tqk::stc::kQ;
     tqk::stc::Args m{};
     m.nq = nq; m.nq_pad = nq_pad; m.d = h->d; m.k = k; m.norm_dtype = h->norm_dtype; m.codes_B = h->codes_B;
@@ -1435,11 +1413,16 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
       if (e != cudaSuccess) return cuda_fail(e, "search_tc_qprep_kernel");
     }
     if ((st = launch_check("search_tc_qprep_kernel"))) return st;
-    auto kern = h->bits == 1 ? tqk::stc::search_tc_kernel<1>
-              : h->bits == 2 ? tqk::stc::search_tc_kernel<2>
-              : h->bits == 3 ? tqk::stc::search_tc_kernel<3>
-                             : tqk::stc::search_tc_kernel<4>;
-    if (once_per_device(16 + h->bits, h->device))
+    // the running lists hold 16 entries for k <= 16, else 32
+    using Kern = void (*)(const CUtensorMap, tqk::stc::Args);
+    static const Kern kerns[2][4] = {
+        {tqk::stc::search_tc_kernel<1, 16>, tqk::stc::search_tc_kernel<2, 16>, tqk::stc::search_tc_kernel<3, 16>,
+         tqk::stc::search_tc_kernel<4, 16>},
+        {tqk::stc::search_tc_kernel<1, 32>, tqk::stc::search_tc_kernel<2, 32>, tqk::stc::search_tc_kernel<3, 32>,
+         tqk::stc::search_tc_kernel<4, 32>}};
+    const int big = k > 16 ? 1 : 0;
+    auto kern = kerns[big][h->bits - 1];
+    if (once_per_device(16 + 4 * big + h->bits, h->device))
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tqk::stc::kSmemBytes);
     {
       KernelScope ks("search", s);
@@ -1452,63 +1435,9 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
     tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
     return launch_check("topk_merge_kernel");
   }
-  // int8 tensor-core bit-plane scores: 2-bit codes with d % 128 == 0, or 4-bit codes (symmetric
-  // codebook, Walsh planes) with d % 64 == 0; d <= 1536, k <= 32
-  const bool tc_ok = !std::getenv("TQ_SIMT") && h->d <= 1536 && k <= tqk::sm2::kMaxK && n < (int64_t(1) << 31);
-  const bool mma2 = tc_ok && h->bits == 2 && h->d % 128 == 0 &&
-                    std::fabs(h->cent[3] - h->cent[2] - h->cent[1] + h->cent[0]) < 1e-12;
-  float w4[8], c04 = 0.f;
-  const bool mma4 = tc_ok && h->bits == 4 && h->d % 64 == 0 && plane_coeffs4(h->cent, &c04, w4);
-  search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk,
-                   mma2 ? tqk::sm2::kQT : mma4 ? tqk::sm4::kQT : 0);
+  search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk, false);
   int st = launch_qprep(h, q, TQ_F32, nq, qr, nullptr, s);
   if (st) return st;
-  if (mma4) {
-    tqk::sm4::Args m{};
-    m.qr = qr; m.nq = nq; m.d = h->d; m.codes_B = h->codes_B; m.k = k; m.norm_dtype = h->norm_dtype;
-    m.norms = norms; m.n = n; m.chunk = chunk; m.c0 = c04;
-    for (int i = 0; i < 8; ++i) m.w[i] = w4[i];
-    m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
-    CUtensorMap cmap;
-    if ((st = codes_map_2d(codes, n, h->codes_B, tqk::sm4::kSlice, tqk::sm4::kVB, &cmap))) return st;
-    const size_t msmem = tqk::sm4::smem_bytes();
-    if (once_per_device(13, h->device))
-      cudaFuncSetAttribute(tqk::sm4::search_mma4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
-    {
-      KernelScope ks("search", s);
-      const cudaError_t e = launch_pdl(tqk::sm4::search_mma4_kernel,
-                                       dim3((unsigned)nchunks, (unsigned)((nq + tqk::sm4::kQT - 1) / tqk::sm4::kQT)),
-                                       dim3(tqk::sm4::kThreads), msmem, s, cmap, m);
-      if (e != cudaSuccess) return cuda_fail(e, "search_mma4_kernel");
-    }
-    if ((st = launch_check("search_mma4_kernel"))) return st;
-    KernelScope ks("topk_merge", s);
-    tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
-    return launch_check("topk_merge_kernel");
-  }
-  if (mma2) {
-    tqk::sm2::Args m{};
-    m.qr = qr; m.nq = nq; m.d = h->d; m.codes_B = h->codes_B; m.k = k; m.norm_dtype = h->norm_dtype;
-    m.codes = codes; m.norms = norms; m.n = n; m.chunk = chunk;
-    m.c0 = (float)h->cent[0]; m.w0 = (float)(h->cent[1] - h->cent[0]); m.w1 = (float)(h->cent[2] - h->cent[0]);
-    m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
-    CUtensorMap cmap;
-    if ((st = codes_map_2d(codes, n, h->codes_B, tqk::sm2::kSlice, tqk::sm2::kBoxRows, &cmap))) return st;
-    const size_t msmem = tqk::sm2::smem_bytes();
-    if (once_per_device(12, h->device))
-      cudaFuncSetAttribute(tqk::sm2::search_mma2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
-    {
-      KernelScope ks("search", s);
-      const cudaError_t e = launch_pdl(tqk::sm2::search_mma2_kernel,
-                                       dim3((unsigned)nchunks, (unsigned)((nq + tqk::sm2::kQT - 1) / tqk::sm2::kQT)),
-                                       dim3(tqk::sm2::kThreads), msmem, s, cmap, m);
-      if (e != cudaSuccess) return cuda_fail(e, "search_mma2_kernel");
-    }
-    if ((st = launch_check("search_mma2_kernel"))) return st;
-    KernelScope ks("topk_merge", s);
-    tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
-    return launch_check("topk_merge_kernel");
-  }
   tqk::SearchArgs a{};
   a.qr = qr; a.nq = nq; a.d = h->d; a.bits = h->bits; a.norm_dtype = h->norm_dtype; a.codes_B = h->codes_B;
   a.k = k; a.codes = codes; a.norms = norms; a.n = n; a.chunk = chunk; a.cent = h->dcent; a.cand_s = cs; a.cand_i = ci;

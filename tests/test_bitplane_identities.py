@@ -150,9 +150,8 @@ def test_int32_accumulation_cannot_overflow_at_the_largest_shapes():
     assert 1024 * 255 * 16 < 2 ** 31 and 1024 * 65535 < 2 ** 31
     # the 4-bit kernel's hi sum over 8 planes x 128 coordinates is formed in float (exact below 2^24)
     assert 8 * 128 * 127 < 2 ** 24
-    # 4-bit search at d = 1536: 8 planes x d coordinates of 0/1 (or 16) bytes against |piece| <= 127
-    worst = 16 * 127 * 8 * 1536
-    assert worst < 2 ** 31
+    # tcgen05 search at its largest d (65536): acc_hi = sum C_h Q_h and acc_mid = sum (C_h Q_l + C_l Q_h)
+    assert 65536 * 127 * 127 < 2 ** 31 and 65536 * (127 * 64 + 64 * 127) < 2 ** 31
     # the x16 family's sums are multiples of 16, so the exact division by 16 loses nothing
     for parts in itertools.product([0, 16, 32, 48], repeat=3):
         assert sum(parts) % 16 == 0
@@ -163,3 +162,17 @@ def test_fast_layout_decoder_of_the_tests_matches_the_oracle_unpack(bits, d):
     from gpu_util import unpack_fast
     rows = np.random.default_rng(bits * 1000 + d).integers(0, 256, size=(300, (d * bits + 7) // 8), dtype=np.uint8)
     assert np.array_equal(unpack_fast(rows, d, bits).astype(np.int64), quant.unpack(rows, d, bits))
+
+
+def test_search_piece_split_covers_the_15_bit_range():
+    """The tcgen05 search rounds centroids and queries to |x| <= 16319 and splits x = 128 h + l
+    with h = floor((x + 64) / 128): h and l must fit its int8 operands (|h| <= 127, l in
+    [-64, 63]); the dropped l_c l_q term is at most 64 * 64 per coordinate, 1.6e-5 of the
+    largest product 16319^2 (max |c| max |q'|)."""
+    x = np.arange(-16319, 16320)
+    h = np.floor((x + 64) / 128).astype(np.int64)
+    assert np.array_equal((x + 64) >> 7, h)   # the kernel's arithmetic shift
+    l = x - 128 * h
+    assert h.min() == -127 and h.max() == 127 and l.min() == -64 and l.max() == 63
+    assert np.array_equal(128 * h + l, x)
+    assert 64 * 64 / 16319 ** 2 < 1.6e-5

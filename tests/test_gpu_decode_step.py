@@ -1,5 +1,7 @@
 """tq_decode_step (append K and V at slot len[b], attend over len[b] + 1 tokens, advance
-len) against the same work done by separate calls, and against the oracle
+len) against the same work done by separate calls, and against the oracle. With Hkv in
+{2, 4, 8} the step's appends are column-sliced over a cluster of Hkv CTAs; their rows must
+be bit-identical to the per-vector append of tq_append
 ("Google TurboQuant: 6x KV-cache compression", "Stage 1" / "Stage 2"; "TurboQuant /
 PolarQuant / QJL technical deep dive", "Scaled dot-product attention")."""
 
@@ -55,6 +57,9 @@ def _step(tq, hk, hv, q, k_new, v_new, kc, vc, lens, scale):
     (3, 0, 2, 2, 4, 1024, [700, 1023], False),      # MSE-only K/V: the SIMT attention kernel
     (4, 0, 1, 2, 2, 512, [3], False),
     (4, 0, 2, 2, 4, 3072, [3000, 1024], True),       # 4-bit MSE, fp16 norms: the Walsh-plane kernel
+    (1, 128, 2, 4, 2, 512, [100, 511], False),       # QJL-only K/V (no MSE bits)
+    (3, 128, 1, 1, 4, 640, [639], False),            # Hkv = 1: the per-vector append (no column slices)
+    (2, 64, 1, 16, 2, 256, [200], False),            # Hkv = 16: above the cluster size, per-vector append
 ])
 def test_decode_step_equals_separate_calls(tq, bits, m, B, Hkv, G, L_cap, L0, f16):
     hk, hv, caches, q, k_new, v_new = _setup(tq, bits, m, B, Hkv, G, L_cap, L0, seed=bits * 10 + B,
@@ -76,9 +81,9 @@ def test_decode_step_equals_separate_calls(tq, bits, m, B, Hkv, G, L_cap, L0, f1
     assert s1 == s2 and (s1[0] == tq.TQ_ECAPACITY) == full
     assert lens1.cpu().tolist() == lens2.cpu().tolist() == [min(x + 1, L_cap) for x in L0]
     for a, b in [(kc1, kc2), (vc1, vc2)]:
-        assert torch.equal(a.codes, b.codes) and torch.equal(a.norms, b.norms)
-        if m:
-            assert torch.equal(a.signs, b.signs) and torch.equal(a.rnorms, b.rnorms)
+        for name in ("codes", "norms", "signs", "rnorms"):   # QJL-only rows have no codes or rnorms
+            x, y = getattr(a, name), getattr(b, name)
+            assert (x is None) == (y is None) and (x is None or torch.equal(x, y)), name
     assert torch.equal(o1, o2)
 
 

@@ -313,10 +313,9 @@ def test_attention_mse4_tensor_core_path_matches_simt_and_oracle(tq, B, Hkv, L, 
 @pytest.mark.parametrize("d,n,nq,k", [(512, 50000, 40, 32), (1536, 9000, 17, 1), (128, 700, 3, 10),
                                      (640, 3000, 16, 10), (1024, 300, 64, 5), (256, 100, 5, 7)])
 def test_search_tensor_core_path_matches_simt_and_oracle(tq, d, n, nq, k):
-    """2-bit codes: the int8 tensor-core search (several 256-vector blocks and chunks, code
-    rows of one, two and three 128-byte slices and a partial last slice (d = 640), a
-    database shorter than one block, partial query tiles, k = 1 and 32) and the SIMT kernel
-    (TQ_SIMT=1) against the oracle.
+    """2-bit codes: the tcgen05 search (several 256-vector tiles and chunks, one to twelve
+    K-chunks of 128 coordinates, a database shorter than one tile, partial query tiles, k = 1
+    and 32) and the SIMT kernel (TQ_SIMT=1) against the oracle.
     Exact duplicate database rows score identically on either path, so the lower index
     must be returned first."""
     import os
@@ -358,11 +357,10 @@ def test_search_tensor_core_path_matches_simt_and_oracle(tq, d, n, nq, k):
 
 @pytest.mark.parametrize("d,n,nq,k", [(1536, 6000, 9, 10), (320, 3000, 13, 32), (128, 200, 4, 1), (512, 20000, 70, 10)])
 def test_search_4bit_tensor_core_path_matches_simt_and_oracle(tq, d, n, nq, k):
-    """4-bit codes: the int8 tensor-core search over the eight Walsh planes of the symmetric
-    codebook (code rows of one to six 128-byte slices, a partial last slice at d = 320, a
-    database shorter than one 256-vector block, partial query tiles of 4, k = 1 and 32) and
-    the SIMT kernel (TQ_SIMT=1) against the oracle; planted duplicates of a best vector must
-    come back lower index first."""
+    """4-bit codes: the tcgen05 search (one to twelve K-chunks, a half last K-chunk at d = 320,
+    a database shorter than one 256-vector tile, partial query tiles, k = 1 and 32) and the
+    SIMT kernel (TQ_SIMT=1) against the oracle; planted duplicates of a best vector must come
+    back lower index first."""
     import os
     h = tq.Handle(d, 4, 11)
     oh = OracleHandle(d, 4, 11)

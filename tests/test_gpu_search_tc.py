@@ -3,11 +3,11 @@ queries x 256 vectors per tile, any 1- to 4-bit codebook through byte-permute ta
 against the oracle ("TurboQuant: redefining AI efficiency", "Impact on high-dimensional
 vector search": s = ||x|| <Pi q, c[idx]>, ranked by score, equal scores lower index first).
 
-Shapes cover every code width, several K-chunks per tile (d = 128 .. 1536), ragged database
-tiles and chunks, a ragged second query tile (nq = 130 and 300), forced chunk lengths
-(TQ_SPLITK), k = 1 and 32, fp16 norms and planted exact duplicates. The legacy int8 kernels
-(TQ_SEARCH_MMA=1) and the SIMT kernel (TQ_SIMT=1) are checked on the same data where they
-apply. Rule: every returned index scores (oracle) within the tolerance of the k-th best, the
+Shapes cover every code width, several K-chunks per tile (d = 128 .. 1536), a last K-chunk of
+64 coordinates (d = 192, 320, 704: code rows only 8-byte aligned), ragged database tiles and
+chunks, a ragged second query tile (nq = 130 and 300), forced chunk lengths (TQ_SPLITK), k = 1
+and 32, fp16 norms and planted exact duplicates. The SIMT kernel (TQ_SIMT=1) is checked on the
+same data. Rule: every returned index scores (oracle) within the tolerance of the k-th best, the
 returned scores match the oracle's within the score tolerance, scores are non-increasing and
 equal scores come lower index first."""
 
@@ -101,6 +101,9 @@ def _run(tq, bits, d, n, nq, k, seed, norm_dtype="f32", sample=None, force=None)
     (1, 256, 2000, 40, 1),       # 1-bit, k = 1
     (4, 128, 100, 5, 7),         # one K-chunk, a database shorter than one tile
     (2, 512, 20000, 257, 16),    # many tiles per chunk, 257 queries
+    (1, 192, 3000, 33, 10),      # d % 128 = 64: a half last K-chunk, 24-byte rows
+    (3, 320, 2500, 70, 10),      # 120-byte rows
+    (4, 704, 1000, 129, 32),     # 352-byte rows, 129 queries
 ])
 def test_search_tc_matches_oracle(tq, bits, d, n, nq, k):
     _run(tq, bits, d, n, nq, k, seed=bits * 100 + d + nq)
@@ -113,16 +116,15 @@ def test_search_tc_forced_chunks_and_f16_norms(tq, bits, force):
     _run(tq, bits, 256, 7001, 19, 32, seed=70 + bits, norm_dtype="f16", force=force)
 
 
-def test_search_tc_agrees_with_legacy_and_simt(tq):
-    """2- and 4-bit codes at d = 1536: the tcgen05 kernel, the legacy int8 kernels
-    (TQ_SEARCH_MMA=1) and the SIMT kernel (TQ_SIMT=1) return valid top-k lists for the oracle."""
+def test_search_tc_agrees_with_simt(tq):
+    """2- and 4-bit codes at d = 1536: the tcgen05 kernel and the SIMT kernel (TQ_SIMT=1) both
+    return valid top-k lists for the oracle."""
     for bits in (2, 4):
         h, codes, norms, qg, _, (S, Q, e, rows) = _run(tq, bits, 1536, 4000, 20, 10, seed=500 + bits)
-        for var in ("TQ_SEARCH_MMA", "TQ_SIMT"):
-            with env(**{var: 1}):
-                idx, sc = (x.cpu().numpy() for x in h.search_topk(qg, codes, norms, 10))
-            assert h.status() == tq.TQ_OK
-            _check(idx, sc, S, Q, e, 10, 1536, 4000, rows)
+        with env(TQ_SIMT=1):
+            idx, sc = (x.cpu().numpy() for x in h.search_topk(qg, codes, norms, 10))
+        assert h.status() == tq.TQ_OK
+        _check(idx, sc, S, Q, e, 10, 1536, 4000, rows)
 
 
 def test_search_tc_full_query_tiles_sampled(tq):

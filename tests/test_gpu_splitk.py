@@ -9,7 +9,7 @@ two blocks, so the ring never wraps. Here every kernel runs chunks of several bl
   blocks with one barrier each), plus a ragged length and forced 512-token chunks;
 * attn_mse4_kernel with 896-token chunks (4 + 4 blocks on its 4-stage ring);
 * score_prod2_kernel with 5- and 10-block chunks on its 4-stage ring (TQ_SPLITK);
-* search_mma2_kernel / search_mma4_kernel with 3 to 6 blocks per chunk.
+* search_tc_kernel with 3 to 12 tiles of 256 vectors per chunk.
 
 Caches hold the oracle's codes ("Google TurboQuant: 6x KV-cache compression", "Stage 1"
 and "Stage 2"; "TurboQuant / PolarQuant / QJL technical deep dive", "Scaled dot-product
@@ -232,15 +232,15 @@ def _search_case(tq, bits, d, n, nq, k, seed, sample=None):
 
 @pytest.mark.parametrize("bits", [2, 4])
 def test_search_multiblock_chunks_natural_split(tq, bits):
-    """1024 queries over 50,000 vectors at d = 256: the search's own split gives 37 chunks of
-    1536 vectors, i.e. 4 blocks of 384 (2-bit) or 6 blocks of 256 (4-bit) per chunk, and a
-    shorter last chunk; 64 sampled queries are checked against the oracle."""
+    """1024 queries over 50,000 vectors at d = 256: the search's own split gives 8 query tiles
+    x 33 chunks of 1536 vectors (6 tiles of 256) and a shorter last chunk; 64 sampled queries
+    are checked against the oracle."""
     _search_case(tq, bits, 256, 50000, 1024, 10, seed=60 + bits, sample=np.arange(0, 1024, 16))
 
 
 @pytest.mark.parametrize("bits,force", [(2, 1152), (4, 768), (2, 3000)])
 def test_search_multiblock_chunks_forced(tq, bits, force):
-    """A partial query tile (19 queries) with forced chunks of 3 or more blocks (TQ_SPLITK),
-    a ragged last chunk, k = 32."""
+    """A partial query tile (19 queries) with forced chunks of 3 to 12 tiles (TQ_SPLITK), a
+    ragged last chunk, k = 32."""
     with splitk(force):
         _search_case(tq, bits, 512, 7001, 19, 32, seed=70 + bits)
