@@ -29,10 +29,12 @@
 //   warps 2-9        expansion: thread p owns vector row p of the tile, keeps its packed codes of
 //                    the next K-chunk in flight in registers, and writes C_h and C_l of all 128
 //                    coordinates into the swizzled B tiles of a 2-stage ring
-//   warps 10-13      epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31, so thread t owns
-//                    query 32 (w % 4) + lane: it turns the row's 2 x 256 accumulators into scores and
-//                    keeps the query's running top-k (k <= 16 or <= 32) as a sorted list in registers.
-// Per query and chunk the list goes to the candidate arrays, which topk_merge_kernel reduces.
+//   warps 10-17      epilogue: warp w reads tensor-memory lanes 32 (w % 4) .. + 31 and columns of
+//                    half (w - 10) / 4 of the tile, so thread t owns query 32 (w % 4) + lane on those
+//                    128 vectors: it turns the accumulators into scores and keeps the query's running
+//                    top-k (k <= 16 or <= 32) over its half as a sorted list in registers.
+// Per query, chunk and half the list goes to the candidate arrays ([chunk][half] counts as one
+// chunk), which topk_merge_kernel reduces.
 // Every wait is bounded; a wait that runs out sets an abort flag (checked by every loop) and the
 // error word's kErrTimeout bit; the kernel then waits (bounded) for its own copies and MMAs and
 // frees its tensor memory.
@@ -64,8 +66,10 @@ constexpr int kVS = 2;           // vector-operand stages
 constexpr int kMaxK = 32;        // list entries per query
 constexpr int kMaxBits = 4;
 constexpr int kCMax = 16319;     // |C|, |Q| bound: 128 * 127 + 63
-constexpr int kThreads = 448;    // 14 warps
-constexpr int kExpandWarp0 = 2, kEpiWarp0 = 10;   // eight expansion warps, four epilogue warps
+constexpr int kExpandWarp0 = 2, kEpiWarp0 = 10;   // eight expansion warps, then the epilogue warps
+constexpr int kEpiWarps = 8;     // two per tensor-memory lane quarter: one per half of the tile's columns
+constexpr int kHalves = kEpiWarps / 4;
+constexpr int kThreads = 32 * (kEpiWarp0 + kEpiWarps);   // 18 warps
 constexpr uint32_t kTmemCols = 512;
 
 constexpr uint32_t kQStage = 2u * kQ * kKC;              // 32 KB: Q_h box, then Q_l box
@@ -282,7 +286,7 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
       bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + kVS + s, 1);
     }
     bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + 2 * kVS, 1);       // acc_full: commit
-    bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + 2 * kVS + 1, 4);   // acc_empty: epilogue warps
+    bar_init(reinterpret_cast<uint64_t*>(smem + kOffBars) + 2 * kQS + 2 * kVS + 1, kEpiWarps);   // acc_empty
     asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
   }
   if (warp == 1) {
@@ -400,7 +404,9 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
   } else {
     // ---------------- epilogue: scores and running top-k, one query per thread
     const int quarter = warp & 3, ql = 32 * quarter + lane, q = q0 + ql;
-    const int e = tid - 32 * kEpiWarp0;   // 0 .. 127
+    const int e = tid - 32 * kEpiWarp0;   // 0 .. 32 kEpiWarps - 1
+    const int half = (warp - kEpiWarp0) >> 2;
+    constexpr int kStepsPerHalf = kV / 8 / kHalves;
     const bool qok = q < a.nq;
     const float qscale128 = qok ? 128.f * a.qscale[q] : 0.f;
     const uint32_t lane_addr = tmem + ((uint32_t)(32 * quarter) << 16);
@@ -449,50 +455,58 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
       const int64_t v0 = c0 + (int64_t)t * kV;
       const int nv = (int)min((int64_t)kV, c1 - v0);
       float* nb = nrm_s + (t & 1) * kV;
-#pragma unroll
-      for (int r = 0; r < 2; ++r) {
-        const int j = e + 128 * r;
-        nb[j] = j < nv ? load_norm(a.norms, a.norm_dtype, v0 + j) : 0.f;
-      }
+      for (int j = e; j < kV; j += 32 * kEpiWarps) nb[j] = j < nv ? load_norm(a.norms, a.norm_dtype, v0 + j) : 0.f;
       bool ok = !*abort_flag;
       if (ok && !wait_bar(acc_full, t & 1)) { fail_wait(); ok = false; }
-      // one decision for all four warps (this barrier also publishes the norms): tcgen05.ld is
-      // warp-collective and every epilogue warp must reach the same barriers
-      if (bar_red_or(1, 128, !ok)) break;
+      // one decision for all epilogue warps (this barrier also publishes the norms): tcgen05.ld
+      // is warp-collective and every epilogue warp must reach the same barriers
+      if (bar_red_or(1, 32 * kEpiWarps, !ok)) break;
       tc_fence_after();
       // 8 columns per step; the next step's accumulators load while this step is scored
       // (tcgen05.wait::ld waits for every load of the thread, so the loaded registers are copied
       // out before the next loads are issued into them)
-      const int nsteps = (nv + 7) / 8;   // the same for the whole warp
+      // this warp's steps: [st0, st1) of the tile's (nv + 7) / 8 (the same for the whole warp)
+      const int st0 = half * kStepsPerHalf, st1 = min((nv + 7) / 8, st0 + kStepsPerHalf);
       uint32_t hA[8], mA[8];
-      if (nsteps > 0) {
-        tmem_ld8(lane_addr, hA);
-        tmem_ld8(lane_addr + kV, mA);
+      if (st0 < st1) {
+        tmem_ld8(lane_addr + 8 * st0, hA);
+        tmem_ld8(lane_addr + kV + 8 * st0, mA);
       }
 #pragma unroll 1
-      for (int st = 0; st < nsteps; ++st) {
+      for (int st = st0; st < st1; ++st) {
         tmem_wait_ld8x2(hA, mA);
         uint32_t h[8], mm[8];
 #pragma unroll
         for (int j = 0; j < 8; ++j) h[j] = hA[j], mm[j] = mA[j];
-        if (st + 1 < nsteps) {
+        if (st + 1 < st1) {
           tmem_ld8(lane_addr + 8 * (st + 1), hA);
           tmem_ld8(lane_addr + kV + 8 * (st + 1), mA);
         }
         const int c = 8 * st;
         const float4 n0 = *reinterpret_cast<const float4*>(nb + c), n1 = *reinterpret_cast<const float4*>(nb + c + 4);
         const float nr[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+        // scores and a candidate mask without branches; the rare step with a candidate in any lane
+        // pushes them (in index order: an equal score ranks after) into the buffer
+        float sv[8];
+        uint32_t cand = 0;
 #pragma unroll
         for (int j = 0; j < 8; ++j) {
           // 16384 acc_hi + 128 acc_mid = 128 (128 acc_hi + acc_mid)
-          const float sj = fmaf(128.f, (float)(int)h[j], (float)(int)mm[j]) * (qscale128 * nr[j]);
-          if (qok && c + j < nv && sj > thr) {   // visited in index order: an equal score ranks after
-            bs[nbuf] = sj;
-            bi[nbuf] = (int)(v0 + c + j);
-            ++nbuf;
-          }
+          sv[j] = fmaf(128.f, (float)(int)h[j], (float)(int)mm[j]) * (qscale128 * nr[j]);
+          cand |= (sv[j] > thr) ? (1u << j) : 0u;
         }
-        if (nbuf >= 8) flush();
+        if (nv - c < 8) cand &= (1u << max(nv - c, 0)) - 1u;
+        if (!qok) cand = 0u;
+        if (__any_sync(0xffffffffu, cand != 0u)) {
+#pragma unroll
+          for (int j = 0; j < 8; ++j)
+            if (cand >> j & 1u) {
+              bs[nbuf] = sv[j];
+              bi[nbuf] = (int)(v0 + c + j);
+              ++nbuf;
+            }
+          if (nbuf >= 8) flush();
+        }
       }
       tc_fence_before();
       __syncwarp();
@@ -500,7 +514,7 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
       if (__any_sync(0xffffffffu, nbuf > 0)) flush();
     }
     if (qok && !*abort_flag) {
-      const size_t o = ((size_t)blockIdx.x * a.nq + q) * k - (KMAX - k);
+      const size_t o = (((size_t)blockIdx.x * kHalves + half) * a.nq + q) * k - (KMAX - k);
 #pragma unroll
       for (int x = 0; x < KMAX; ++x)
         if (x >= KMAX - k) {

@@ -644,6 +644,7 @@ size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base
     search_split(nq, n, &nc, &ch);
   if (nchunks) *nchunks = nc;
   if (chunk) *chunk = ch;
+  if (tc) nc *= tqk::stc::kHalves;   // one candidate list per chunk and column half
   size_t off = 0;
   if (qr) *qr = reinterpret_cast<float*>(base + off);
   off += round_up((size_t)nq * h->d * 4, 256);
@@ -1432,7 +1433,8 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
     }
     if ((st = launch_check("search_tc_kernel"))) return st;
     KernelScope ks("topk_merge", s);
-    tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
+    tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks * tqk::stc::kHalves, nq, k, score,
+                                                                 idx);
     return launch_check("topk_merge_kernel");
   }
   search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk, false);
