@@ -132,33 +132,56 @@ __global__ void __launch_bounds__(kSearchThreads) search_simt_kernel(SearchArgs 
   }
 }
 
-// Merge the per-chunk lists of one query (one warp per query; lane 0 inserts).
-__global__ void topk_merge_kernel(const float* cand_s, const int64_t* cand_i, int nchunks, int nq,
-                                  int K, float* out_s, int64_t* out_i) {
+// Merge the per-chunk lists of one query: one warp per query, a k-way merge of the sorted lists
+// (best first; an entry with index < 0 ends a list). Lane l owns lists l, l + 32, ...; their
+// read positions live in shared memory and each lane keeps the best current head of its lists.
+// Every round the warp picks the best head over the lanes ((score, index): higher score, then
+// lower index), writes it, and only the owning lane advances that list and rescans its own.
+__global__ void topk_merge_kernel(const float* cand_s, const int64_t* cand_i, int nchunks, int nq, int K,
+                                  float* out_s, int64_t* out_i) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
-  const int q = blockIdx.x;
-  int64_t* ti = reinterpret_cast<int64_t*>(smem_raw);
-  float* ts = reinterpret_cast<float*>(ti + K);
-  if (threadIdx.x != 0) return;
-  for (int i = 0; i < K; ++i) { ts[i] = -INFINITY; ti[i] = -1; }
-  for (int c = 0; c < nchunks; ++c) {
-    for (int r = 0; r < K; ++r) {
-      const size_t o = ((size_t)c * nq + q) * K + r;
-      const int64_t idx = cand_i[o];
-      if (idx < 0) break;
-      const float s = cand_s[o];
-      if (ti[K - 1] >= 0 && !ranks_before(s, idx, ts[K - 1], ti[K - 1])) break;  // lists are sorted
-      int pos = K - 1;
-      while (pos > 0 && (ti[pos - 1] < 0 || ranks_before(s, idx, ts[pos - 1], ti[pos - 1]))) {
-        ts[pos] = ts[pos - 1];
-        ti[pos] = ti[pos - 1];
-        --pos;
-      }
-      ts[pos] = s;
-      ti[pos] = idx;
+  int* pos = reinterpret_cast<int*>(smem_raw);   // [nchunks]
+  const int q = blockIdx.x, lane = threadIdx.x;
+  for (int c = lane; c < nchunks; c += 32) pos[c] = 0;
+  __syncwarp();
+  auto entry = [&](int c, int r) { return ((size_t)c * nq + q) * K + r; };
+  float bs = -INFINITY;
+  int64_t bi = -1;
+  int bc = -1;
+  auto rescan = [&]() {
+    bs = -INFINITY, bi = -1, bc = -1;
+    for (int c = lane; c < nchunks; c += 32) {
+      const int r = pos[c];
+      if (r >= K) continue;
+      const int64_t i = cand_i[entry(c, r)];
+      if (i < 0) continue;
+      const float sv = cand_s[entry(c, r)];
+      if (bc < 0 || ranks_before(sv, i, bs, bi)) bs = sv, bi = i, bc = c;
     }
+  };
+  rescan();
+  for (int r = 0; r < K; ++r) {
+    float ws = bs;
+    int64_t wi = bi;
+    int wl = bc >= 0 ? lane : 32;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      const float os = __shfl_xor_sync(0xffffffffu, ws, o);
+      const int64_t oi = __shfl_xor_sync(0xffffffffu, wi, o);
+      const int ol = __shfl_xor_sync(0xffffffffu, wl, o);
+      const bool take = ol < 32 && (wl == 32 || ranks_before(os, oi, ws, wi) || (os == ws && oi == wi && ol < wl));
+      if (take) ws = os, wi = oi, wl = ol;
+    }
+    if (lane == 0) {
+      out_s[(size_t)q * K + r] = wl < 32 ? ws : -INFINITY;
+      out_i[(size_t)q * K + r] = wl < 32 ? wi : -1;
+    }
+    if (wl == lane) {
+      ++pos[bc];
+      rescan();
+    }
+    __syncwarp();
   }
-  for (int i = 0; i < K; ++i) { out_s[(size_t)q * K + i] = ts[i]; out_i[(size_t)q * K + i] = ti[i]; }
 }
 
 }  // namespace tqk

@@ -34,7 +34,10 @@
 //                    128 vectors: it turns the accumulators into scores and keeps the query's running
 //                    top-k (k <= 16 or <= 32) over its half as a sorted list in registers.
 // Per query, chunk and half the list goes to the candidate arrays ([chunk][half] counts as one
-// chunk), which topk_merge_kernel reduces.
+// chunk), which topk_merge_kernel reduces. Every list's k-th best score is a lower bound of the
+// query's final k-th best, so each list publishes it (atomicMax into gbound) once full, and every
+// list reads the query's bound once per tile: a vector scoring below it cannot be in the final
+// top-k and is not considered (equal scores still are: the lower index may win them).
 // Every wait is bounded; a wait that runs out sets an abort flag (checked by every loop) and the
 // error word's kErrTimeout bit; the kernel then waits (bounded) for its own copies and MMAs and
 // frees its tensor memory.
@@ -92,10 +95,18 @@ struct Args {
   const float* qscale;     // [nq]: step_q * step_c
   int64_t n, chunk;        // database rows, rows per CTA chunk (a multiple of kV)
   uint32_t th[4], tl[4];   // C_h[idx], C_l[idx] as bytes, idx = 0 .. 15
-  float* cand_s;           // [nchunks][nq][k]
+  float* cand_s;           // [nchunks][kHalves][nq][k]
   int64_t* cand_i;
+  int* gbound;             // [nq]: the largest k-th best score any list has reached, as an ordered int
   int* err;
 };
+
+// Order-preserving map between floats and ints (its own inverse), for atomicMax on scores.
+__device__ __forceinline__ int float_ord(float f) {
+  const int i = __float_as_int(f);
+  return i >= 0 ? i : i ^ 0x7FFFFFFF;
+}
+__device__ __forceinline__ float ord_float(int i) { return __int_as_float(i >= 0 ? i : i ^ 0x7FFFFFFF); }
 
 // 16-entry table lookup of four 4-bit indices (nibbles 0..3 of x) -> four bytes: two 8-entry
 // permutes, then a permute that takes byte j from the second when bit 3 of nibble j is set.
@@ -219,6 +230,12 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, uint32_t (&v)[8]) {
   asm volatile("tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0,%1,%2,%3,%4,%5,%6,%7}, [%8];\n"
                : "=r"(v[0]), "=r"(v[1]), "=r"(v[2]), "=r"(v[3]), "=r"(v[4]), "=r"(v[5]), "=r"(v[6]), "=r"(v[7])
                : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_ld1x2(uint32_t ta, uint32_t tb, uint32_t& x, uint32_t& y) {
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n" : "=r"(x) : "r"(ta));
+  asm volatile("tcgen05.ld.sync.aligned.32x32b.x1.b32 {%0}, [%1];\n" : "=r"(y) : "r"(tb));
+  asm volatile("tcgen05.wait::ld.sync.aligned;\n" : "+r"(x), "+r"(y) : : "memory");
 }
 
 // Waits for this thread's tensor-memory loads; the loaded registers are operands, so that no use
@@ -441,20 +458,12 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
       }
       thr = ls[KMAX - 1];
     };
-    // candidates above the threshold wait in a small buffer (in index order) and are inserted
-    // once 8 have gathered, and at the end of each tile (one copy of the insertion code)
-    constexpr int kBuf = 16;
-    float bs[kBuf];
-    int bi[kBuf];
-    int nbuf = 0;
-    auto flush = [&]() {
-      for (int x = 0; x < nbuf; ++x) insert(bs[x], bi[x]);
-      nbuf = 0;
-    };
+    float gb = -INFINITY;   // the query's shared lower bound, read once per tile
     for (int t = 0; t < ntiles; ++t) {
       const int64_t v0 = c0 + (int64_t)t * kV;
       const int nv = (int)min((int64_t)kV, c1 - v0);
       float* nb = nrm_s + (t & 1) * kV;
+      if (qok) gb = fmaxf(gb, ord_float(*reinterpret_cast<volatile int*>(a.gbound + q)));
       for (int j = e; j < kV; j += 32 * kEpiWarps) nb[j] = j < nv ? load_norm(a.norms, a.norm_dtype, v0 + j) : 0.f;
       bool ok = !*abort_flag;
       if (ok && !wait_bar(acc_full, t & 1)) { fail_wait(); ok = false; }
@@ -465,53 +474,70 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
       // 8 columns per step; the next step's accumulators load while this step is scored
       // (tcgen05.wait::ld waits for every load of the thread, so the loaded registers are copied
       // out before the next loads are issued into them)
-      // this warp's steps: [st0, st1) of the tile's (nv + 7) / 8 (the same for the whole warp)
+      // this warp's steps: [st0, st1) of the tile's (nv + 7) / 8 (the same for the whole warp).
+      // Pass 1 scores every column against the threshold and bound as they stood at the start of
+      // the tile and keeps one bit per candidate; pass 2 (rare: a candidate in any lane) reloads
+      // those columns, in index order, and inserts what still qualifies.
       const int st0 = half * kStepsPerHalf, st1 = min((nv + 7) / 8, st0 + kStepsPerHalf);
+      uint64_t cbits[kStepsPerHalf / 8];
       uint32_t hA[8], mA[8];
       if (st0 < st1) {
         tmem_ld8(lane_addr + 8 * st0, hA);
         tmem_ld8(lane_addr + kV + 8 * st0, mA);
       }
-#pragma unroll 1
-      for (int st = st0; st < st1; ++st) {
-        tmem_wait_ld8x2(hA, mA);
-        uint32_t h[8], mm[8];
 #pragma unroll
-        for (int j = 0; j < 8; ++j) h[j] = hA[j], mm[j] = mA[j];
-        if (st + 1 < st1) {
-          tmem_ld8(lane_addr + 8 * (st + 1), hA);
-          tmem_ld8(lane_addr + kV + 8 * (st + 1), mA);
-        }
-        const int c = 8 * st;
-        const float4 n0 = *reinterpret_cast<const float4*>(nb + c), n1 = *reinterpret_cast<const float4*>(nb + c + 4);
-        const float nr[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
-        // scores and a candidate mask without branches; the rare step with a candidate in any lane
-        // pushes them (in index order: an equal score ranks after) into the buffer
-        float sv[8];
-        uint32_t cand = 0;
+      for (int gr = 0; gr < kStepsPerHalf / 8; ++gr) {
+        uint64_t bits = 0;
 #pragma unroll
-        for (int j = 0; j < 8; ++j) {
-          // 16384 acc_hi + 128 acc_mid = 128 (128 acc_hi + acc_mid)
-          sv[j] = fmaf(128.f, (float)(int)h[j], (float)(int)mm[j]) * (qscale128 * nr[j]);
-          cand |= (sv[j] > thr) ? (1u << j) : 0u;
-        }
-        if (nv - c < 8) cand &= (1u << max(nv - c, 0)) - 1u;
-        if (!qok) cand = 0u;
-        if (__any_sync(0xffffffffu, cand != 0u)) {
+        for (int i = 0; i < 8; ++i) {
+          const int st = st0 + 8 * gr + i;
+          if (st < st1) {   // the same for the whole warp
+            tmem_wait_ld8x2(hA, mA);
+            uint32_t h[8], mm[8];
 #pragma unroll
-          for (int j = 0; j < 8; ++j)
-            if (cand >> j & 1u) {
-              bs[nbuf] = sv[j];
-              bi[nbuf] = (int)(v0 + c + j);
-              ++nbuf;
+            for (int j = 0; j < 8; ++j) h[j] = hA[j], mm[j] = mA[j];
+            if (st + 1 < st1) {
+              tmem_ld8(lane_addr + 8 * (st + 1), hA);
+              tmem_ld8(lane_addr + kV + 8 * (st + 1), mA);
             }
-          if (nbuf >= 8) flush();
+            const int c = 8 * st;
+            const float4 n0 = *reinterpret_cast<const float4*>(nb + c);
+            const float4 n1 = *reinterpret_cast<const float4*>(nb + c + 4);
+            const float nr[8] = {n0.x, n0.y, n0.z, n0.w, n1.x, n1.y, n1.z, n1.w};
+            uint32_t cand = 0;
+#pragma unroll
+            for (int j = 0; j < 8; ++j) {
+              // 16384 acc_hi + 128 acc_mid = 128 (128 acc_hi + acc_mid)
+              const float sj = fmaf(128.f, (float)(int)h[j], (float)(int)mm[j]) * (qscale128 * nr[j]);
+              cand |= (sj > thr && sj >= gb) ? (1u << j) : 0u;
+            }
+            if (nv - c < 8) cand &= (1u << max(nv - c, 0)) - 1u;
+            bits |= (uint64_t)cand << (8 * i);
+          }
+        }
+        cbits[gr] = qok ? bits : 0ull;
+      }
+#pragma unroll
+      for (int gr = 0; gr < kStepsPerHalf / 8; ++gr) {
+        const uint32_t lo = __reduce_or_sync(0xffffffffu, (uint32_t)cbits[gr]);
+        const uint32_t hi = __reduce_or_sync(0xffffffffu, (uint32_t)(cbits[gr] >> 32));
+        uint64_t any = ((uint64_t)hi << 32) | lo;
+        while (any) {   // the same for the whole warp
+          const int bit = __ffsll((long long)any) - 1;
+          any &= any - 1;
+          const int col = 8 * st0 + 64 * gr + bit;
+          uint32_t x, y;
+          tmem_ld1x2(lane_addr + col, lane_addr + kV + col, x, y);
+          if (cbits[gr] >> bit & 1ull) {
+            const float sj = fmaf(128.f, (float)(int)x, (float)(int)y) * (qscale128 * nb[col]);
+            if (sj > thr && sj >= gb) insert(sj, (int)(v0 + col));   // an equal score ranks after
+          }
         }
       }
       tc_fence_before();
       __syncwarp();
       if (lane == 0) bar_arrive(acc_empty);
-      if (__any_sync(0xffffffffu, nbuf > 0)) flush();
+      if (qok && thr > -INFINITY) atomicMax(a.gbound + q, float_ord(thr));
     }
     if (qok && !*abort_flag) {
       const size_t o = (((size_t)blockIdx.x * kHalves + half) * a.nq + q) * k - (KMAX - k);
@@ -534,10 +560,10 @@ __global__ void __launch_bounds__(kThreads, 1) search_tc_kernel(const __grid_con
 }
 
 // Query pieces: row q of qr (rotated queries, fp32) -> Q_h (row q) and Q_l (row nq_pad + q) of
-// `pieces`, Q = rint(q' / step_q) with step_q = max_j |q'_j| / 16319; qscale[q] = step_q * step_c.
-// Rows nq .. nq_pad - 1 are zero. One warp per row.
+// `pieces`, Q = rint(q' / step_q) with step_q = max_j |q'_j| / 16319; qscale[q] = step_q * step_c;
+// gbound[q] starts at -inf. Rows nq .. nq_pad - 1 are zero. One warp per row.
 __global__ void search_tc_qprep_kernel(const float* qr, int nq, int nq_pad, int d, float step_c, int8_t* pieces,
-                                       float* qscale) {
+                                       float* qscale, int* gbound) {
   grid_dep_launch();
   grid_dep_wait();   // qr comes from the rotation kernel before this one
   const int lane = threadIdx.x & 31;
@@ -561,7 +587,16 @@ __global__ void search_tc_qprep_kernel(const float* qr, int nq, int nq_pad, int 
     ph[j] = (int8_t)h;
     pl[j] = (int8_t)(x - 128 * h);
   }
-  if (lane == 0) qscale[q] = mx > 0.f ? (mx / (float)kCMax) * step_c : 0.f;
+  if (lane == 0) {
+    qscale[q] = mx > 0.f ? (mx / (float)kCMax) * step_c : 0.f;
+    gbound[q] = float_ord(-INFINITY);
+  }
+}
+
+// The bound pass's result: gbound[q] = the k-th best score of the sample (when it has k vectors).
+__global__ void search_tc_bound_kernel(const float* ts, const int64_t* ti, int nq, int k, int* gbound) {
+  const int q = blockIdx.x * blockDim.x + threadIdx.x;
+  if (q < nq && ti[(size_t)q * k + k - 1] >= 0) atomicMax(gbound + q, float_ord(ts[(size_t)q * k + k - 1]));
 }
 
 }  // namespace stc

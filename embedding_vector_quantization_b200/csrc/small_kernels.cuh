@@ -200,6 +200,77 @@ __global__ void __launch_bounds__(kSmallThreads) qprep_wide_kernel(const void* q
   qprep_tile(q, q_dtype, rows, d, PiT, ST, m, out_r, out_s, blockIdx.x, blockIdx.y, rpc, smem_raw);
 }
 
+// ---------------------------------------------------------------- batched query rotation
+
+// C = X B for a batch of fp32 query rows (X [rows][K] row-major, B [K][N] row-major: Pi^T or
+// S^T), C [rows][N]: 128 x 128 output tiles per CTA, 8 x 8 per thread, K in steps of 16 through
+// shared memory (X transposed on the way in). For the large query batches of the search, where
+// the per-row kernels above re-read B once per row group. K % 16 == 0 and N % 4 == 0; rows and
+// N need not be multiples of the tile.
+constexpr int kRotBM = 128, kRotBN = 128, kRotBK = 16;
+__global__ void __launch_bounds__(256) rotate_tiled_kernel(const float* __restrict__ X, int rows, int K,
+                                                           const float* __restrict__ B, int N,
+                                                           float* __restrict__ C) {
+  __shared__ __align__(16) float As[kRotBK][kRotBM];
+  __shared__ __align__(16) float Bs[kRotBK][kRotBN];
+  grid_dep_launch();
+  const int tid = threadIdx.x, tx = tid & 15, ty = tid >> 4;
+  const int m0 = blockIdx.y * kRotBM, n0 = blockIdx.x * kRotBN;
+  float acc[8][8];
+#pragma unroll
+  for (int i = 0; i < 8; ++i)
+#pragma unroll
+    for (int j = 0; j < 8; ++j) acc[i][j] = 0.f;
+  for (int k0 = 0; k0 < K; k0 += kRotBK) {
+    // X tile: 128 rows x 16 k, two float4 per thread, stored transposed
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int e = tid + 256 * r, row = e >> 2, kq = (e & 3) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (m0 + row < rows) v = *reinterpret_cast<const float4*>(X + (size_t)(m0 + row) * K + k0 + kq);
+      As[kq][row] = v.x;
+      As[kq + 1][row] = v.y;
+      As[kq + 2][row] = v.z;
+      As[kq + 3][row] = v.w;
+    }
+    // B tile: 16 k x 128 columns, two float4 per thread
+#pragma unroll
+    for (int r = 0; r < 2; ++r) {
+      const int e = tid + 256 * r, kk = e >> 5, c = (e & 31) * 4;
+      float4 v = make_float4(0.f, 0.f, 0.f, 0.f);
+      if (n0 + c < N) v = *reinterpret_cast<const float4*>(B + (size_t)(k0 + kk) * N + n0 + c);
+      *reinterpret_cast<float4*>(&Bs[kk][c]) = v;
+    }
+    __syncthreads();
+#pragma unroll
+    for (int kk = 0; kk < kRotBK; ++kk) {
+      const float4 a0 = *reinterpret_cast<const float4*>(&As[kk][ty * 8]);
+      const float4 a1 = *reinterpret_cast<const float4*>(&As[kk][ty * 8 + 4]);
+      const float4 b0 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8]);
+      const float4 b1 = *reinterpret_cast<const float4*>(&Bs[kk][tx * 8 + 4]);
+      const float av[8] = {a0.x, a0.y, a0.z, a0.w, a1.x, a1.y, a1.z, a1.w};
+      const float bv[8] = {b0.x, b0.y, b0.z, b0.w, b1.x, b1.y, b1.z, b1.w};
+#pragma unroll
+      for (int i = 0; i < 8; ++i)
+#pragma unroll
+        for (int j = 0; j < 8; ++j) acc[i][j] = fmaf(av[i], bv[j], acc[i][j]);
+    }
+    __syncthreads();
+  }
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    const int row = m0 + ty * 8 + i;
+    if (row >= rows) continue;
+#pragma unroll
+    for (int j = 0; j < 8; j += 4) {
+      const int col = n0 + tx * 8 + j;
+      if (col < N)
+        *reinterpret_cast<float4*>(C + (size_t)row * N + col) =
+            make_float4(acc[i][j], acc[i][j + 1], acc[i][j + 2], acc[i][j + 3]);
+    }
+  }
+}
+
 // ---------------------------------------------------------------- decode-step prologue
 
 // One launch for the independent first half of a decode step: CTAs [0, nvec) append the

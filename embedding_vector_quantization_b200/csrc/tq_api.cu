@@ -631,11 +631,25 @@ size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, i
 }
 
 // mma: 0 for the SIMT kernel, else the queries per CTA of the tensor-core kernel.
-// tc: the tcgen05 search, which also takes the int8 query pieces [2][nq_pad][d] and their
-// scales [nq_pad] (pieces / qscale, else unused); otherwise the SIMT search.
+// The bound pass of the tcgen05 search: the first kSearchSample vectors are searched first, and
+// their exact k-th best score per query (a lower bound of the whole database's) seeds the score
+// bound of the full pass, which then sets aside far fewer candidates. Only for n >= 4 samples.
+constexpr int64_t kSearchSample = 32768;
+struct SampleWs {
+  int nchunks = 0;
+  int64_t chunk = 0;
+  float* cs = nullptr;     // [nchunks][halves][nq][k]
+  int64_t* ci = nullptr;
+  float* ts = nullptr;     // [nq][k]: the sample's top-k
+  int64_t* ti = nullptr;
+};
+
+// tc: the tcgen05 search, which also takes the int8 query pieces [2][nq_pad][d], their scales
+// [nq_pad], the per-query score bounds [nq_pad] and the bound pass's arrays (pieces / qscale /
+// gbound / sample, else unused); otherwise the SIMT search.
 size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base, float** qr, float** cs,
                         int64_t** ci, int* nchunks, int64_t* chunk, bool tc, int8_t** pieces = nullptr,
-                        float** qscale = nullptr) {
+                        float** qscale = nullptr, int** gbound = nullptr, SampleWs* sample = nullptr) {
   int nc;
   int64_t ch;
   if (tc)
@@ -654,6 +668,22 @@ size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base
     off += round_up(2 * nq_pad * h->d, 256);
     if (qscale) *qscale = reinterpret_cast<float*>(base + off);
     off += round_up(nq_pad * 4, 256);
+    if (gbound) *gbound = reinterpret_cast<int*>(base + off);
+    off += round_up(nq_pad * 4, 256);
+    if (n >= 4 * kSearchSample) {
+      SampleWs sw;
+      search_tc_split(nq, kSearchSample, sm_count(h->device), &sw.nchunks, &sw.chunk);
+      const size_t lists = (size_t)sw.nchunks * tqk::stc::kHalves * nq * k;
+      sw.cs = reinterpret_cast<float*>(base + off);
+      off += round_up(lists * 4, 256);
+      sw.ci = reinterpret_cast<int64_t*>(base + off);
+      off += round_up(lists * 8, 256);
+      sw.ts = reinterpret_cast<float*>(base + off);
+      off += round_up((size_t)nq * k * 4, 256);
+      sw.ti = reinterpret_cast<int64_t*>(base + off);
+      off += round_up((size_t)nq * k * 8, 256);
+      if (sample) *sample = sw;
+    }
   }
   if (cs) *cs = reinterpret_cast<float*>(base + off);
   off += round_up((size_t)nc * nq * k * 4, 256);
@@ -664,6 +694,19 @@ size_t search_ws_layout(const tq_handle* h, int nq, int64_t n, int k, char* base
 
 int launch_qprep(const tq_handle* h, const void* q, int q_dtype, int rows, float* qr, float* qs, cudaStream_t s) {
   if (rows == 0) return TQ_OK;
+  // large fp32 batches (the search's queries): the tiled kernel
+  if (rows >= 256 && q_dtype == TQ_F32 && aligned(q, 16) && h->d % tqk::kRotBK == 0 && h->d % 4 == 0 &&
+      h->m % 4 == 0) {
+    KernelScope ks("qprep", s);
+    const float* X = static_cast<const float*>(q);
+    const dim3 gr((unsigned)((h->d + tqk::kRotBN - 1) / tqk::kRotBN), (unsigned)((rows + tqk::kRotBM - 1) / tqk::kRotBM));
+    tqk::rotate_tiled_kernel<<<gr, 256, 0, s>>>(X, rows, h->d, h->dPiT, h->d, qr);
+    if (qs && h->m > 0) {
+      const dim3 gs((unsigned)((h->m + tqk::kRotBN - 1) / tqk::kRotBN), gr.y);
+      tqk::rotate_tiled_kernel<<<gs, 256, 0, s>>>(X, rows, h->d, h->dST, h->m, qs);
+    }
+    return launch_check("rotate_tiled_kernel");
+  }
   if (h->d <= tqk::kWideMaxD && h->m <= tqk::kWideMaxD) {
     if (once_per_device(6, h->device))
       cudaFuncSetAttribute(tqk::qprep_wide_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, 200 * 1024);
@@ -1393,13 +1436,15 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
   if (search_tc_ok(h, n, k)) {
     int8_t* pieces;
     float* qscale;
+    int* gbound;
+    SampleWs sw;
     search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk, true, &pieces,
-                     &qscale);
+                     &qscale, &gbound, &sw);
     const int nq_pad = (nq + tqk::stc::kQ - 1) / tqk::stc::kQ * tqk::stc::kQ;
     tqk::stc::Args m{};
     m.nq = nq; m.nq_pad = nq_pad; m.d = h->d; m.k = k; m.norm_dtype = h->norm_dtype; m.codes_B = h->codes_B;
     m.codes = codes; m.norms = norms; m.qscale = qscale; m.n = n; m.chunk = chunk;
-    m.cand_s = cs; m.cand_i = ci; m.err = h->derr;
+    m.cand_s = cs; m.cand_i = ci; m.gbound = gbound; m.err = h->derr;
     float step_c;
     centroid_pieces(h->cent, &step_c, m.th, m.tl);
     CUtensorMap qmap;
@@ -1410,7 +1455,7 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
     {
       KernelScope ks("search_qprep", s);
       const cudaError_t e = launch_pdl(tqk::stc::search_tc_qprep_kernel, dim3((unsigned)(nq_pad / 8)), dim3(256), 0,
-                                       s, (const float*)qr, nq, nq_pad, h->d, step_c, pieces, qscale);
+                                       s, (const float*)qr, nq, nq_pad, h->d, step_c, pieces, qscale, gbound);
       if (e != cudaSuccess) return cuda_fail(e, "search_tc_qprep_kernel");
     }
     if ((st = launch_check("search_tc_qprep_kernel"))) return st;
@@ -1425,6 +1470,26 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
     auto kern = kerns[big][h->bits - 1];
     if (once_per_device(16 + 4 * big + h->bits, h->device))
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tqk::stc::kSmemBytes);
+    const char* sample_env = std::getenv("TQ_SEARCH_SAMPLE");   // "0": no bound pass (tests compare both)
+    if (sample_env && std::strcmp(sample_env, "0") == 0) sw.nchunks = 0;
+    if (sw.nchunks > 0) {   // bound pass over the first kSearchSample vectors
+      tqk::stc::Args ms = m;
+      ms.n = kSearchSample; ms.chunk = sw.chunk; ms.cand_s = sw.cs; ms.cand_i = sw.ci;
+      {
+        KernelScope ks("search_sample", s);
+        const cudaError_t e = launch_pdl(kern, dim3((unsigned)sw.nchunks, (unsigned)(nq_pad / tqk::stc::kQ)),
+                                         dim3(tqk::stc::kThreads), (size_t)tqk::stc::kSmemBytes, s, qmap, ms);
+        if (e != cudaSuccess) return cuda_fail(e, "search_tc_kernel");
+      }
+      if ((st = launch_check("search_tc_kernel"))) return st;
+      {
+        KernelScope ks("search_sample", s);
+        const int nl = sw.nchunks * tqk::stc::kHalves;
+        tqk::topk_merge_kernel<<<nq, 32, (size_t)nl * 4 + 16, s>>>(sw.cs, sw.ci, nl, nq, k, sw.ts, sw.ti);
+        tqk::stc::search_tc_bound_kernel<<<(nq + 255) / 256, 256, 0, s>>>(sw.ts, sw.ti, nq, k, gbound);
+      }
+      if ((st = launch_check("search_tc_bound_kernel"))) return st;
+    }
     {
       KernelScope ks("search", s);
       const cudaError_t e = launch_pdl(kern, dim3((unsigned)nchunks, (unsigned)(nq_pad / tqk::stc::kQ)),
@@ -1433,8 +1498,8 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
     }
     if ((st = launch_check("search_tc_kernel"))) return st;
     KernelScope ks("topk_merge", s);
-    tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks * tqk::stc::kHalves, nq, k, score,
-                                                                 idx);
+    const int nl = nchunks * tqk::stc::kHalves;
+    tqk::topk_merge_kernel<<<nq, 32, (size_t)nl * 4 + 16, s>>>(cs, ci, nl, nq, k, score, idx);
     return launch_check("topk_merge_kernel");
   }
   search_ws_layout(h, nq, n, k, static_cast<char*>(workspace), &qr, &cs, &ci, &nchunks, &chunk, false);
@@ -1453,7 +1518,7 @@ int tq_search_topk(const tq_handle* h, const float* q, int nq, const uint8_t* co
   }
   if ((st = launch_check("search_simt_kernel"))) return st;
   KernelScope ks("topk_merge", s);
-  tqk::topk_merge_kernel<<<nq, 32, (size_t)k * 12 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
+  tqk::topk_merge_kernel<<<nq, 32, (size_t)nchunks * 4 + 16, s>>>(cs, ci, nchunks, nq, k, score, idx);
   return launch_check("topk_merge_kernel");
 }
 

@@ -131,3 +131,15 @@ def test_search_tc_full_query_tiles_sampled(tq):
     """1024 queries (8 query tiles of 128) over 60,000 vectors at d = 768: the natural split
     (whole waves of one CTA per SM); 64 sampled queries against the oracle."""
     _run(tq, 2, 768, 60000, 1024, 10, seed=901, sample=np.arange(0, 1024, 16))
+
+
+def test_search_tc_bound_pass_changes_nothing(tq):
+    """From 131,072 vectors on, a bound pass over the first 32,768 seeds each query's score bound
+    with their exact k-th best; the full pass then skips vectors below it. The result must equal
+    the search without the bound pass (TQ_SEARCH_SAMPLE=0) exactly, and be valid for the oracle."""
+    h, codes, norms, qg, (idx, sc), (S, Q, e, rows) = _run(tq, 2, 256, 140000, 200, 10, seed=77,
+                                                            sample=np.arange(0, 200, 8))
+    with env(TQ_SEARCH_SAMPLE=0):
+        idx0, sc0 = (x.cpu().numpy() for x in h.search_topk(qg, codes, norms, 10))
+    assert h.status() == tq.TQ_OK
+    assert np.array_equal(idx, idx0) and np.array_equal(sc, sc0)
