@@ -42,6 +42,7 @@
 #include "encode_tc.cuh"
 #include "attn_mse4.cuh"
 #include "search_tc.cuh"
+#include "encode_big_tc.cuh"
 #include "polar.cuh"
 
 struct tq_handle {
@@ -59,6 +60,7 @@ struct tq_handle {
   float* dbnd = nullptr;  // [2^bits - 1]
   int* derr = nullptr;    // device error word
   uint8_t* dOps = nullptr; // d = 128: pre-swizzled 16-bit hi/lo operands of the tensor-core encode
+  uint16_t* dPiB = nullptr; // MSE, d % 256 = 0, 256 <= d <= 4096: Pi as a bf16 pair, [2][d][d] (hi rows, lo rows)
   // recursive polar transform handles (tq_create_polar): per-level angle codebooks
   int polar = 0;
   tqk::polar::Layout play{};
@@ -188,6 +190,8 @@ void free_device(tq_handle* h) {
   cudaFree(h->dbnd);
   cudaFree(h->derr);
   cudaFree(h->dOps);
+  cudaFree(h->dPiB);
+  h->dPiB = nullptr;
   cudaFree(h->dTab);
   h->dPi = h->dPiT = h->dS = h->dST = h->dMT = h->dcent = h->dbnd = nullptr;
   h->derr = nullptr;
@@ -303,11 +307,31 @@ int create_common(int d, int bits_mse, int m, uint64_t seed, int norm_dtype, tq_
     }
   std::vector<uint8_t> ops;
   if (d == tqk::etc::kD && (m == 0 || m == tqk::etc::kD)) ops = tc_operands(h->Pi, M);
+  // Pi = Pi_h + Pi_l as bf16 (round to nearest even), for the tensor-core encode of large d
+  std::vector<uint16_t> pib;
+  if (m == 0 && bits_mse > 0 && d % tqk::ebig::kN == 0 && d >= tqk::ebig::kMinD && d <= tqk::ebig::kMaxD) {
+    pib.resize((size_t)2 * d * d);
+    auto bf16 = [](float f) {
+      uint32_t u;
+      std::memcpy(&u, &f, 4);
+      u += 0x7FFFu + ((u >> 16) & 1u);
+      return (uint16_t)(u >> 16);
+    };
+    for (size_t i = 0; i < (size_t)d * d; ++i) {
+      const float v = (float)h->Pi[i];
+      const uint16_t hi = bf16(v);
+      const uint32_t hb = (uint32_t)hi << 16;
+      float hf;
+      std::memcpy(&hf, &hb, 4);
+      pib[i] = hi;
+      pib[(size_t)d * d + i] = bf16((float)(h->Pi[i] - (double)hf));
+    }
+  }
   int st = TQ_OK;
   if ((st = upload(&h->dPi, Pi, "Pi")) || (st = upload(&h->dPiT, PiT, "PiT")) ||
       (st = upload(&h->dS, S, "S")) || (st = upload(&h->dST, ST, "ST")) || (st = upload(&h->dMT, MT, "MT")) ||
       (st = upload(&h->dcent, cent, "centroids")) || (st = upload(&h->dbnd, bnd, "bounds")) ||
-      (st = upload(&h->dOps, ops, "tensor-core operands"))) {
+      (st = upload(&h->dOps, ops, "tensor-core operands")) || (st = upload(&h->dPiB, pib, "bf16 rotation pair"))) {
     free_device(h);
     delete h;
     return st;
@@ -847,8 +871,43 @@ int encode_tc_launch(const tq_handle* h, const tqk::EncodeArgs& a, cudaStream_t 
   return n32 ? tc_launch_bits<false, true>(h, map, ea, f16, grid, s) : tc_launch_bits<false, false>(h, map, ea, f16, grid, s);
 }
 
+// The tensor-core encode of large vectors: MSE handles with d % 256 == 0 (256 .. 4096), at least
+// 256 rows, not an append.
+bool big_tc_ok(const tq_handle* h, const tqk::EncodeArgs& a) {
+  return !std::getenv("TQ_SIMT") && h->dPiB && a.len == nullptr && a.rows >= 256 && a.rows < ((int64_t)1 << 31);
+}
+
+int encode_big_tc_launch(const tq_handle* h, const tqk::EncodeArgs& a, cudaStream_t s) {
+  PFN_cuTensorMapEncodeTiled enc = tensor_map_encoder();
+  if (!enc) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled is not available from the driver");
+  const int d = h->d;
+  CUtensorMap pmap;
+  const cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)2 * d};
+  const cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  const cuuint32_t box[2] = {(cuuint32_t)tqk::ebig::kKC, (cuuint32_t)tqk::ebig::kN};
+  const cuuint32_t estr[2] = {1, 1};
+  const CUresult r = enc(&pmap, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, h->dPiB, dims, strides, box, estr,
+                         CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                         CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  if (r != CUDA_SUCCESS) return fail(TQ_ECUDA, "cuTensorMapEncodeTiled failed (%d)", (int)r);
+  tqk::ebig::Args ea{};
+  ea.x = a.x; ea.x_dtype = a.x_dtype; ea.rows = a.rows; ea.d = d; ea.bits = h->bits; ea.norm_dtype = a.norm_dtype;
+  ea.codes_B = h->codes_B; ea.bnd = h->dbnd; ea.codes = a.codes; ea.norms = a.norms; ea.err = h->derr;
+  auto kern = a.x_dtype == TQ_F32 ? tqk::ebig::encode_big_tc_kernel<TQ_F32>
+            : a.x_dtype == TQ_BF16 ? tqk::ebig::encode_big_tc_kernel<TQ_BF16>
+                                   : tqk::ebig::encode_big_tc_kernel<TQ_F16>;
+  if (once_per_device(25 + a.x_dtype, h->device))
+    cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)tqk::ebig::kSmemBytes);
+  const int64_t ntiles = (a.rows + tqk::ebig::kM - 1) / tqk::ebig::kM;
+  const unsigned grid = (unsigned)std::min<int64_t>(ntiles, sm_count(h->device));
+  KernelScope ks("encode", s);
+  kern<<<grid, tqk::ebig::kThreads, tqk::ebig::kSmemBytes, s>>>(pmap, ea);
+  return launch_check("encode_big_tc_kernel");
+}
+
 int encode_launch(const tq_handle* h, tqk::EncodeArgs& a, cudaStream_t s) {
   if (tc_encode_ok(h, a)) return encode_tc_launch(h, a, s);
+  if (big_tc_ok(h, a)) return encode_big_tc_launch(h, a, s);
   if (a.len == nullptr && a.rows <= 256 && rows_kernel_ok(h, 1))
     return encode_rows_launch(h, a, (unsigned)((a.rows + tqk::kRowsMax - 1) / tqk::kRowsMax), 0, s);
   const size_t smem = tqk::encode_smem_bytes(h->m);

@@ -180,3 +180,40 @@ def test_encode_tc_matches_simt(tq, monkeypatch):
     # fp16 norms: the tensor-core path takes ||(Pi_hi + Pi_lo) x||, within 1 ulp of ||x||
     ulp = (a["norms"].float() - b["norms"].float()).abs() / torch.finfo(torch.float16).eps / b["norms"].float().abs()
     assert ulp.max().item() <= 1.0
+
+
+@pytest.mark.parametrize("d,bits,n,dtype", [
+    (1536, 2, 3000, torch.float32),    # 6 passes of 256 coordinates, a ragged last tile
+    (1536, 4, 1200, torch.bfloat16),   # bf16 input: the x_l contraction is skipped
+    (512, 3, 2000, torch.float16),     # 3-bit fields straddle words
+    (256, 1, 40000, torch.float32),    # one pass; more tiles than SMs (several per CTA)
+    (768, 2, 300, torch.float32),      # a single, partial tile
+])
+def test_encode_large_d_tensor_core_path(tq, d, bits, n, dtype):
+    """The tcgen05 encode of large vectors (MSE, d % 256 = 0): indices within the boundary band of
+    the oracle's, norms within an ulp; zero rows and huge / tiny scales included; and the same
+    rows as the SIMT kernel (TQ_SIMT=1) outside that band."""
+    import os
+    g = torch.Generator().manual_seed(d + bits)
+    x = torch.randn(n, d, generator=g) * torch.exp(0.5 * torch.randn(n, 1, generator=g))
+    x[0] = 0
+    x[min(5, n - 1)] *= 1e4
+    x[min(9, n - 1)] *= 1e-4
+    x = x.to(dtype)
+    frac, _ = _encode_and_check(tq, x, d, bits, seed=d)
+    print(f"large-d encode d={d} bits={bits} n={n} {dtype}: index mismatch fraction {frac:.2e}")
+    assert frac < 1e-3
+    h = tq.Handle(d, bits, d)
+    fast = h.encode(x.cuda())
+    os.environ["TQ_SIMT"] = "1"
+    try:
+        simt = h.encode(x.cuda())
+    finally:
+        del os.environ["TQ_SIMT"]
+    from gpu_util import unpack_fast
+    a = unpack_fast(fast["codes"].cpu().numpy().reshape(n, -1), d, bits)
+    b = unpack_fast(simt["codes"].cpu().numpy().reshape(n, -1), d, bits)
+    differ = (a != b).mean()
+    # the two kernels round y differently by ~1e-7: only coordinates at a decision boundary differ
+    assert differ < 1e-4, differ
+    assert torch.equal(fast["norms"], simt["norms"]) or torch.allclose(fast["norms"], simt["norms"], rtol=2e-7)
