@@ -296,7 +296,10 @@ __device__ __forceinline__ void prepare_query(const float* qr_rows, const float*
 // fragments qb held in registers) and n tile 1 (lo: lo(k-step, register) returns this thread's
 // fragment word, from registers or shared memory), the sign bit planes against the two pieces of
 // S q in n tile 0.
-template <int NT, typename LoFn>
+// LO: the code side uses all three query pieces (22-bit queries, what the attention needs so that
+// softmax does not amplify the rounding); without it the lo piece is skipped and the code-side
+// query is the 15-bit hi/mid value, which raw scores are accurate enough with (about 3e-5 relative).
+template <int NT, bool LO, typename LoFn>
 __device__ __forceinline__ void mtile_scores(const unsigned char* codes, const unsigned char* signs, const __half* nrm,
                                              const __half* rnm, const int (&kbase)[NT], const uint32_t (&qb)[12][2],
                                              LoFn lo, float c0h, float dmh, float dsh, float ssh, float (&sc)[NT][2]) {
@@ -322,8 +325,10 @@ __device__ __forceinline__ void mtile_scores(const unsigned char* codes, const u
       const uint32_t b0 = x0 & 0x10101010u, b1 = x2 & 0x10101010u, b2 = x1 & 0x10101010u, b3 = x3 & 0x10101010u;
       mma_s8(dm1[i], a0, a1, a2, a3, qb[s][0], qb[s][1]);
       mma_s8(dm16[i], b0, b1, b2, b3, qb[4 + s][0], qb[4 + s][1]);
-      mma_s8(lm1[i], a0, a1, a2, a3, lo(s, 0), lo(s, 1));
-      mma_s8(lm16[i], b0, b1, b2, b3, lo(4 + s, 0), lo(4 + s, 1));
+      if (LO) {
+        mma_s8(lm1[i], a0, a1, a2, a3, lo(s, 0), lo(s, 1));
+        mma_s8(lm16[i], b0, b1, b2, b3, lo(4 + s, 0), lo(4 + s, 1));
+      }
     }
   }
   // sign words: sw[0] = key g word t, sw[1] = key g+8 word t
@@ -347,7 +352,7 @@ __device__ __forceinline__ void mtile_scores(const unsigned char* codes, const u
       const int hi = 2 * r, md = 2 * r + 1;   // tile 0: columns 2t (hi) and 2t + 1 (mid); tile 1: column 2t (lo)
       // exact in int32: at most 256 code positions of |piece| <= 127 each, times 2^14
       const int mse = (dm1[i][hi] + (dm16[i][hi] >> 4)) * 16384 + (dm1[i][md] + (dm16[i][md] >> 4)) * 128 +
-                      lm1[i][hi] + (lm16[i][hi] >> 4);
+                      (LO ? lm1[i][hi] + (lm16[i][hi] >> 4) : 0);
       // column 2t + 1 holds the lo piece of S q here
       const int qjl = (ds1[i][hi] + (ds16[i][hi] >> 4)) * 128 + ds1[i][md] + (ds16[i][md] >> 4);
       const float n = __half2float(nrm[key]), rn = __half2float(rnm[key]);
@@ -498,11 +503,11 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
     float sc[2][2];
     if (16 * warp + 128 < nvalid) {
       const int kb2[2] = {16 * warp, 128 + 16 * warp};
-      mtile_scores<2>(kc, ks, nrm, rnm, kb2, qb, lo_reg, c0h, dmh, dsh, ssh, sc);
+      mtile_scores<2, true>(kc, ks, nrm, rnm, kb2, qb, lo_reg, c0h, dmh, dsh, ssh, sc);
     } else if (16 * warp < nvalid) {
       const int kb1[1] = {16 * warp};
       float sc1[1][2];
-      mtile_scores<1>(kc, ks, nrm, rnm, kb1, qb, lo_reg, c0h, dmh, dsh, ssh, sc1);
+      mtile_scores<1, true>(kc, ks, nrm, rnm, kb1, qb, lo_reg, c0h, dmh, dsh, ssh, sc1);
       sc[0][0] = sc1[0][0], sc[0][1] = sc1[0][1], sc[1][0] = sc[1][1] = 0.f;
     }
 #pragma unroll
@@ -861,7 +866,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
       for (int mt = 0; mt < 2; ++mt) {
         const int kb1[1] = {128 * mt + 16 * warp};
         float sc1[1][2];
-        mtile_scores<1>(st, st + kStageCodes, nrm, rnm, kb1, qb, lo_smem, c0h, dmh, dsh, ssh, sc1);
+        mtile_scores<1, false>(st, st + kStageCodes, nrm, rnm, kb1, qb, lo_smem, c0h, dmh, dsh, ssh, sc1);
         sc[mt][0] = sc1[0][0], sc[mt][1] = sc1[0][1];
       }
     }
