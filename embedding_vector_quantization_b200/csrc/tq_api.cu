@@ -38,6 +38,7 @@
 #include "score_attn_simt.cuh"
 #include "search_simt.cuh"
 #include "attn_mma.cuh"
+#include "attn_tc.cuh"
 #include "small_kernels.cuh"
 #include "encode_tc.cuh"
 #include "attn_mse4.cuh"
@@ -505,6 +506,22 @@ void attn_split(int B, int Hkv, int64_t L_cap, int* nsplit, int64_t* chunk) {
   *nsplit = (int)((L_cap + ch - 1) / ch);
 }
 
+// Split of the tcgen05 3-bit attention (one persistent CTA per SM): about one item
+// (sequence, KV head, chunk) per SM when the batch has fewer KV heads than SMs, chunks a
+// multiple of 128 tokens and at most 2048 tokens long (the logits of a chunk stay in
+// shared memory).
+void attn_tc_split(int B, int Hkv, int64_t L_cap, int sms, int* nsplit, int64_t* chunk) {
+  constexpr int64_t kMax = tqk::atc::kMaxChunk;
+  const int64_t units = std::max<int64_t>(1, (int64_t)B * Hkv);
+  const int64_t per = std::max<int64_t>(1, sms / units);
+  const int64_t ns = std::max<int64_t>(per, (L_cap + kMax - 1) / kMax);
+  int64_t ch = (L_cap + ns - 1) / ns;
+  ch = std::min<int64_t>(kMax, std::max<int64_t>(128, (ch + 127) / 128 * 128));
+  if (const int64_t f = splitk_override()) ch = round_chunk(f, 128, 128, kMax);
+  *chunk = ch;
+  *nsplit = (int)((L_cap + ch - 1) / ch);
+}
+
 void search_split(int nq, int64_t n, int* nchunks, int64_t* chunk) {
   const int64_t qt = (nq + tqk::kSQ - 1) / tqk::kSQ;
   int64_t nc = (2 * 148 + qt - 1) / qt;
@@ -644,13 +661,15 @@ size_t score_ws_layout(const tq_handle* h, int rows, char* base, ScoreWs* w) {
 size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, int Hkv, int64_t L_cap,
                       char* base, ScoreWs* w, float** part, int* nsplit, int64_t* chunk) {
   size_t off = score_ws_layout(hk, B * Hq, base, w);
-  int ns;
-  int64_t ch;
+  int ns, ns_tc;
+  int64_t ch, ch_tc;
   attn_split(B, Hkv, L_cap, &ns, &ch);
   if (nsplit) *nsplit = ns;
   if (chunk) *chunk = ch;
   if (part) *part = reinterpret_cast<float*>(base + off);
-  off += round_up((size_t)B * Hq * ns * tqk::partial_stride(hv->d, hv->m) * 4, 256);
+  // room for the partials of either split (the tcgen05 3-bit kernel has its own)
+  attn_tc_split(B, Hkv, L_cap, sm_count(hk->device), &ns_tc, &ch_tc);
+  off += round_up((size_t)B * Hq * std::max(ns, ns_tc) * tqk::partial_stride(hv->d, hv->m) * 4, 256);
   return off;
 }
 
@@ -1321,6 +1340,14 @@ int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dty
   const int G = Hq / Hkv;
   if (attn_prod2_fast_path(hk, hv, G, k, v)) {
     tqk::amma::Args m{};
+    // TQ_ATTN_TC=1: the tcgen05 kernel (attn_tc.cuh), measured slower than this mma.sync one at
+    // these shapes (each of its small MMAs costs the tensor pipe about as much as a full-width one)
+    const char* tce = std::getenv("TQ_ATTN_TC");
+    const bool tc = tce && *tce && *tce != '0';
+    if (tc) {
+      const int sms = sm_count(hk->device);
+      attn_tc_split(B, Hkv, k->L_cap, sms, &nsplit, &chunk);
+    }
     m.qr = w.qr; m.qs = w.qs; m.B = B; m.Hq = Hq; m.Hkv = Hkv;
     m.kcodes = k->codes; m.ksigns = k->signs; m.knorm = static_cast<const __half*>(k->norms);
     m.krn = static_cast<const __half*>(k->rnorms);
@@ -1330,6 +1357,21 @@ int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dty
     m.kc0 = (float)hk->cent[0]; m.kb0 = (float)(hk->cent[1] - hk->cent[0]); m.kb1 = (float)(hk->cent[2] - hk->cent[0]);
     m.vc0 = (float)hv->cent[0]; m.vb0 = (float)(hv->cent[1] - hv->cent[0]); m.vb1 = (float)(hv->cent[2] - hv->cent[0]);
     m.scale = scale; m.part = part; m.err = hk->derr;
+    m.prefetch_ahead = tc ? 0 : 2 * sm_count(hk->device);   // two CTAs per SM
+    if (tc) {
+      const int nitems = B * Hkv * nsplit;
+      const int grid = std::max(1, std::min(nitems, sm_count(hk->device)));
+      if (once_per_device(12, hk->device))
+        cudaFuncSetAttribute(tqk::atc::attn_prod2_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             (int)tqk::atc::kSmemBytes);
+      {
+        KernelScope ks("attn_split", s);
+        const cudaError_t e = launch_pdl(tqk::atc::attn_prod2_tc_kernel, dim3((unsigned)grid),
+                                         dim3(tqk::atc::kThreads), (size_t)tqk::atc::kSmemBytes, s, m, nitems);
+        if (e != cudaSuccess) return cuda_fail(e, "attn_prod2_tc_kernel");
+      }
+      if ((st = launch_check("attn_prod2_tc_kernel"))) return st;
+    } else {
     const size_t msmem = sizeof(tqk::amma::Smem);
     if (once_per_device(2, hk->device)) {
       cudaFuncSetAttribute(tqk::amma::attn_prod2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
@@ -1342,6 +1384,7 @@ int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dty
       if (e != cudaSuccess) return cuda_fail(e, "attn_prod2_kernel");
     }
     if ((st = launch_check("attn_prod2_kernel"))) return st;
+    }
   } else if (attn_mse4_fast_path(hk, hv, G, k, v)) {
     tqk::am4::Args m4{};
     m4.qr = w.qr; m4.B = B; m4.Hq = Hq; m4.Hkv = Hkv;
@@ -1351,6 +1394,7 @@ int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dty
     plane_coeffs4(hk->cent, &m4.kc0, m4.kw);
     plane_coeffs4(hv->cent, &m4.vc0, m4.vw);
     m4.scale = scale; m4.part = part; m4.err = hk->derr;
+    m4.prefetch_ahead = 2 * sm_count(hk->device);
     const size_t msmem = sizeof(tqk::am4::Smem);
     if (once_per_device(11, hk->device)) {
       cudaFuncSetAttribute(tqk::am4::attn_mse4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
