@@ -90,8 +90,6 @@ struct Args {
   float scale;          // softmax scale
   float* part;          // [B*Hq][nsplit][d + m + 2]
   int* err;
-  int prefetch_ahead;   // CTAs resident at once: each CTA asks the L2 for the chunk of the CTA that
-                        // many places after it in launch order (0: none)
 };
 
 // Key-pass data of the chunk; after the key pass its codes and signs are dead and hold the
@@ -438,35 +436,6 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
   const bool holds_new = a.len_extra && slot >= start && slot < end;
   const int s_loc = holds_new ? (int)(slot - start) : -1, s_blk = holds_new ? s_loc / kBlk : -1;
   issue_all();
-  // The CTA one wave later in launch order will most likely run on this SM's slot next: its chunk
-  // is requested into L2 now, so that its copies hit L2 and the cold read streams without gaps
-  // between waves.
-  if (a.prefetch_ahead > 0 && warp == 0 && lane < 8) {
-    const int64_t c2 = (int64_t)blockIdx.y * gridDim.x + blockIdx.x + a.prefetch_ahead;
-    if (c2 < (int64_t)gridDim.x * gridDim.y) {
-      const int bh2 = (int)(c2 % gridDim.x), split2 = (int)(c2 / gridDim.x), b2 = bh2 / a.Hkv;
-      const int64_t L2 = min((int64_t)max(a.len[b2], 0) + a.len_extra, a.L_cap);
-      const int64_t st2 = (int64_t)split2 * a.chunk;
-      const int64_t n2 = min(L2, st2 + a.chunk) - st2;
-      if (n2 > 0) {
-        const int64_t r2 = (int64_t)bh2 * a.L_cap + st2;
-        const uint32_t n = (uint32_t)n2, n8 = (n + 7u) & ~7u;
-        const void* p = nullptr;
-        uint32_t nb = n8 * 2u;   // the four norm rows (whole 8-token groups)
-        switch (lane) {
-          case 0: p = a.kcodes + r2 * kCodesB; nb = n * kCodesB; break;
-          case 1: p = a.ksigns + r2 * kSignsB; nb = n * kSignsB; break;
-          case 2: p = a.knorm + r2; break;
-          case 3: p = a.krn + r2; break;
-          case 4: p = a.vnorm + r2; break;
-          case 5: p = a.vrn + r2; break;
-          case 6: p = a.vcodes + r2 * kCodesB; nb = n * kCodesB; break;
-          default: p = a.vsigns + r2 * kSignsB; nb = n * kSignsB; break;
-        }
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(nb) : "memory");
-      }
-    }
-  }
   grid_dep_wait();
   // this token's rows as the previous kernel wrote them (key side: codes, signs, the four norms;
   // value side: codes, signs); called with the block's data resident, followed by a CTA barrier

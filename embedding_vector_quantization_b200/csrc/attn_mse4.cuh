@@ -70,7 +70,6 @@ struct Args {
   float scale;
   float* part;             // [B*Hq][nsplit][partial_stride(128, 0)]
   int* err;
-  int prefetch_ahead;      // CTAs resident at once (0: no prefetch of a later CTA's chunk)
 };
 
 struct __align__(16) Smem {
@@ -287,31 +286,6 @@ __global__ void __launch_bounds__(kThreads, 2) attn_mse4_kernel(Args a) {
   };
   const int njobs = 2 * nblk;
   constexpr int kAhead = kStages - 2;
-  // The ring keeps only kAhead blocks in flight, so the whole chunk (lanes 0-3) and the chunk of
-  // the CTA one wave later in launch order (lanes 4-7) are requested into L2 at launch: the cold
-  // read streams at full rate and the ring's copies hit L2.
-  if (warp == 0 && lane < 8) {
-    const int64_t c2 = (int64_t)blockIdx.y * gridDim.x + blockIdx.x + (lane >= 4 ? a.prefetch_ahead : 0);
-    if ((lane < 4 || a.prefetch_ahead > 0) && c2 < (int64_t)gridDim.x * gridDim.y) {
-      const int bh2 = (int)(c2 % gridDim.x), split2 = (int)(c2 / gridDim.x), b2 = bh2 / a.Hkv;
-      const int64_t L2 = min((int64_t)max(a.len[b2], 0) + a.len_extra, a.L_cap);
-      const int64_t st2 = (int64_t)split2 * a.chunk;
-      const int64_t n2 = min(L2, st2 + a.chunk) - st2;
-      if (n2 > 0) {
-        const int64_t r2 = (int64_t)bh2 * a.L_cap + st2;
-        const uint32_t n = (uint32_t)n2, n8 = (n + 7u) & ~7u;   // whole 8-token groups of the norm rows
-        const void* p;
-        uint32_t nb;
-        switch (lane & 3) {
-          case 0: p = a.kcodes + r2 * kCodesB; nb = n * kCodesB; break;
-          case 1: p = a.knorm + r2; nb = n8 * 2u; break;
-          case 2: p = a.vcodes + r2 * kCodesB; nb = n * kCodesB; break;
-          default: p = a.vnorm + r2; nb = n8 * 2u; break;
-        }
-        asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;\n" ::"l"(p), "r"(nb) : "memory");
-      }
-    }
-  }
   grid_dep_launch();
   // in a decode step the kernel before this one writes only slot len[b] and the queries
   const int64_t slot = (int64_t)max(a.len[b], 0);

@@ -1357,7 +1357,6 @@ int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dty
     m.kc0 = (float)hk->cent[0]; m.kb0 = (float)(hk->cent[1] - hk->cent[0]); m.kb1 = (float)(hk->cent[2] - hk->cent[0]);
     m.vc0 = (float)hv->cent[0]; m.vb0 = (float)(hv->cent[1] - hv->cent[0]); m.vb1 = (float)(hv->cent[2] - hv->cent[0]);
     m.scale = scale; m.part = part; m.err = hk->derr;
-    m.prefetch_ahead = tc ? 0 : 2 * sm_count(hk->device);   // two CTAs per SM
     if (tc) {
       const int nitems = B * Hkv * nsplit;
       const int grid = std::max(1, std::min(nitems, sm_count(hk->device)));
@@ -1394,7 +1393,6 @@ int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dty
     plane_coeffs4(hk->cent, &m4.kc0, m4.kw);
     plane_coeffs4(hv->cent, &m4.vc0, m4.vw);
     m4.scale = scale; m4.part = part; m4.err = hk->derr;
-    m4.prefetch_ahead = 2 * sm_count(hk->device);
     const size_t msmem = sizeof(tqk::am4::Smem);
     if (once_per_device(11, hk->device)) {
       cudaFuncSetAttribute(tqk::am4::attn_mse4_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
