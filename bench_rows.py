@@ -860,6 +860,30 @@ def run_cfg1(args):
                          "max_score_error_on_gpu_codes_rel_to_floor": float(np.max(np.abs(scores - sg) / floor)),
                          "max_abs_score_difference_end_to_end": float(np.max(np.abs(scores - so))),
                          "oracle_seconds": el, "kind": "oracle", "cores": bench.blas_threads()}
+        # the same keys through the 3-bit prod encode (2-bit codes + 128 QJL signs, fp16 norms; the
+        # tensor-core encode at d = 128): index and sign mismatch fractions against the oracle's
+        # encode. An index may differ only within 1e-5 of a boundary, a sign only for a projection
+        # within 1e-5 ||x|| of zero (or in a row whose index differs, which moves the residual).
+        hp = tq.Handle(d, 3, 0, qjl_m=128)
+        pc = tq.Cache(hp, 1, 1, n)
+        pc.fill(xg.view(1, 1, n, d))
+        torch.cuda.synchronize()
+        pidx = _unpack_rows(pc.codes.cpu().numpy().reshape(n, -1), d, 2)
+        psig = np.unpackbits(pc.signs.cpu().numpy().reshape(n, -1), axis=1, bitorder="little")[:, :128]
+        Pip, Sp = rotation.rotation(d, 0, 128)
+        cp_, bp_ = codebook.lloyd_max(d, 2)
+        ep = quant.encode_prod(xd, Pip, Sp, cp_, bp_, "f16")
+        imis = pidx != ep["idx"]
+        inear = (np.abs(ep["y"][imis] - bp_[np.minimum(pidx[imis], ep["idx"][imis])])
+                 if imis.any() else np.zeros(0))
+        smis = psig.astype(np.int64) != ep["sigma"]
+        smis[np.any(imis, axis=1)] = False
+        r_, j_ = np.nonzero(smis)
+        snear = np.abs(ep["z"][r_, j_]) < 1e-5 * ep["n_exact"][r_]
+        rec["oracle"]["prod_3bit"] = {"index_mismatch_fraction": float(imis.mean()),
+                                      "index_mismatches_within_1e-5_of_a_boundary": bool(np.all(inear < 1e-5)),
+                                      "sign_mismatch_fraction": float(smis.mean()),
+                                      "sign_mismatches_within_1e-5_of_zero": bool(np.all(snear))}
     if COLLECT is not None:
         COLLECT.append({"metric": "cfg1", "record": rec})
     else:
