@@ -754,11 +754,11 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 // The key pass above on its own: raw scores s = ||k|| <q', c[idx]> + rnorm sqrt(pi/2)/m
 // <S q, 2 sigma - 1> of every key of the chunk for the 4 query heads of a KV head,
 // written to logits [B][Hq][L_cap] ("TurboQuant: redefining AI efficiency", "QJL";
-// "Google TurboQuant", "Stage 2"). Key blocks of 256 stream through a 4-stage TMA ring;
+// "Google TurboQuant", "Stage 2"). Key blocks of 256 stream through a 5-stage TMA ring;
 // every thread stores its scores directly: per store instruction a warp writes 8
 // consecutive keys of each of the 4 heads, i.e. whole 32-byte sectors.
 
-constexpr int kSStages = 4;
+constexpr int kSStages = 5;   // 5 x 13 KB: three CTAs still fit an SM, three blocks in flight per CTA
 constexpr int kSStageBytes = kStageCodes + kStageSigns + 2 * kBlk * 2;  // codes, signs, norms, rnorms: 13312
 
 struct ScoreArgs {

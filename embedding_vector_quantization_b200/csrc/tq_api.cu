@@ -1268,8 +1268,10 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const 
     m.kc0 = (float)hk->cent[0]; m.kb0 = (float)(hk->cent[1] - hk->cent[0]); m.kb1 = (float)(hk->cent[2] - hk->cent[0]);
     m.logits = logits; m.err = hk->derr;
     const size_t msmem = sizeof(tqk::amma::ScoreSmem);
-    if (once_per_device(10, hk->device))
+    if (once_per_device(10, hk->device)) {
       cudaFuncSetAttribute(tqk::amma::score_prod2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+      cudaFuncSetAttribute(tqk::amma::score_prod2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    }
     KernelScope ks("score", s);
     const cudaError_t e = launch_pdl(tqk::amma::score_prod2_kernel, dim3((unsigned)units, (unsigned)nsp),
                                      dim3(tqk::amma::kThreads), msmem, s, m);

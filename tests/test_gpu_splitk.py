@@ -8,7 +8,7 @@ two blocks, so the ring never wraps. Here every kernel runs chunks of several bl
   heads, context 32768: 37 chunks of 896 tokens, each staged whole as 4 key and 4 value
   blocks with one barrier each), plus a ragged length and forced 512-token chunks;
 * attn_mse4_kernel with 896-token chunks (4 + 4 blocks on its 4-stage ring);
-* score_prod2_kernel with 5- and 10-block chunks on its 4-stage ring (TQ_SPLITK);
+* score_prod2_kernel with 4-, 5- and 10-block chunks on its 5-stage ring (TQ_SPLITK);
 * search_tc_kernel with 3 to 12 tiles of 256 vectors per chunk.
 
 Caches hold the oracle's codes ("Google TurboQuant: 6x KV-cache compression", "Stage 1"
@@ -180,8 +180,8 @@ def test_attn_mse4_multiblock_chunks_match_oracle(tq, lens, force):
 
 @pytest.mark.parametrize("force,lens", [(2560, [8192, 6001]), (1280, [8192, 2561]), (1024, [8192, 7937])])
 def test_score_prod2_ring_wraps(tq, force, lens):
-    """score_prod2_kernel with chunks of 10, 5 and 4 blocks of 256 keys (its TMA ring has 4
-    stages), ragged lengths; the untouched tail stays zero."""
+    """score_prod2_kernel with chunks of 10, 5 and 4 blocks of 256 keys (its TMA ring has 5
+    stages, 3 blocks in flight), ragged lengths; the untouched tail stays zero."""
     B, Hkv, G, L, d = 2, 8, 4, 8192, 128
     h = tq.Handle(d, 3, 21, qjl_m=128)
     oh = OracleHandle(d, 2, 21, 128)
