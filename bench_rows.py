@@ -325,7 +325,11 @@ def run_attn3big(args):
         S5A["B"] = 8        # 109 MB of packed K/V
     hk = tq.Handle(S5A["d"], S5A["bits"], 0, qjl_m=S5A["m"])
     hv = tq.Handle(S5A["d"], S5A["bits"], 1, qjl_m=S5A["m"])
-    spec = dict(S5A, bytes_per_token=2 * (32 + 16 + 2 + 2), kernel="attn_prod2_kernel", scaled=False,
+    # caches of 256 MB and more take the two-kernel form (scores, then values; timed together)
+    two = S5A["B"] * S5A["Hkv"] * S5A["L"] * 104 >= 256e6 and os.environ.get("TQ_ATTN_2K", "") != "0"
+    spec = dict(S5A, bytes_per_token=2 * (32 + 16 + 2 + 2),
+                kernel="score_prod2_kernel<true> + value_prod2_kernel" if two else "attn_prod2_kernel",
+                scaled=False,
                 workload="GQA decode step, TurboQuant prod 3-bit (2-bit Lloyd-Max + 1-bit QJL m=128), d=128, "
                          "B=%d, 8 KV heads / 32 query heads, context 16384, bf16 K/V N(0,1)" % S5A["B"],
                 dtype="s8xs8->s32 MMA (22-bit fixed-point queries), u8xu8->s32 MMA (16-bit weights), "

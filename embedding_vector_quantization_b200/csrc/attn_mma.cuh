@@ -771,6 +771,7 @@ struct ScoreArgs {
   const __half* krn;
   int64_t L_cap, chunk;
   const int32_t* len;
+  int len_extra;    // 1 inside a decode step: the key appended at slot len[b] by the kernel before counts
   float kc0, kb0, kb1;
   float* logits;    // [B][Hq][L_cap]
   int* err;
@@ -785,6 +786,8 @@ struct __align__(16) ScoreSmem {
   int abort_flag;
 };
 
+// LO: 22-bit code-side queries (the attention's logits), else 15-bit (raw scores).
+template <bool LO>
 __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
   ScoreSmem& sm = *reinterpret_cast<ScoreSmem*>(smem_raw);
@@ -792,13 +795,17 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
   const int g = lane >> 2, t = lane & 3;
   const int bh = blockIdx.x, split = blockIdx.y;
   const int b = bh / a.Hkv, hk = bh % a.Hkv, h0 = hk * kG;
-  const int64_t L = min((int64_t)max(a.len[b], 0), a.L_cap);
+  const int64_t L = min((int64_t)max(a.len[b], 0) + a.len_extra, a.L_cap);
   const int64_t start = (int64_t)split * a.chunk;
   const int64_t end = min(L, start + a.chunk);
   const int ntok = (int)max((int64_t)0, end - start);
   const int nblk = (ntok + kBlk - 1) / kBlk;
   const int64_t row0 = (int64_t)bh * a.L_cap + start;
   if (nblk == 0) return;
+  // inside a decode step the kernel before this one writes slot len[b]; copies issued before the
+  // wait below may hold that key's old rows, so the one warp that scores it reads them again
+  const int64_t slot = (int64_t)max(a.len[b], 0);
+  const int s_loc = (a.len_extra && slot >= start && slot < end) ? (int)(slot - start) : -1;
 
   if (tid == 0) {
     for (int s = 0; s < kSStages; ++s) {
@@ -857,6 +864,22 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
     }
     if (!aborted && !mbar_wait(&sm.full[j % kSStages], (j / kSStages) & 1)) sm.abort_flag = 1;
     const unsigned char* st = sm.stage[j % kSStages];
+    if (!aborted && s_loc >= 0 && s_loc / kBlk == j && warp == ((s_loc % kBlk) % 128) / 16) {
+      // the warp whose m-tiles hold the appended key (rows 16w.. and 128 + 16w..) patches its rows
+      const int kk = s_loc & (kBlk - 1);
+      const int64_t r = row0 + s_loc;
+      unsigned char* sw = sm.stage[j % kSStages];
+      if (lane < 8)
+        reinterpret_cast<uint32_t*>(sw + kk * kCodesB)[lane] = __ldcg(reinterpret_cast<const uint32_t*>(a.kcodes + r * kCodesB) + lane);
+      else if (lane < 12)
+        reinterpret_cast<uint32_t*>(sw + kStageCodes + kk * kSignsB)[lane - 8] =
+            __ldcg(reinterpret_cast<const uint32_t*>(a.ksigns + r * kSignsB) + lane - 8);
+      else if (lane == 12)
+        reinterpret_cast<__half*>(sw + kStageCodes + kStageSigns)[kk] = __ldcg(a.knorm + r);
+      else if (lane == 13)
+        reinterpret_cast<__half*>(sw + kStageCodes + kStageSigns)[kBlk + kk] = __ldcg(a.krn + r);
+      __syncwarp();
+    }
     const __half* nrm = reinterpret_cast<const __half*>(st + kStageCodes + kStageSigns);
     const __half* rnm = nrm + kBlk;
     const int tb = j * kBlk, nvalid = min(kBlk, ntok - tb);
@@ -866,7 +889,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
       for (int mt = 0; mt < 2; ++mt) {
         const int kb1[1] = {128 * mt + 16 * warp};
         float sc1[1][2];
-        mtile_scores<1, false>(st, st + kStageCodes, nrm, rnm, kb1, qb, lo_smem, c0h, dmh, dsh, ssh, sc1);
+        mtile_scores<1, LO>(st, st + kStageCodes, nrm, rnm, kb1, qb, lo_smem, c0h, dmh, dsh, ssh, sc1);
         sc[mt][0] = sc1[0][0], sc[mt][1] = sc1[0][1];
       }
     }
@@ -886,6 +909,303 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
   if (sm.abort_flag && tid == 0) {
     report_error(a.err, kErrTimeout);
     for (int jx = max(0, issued - kSStages); jx < issued; ++jx) (void)mbar_wait(&sm.full[jx % kSStages], (jx / kSStages) & 1);
+  }
+}
+
+
+// ================================================================ value pass over stored scores
+//
+// The second half of a two-kernel form of attn_prod2_kernel for caches much larger than L2: the
+// score kernel above (22-bit queries, the same logits as the fused kernel's key pass) writes every
+// key's raw score, and this kernel turns a chunk's scores into the same 16-bit integer weights
+// (against each head's largest p ||v|| and p rnorm in the chunk) and runs the same value pass over
+// value blocks streamed through a TMA ring, writing the same partial results. Both halves stream
+// through small rings with three CTAs per SM, which keeps more of the cold read in flight than the
+// fused kernel's whole-chunk staging (two CTAs per SM).
+struct VArgs {
+  const float* logits;  // [B][Hq][L_cap] raw scores (score_prod2_kernel<true>)
+  int B, Hq, Hkv;
+  const uint8_t* vcodes;
+  const uint8_t* vsigns;
+  const __half* vnorm;
+  const __half* vrn;
+  int64_t L_cap, chunk;
+  int nsplit;
+  const int32_t* len;
+  int len_extra;
+  float vc0, vb0, vb1;  // V codebook
+  float scale;
+  float* part;          // [B*Hq][nsplit][d + m + 2]
+  int* err;
+};
+
+constexpr int kVStages = 4;
+constexpr int kVStageBytes = kStageCodes + kStageSigns;   // 12288
+constexpr int kVAhead = kVStages - 2;
+
+struct __align__(16) VSmem {
+  unsigned char stage[kVStages][kVStageBytes];
+  uint8_t pw[2][2][8][kPwRow];   // [buffer][0: value weights, 1: QJL weights][col = head*2+piece][token]
+  float vacc[3][kG][128];
+  float red[kWarps][3][kG];
+  int red_i[kWarps][2 * kG];
+  float hmax[kG];
+  float dv[2][kG];
+  float inv[2][kG];
+  int W[2][kG];
+  uint64_t full[kVStages];
+  uint64_t empty[kVStages];
+  int abort_flag;
+};
+
+__global__ void __launch_bounds__(kThreads, 3) value_prod2_kernel(VArgs a) {
+  extern __shared__ __align__(128) unsigned char smem_raw[];
+  VSmem& sm = *reinterpret_cast<VSmem*>(smem_raw);
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int g = lane >> 2, t = lane & 3;
+  const int bh = blockIdx.x, split = blockIdx.y;
+  const int b = bh / a.Hkv, hk = bh % a.Hkv, h0 = hk * kG;
+  // the scores and, in a decode step, the appended value come from the kernels before this one
+  // (which this one starts after: the score kernel triggers nothing early)
+  grid_dep_wait();
+  const int64_t L = min((int64_t)max(a.len[b], 0) + a.len_extra, a.L_cap);
+  const int64_t start = (int64_t)split * a.chunk;
+  const int64_t end = min(L, start + a.chunk);
+  const int ntok = (int)max((int64_t)0, end - start);
+  const int nblk = (ntok + kBlk - 1) / kBlk;
+  const int64_t row0 = (int64_t)bh * a.L_cap + start;
+  const int stride = partial_stride(kD, kM);
+  if (ntok == 0) {   // an empty chunk: zero sums, max -inf
+    for (int i = tid; i < kG * stride; i += kThreads) {
+      const int h = i / stride, j = i - h * stride;
+      a.part[(((size_t)b * a.Hq + h0 + h) * a.nsplit + split) * stride + j] = (j == kD + kM) ? -INFINITY : 0.f;
+    }
+    return;
+  }
+  if (tid == 0) {
+    for (int s = 0; s < kVStages; ++s) {
+      mbar_init(&sm.full[s], 1);
+      mbar_init(&sm.empty[s], kWarps);
+    }
+    sm.abort_flag = 0;
+    asm volatile("fence.mbarrier_init.release.cluster;\n" ::: "memory");
+  }
+  __syncthreads();
+  auto issue = [&](int j) {
+    const int64_t tok0 = (int64_t)j * kBlk;
+    const int ncopy = (int)min((int64_t)kBlk, a.L_cap - (start + tok0));   // multiple of 8 (L_cap % 8 == 0)
+    const int64_t r = row0 + tok0;
+    unsigned char* st = sm.stage[j % kVStages];
+    uint64_t* bar = &sm.full[j % kVStages];
+    mbar_expect_tx(bar, (uint32_t)ncopy * (kCodesB + kSignsB));
+    tma_bulk_g2s(st, a.vcodes + r * kCodesB, ncopy * kCodesB, bar);
+    tma_bulk_g2s(st + kStageCodes, a.vsigns + r * kSignsB, ncopy * kSignsB, bar);
+  };
+  if (tid == 0)
+    for (int j = 0; j < min(kVAhead, nblk); ++j) issue(j);
+  int issued = min(kVAhead, nblk);
+
+  // ---- per head over the chunk: the largest l, l + log2 ||v|| and l + log2 rnorm (l = the score
+  // in log2 units), so that the weight steps max p ||v|| / 65535 and max p rnorm / 65535 are known
+  // before the first value block
+  const float scale2 = a.scale * 1.4426950408889634f;
+  const float* lg = a.logits + ((size_t)b * a.Hq + h0) * a.L_cap + start;   // head h: lg + h * L_cap
+  {
+    const int h = t;
+    float m = -INFINITY, m1 = -INFINITY, m2 = -INFINITY;
+    for (int tok = tid >> 2; tok < ntok; tok += kThreads / 4) {
+      const float l = lg[(size_t)h * a.L_cap + tok] * scale2;
+      const float vn = __half2float(a.vnorm[row0 + tok]), vr = __half2float(a.vrn[row0 + tok]);
+      m = fmaxf(m, l);
+      m1 = fmaxf(m1, l + __log2f(vn));
+      m2 = fmaxf(m2, l + __log2f(vr));
+    }
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, o));
+      m1 = fmaxf(m1, __shfl_xor_sync(0xffffffffu, m1, o));
+      m2 = fmaxf(m2, __shfl_xor_sync(0xffffffffu, m2, o));
+    }
+    if (g == 0) sm.red[warp][0][h] = m, sm.red[warp][1][h] = m1, sm.red[warp][2][h] = m2;
+  }
+  __syncthreads();
+  if (tid < kG) {
+    float m = -INFINITY, m1 = -INFINITY, m2 = -INFINITY;
+    for (int w = 0; w < kWarps; ++w) {
+      m = fmaxf(m, sm.red[w][0][tid]);
+      m1 = fmaxf(m1, sm.red[w][1][tid]);
+      m2 = fmaxf(m2, sm.red[w][2][tid]);
+    }
+    sm.hmax[tid] = m;
+    const float s1 = exp2f(m1 - m) / 65535.f, s2 = exp2f(m2 - m) / 65535.f;
+    sm.dv[0][tid] = s1 > 0.f ? s1 : 1.f;
+    sm.inv[0][tid] = s1 > 0.f ? 1.f / s1 : 0.f;
+    sm.dv[1][tid] = s2 > 0.f ? s2 : 1.f;
+    sm.inv[1][tid] = s2 > 0.f ? 1.f / s2 : 0.f;
+  }
+  __syncthreads();
+  // ---- value blocks: weights of the block (all threads) into one of two weight buffers, then
+  // the value MMAs (warps 0..5: three byte groups x two token halves), exactly as in the fused kernel
+  const int h = tid & 3, q4 = (tid >> 2) * 4;
+  const float hm = sm.hmax[h], inv1 = sm.inv[0][h], inv2 = sm.inv[1][h];
+  // round to nearest (even) through the float adder (0 <= x < 2^22)
+  auto to_int = [](float x) { return __float_as_int(x + 12582912.f) - 0x4B400000; };
+  float lsum = 0.f;
+  int wsum[2] = {0, 0};
+  int vacc[8][4];
+#pragma unroll
+  for (int u = 0; u < 8; ++u) vacc[u][0] = vacc[u][1] = vacc[u][2] = vacc[u][3] = 0;
+  const int bg = warp % 3, half = warp / 3;
+  for (int jj = 0; jj < nblk; ++jj) {
+    const bool aborted = __syncthreads_or(*(volatile int*)&sm.abort_flag != 0);   // uniform decision
+    if (aborted) break;
+    if (tid == 0 && jj + kVAhead < nblk) {
+      const int jo = jj + kVAhead - kVStages;   // the stage's previous block
+      if (jo >= 0 && !mbar_wait(&sm.empty[jo % kVStages], (jo / kVStages) & 1)) {
+        sm.abort_flag = 1;
+      } else {
+        issue(jj + kVAhead);
+        issued = jj + kVAhead + 1;
+      }
+    }
+    {
+      const int tb = jj * kBlk, nval = min(kBlk, ntok - tb);
+      uint32_t w1h = 0, w1l = 0, w2h = 0, w2l = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        const int tok = tb + q4 + q;
+        if (q4 + q < nval) {   // tokens past the chunk's end get zero weight
+          const float l = lg[(size_t)h * a.L_cap + tok] * scale2;
+          const float pp = exp2_approx(l - hm);
+          lsum += pp;
+          const float vn = __half2float(a.vnorm[row0 + tok]), vr = __half2float(a.vrn[row0 + tok]);
+          const int w1 = min(to_int(pp * vn * inv1), 65535), w2 = min(to_int(pp * vr * inv2), 65535);
+          w1h |= (uint32_t)(w1 >> 8) << (8 * q);
+          w1l |= (uint32_t)(w1 & 255) << (8 * q);
+          w2h |= (uint32_t)(w2 >> 8) << (8 * q);
+          w2l |= (uint32_t)(w2 & 255) << (8 * q);
+          wsum[0] += w1;
+          wsum[1] += w2;
+        }
+      }
+      uint8_t* blk = &sm.pw[jj & 1][0][0][0];
+      *reinterpret_cast<uint32_t*>(blk + (2 * h) * kPwRow + q4) = w1h;
+      *reinterpret_cast<uint32_t*>(blk + (2 * h + 1) * kPwRow + q4) = w1l;
+      *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h) * kPwRow + q4) = w2h;
+      *reinterpret_cast<uint32_t*>(blk + (8 + 2 * h + 1) * kPwRow + q4) = w2l;
+    }
+    bool ok = true;
+    if (warp < 6 && !mbar_wait(&sm.full[jj % kVStages], (jj / kVStages) & 1)) ok = false;
+    if (!ok && lane == 0) sm.abort_flag = 1;
+    __syncthreads();   // the block's weights are written (and the previous block's MMAs are done)
+    if (warp < 6 && __all_sync(0xffffffffu, ok)) {
+      const uint8_t* pw = &sm.pw[jj & 1][bg == 2 ? 1 : 0][0][0];
+      const unsigned char* vc = sm.stage[jj % kVStages];
+      const unsigned char* vs = vc + kStageCodes;
+      const int nvalv = min(kBlk, ntok - jj * kBlk);
+#pragma unroll
+      for (int kq = 0; kq < 4; ++kq) {
+        const int tk = 128 * half + 32 * kq;  // first token of this 32-token k-step
+        if (tk >= nvalv) break;               // past the chunk's end (weights 0; warp-uniform)
+        uint32_t r[4];
+        const int tok = tk + (lane & 15) + 16 * (lane >> 4);
+        const unsigned char* rowp = (bg < 2) ? vc + tok * kCodesB + 16 * bg : vs + tok * kSignsB;
+        ldsm_t8_x2(r, rowp);
+        const uint32_t b0 = *reinterpret_cast<const uint32_t*>(pw + g * kPwRow + tk + 4 * t);
+        const uint32_t b1 = *reinterpret_cast<const uint32_t*>(pw + g * kPwRow + tk + 16 + 4 * t);
+#pragma unroll
+        for (int s4 = 0; s4 < 4; ++s4) {
+          const uint32_t x0 = r[0] >> s4, x1 = r[1] >> s4, x2 = r[2] >> s4, x3 = r[3] >> s4;
+          mma_u8(vacc[s4], x0 & 0x01010101u, x1 & 0x01010101u, x2 & 0x01010101u, x3 & 0x01010101u, b0, b1);
+          mma_u8(vacc[4 + s4], x0 & 0x10101010u, x1 & 0x10101010u, x2 & 0x10101010u, x3 & 0x10101010u, b0, b1);
+        }
+      }
+    }
+    __syncwarp();
+    if (lane == 0) asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];\n" ::"r"(smem_u32(&sm.empty[jj % kVStages])) : "memory");
+  }
+
+  __syncthreads();
+  if (sm.abort_flag) {
+    // a copy never completed: record it, then wait (bounded) for the copies that may still be in
+    // flight into this CTA's shared memory before leaving
+    if (tid == 0) {
+      report_error(a.err, kErrTimeout);
+      for (int jx = max(0, issued - kVStages); jx < issued; ++jx)
+        (void)mbar_wait(&sm.full[jx % kVStages], (jx / kVStages) & 1);
+    }
+    __syncthreads();
+    return;
+  }
+
+  // ---- sums of p and integer weights per head, value sums of the two token halves
+  {
+    float l = lsum;
+    int w1 = wsum[0], w2 = wsum[1];
+#pragma unroll
+    for (int o = 4; o < 32; o <<= 1) {
+      l += __shfl_xor_sync(0xffffffffu, l, o);
+      w1 += __shfl_xor_sync(0xffffffffu, w1, o);
+      w2 += __shfl_xor_sync(0xffffffffu, w2, o);
+    }
+    if (lane < kG) {
+      sm.red[warp][0][lane] = l;
+      sm.red_i[warp][lane] = w1;
+      sm.red_i[warp][kG + lane] = w2;
+    }
+  }
+  if (warp >= 3 && warp < 6) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int f = (u < 4) ? 0 : 4;
+      const float v0 = 256.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
+      const float v1 = 256.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
+      sm.vacc[bg][t][g * 8 + u] = v0;          // byte g, bit u
+      sm.vacc[bg][t][64 + g * 8 + u] = v1;     // byte g + 8, bit u
+    }
+  }
+  __syncthreads();
+  if (warp < 3) {
+#pragma unroll
+    for (int u = 0; u < 8; ++u) {
+      const int f = (u < 4) ? 0 : 4;
+      const float v0 = 256.f * (float)(vacc[u][0] >> f) + (float)(vacc[u][1] >> f);
+      const float v1 = 256.f * (float)(vacc[u][2] >> f) + (float)(vacc[u][3] >> f);
+      sm.vacc[bg][t][g * 8 + u] += v0;
+      sm.vacc[bg][t][64 + g * 8 + u] += v1;
+    }
+  }
+  if (tid < 2 * kG) {
+    int W = 0;
+    for (int w = 0; w < kWarps; ++w) W += sm.red_i[w][tid];
+    sm.W[tid / kG][tid % kG] = W;
+  }
+  __syncthreads();
+
+  // ---- partial outputs: rotated-domain value sum, QJL sum, max (natural-log units), sum of p
+  for (int i = tid; i < kG * (kD + kM); i += kThreads) {
+    const int hh = i / (kD + kM), j = i % (kD + kM);
+    const int W1 = sm.W[0][hh], W2 = sm.W[1][hh];
+    float v;
+    if (j < kD) {
+      // code c = j: byte c / 4 (group c / 64), bits 2(c % 4) (plane 0) and 2(c % 4) + 1 (plane 1)
+      const int byte = j >> 2, grp = byte >> 4, bl = byte & 15, u0 = 2 * (j & 3);
+      const int idx = (bl < 8) ? bl * 8 : 64 + (bl - 8) * 8;
+      const float d0 = sm.vacc[grp][hh][idx + u0], d1 = sm.vacc[grp][hh][idx + u0 + 1];
+      v = sm.dv[0][hh] * (a.vc0 * (float)W1 + a.vb0 * d0 + a.vb1 * d1);
+    } else {
+      const int p = j - kD, byte = p >> 3, u = p & 7;
+      const int idx = (byte < 8) ? byte * 8 + u : 64 + (byte - 8) * 8 + u;
+      v = sm.dv[1][hh] * (2.f * sm.vacc[2][hh][idx] - (float)W2);
+    }
+    a.part[(((size_t)b * a.Hq + h0 + hh) * a.nsplit + split) * stride + j] = v;
+  }
+  if (tid < kG) {
+    float l = 0.f;
+    for (int w = 0; w < kWarps; ++w) l += sm.red[w][0][tid];
+    float* o = a.part + (((size_t)b * a.Hq + h0 + tid) * a.nsplit + split) * stride;
+    o[kD + kM] = sm.hmax[tid] * 0.6931471805599453f;   // back to natural-log units
+    o[kD + kM + 1] = l;
   }
 }
 

@@ -522,6 +522,32 @@ void attn_tc_split(int B, int Hkv, int64_t L_cap, int sms, int* nsplit, int64_t*
   *nsplit = (int)((L_cap + ch - 1) / ch);
 }
 
+// The two-kernel 3-bit attention (score kernel, then value kernel) for caches much larger than
+// L2: prod 2+1 handles of the fast path's format, at least 256 MB of packed K and V
+// (TQ_ATTN_2K=1 forces it for any such shape, TQ_ATTN_2K=0 disables it). It needs a scores
+// buffer in the workspace, so it runs only when the caller's workspace holds one.
+bool attn_2k_wanted(const tq_handle* hk, const tq_handle* hv, int B, int Hq, int Hkv, int64_t L_cap) {
+  auto fmt = [](const tq_handle* h) {
+    return h->d == 128 && h->m == 128 && h->bits == 2 && h->norm_dtype == TQ_F16 &&
+           std::fabs(h->cent[3] - h->cent[2] - h->cent[1] + h->cent[0]) < 1e-12;
+  };
+  if (Hkv < 1 || Hq != 4 * Hkv || !fmt(hk) || !fmt(hv)) return false;
+  const char* e = std::getenv("TQ_ATTN_2K");
+  if (e && *e) return *e != '0';
+  return (double)B * Hkv * (double)L_cap * 104.0 >= 256e6;
+}
+
+// Split of its value kernel (three CTAs per SM): about four waves, chunks whole 256-token blocks.
+void attn_2k_split(int B, int Hkv, int64_t L_cap, int sms, int* nsplit, int64_t* chunk) {
+  const int64_t units = std::max<int64_t>(1, (int64_t)B * Hkv);
+  const int64_t ns = std::max<int64_t>(1, (4 * 3 * (int64_t)sms + units - 1) / units);
+  int64_t ch = (L_cap + ns - 1) / ns;
+  ch = std::max<int64_t>(256, (ch + 255) / 256 * 256);
+  if (const int64_t f = splitk_override()) ch = round_chunk(f, 256, 256, (L_cap + 255) / 256 * 256);
+  *chunk = ch;
+  *nsplit = (int)((L_cap + ch - 1) / ch);
+}
+
 void search_split(int nq, int64_t n, int* nchunks, int64_t* chunk) {
   const int64_t qt = (nq + tqk::kSQ - 1) / tqk::kSQ;
   int64_t nc = (2 * 148 + qt - 1) / qt;
@@ -658,8 +684,10 @@ size_t score_ws_layout(const tq_handle* h, int rows, char* base, ScoreWs* w) {
   return off;
 }
 
+// with_2k: room for the two-kernel attention too (its partials and the [B*Hq][L_cap] scores).
 size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, int Hkv, int64_t L_cap,
-                      char* base, ScoreWs* w, float** part, int* nsplit, int64_t* chunk) {
+                      char* base, ScoreWs* w, float** part, int* nsplit, int64_t* chunk, bool with_2k = false,
+                      float** logits = nullptr) {
   size_t off = score_ws_layout(hk, B * Hq, base, w);
   int ns, ns_tc;
   int64_t ch, ch_tc;
@@ -667,9 +695,20 @@ size_t attn_ws_layout(const tq_handle* hk, const tq_handle* hv, int B, int Hq, i
   if (nsplit) *nsplit = ns;
   if (chunk) *chunk = ch;
   if (part) *part = reinterpret_cast<float*>(base + off);
-  // room for the partials of either split (the tcgen05 3-bit kernel has its own)
+  // room for the partials of every split (the tcgen05 3-bit kernel and the two-kernel form have their own)
   attn_tc_split(B, Hkv, L_cap, sm_count(hk->device), &ns_tc, &ch_tc);
-  off += round_up((size_t)B * Hq * std::max(ns, ns_tc) * tqk::partial_stride(hv->d, hv->m) * 4, 256);
+  int ns_max = std::max(ns, ns_tc);
+  if (with_2k) {
+    int ns_2k;
+    int64_t ch_2k;
+    attn_2k_split(B, Hkv, L_cap, sm_count(hk->device), &ns_2k, &ch_2k);
+    ns_max = std::max(ns_max, ns_2k);
+  }
+  off += round_up((size_t)B * Hq * ns_max * tqk::partial_stride(hv->d, hv->m) * 4, 256);
+  if (with_2k) {
+    if (logits) *logits = reinterpret_cast<float*>(base + off);
+    off += round_up((size_t)B * Hq * (size_t)L_cap * 4, 256);
+  }
   return off;
 }
 
@@ -1201,7 +1240,14 @@ size_t tq_score_workspace_bytes(const tq_handle* hk, int B, int Hq) {
 
 size_t tq_attn_workspace_bytes(const tq_handle* hk, const tq_handle* hv, int B, int Hq, int Hkv, int64_t L_cap) {
   if (!hk || !hv || B < 0 || Hq < 1 || Hkv < 1 || L_cap < 1) return 0;
-  return attn_ws_layout(hk, hv, B, Hq, Hkv, L_cap, nullptr, nullptr, nullptr, nullptr, nullptr);
+  return attn_ws_layout(hk, hv, B, Hq, Hkv, L_cap, nullptr, nullptr, nullptr, nullptr, nullptr,
+                        attn_2k_wanted(hk, hv, B, Hq, Hkv, L_cap));
+}
+
+size_t tq_internal_attn_workspace_min_bytes(const tq_handle* hk, const tq_handle* hv, int B, int Hq, int Hkv,
+                                            int64_t L_cap) {
+  if (!hk || !hv || B < 0 || Hq < 1 || Hkv < 1 || L_cap < 1) return 0;
+  return attn_ws_layout(hk, hv, B, Hq, Hkv, L_cap, nullptr, nullptr, nullptr, nullptr, nullptr, false);
 }
 
 size_t tq_search_workspace_bytes(const tq_handle* h, int nq, int64_t n, int k) {
@@ -1269,11 +1315,11 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv, const 
     m.logits = logits; m.err = hk->derr;
     const size_t msmem = sizeof(tqk::amma::ScoreSmem);
     if (once_per_device(10, hk->device)) {
-      cudaFuncSetAttribute(tqk::amma::score_prod2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
-      cudaFuncSetAttribute(tqk::amma::score_prod2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      cudaFuncSetAttribute(tqk::amma::score_prod2_kernel<false>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)msmem);
+      cudaFuncSetAttribute(tqk::amma::score_prod2_kernel<false>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
     }
     KernelScope ks("score", s);
-    const cudaError_t e = launch_pdl(tqk::amma::score_prod2_kernel, dim3((unsigned)units, (unsigned)nsp),
+    const cudaError_t e = launch_pdl(tqk::amma::score_prod2_kernel<false>, dim3((unsigned)units, (unsigned)nsp),
                                      dim3(tqk::amma::kThreads), msmem, s, m);
     if (e != cudaSuccess) return cuda_fail(e, "score_prod2_kernel");
     return launch_check("score_prod2_kernel");
@@ -1314,7 +1360,8 @@ int attn_check(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dt
   if ((st = check_cache(hv, v, "value"))) return st;
   if (k->L_cap != v->L_cap) return fail(TQ_EINVAL, "K and V caches differ in L_cap");
   if (!q || !len || !out || !workspace) return fail(TQ_EINVAL, "NULL pointer");
-  const size_t need = tq_attn_workspace_bytes(hk, hv, B, Hq, Hkv, k->L_cap);
+  // the minimum (without the two-kernel attention's scores buffer, which is used when present)
+  const size_t need = tq_internal_attn_workspace_min_bytes(hk, hv, B, Hq, Hkv, k->L_cap);
   if (ws_bytes < need) return fail(TQ_EINVAL, "workspace %zu < %zu bytes", ws_bytes, need);
   if (!aligned(workspace, 16)) return fail(TQ_EINVAL, "workspace misaligned");
   if (!std::isfinite(scale)) return fail(TQ_EINVAL, "scale is not finite");
@@ -1327,7 +1374,7 @@ int attn_check(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dt
 // advances len[b] once everything that reads it is done.
 int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, int B, int Hq, int Hkv,
               const tq_cache* k, const tq_cache* v, int32_t* len, float scale, float* out, void* workspace,
-              cudaStream_t s, bool fused) {
+              size_t ws_bytes, cudaStream_t s, bool fused) {
   ScoreWs w;
   float* part;
   int nsplit;
@@ -1340,7 +1387,55 @@ int attn_impl(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dty
   a.k = view_of(hk, k); a.v = view_of(hv, v); a.L_cap = k->L_cap; a.chunk = chunk; a.nsplit = nsplit;
   a.len = len; a.len_extra = fused ? 1 : 0; a.scale = scale; a.part = part;
   const int G = Hq / Hkv;
-  if (attn_prod2_fast_path(hk, hv, G, k, v)) {
+  const char* tce0 = std::getenv("TQ_ATTN_TC");
+  const bool tc0 = tce0 && *tce0 && *tce0 != '0';
+  if (!tc0 && attn_prod2_fast_path(hk, hv, G, k, v) && attn_2k_wanted(hk, hv, B, Hq, Hkv, k->L_cap) &&
+      ws_bytes >= attn_ws_layout(hk, hv, B, Hq, Hkv, k->L_cap, nullptr, nullptr, nullptr, nullptr, nullptr, true)) {
+    // two kernels: every key's score (22-bit queries) into the workspace, then the value pass
+    // (timed together as the split attention)
+    float* logits = nullptr;
+    attn_ws_layout(hk, hv, B, Hq, Hkv, k->L_cap, static_cast<char*>(workspace), nullptr, nullptr, nullptr, nullptr,
+                   true, &logits);
+    const int sms = sm_count(hk->device);
+    const int64_t units = (int64_t)B * Hkv;
+    const int64_t target = 8 * 3 * (int64_t)sms;   // scores: about eight waves of 3 CTAs per SM
+    int64_t sch = ((units * k->L_cap + target - 1) / target + 255) / 256 * 256;
+    sch = std::max<int64_t>(256, std::min<int64_t>(sch, (k->L_cap + 255) / 256 * 256));
+    const int64_t nsp = (k->L_cap + sch - 1) / sch;
+    tqk::amma::ScoreArgs ms{};
+    ms.qr = w.qr; ms.qs = w.qs; ms.B = B; ms.Hq = Hq; ms.Hkv = Hkv;
+    ms.kcodes = k->codes; ms.ksigns = k->signs; ms.knorm = static_cast<const __half*>(k->norms);
+    ms.krn = static_cast<const __half*>(k->rnorms);
+    ms.L_cap = k->L_cap; ms.chunk = sch; ms.len = len; ms.len_extra = fused ? 1 : 0;
+    ms.kc0 = (float)hk->cent[0]; ms.kb0 = (float)(hk->cent[1] - hk->cent[0]); ms.kb1 = (float)(hk->cent[2] - hk->cent[0]);
+    ms.logits = logits; ms.err = hk->derr;
+    int64_t vch;
+    attn_2k_split(B, Hkv, k->L_cap, sms, &nsplit, &vch);
+    tqk::amma::VArgs mv{};
+    mv.logits = logits; mv.B = B; mv.Hq = Hq; mv.Hkv = Hkv;
+    mv.vcodes = v->codes; mv.vsigns = v->signs; mv.vnorm = static_cast<const __half*>(v->norms);
+    mv.vrn = static_cast<const __half*>(v->rnorms);
+    mv.L_cap = k->L_cap; mv.chunk = vch; mv.nsplit = nsplit; mv.len = len; mv.len_extra = fused ? 1 : 0;
+    mv.vc0 = (float)hv->cent[0]; mv.vb0 = (float)(hv->cent[1] - hv->cent[0]); mv.vb1 = (float)(hv->cent[2] - hv->cent[0]);
+    mv.scale = scale; mv.part = part; mv.err = hk->derr;
+    const size_t ssmem = sizeof(tqk::amma::ScoreSmem), vsmem = sizeof(tqk::amma::VSmem);
+    if (once_per_device(13, hk->device)) {
+      cudaFuncSetAttribute(tqk::amma::score_prod2_kernel<true>, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)ssmem);
+      cudaFuncSetAttribute(tqk::amma::score_prod2_kernel<true>, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+      cudaFuncSetAttribute(tqk::amma::value_prod2_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)vsmem);
+      cudaFuncSetAttribute(tqk::amma::value_prod2_kernel, cudaFuncAttributePreferredSharedMemoryCarveout, 100);
+    }
+    {
+      KernelScope ks("attn_split", s);
+      cudaError_t e = launch_pdl(tqk::amma::score_prod2_kernel<true>, dim3((unsigned)units, (unsigned)nsp),
+                                 dim3(tqk::amma::kThreads), ssmem, s, ms);
+      if (e != cudaSuccess) return cuda_fail(e, "score_prod2_kernel");
+      e = launch_pdl(tqk::amma::value_prod2_kernel, dim3((unsigned)units, (unsigned)nsplit), dim3(tqk::amma::kThreads),
+                     vsmem, s, mv);
+      if (e != cudaSuccess) return cuda_fail(e, "value_prod2_kernel");
+    }
+    if ((st = launch_check("value_prod2_kernel"))) return st;
+  } else if (attn_prod2_fast_path(hk, hv, G, k, v)) {
     tqk::amma::Args m{};
     // TQ_ATTN_TC=1: the tcgen05 kernel (attn_tc.cuh), measured slower than this mma.sync one at
     // these shapes (each of its small MMAs costs the tensor pipe about as much as a full-width one)
@@ -1463,7 +1558,7 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
   if (st || B == 0) return st;
   if ((st = pre_launch(hk, len, B, k->L_cap, static_cast<cudaStream_t>(stream)))) return st;
   return attn_impl(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, const_cast<int32_t*>(len), scale, out, workspace,
-                   static_cast<cudaStream_t>(stream), false);
+                   ws_bytes, static_cast<cudaStream_t>(stream), false);
 }
 
 int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype, const void* k_new,
@@ -1513,7 +1608,7 @@ int tq_decode_step(const tq_handle* hk, const tq_handle* hv, const void* q, int 
     tqk::decode_prologue_kernel<<<grid, tqk::kSmallThreads, smem, s>>>(p);
   }
   if ((st = launch_check("decode_prologue_kernel"))) return st;
-  return attn_impl(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, len, scale, out, workspace, s, true);
+  return attn_impl(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, len, scale, out, workspace, ws_bytes, s, true);
 }
 
 

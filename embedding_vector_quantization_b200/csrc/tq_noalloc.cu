@@ -43,7 +43,7 @@ extern "C" int tq_attn_decode_noalloc(const tq_handle* hk, const tq_handle* hv, 
   // nothing to attend: tq_attn_decode checks the rest and returns without touching any buffer
   if (B == 0) return tq_attn_decode(hk, hv, q, q_dtype, B, Hq, Hkv, k, v, len, scale, out, nullptr, 0, stream);
   if (!k) return tq_internal_fail(TQ_EINVAL, "tq_attn_decode_noalloc: key cache is NULL");
-  const size_t need = tq_attn_workspace_bytes(hk, hv, B, Hq, Hkv, k->L_cap);
+  const size_t need = tq_internal_attn_workspace_min_bytes(hk, hv, B, Hq, Hkv, k->L_cap);
   if (need == 0) return tq_internal_fail(TQ_EINVAL, "tq_attn_decode_noalloc: invalid shape");
   if (need > kNoAllocScratchBytes)
     return tq_internal_fail(TQ_EINVAL,

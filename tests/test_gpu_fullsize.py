@@ -1,7 +1,7 @@
 """Oracle parity at the full sizes of the bench's workloads, on sampled outputs.
 
 The caches and databases here are full size (the 4-bit decode workload: 4 sequences x 8
-KV heads x 131072 tokens; the streaming score workload: 64 x 8 heads at 16385 keys in
+KV heads x 131072 tokens; the 3-bit big-cache decode workload: 64 x 8 x 16640; the streaming score workload: 64 x 8 heads at 16385 keys in
 16640 slots; the search workload: 1,000,000 vectors at d = 1536, 1024 queries), so the
 kernels run in exactly the launch configuration the bench times. An fp64 encode of that
 many vectors would take minutes, so the packed rows are uniformly random bytes (every bit
@@ -103,6 +103,54 @@ def test_score_prod2_full_size_sampled(tq):
         assert np.all(got[b, hq, Lb:] == 0)
         worst = max(worst, max_rel_score_error(got[b, hq, :Lb], ref, np.linalg.norm(qn[b, hq]), nn, d))
     print(f"score, full size: max relative score error above the floor {worst:.2e}")
+
+
+def test_attn_prod3_big_cache_full_size_sampled(tq):
+    """3-bit prod K and V (m = 128, fp16 norms), 64 sequences x 8 KV heads in 16640 slots (the
+    872 MB cache of the big-cache decode row, which takes the two-kernel path: scores, then
+    values), ragged lengths: every query head of five sampled (sequence, KV head) units against
+    the oracle's attention over the same rows."""
+    B, Hkv, G, Lcap, d = 64, 8, 4, 16640, 128
+    lens = [16385 - (b % 7) * 1501 for b in range(B)]
+    hk, hv = tq.Handle(d, 3, 0, qjl_m=128), tq.Handle(d, 3, 1, qjl_m=128)
+    ohk, ohv = OracleHandle(d, 2, 0, 128), OracleHandle(d, 2, 1, 128)
+    rows = {}
+    caches = []
+    for name, h, seed in (("k", hk, 80), ("v", hv, 90)):
+        codes = workloads.random_rows((B, Hkv, Lcap), 32, seed)
+        signs = workloads.random_rows((B, Hkv, Lcap), 16, seed + 1)
+        n = workloads.random_norms((B, Hkv, Lcap), d, seed + 2)
+        rn = (n.astype(np.float64) * np.random.default_rng(seed + 3).uniform(0.2, 0.5, size=(B, Hkv, Lcap))).astype(
+            np.float16)
+        c = tq.Cache(h, B, Hkv, Lcap)
+        c.codes.copy_(torch.from_numpy(codes))
+        c.signs.copy_(torch.from_numpy(signs))
+        c.norms.copy_(torch.from_numpy(n))
+        c.rnorms.copy_(torch.from_numpy(rn))
+        rows[name] = (codes, signs, n, rn)
+        caches.append(c)
+    q = workloads.queries((B, Hkv * G, d), 85)
+    o = tq.attn_decode(hk, hv, q.cuda(), caches[0], caches[1], torch.tensor(lens, dtype=torch.int32).cuda(),
+                       1.0 / np.sqrt(d)).cpu().numpy()
+    assert hk.status() == tq.TQ_OK
+    del caches
+    worst = 0.0
+    for b, h in ((0, 0), (1, 5), (20, 3), (41, 7), (63, 2)):
+        Lb = lens[b]
+        od = []
+        for name, oh in (("k", ohk), ("v", ohv)):
+            codes, signs, n, rn = rows[name]
+            od.append({"idx": unpack_fast(codes[b, h, :Lb], d, 2)[None, None], "n": n[b, h, :Lb][None, None],
+                       "sigma": unpack_fast(signs[b, h, :Lb], 128, 1)[None, None],
+                       "rnorm": rn[b, h, :Lb][None, None], "Pi": oh.Pi, "S": oh.S, "c": oh.c})
+        qq = q[b:b + 1, h * G:(h + 1) * G].double().numpy()
+        ref = ops.decode_attention(qq, od[0], od[1], [Lb], 1.0 / np.sqrt(d))
+        for g in range(G):
+            nr = np.linalg.norm(ref[0, g])
+            err = np.linalg.norm(o[b, h * G + g] - ref[0, g])
+            worst = max(worst, err / nr)
+            assert err <= ATTN_RTOL * nr, (b, h, g, err / nr)
+    print(f"3-bit attention over the 872 MB cache, full size: max relative error over the sampled heads {worst:.2e}")
 
 
 @pytest.mark.parametrize("bits", [2, 4])
