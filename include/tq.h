@@ -193,7 +193,11 @@ int tq_pack_indices(const tq_handle* h, const uint8_t* idx, int64_t n, uint8_t* 
 int tq_append(const tq_handle* h, const void* x_new, int x_dtype, int B, int Hkv,
               const tq_cache* cache, int32_t* len, int advance, void* stream);
 
-/* Workspace sizes (bytes) for the calls below; 0 is never returned for a valid call. */
+/* Workspace sizes (bytes) for the calls below; 0 is never returned for a valid call.
+ * tq_attn_workspace_bytes is the recommended size: for 3-bit prod caches of 256 MB and
+ * more it includes a [B][Hq][L_cap] fp32 scores buffer for the two-kernel attention
+ * (scores, then values); tq_attn_decode and tq_decode_step accept any workspace of at
+ * least the size without it and then run the single-kernel attention. */
 size_t tq_score_workspace_bytes(const tq_handle* hk, int B, int Hq);
 size_t tq_attn_workspace_bytes(const tq_handle* hk, const tq_handle* hv, int B, int Hq, int Hkv,
                                int64_t L_cap);
@@ -220,7 +224,8 @@ int tq_score(const tq_handle* hk, const float* q, int B, int Hq, int Hkv,
  *  q        device [B][Hq][d] fp32 (q_dtype TQ_F32) or bf16 (TQ_BF16)
  *  k, v     caches of hk and hv (same d; any bits/prod mix)
  *  out      device fp32 [B][Hq][d]; a sequence with len[b] == 0 gets zeros
- *  workspace device scratch of tq_attn_workspace_bytes(hk, hv, B, Hq, Hkv, L_cap) bytes */
+ *  workspace device scratch of tq_attn_workspace_bytes(hk, hv, B, Hq, Hkv, L_cap) bytes
+ *           (see the workspace sizes above for the smaller size that is also accepted) */
 int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int q_dtype,
                    int B, int Hq, int Hkv, const tq_cache* k, const tq_cache* v,
                    const int32_t* len, float scale, float* out,
@@ -233,8 +238,9 @@ int tq_attn_decode(const tq_handle* hk, const tq_handle* hv, const void* q, int 
  * serving loop whose allocator is frozen after start-up. The split-K scratch
  * comes from a fixed 4 MiB array compiled into libtq.so (every GPU that loads
  * the library holds it until the process exits); nothing is allocated.
- *  - A shape whose tq_attn_workspace_bytes exceeds 4 MiB is rejected with
- *    TQ_EINVAL (e.g. B*Hq*nsplit*(d+m+2)*4 bytes of partial sums too large).
+ *  - A shape whose minimum attention workspace (without the two-kernel scores
+ *    buffer) exceeds 4 MiB is rejected with TQ_EINVAL (e.g. B*Hq*nsplit*(d+m+2)*4
+ *    bytes of partial sums too large).
  *  - B == 0 returns TQ_OK without touching any buffer, as tq_attn_decode does.
  *  - The first call on a device looks up the array's device address with that
  *    device current; make that first call before any stream capture. The
