@@ -786,7 +786,8 @@ struct __align__(16) ScoreSmem {
   int abort_flag;
 };
 
-// LO: 22-bit code-side queries (the attention's logits), else 15-bit (raw scores).
+// LO: 22-bit code-side queries and the decode-step slot handling (the two-kernel attention's
+// scores), else 15-bit queries (tq_score's raw scores).
 template <bool LO>
 __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
   extern __shared__ __align__(128) unsigned char smem_raw[];
@@ -795,7 +796,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
   const int g = lane >> 2, t = lane & 3;
   const int bh = blockIdx.x, split = blockIdx.y;
   const int b = bh / a.Hkv, hk = bh % a.Hkv, h0 = hk * kG;
-  const int64_t L = min((int64_t)max(a.len[b], 0) + a.len_extra, a.L_cap);
+  const int64_t L = min((int64_t)max(a.len[b], 0) + (LO ? a.len_extra : 0), a.L_cap);
   const int64_t start = (int64_t)split * a.chunk;
   const int64_t end = min(L, start + a.chunk);
   const int ntok = (int)max((int64_t)0, end - start);
@@ -805,7 +806,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
   // inside a decode step the kernel before this one writes slot len[b]; copies issued before the
   // wait below may hold that key's old rows, so the one warp that scores it reads them again
   const int64_t slot = (int64_t)max(a.len[b], 0);
-  const int s_loc = (a.len_extra && slot >= start && slot < end) ? (int)(slot - start) : -1;
+  const int s_loc = (LO && a.len_extra && slot >= start && slot < end) ? (int)(slot - start) : -1;
 
   if (tid == 0) {
     for (int s = 0; s < kSStages; ++s) {
@@ -864,7 +865,7 @@ __global__ void __launch_bounds__(kThreads, 3) score_prod2_kernel(ScoreArgs a) {
     }
     if (!aborted && !mbar_wait(&sm.full[j % kSStages], (j / kSStages) & 1)) sm.abort_flag = 1;
     const unsigned char* st = sm.stage[j % kSStages];
-    if (!aborted && s_loc >= 0 && s_loc / kBlk == j && warp == ((s_loc % kBlk) % 128) / 16) {
+    if (LO && !aborted && s_loc >= 0 && s_loc / kBlk == j && warp == ((s_loc % kBlk) % 128) / 16) {
       // the warp whose m-tiles hold the appended key (rows 16w.. and 128 + 16w..) patches its rows
       const int kk = s_loc & (kBlk - 1);
       const int64_t r = row0 + s_loc;
