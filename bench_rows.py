@@ -326,7 +326,8 @@ def run_attn3big(args):
     hk = tq.Handle(S5A["d"], S5A["bits"], 0, qjl_m=S5A["m"])
     hv = tq.Handle(S5A["d"], S5A["bits"], 1, qjl_m=S5A["m"])
     # caches of 256 MB and more take the two-kernel form (scores, then values; timed together)
-    two = S5A["B"] * S5A["Hkv"] * S5A["L"] * 104 >= 256e6 and os.environ.get("TQ_ATTN_2K", "") != "0"
+    env2k = os.environ.get("TQ_ATTN_2K", "")
+    two = env2k not in ("", "0") or (env2k == "" and S5A["B"] * S5A["Hkv"] * S5A["L"] * 104 >= 256e6)
     spec = dict(S5A, bytes_per_token=2 * (32 + 16 + 2 + 2),
                 kernel="score_prod2_kernel<true> + value_prod2_kernel" if two else "attn_prod2_kernel",
                 scaled=False,
