@@ -92,14 +92,13 @@ def test_attn_2k_matches_oracle(tq, B, Hkv, lens, force):
 
 def test_attn_2k_decode_step_rereads_the_appended_key(tq):
     """tq_decode_step on the two-kernel path with the appended slot inside a key block whose copy
-    was issued before the append finished: equal to tq_attn_decode over the cache the step
-    leaves behind, and within the tolerance of the oracle over the step's own codes."""
+    was issued before the append finished (the slots hold garbage bytes before the step): equal
+    to tq_attn_decode over the cache the step leaves behind."""
     B, Hkv, Hq, d = 2, 8, 32, 128
     lens0 = [3000, 701]
     hk, hv, kc, vc, kod, vod, q = _case(tq, B, Hkv, [x + 1 for x in lens0], seed=70)
     k_new = workloads.outlier_kv(B, Hkv, 1, d, seed=75)[:, :, 0].contiguous().cuda()
     v_new = workloads.outlier_kv(B, Hkv, 1, d, seed=76)[:, :, 0].contiguous().cuda()
-    # the slots hold the oracle's codes of other tokens: garbage from the step's point of view
     for c in (kc, vc):
         for b, l0 in enumerate(lens0):
             c.codes[b, :, l0].fill_(0xA5)
@@ -118,3 +117,29 @@ def test_attn_2k_decode_step_rereads_the_appended_key(tq):
         again = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens, scale)
     assert hk.status() == tq.TQ_OK and hv.status() == tq.TQ_OK
     assert torch.equal(out, again)
+
+
+def test_attn_2k_needs_the_scores_buffer(tq):
+    """The two-kernel form runs only when the workspace holds its scores buffer: with the
+    minimum workspace (the size asked for when the form is off) the call runs the single-kernel
+    attention and returns exactly its result; with tq_attn_workspace_bytes' size it runs the
+    two kernels (a result that differs in the last bits, within the tolerance)."""
+    B, Hkv, Hq, d = 2, 8, 32, 128
+    lens = [2000, 1500]
+    hk, hv, kc, vc, kod, vod, q = _case(tq, B, Hkv, lens, seed=40)
+    lens_t = torch.tensor(lens, dtype=torch.int32).cuda()
+    L = kc.codes.shape[2]
+    scale = 1.0 / np.sqrt(d)
+    with two_kernels(False):
+        n_min = tq.tq_attn_workspace_bytes(hk.ptr, hv.ptr, B, Hq, Hkv, L)
+        o_single = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens_t, scale)
+    with two_kernels(True):
+        n_two = tq.tq_attn_workspace_bytes(hk.ptr, hv.ptr, B, Hq, Hkv, L)
+        assert n_two >= n_min + B * Hq * L * 4
+        ws_min = torch.empty(n_min, dtype=torch.uint8, device="cuda")
+        o_min = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens_t, scale, workspace=ws_min)
+        o_two = tq.attn_decode(hk, hv, q.cuda(), kc, vc, lens_t, scale)
+    assert hk.status() == tq.TQ_OK and hv.status() == tq.TQ_OK
+    assert torch.equal(o_min, o_single)
+    ref = ops.decode_attention(q.double().numpy(), kod, vod, lens, scale)
+    _check_attention(o_two.cpu().numpy(), ref, lens)
