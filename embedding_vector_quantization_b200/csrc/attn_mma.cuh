@@ -756,7 +756,8 @@ __global__ void __launch_bounds__(kThreads, 2) attn_prod2_kernel(Args a) {
 // written to logits [B][Hq][L_cap] ("TurboQuant: redefining AI efficiency", "QJL";
 // "Google TurboQuant", "Stage 2"). Key blocks of 256 stream through a 5-stage TMA ring;
 // every thread stores its scores directly: per store instruction a warp writes 8
-// consecutive keys of each of the 4 heads, i.e. whole 32-byte sectors.
+// consecutive keys of each of the 4 heads, i.e. whole 32-byte sectors. tq_score runs it with
+// 15-bit code-side queries; the two-kernel attention below with the fused kernel's 22-bit ones.
 
 constexpr int kSStages = 5;   // 5 x 13 KB: three CTAs still fit an SM, three blocks in flight per CTA
 constexpr int kSStageBytes = kStageCodes + kStageSigns + 2 * kBlk * 2;  // codes, signs, norms, rnorms: 13312
